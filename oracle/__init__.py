@@ -1,0 +1,138 @@
+"""CPU oracle for the SALAD hybrid attention layer (fp64, plain C via ctypes).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference leg may import this package.  It shares no
+code with the CUDA library and never imports it.
+
+Functions follow the definitions in ``salad_oracle.c`` (whose header lists the
+SALAD page passages each step follows and the readings taken where the pages
+are silent).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "salad_oracle.c")
+_LIB = os.path.join(_HERE, "libsalad_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
+                               "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        lib.oracle_block_mask.restype = ctypes.c_int64
+        lib.oracle_block_mask.argtypes = [ctypes.c_int] * 5 + [P, P, P, ctypes.c_int64]
+        lib.oracle_linear_state.restype = None
+        lib.oracle_linear_state.argtypes = [P, P] + [ctypes.c_int] * 4 + [P, P]
+        lib.oracle_forward_blocks.restype = None
+        lib.oracle_forward_blocks.argtypes = ([P, P, P] + [ctypes.c_int] * 5 + [P, P, P, P]
+                                              + [ctypes.c_double] * 2 + [P, P, P, ctypes.c_int]
+                                              + [P, P, P])
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def block_mask(T, H, W, block, windows):
+    """Per-head CSR of kept key blocks: (row_ptr int32 [Hh*nb+1], col_idx int32 [nnz])."""
+    windows = np.ascontiguousarray(windows, dtype=np.int32).reshape(-1, 3)
+    Hh = windows.shape[0]
+    nb = (T * H * W + block - 1) // block
+    row_ptr = np.zeros(Hh * nb + 1, dtype=np.int32)
+    lib = _load()
+    nnz = lib.oracle_block_mask(T, H, W, block, Hh, _ptr(windows), _ptr(row_ptr), None, 0)
+    col_idx = np.zeros(max(nnz, 1), dtype=np.int32)
+    nnz2 = lib.oracle_block_mask(T, H, W, block, Hh, _ptr(windows), _ptr(row_ptr),
+                                 _ptr(col_idx), nnz)
+    assert nnz2 == nnz
+    return row_ptr, col_idx[:nnz]
+
+
+def linear_state(k, v):
+    """S fp64 [B*Hh][d][d] and z fp64 [B*Hh][d] over all tokens (bf16-bit inputs)."""
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    B, N, Hh, d = k.shape
+    S = np.zeros((B * Hh, d, d), dtype=np.float64)
+    z = np.zeros((B * Hh, d), dtype=np.float64)
+    _load().oracle_linear_state(_ptr(k), _ptr(v), B, N, Hh, d, _ptr(S), _ptr(z))
+    return S, z
+
+
+def forward_blocks(q, k, v, block, row_ptr, col_idx, w_proj, gate, pairs, tau=None,
+                   eps=1e-6, S=None, z=None, want_branches=False):
+    """Layer output for the listed (b*Hh+h, I) query blocks.
+
+    Returns out fp64 [npairs][block][d] (and o_sp, o_lin when want_branches).
+    Rows of a partial last block past N hold NaN.
+    """
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    B, N, Hh, d = q.shape
+    if tau is None:
+        tau = 1.0 / np.sqrt(d)
+    gate = np.ascontiguousarray(gate, dtype=np.float32).reshape(B, Hh)
+    w_proj = np.ascontiguousarray(w_proj, dtype=np.uint16).reshape(d, d)
+    pairs = np.ascontiguousarray(pairs, dtype=np.int32).reshape(-1, 2)
+    need_lin = want_branches or bool(np.any(gate.reshape(-1)[pairs[:, 0]] != 0))
+    if need_lin and S is None:
+        S, z = linear_state(k, v)
+    n = pairs.shape[0]
+    out = np.full((n, block, d), np.nan, dtype=np.float64)
+    o_sp = np.full_like(out, np.nan) if want_branches else None
+    o_lin = np.full_like(out, np.nan) if want_branches else None
+    _load().oracle_forward_blocks(
+        _ptr(q), _ptr(k), _ptr(v), B, N, Hh, d, block,
+        _ptr(np.ascontiguousarray(row_ptr, dtype=np.int32)),
+        _ptr(np.ascontiguousarray(col_idx, dtype=np.int32)),
+        _ptr(w_proj), _ptr(gate), float(tau), float(eps),
+        _ptr(S), _ptr(z), _ptr(pairs), n, _ptr(out), _ptr(o_sp), _ptr(o_lin))
+    if want_branches:
+        return out, o_sp, o_lin
+    return out
+
+
+def all_pairs(B, Hh, nb):
+    bh, i = np.meshgrid(np.arange(B * Hh), np.arange(nb), indexing="ij")
+    return np.stack([bh.ravel(), i.ravel()], axis=1).astype(np.int32)
+
+
+def forward(q, k, v, block, row_ptr, col_idx, w_proj, gate, tau=None, eps=1e-6,
+            want_branches=False):
+    """Full layer output fp64 [B, N, Hh, d] (every query block)."""
+    B, N, Hh, d = q.shape
+    nb = (N + block - 1) // block
+    pairs = all_pairs(B, Hh, nb)
+    res = forward_blocks(q, k, v, block, row_ptr, col_idx, w_proj, gate, pairs, tau, eps,
+                         want_branches=want_branches)
+    outs = res if want_branches else (res,)
+    full = []
+    for o in outs:
+        o = o.reshape(B, Hh, nb * block, d)[:, :, :N, :]
+        full.append(np.ascontiguousarray(o.transpose(0, 2, 1, 3)))
+    return tuple(full) if want_branches else full[0]

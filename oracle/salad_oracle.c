@@ -1,0 +1,251 @@
+/*
+ * CPU oracle for the SALAD hybrid attention layer.  TEST INFRASTRUCTURE ONLY:
+ * only the tests, the smoke check and the benchmark's CPU-baseline leg may load
+ * this library.  It shares no code with the CUDA path.
+ *
+ * Plain fp64 C, written from the definitions in the SALAD pages:
+ *   - the parallel dual-branch layer and the shared Q/K/V
+ *     (SALAD technical summary, section 2.1 "Architecture design");
+ *   - the sparse branch as static spatio-temporal sliding-window attention
+ *     (ST-SWA, named in Figure 1 of the sciencestack SALAD page and in the
+ *     summary's "Significance" section as "static sparse attention such as a
+ *     sliding window");
+ *   - the ReLU-based O(N) linear branch (summary section 2.1);
+ *   - the static projection on the linear output (summary section 2.2, LWSS);
+ *   - the input-dependent gate in (0,1) on the linear branch (summary section
+ *     2.2, ITADS; sciencestack TL;DR "input-dependent scalar gate");
+ *   - dropping the linear branch when the gate is 0 (summary section 2.3).
+ * The pages give no formula; the readings taken where they are silent are:
+ *   token n <-> (t, y, x) with n = (t*H + y)*W + x; key/query block I holds
+ *   tokens [I*blk, min(N, (I+1)*blk)); block pair (I, J) is kept when some real
+ *   token pair i in I, j in J has |dt| <= wt, |dy| <= wh, |dx| <= ww; softmax
+ *   scale tau (1/sqrt(d) by default); phi = ReLU on q and k; denominator
+ *   phi(q).z + eps; y = o_lin W (row vector times W[c][e]); out = o_sp + g*y,
+ *   with out = o_sp exactly when g == 0.
+ *
+ * Parity pins (tests/test_oracle_*.py): token-pair brute force for the mask,
+ * dense element-masked attention, torch SDPA for the full window, the naive
+ * O(N^2) linear attention, and the closed-form limits.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_to_double(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/*
+ * Block mask.  For every head h and query block I: visit every real token i of
+ * I, every grid point j inside i's window box, and mark the key block holding
+ * j.  The x-extent of the box on one (t, y) row is a contiguous token range, so
+ * the blocks that range touches are marked directly.
+ *
+ * windows: int32 [Hh][3] = (wt, wh, ww).  row_ptr: int32 [Hh*nb + 1], global
+ * offsets into col_idx.  col_idx: int32 [cap] (may be NULL when cap == 0).
+ * Returns the total number of kept block pairs; col_idx is only written when
+ * it fits (the caller compares the return value with cap).
+ */
+int64_t oracle_block_mask(int T, int H, int W, int blk, int Hh, const int32_t *windows,
+                          int32_t *row_ptr, int32_t *col_idx, int64_t cap) {
+    const int64_t N = (int64_t)T * H * W;
+    const int64_t nb = (N + blk - 1) / blk;
+    unsigned char *mark = (unsigned char *)malloc((size_t)(nb * nb));
+    int64_t total = 0;
+    for (int h = 0; h < Hh; ++h) {
+        const int wt = windows[3 * h + 0], wh = windows[3 * h + 1], ww = windows[3 * h + 2];
+        memset(mark, 0, (size_t)(nb * nb));
+#pragma omp parallel for schedule(dynamic)
+        for (int64_t I = 0; I < nb; ++I) {
+            unsigned char *row = mark + I * nb;
+            const int64_t i_end = (I + 1) * blk < N ? (I + 1) * blk : N;
+            for (int64_t i = I * blk; i < i_end; ++i) {
+                const int x = (int)(i % W), y = (int)((i / W) % H), t = (int)(i / ((int64_t)W * H));
+                for (int t2 = t - wt; t2 <= t + wt; ++t2) {
+                    if (t2 < 0 || t2 >= T) continue;
+                    for (int y2 = y - wh; y2 <= y + wh; ++y2) {
+                        if (y2 < 0 || y2 >= H) continue;
+                        const int x_lo = x - ww < 0 ? 0 : x - ww;
+                        const int x_hi = x + ww > W - 1 ? W - 1 : x + ww;
+                        const int64_t base = ((int64_t)t2 * H + y2) * W;
+                        for (int64_t J = (base + x_lo) / blk; J <= (base + x_hi) / blk; ++J)
+                            row[J] = 1;
+                    }
+                }
+            }
+        }
+        for (int64_t I = 0; I < nb; ++I) {
+            row_ptr[h * nb + I] = (int32_t)total;
+            for (int64_t J = 0; J < nb; ++J) {
+                if (mark[I * nb + J]) {
+                    if (col_idx && total < cap) col_idx[total] = (int32_t)J;
+                    ++total;
+                }
+            }
+        }
+    }
+    row_ptr[Hh * nb] = (int32_t)total;
+    free(mark);
+    return total;
+}
+
+/*
+ * Linear-branch state of every (b, h), over all N real tokens (global and
+ * non-causal, as the summary's "global token interaction" says):
+ *   z[c]    = sum_j relu(k_j[c])
+ *   S[c][e] = sum_j relu(k_j[c]) * v_j[e]
+ * q/k/v are bf16 bits [B][N][Hh][d].  S: fp64 [B*Hh][d][d], z: fp64 [B*Hh][d].
+ */
+void oracle_linear_state(const uint16_t *k, const uint16_t *v, int B, int N, int Hh, int d,
+                         double *S, double *z) {
+#pragma omp parallel for schedule(static)
+    for (int bh = 0; bh < B * Hh; ++bh) {
+        const int b = bh / Hh, h = bh % Hh;
+        double *Sb = S + (int64_t)bh * d * d;
+        double *zb = z + (int64_t)bh * d;
+        double *pk = (double *)malloc(sizeof(double) * d);
+        double *pv = (double *)malloc(sizeof(double) * d);
+        for (int64_t i = 0; i < (int64_t)d * d; ++i) Sb[i] = 0.0;
+        for (int c = 0; c < d; ++c) zb[c] = 0.0;
+        for (int64_t j = 0; j < N; ++j) {
+            const int64_t off = (((int64_t)b * N + j) * Hh + h) * d;
+            for (int c = 0; c < d; ++c) {
+                const double kv = bf16_to_double(k[off + c]);
+                pk[c] = kv > 0.0 ? kv : 0.0;
+                pv[c] = bf16_to_double(v[off + c]);
+            }
+            for (int c = 0; c < d; ++c) {
+                zb[c] += pk[c];
+                for (int e = 0; e < d; ++e) Sb[(int64_t)c * d + e] += pk[c] * pv[e];
+            }
+        }
+        free(pk);
+        free(pv);
+    }
+}
+
+/*
+ * Forward pass for a list of (bh, I) query blocks.
+ *   pairs:   int32 [npairs][2] = (b*Hh + h, I)
+ *   S, z:    from oracle_linear_state (may be NULL when every gate of the listed
+ *            pairs is 0)
+ *   w_proj:  bf16 bits [d][d];  gate: float [B][Hh]
+ *   out:     fp64 [npairs][blk][d]; rows past N are left untouched.
+ *   o_sp, o_lin (nullable): same layout, the sparse branch and the normalised
+ *            linear branch before the projection.
+ * For each real query i of the block:
+ *   s_j  = tau * q_i . k_j over all real tokens j of the kept key blocks
+ *   o_sp = sum_j exp(s_j - max s) v_j / sum_j exp(s_j - max s)
+ *   if g == 0: out = o_sp (linear branch dropped)
+ *   else:      u = relu(q_i)^T S, den = relu(q_i) . z, o_lin = u / (den + eps),
+ *              y = o_lin W, out = o_sp + g * y
+ */
+void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int N,
+                           int Hh, int d, int blk, const int32_t *row_ptr, const int32_t *col_idx,
+                           const uint16_t *w_proj, const float *gate, double tau, double eps,
+                           const double *S, const double *z, const int32_t *pairs, int npairs,
+                           double *out, double *o_sp, double *o_lin) {
+    const int nb = (N + blk - 1) / blk;
+    double *W = (double *)malloc(sizeof(double) * d * d);
+    for (int i = 0; i < d * d; ++i) W[i] = bf16_to_double(w_proj[i]);
+#pragma omp parallel for schedule(dynamic)
+    for (int p = 0; p < npairs; ++p) {
+        const int bh = pairs[2 * p], I = pairs[2 * p + 1];
+        const int b = bh / Hh, h = bh % Hh;
+        const double g = (double)gate[bh];
+        const int32_t r0 = row_ptr[h * nb + I], r1 = row_ptr[h * nb + I + 1];
+        /* gather the real key tokens of the kept key blocks, in CSR order */
+        int64_t nkeys = 0;
+        for (int32_t r = r0; r < r1; ++r) {
+            const int64_t J = col_idx[r];
+            const int64_t j_end = (J + 1) * blk < N ? (J + 1) * blk : N;
+            nkeys += j_end - J * blk;
+        }
+        int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (nkeys > 0 ? nkeys : 1));
+        double *s = (double *)malloc(sizeof(double) * (nkeys > 0 ? nkeys : 1));
+        double *qi = (double *)malloc(sizeof(double) * d);
+        double *acc = (double *)malloc(sizeof(double) * d);
+        double *lin = (double *)malloc(sizeof(double) * d);
+        int64_t nk = 0;
+        for (int32_t r = r0; r < r1; ++r) {
+            const int64_t J = col_idx[r];
+            const int64_t j_end = (J + 1) * blk < N ? (J + 1) * blk : N;
+            for (int64_t j = J * blk; j < j_end; ++j) keys[nk++] = j;
+        }
+        const int64_t i_end = (int64_t)(I + 1) * blk < N ? (int64_t)(I + 1) * blk : N;
+        for (int64_t i = (int64_t)I * blk; i < i_end; ++i) {
+            const int64_t qoff = (((int64_t)b * N + i) * Hh + h) * d;
+            for (int c = 0; c < d; ++c) qi[c] = bf16_to_double(q[qoff + c]);
+            /* sparse branch: exact softmax over the kept keys */
+            double m = -INFINITY;
+            for (int64_t t = 0; t < nk; ++t) {
+                const int64_t koff = (((int64_t)b * N + keys[t]) * Hh + h) * d;
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += qi[c] * bf16_to_double(k[koff + c]);
+                s[t] = tau * dot;
+                if (s[t] > m) m = s[t];
+            }
+            double den = 0.0;
+            for (int c = 0; c < d; ++c) acc[c] = 0.0;
+            for (int64_t t = 0; t < nk; ++t) {
+                const double pexp = exp(s[t] - m);
+                const int64_t voff = (((int64_t)b * N + keys[t]) * Hh + h) * d;
+                den += pexp;
+                for (int c = 0; c < d; ++c) acc[c] += pexp * bf16_to_double(v[voff + c]);
+            }
+            const int64_t ooff = ((int64_t)p * blk + (i - (int64_t)I * blk)) * d;
+            for (int c = 0; c < d; ++c) {
+                acc[c] /= den;
+                if (o_sp) o_sp[ooff + c] = acc[c];
+            }
+            /* linear branch, projection and gate */
+            if (g != 0.0 || o_lin) {
+                const double *Sb = S + (int64_t)bh * d * d;
+                const double *zb = z + (int64_t)bh * d;
+                double dn = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    const double pq = qi[c] > 0.0 ? qi[c] : 0.0;
+                    dn += pq * zb[c];
+                }
+                for (int e = 0; e < d; ++e) {
+                    double u = 0.0;
+                    for (int c = 0; c < d; ++c) {
+                        const double pq = qi[c] > 0.0 ? qi[c] : 0.0;
+                        u += pq * Sb[(int64_t)c * d + e];
+                    }
+                    lin[e] = u / (dn + eps);
+                    if (o_lin) o_lin[ooff + e] = lin[e];
+                }
+            }
+            if (g == 0.0) {
+                for (int c = 0; c < d; ++c) out[ooff + c] = acc[c];
+            } else {
+                for (int e = 0; e < d; ++e) {
+                    double y = 0.0;
+                    for (int c = 0; c < d; ++c) y += lin[c] * W[c * d + e];
+                    out[ooff + e] = acc[e] + g * y;
+                }
+            }
+        }
+        free(keys);
+        free(s);
+        free(qi);
+        free(acc);
+        free(lin);
+    }
+    free(W);
+}
+
+/* Threads the OpenMP runtime will use (reported next to the CPU timings). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
