@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the SALAD hybrid attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl salad|reference]
+                    [--workload NAME]
+
+One step = one salad_attn_forward over one batch of the workload (the linear
+branch reduction, then the fused block-sparse attention + linear epilogue).
+Metric: effective TFLOP/s on kept block pairs, sum over (b, h) of
+4 * kept_pairs * d, divided by the step's device time (the layer latency is
+ms_per_step).  Inputs are resident in HBM; L2 is flushed (256 MB write) between
+timed steps, outside the timed events.  Multi-GPU: one process per GPU (launch
+with torch.distributed.run), each rank runs its own batch of the workload
+(weak scaling, no collective on the data path); time = max over ranks.
+
+--impl reference times the CPU oracle (fp64, all host cores) on a bounded sample
+of the same workload; rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import salad_inputs as si  # noqa: E402
+
+METRIC = "hybrid-attn layer latency & effective TFLOP/s (% bf16 TC peak), 32760 tok, 90%"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = si.WAN13B_90.name
+FLUSH_BYTES = 256 << 20
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention-kernel launch,
+# from an ncu capture (see profiles/), keyed by the kernel sources it was taken
+# on; stale entries are ignored.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn.cu", "ptx.cuh"):
+        with open(os.path.join(ROOT, "sparse_linear_hybrid_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def kept_pairs_flops(row_ptr: np.ndarray, col_idx: np.ndarray, wl: si.Workload) -> float:
+    """4 * d * sum over kept (I, J) of |I| * |J| (real tokens), times B."""
+    nb, blk, N = wl.nb, wl.block, wl.N
+    sizes = np.minimum(blk, N - np.arange(nb) * blk).astype(np.float64)
+    rows = np.repeat(np.arange(wl.Hh * nb) % nb, np.diff(row_ptr))
+    pairs = float(np.sum(sizes[rows] * sizes[col_idx]))
+    return 4.0 * wl.d * pairs * wl.B
+
+
+def block_flops(row_ptr, col_idx, wl, pairs):
+    nb, blk, N = wl.nb, wl.block, wl.N
+    sizes = np.minimum(blk, N - np.arange(nb) * blk).astype(np.float64)
+    tot = 0.0
+    for bh, I in pairs:
+        h = int(bh) % wl.Hh
+        r = h * nb + int(I)
+        tot += sizes[I] * float(np.sum(sizes[col_idx[row_ptr[r]:row_ptr[r + 1]]]))
+    return 4.0 * wl.d * tot
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, sampled through NVML while
+    the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # reported, never fatal
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = get_reasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": float(self.max_mhz), "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def config_of(wl: si.Workload, flops: float, nnz: int, world: int):
+    return {"workload": wl.name, "B": wl.B, "heads": wl.Hh, "d": wl.d,
+            "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.N, "block": wl.block,
+            "window_thw": list(wl.window), "block_sparsity": round(1 - nnz / (wl.Hh * wl.nb ** 2), 5),
+            "kept_gflop_per_step": round(flops / 1e9, 3), "parallelism": f"replicas{world}",
+            "l2": "flushed between steps (256 MB write outside the timed events)"}
+
+
+# --------------------------------------------------------------------------- oracle legs
+def oracle_sample_rate(wl, inp, row_ptr, col_idx, budget_s, seed=0):
+    """The CPU oracle on a bounded sample: S and z of every (b, h) once, then
+    seeded query blocks until `budget_s` of forward time.  Returns
+    (TFLOP/s, cores, sample description, seconds charged per sample)."""
+    import oracle
+    t0 = time.perf_counter()
+    S, z = oracle.linear_state(inp.k, inp.v)
+    t_lin = time.perf_counter() - t0
+    total = kept_pairs_flops(row_ptr, col_idx, wl)
+    rng = np.random.default_rng(seed)
+    order = np.stack(np.unravel_index(rng.permutation(wl.B * wl.Hh * wl.nb), (wl.B * wl.Hh, wl.nb)), 1)
+    cores = oracle.num_threads()
+    done, t_fwd, flops = 0, 0.0, 0.0
+    while done < len(order) and t_fwd < budget_s:
+        batch = order[done:done + max(cores, 4)].astype(np.int32)
+        t1 = time.perf_counter()
+        oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate, batch,
+                              S=S, z=z)
+        t_fwd += time.perf_counter() - t1
+        flops += block_flops(row_ptr, col_idx, wl, batch)
+        done += len(batch)
+    frac = flops / total
+    charged = t_fwd + t_lin * frac
+    desc = (f"{done} of {len(order)} query blocks ({100 * frac:.2f}% of kept FLOPs) + the linear-branch state "
+            f"of all heads ({t_lin:.2f}s, charged pro rata)")
+    return flops / charged / 1e12, cores, desc, charged, done
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    inp = si.make_inputs(wl)
+    row_ptr, col_idx = oracle.block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)
+    flops_step = kept_pairs_flops(row_ptr, col_idx, wl)
+    _t = time
+    t0 = _t.perf_counter()
+    S, z = oracle.linear_state(inp.k, inp.v)
+    t_lin = _t.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    order = np.stack(np.unravel_index(rng.permutation(wl.B * wl.Hh * wl.nb), (wl.B * wl.Hh, wl.nb)), 1)
+    cores = oracle.num_threads()
+    # size one step so the whole run stays within about two minutes
+    step_budget = max(0.05, min(1.0, 120.0 / max(1, args.steps + args.warmup)))
+    per = max(cores, 4)
+    t1 = _t.perf_counter()
+    oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate,
+                          order[:per].astype(np.int32), S=S, z=z)
+    per_block = (_t.perf_counter() - t1) / per
+    m = int(max(1, min(len(order), step_budget / max(per_block, 1e-6))))
+    times, flops_list = [], []
+    pos = per
+    for i in range(args.warmup + args.steps):
+        if pos + m > len(order):
+            pos = 0
+        batch = order[pos:pos + m].astype(np.int32)
+        pos += m
+        t1 = _t.perf_counter()
+        oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate, batch,
+                              S=S, z=z)
+        dt = _t.perf_counter() - t1
+        fl = block_flops(row_ptr, col_idx, wl, batch)
+        if i >= args.warmup:
+            times.append(dt + t_lin * fl / flops_step)
+            flops_list.append(fl)
+    value = sum(flops_list) / sum(times) / 1e12
+    desc = (f"{m} query blocks per step (seeded, cycling over all {len(order)}) with the linear-branch state of "
+            f"all heads ({t_lin:.2f}s) charged pro rata to their kept FLOPs")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * flops_step / (value * 1e12), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, flops_step, int(row_ptr[-1]), world),
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU leg
+def run_salad(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_linear_hybrid_b200 as sl
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    my_wl = wl.with_(seed=wl.seed + 1000 * rank)
+    inp = si.make_inputs(my_wl)
+
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v, w = up(inp.q), up(inp.k), up(inp.v), up(inp.w_proj)
+    gate = torch.from_numpy(inp.gate).to(dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    row_ptr, col_idx = sl.build_block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows, device=dev)
+    torch.cuda.synchronize()
+    mask_ms = 1e3 * (time.perf_counter() - t0)
+    rp_h, ci_h = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
+    flops = kept_pairs_flops(rp_h, ci_h, wl)
+    nnz = int(rp_h[-1])
+    ws = sl.new_workspace(wl.B, wl.N, wl.Hh, wl.d, dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        sl.attn_forward(q, k, v, row_ptr, col_idx, w, gate, wl.block, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert sl.check_status(ws) == sl.SALAD_OK
+
+    K = args.steps
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev = [(E(), E(), E(), E(), E()) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    with clocks:
+        for i in range(K):
+            flush.zero_()
+            e_start, e_lin, e_att, e_end, e_stop = ev[i]
+            sl.set_phase_events(e_lin, e_att, e_end)
+            e_start.record()
+            step()
+            e_stop.record()
+        torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier()
+    sl.set_phase_events()
+    status = sl.check_status(ws)
+    if status != sl.SALAD_OK:
+        raise RuntimeError(f"device status after the timed steps: {sl.status_string(status)}")
+    step_ms = [a.elapsed_time(b) for a, _, _, _, b in ev]
+    lin_ms = [b.elapsed_time(c) for _, b, c, _, _ in ev]
+    att_ms = [c.elapsed_time(d) for _, _, c, d, _ in ev]
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / K
+    value = world * K * flops / (total_ms / 1e3) / 1e12
+
+    peaks = load_peaks()
+    timed_s = sum(step_ms) / 1e3
+    use_sustained = timed_s > 2.0
+    peak = peaks["bf16_sustained"] if use_sustained else peaks["bf16"]
+    att_avg_ms = statistics.fmean(att_ms)
+    achieved = flops / (att_avg_ms / 1e3) / 1e12
+    src_hash = kernel_source_hash()
+    trec = NCU_TRAFFIC.get(wl.name)
+    traffic = trec["bytes"] if trec and trec.get("source") == src_hash else None
+    roofline = {"bound": "tensor", "kernel": "salad_attn_kernel", "achieved": round(achieved, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_kind": f"{'sustained' if use_sustained else 'burst'} bf16 cuBLAS, of {peaks['source']}",
+                "algorithmic": "4*d*kept_pairs per launch (all heads)", "ms_per_launch": round(att_avg_ms, 4)}
+    kv_bytes = 2 * wl.B * wl.N * wl.Hh * wl.d * 2
+    lin_avg_ms = statistics.fmean(lin_ms)
+    kernels = {
+        "linear_reduce": {"ms_per_launch_pair": round(lin_avg_ms, 4),
+                          "achieved_gbs": round(kv_bytes / (lin_avg_ms / 1e3) / 1e9, 1),
+                          "peak_gbs": peaks["hbm_gbs"],
+                          "frac": round(kv_bytes / (lin_avg_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                          "algorithmic": "K and V read once: 4*d bytes per token per (b,h)"},
+        "mask_build_ms_once": round(mask_ms, 3),
+        "attention_ms_p10_p50_p90": [round(float(np.percentile(att_ms, p)), 4) for p in (10, 50, 90)],
+    }
+
+    # end to end through the C ABI with host buffers: H2D of the step's inputs
+    # from pinned memory, the forward, D2H of the output, all inside the events
+    pin = {n: t.cpu().pin_memory() for n, t in dict(q=q, k=k, v=v, w=w, gate=gate).items()}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    ke = max(3, min(K, 20))
+    e2e_ev = [(E(), E()) for _ in range(ke + 2)]
+    barrier()
+    for i in range(ke + 2):
+        flush.zero_()
+        a, b = e2e_ev[i]
+        a.record()
+        q.copy_(pin["q"], non_blocking=True)
+        k.copy_(pin["k"], non_blocking=True)
+        v.copy_(pin["v"], non_blocking=True)
+        w.copy_(pin["w"], non_blocking=True)
+        gate.copy_(pin["gate"], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        b.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev[2:]))
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = out_h.numel() * out_h.element_size()
+    e2e = {"value": round(world * ke * flops / (e2e_ms / 1e3) / 1e12, 3), "unit": UNIT,
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+           "ms_per_step": round(e2e_ms / ke, 3)}
+    del pin, out_h
+
+    dense = None
+    if not args.no_dense:
+        dwl = wl.with_(window=(wl.T, wl.H, wl.W))
+        drp, dci = sl.build_block_mask(dwl.T, dwl.H, dwl.W, dwl.block, dwl.windows(), device=dev)
+        zero_gate = torch.zeros_like(gate)
+        dflops = kept_pairs_flops(drp.cpu().numpy(), dci.cpu().numpy(), dwl)
+        dev_ev = [(E(), E()) for _ in range(5)]
+        for i in range(6):
+            flush.zero_()
+            if i > 0:
+                dev_ev[i - 1][0].record()
+            sl.attn_forward(q, k, v, drp, dci, w, zero_gate, wl.block, out=out, workspace=ws)
+            if i > 0:
+                dev_ev[i - 1][1].record()
+        torch.cuda.synchronize()
+        dms = statistics.fmean(a.elapsed_time(b) for a, b in dev_ev)
+        dense = {"window_thw": list(dwl.window), "gate": 0.0, "ms_per_step": round(dms, 3),
+                 "tflops": round(dflops / (dms / 1e3) / 1e12, 2),
+                 "sparse_speedup_vs_dense": round(dms / ms_per_step, 3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, desc, _, _ = oracle_sample_rate(wl, inp, rp_h, ci_h, budget_s=args.cpu_seconds)
+        cpu = {"value": round(rate, 6), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_of(wl, flops, nnz, world),
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * K,
+                "clocks": clocks.summary(), "kernels": kernels, "dense": dense,
+                "wall_ms_per_step_incl_flush": round(1e3 * wall / K, 4),
+                "frac_of_bf16_peak_layer": round(value / world / peak, 4),
+                "kernel_source": src_hash}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["salad", "reference"], default="salad")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(si.WORKLOADS))
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-window comparison run")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle forward budget for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = si.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_salad(args, wl)
+
+
+if __name__ == "__main__":
+    main()

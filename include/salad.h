@@ -1,0 +1,162 @@
+/*
+ * salad.h - C ABI of libsalad, a B200 (sm_100a) implementation of the SALAD
+ * hybrid attention layer of a video diffusion transformer:
+ *
+ *   out = SparseAttn_STSWA(q, k, v) + g[b,h] * ( LinAttn_ReLU(q, k, v) . W )
+ *
+ * Sources, all on the SALAD pages: the parallel sparse + linear branches that
+ * share Q/K/V (SALAD technical summary, section 2.1 "Architecture design";
+ * sciencestack abstract and Figure 3, the SALAD module overview);
+ * ST-SWA static sparsity (sciencestack Figure 1; summary section 5); ReLU
+ * linear attention of O(N) cost (summary section 2.1); the learnable projection
+ * that down-weights the linear output (summary section 2.2, LWSS); the
+ * scalar gate in (0,1) that depends on the input (summary section 2.2, ITADS;
+ * sciencestack TL;DR); dropping the linear branch when its gate is negligible
+ * (summary section 2.3).
+ *
+ * Conventions shared by every call:
+ *   - Token n of a T x H x W latent grid is (t, y, x) with n = (t*H + y)*W + x.
+ *   - Tensors q, k, v, out are bf16, contiguous [B][N][Hh][d] (head-interleaved,
+ *     as a DiT's fused QKV projection writes them).
+ *   - Block I holds tokens [I*block, min(N, (I+1)*block)); nb = ceil(N/block).
+ *   - All device pointers are caller-owned; the library never allocates device
+ *     memory and keeps no state between calls apart from cached driver entry
+ *     points.  Calls are asynchronous on `stream` unless stated otherwise.
+ *   - Every entry point returns a salad_status; argument errors are detected on
+ *     the host before anything is launched.
+ */
+#ifndef SALAD_H_
+#define SALAD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* salad_stream_t;
+
+typedef enum {
+  SALAD_OK = 0,
+  SALAD_ERR_INVALID_ARG = -1,    /* null/misaligned pointer, bad size or window */
+  SALAD_ERR_UNSUPPORTED = -2,    /* valid but not built: d or block not in {64,128}, ... */
+  SALAD_ERR_CAPACITY = -3,       /* col_idx too small for the mask (see nnz_out) */
+  SALAD_ERR_WORKSPACE = -4,      /* workspace smaller than salad_workspace_bytes() */
+  SALAD_ERR_CUDA = -5,           /* a CUDA runtime/driver call or launch failed */
+  SALAD_ERR_DEVICE_TIMEOUT = -6  /* a kernel gave up waiting (see salad_check_status) */
+} salad_status;
+
+/*
+ * Number of blocks nb = ceil(T*H*W / block).  Host only.
+ * Errors: INVALID_ARG for non-positive sizes, N >= 2^31 or nb == NULL.
+ */
+int salad_mask_num_blocks(int T, int H, int W, int block, int* nb);
+
+/*
+ * Static spatio-temporal sliding-window block mask (ST-SWA: sciencestack
+ * Figure 1; the SPADE page's 3-D grid of video blocks describes the same
+ * T x H x W block structure).  For every head h and query block I it lists, in
+ * ascending order, the key blocks J for which SOME real token pair i in I,
+ * j in J satisfies |t_i - t_j| <= wt, |y_i - y_j| <= wh, |x_i - x_j| <= ww.
+ *
+ *   windows   HOST int32 [num_heads][3] = (wt, wh, ww), inclusive half-widths,
+ *             each >= 0.
+ *   row_ptr   DEVICE int32 [num_heads*nb + 1]: row (h, I) is
+ *             col_idx[row_ptr[h*nb+I] .. row_ptr[h*nb+I+1]); offsets are global.
+ *   col_idx   DEVICE int32 [col_capacity]; may be NULL when col_capacity == 0.
+ *   nnz_out   HOST, nullable: receives the total number of kept pairs.
+ * The call synchronises `stream` once (to read the count) and is meant to run
+ * once per (grid, block, windows), outside any timed or captured region.
+ * Errors: INVALID_ARG (sizes, negative window, null row_ptr, num_heads outside
+ * [1, 256]); CAPACITY when col_capacity < nnz (row_ptr is then complete,
+ * col_idx untouched, *nnz_out set); CUDA.
+ */
+int salad_build_block_mask(int T, int H, int W, int block, int num_heads, const int32_t* windows,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int64_t* nnz_out,
+                           salad_stream_t stream);
+
+/*
+ * Bytes of device workspace salad_attn_forward needs for these sizes (0 on bad
+ * arguments).  The workspace holds a status word, the linear-branch state
+ * [S | z] of every (b, h) and the split-N partial sums.  It must be zero-filled
+ * once after allocation (the status word must start at 0); calls leave it
+ * reusable.  One workspace must not be shared by calls that may overlap.
+ */
+size_t salad_workspace_bytes(int B, int N, int num_heads, int d);
+
+/*
+ * The SALAD layer forward (sciencestack abstract and Figure 3; summary
+ * sections 2.1-2.3):
+ *   o_sp_i  = sum_{j in K(i)} softmax_j(scale * q_i . k_j) v_j, where K(i) is
+ *             every real token of the key blocks kept for i's query block
+ *   S, z    = sum_j relu(k_j) v_j^T (d x d),  sum_j relu(k_j)   over all N
+ *   o_lin_i = relu(q_i)^T S / (relu(q_i) . z + eps)
+ *   out_i   = o_sp_i + g[b,h] * (o_lin_i W)      (y_e = sum_c o_lin_c W[c][e])
+ * When g[b,h] == 0 the linear branch of (b, h) is skipped entirely and
+ * out_i = o_sp_i exactly (branch dropping).
+ *
+ *   q, k, v      DEVICE bf16 [B][N][Hh][d], 16-byte aligned.
+ *   d            64 or 128.   block: 64 or 128.   Hh*d*2 bytes % 16 == 0.
+ *   row_ptr, col_idx  DEVICE, from salad_build_block_mask with the same N
+ *                (= T*H*W), block and num_heads; columns ascending.
+ *   w_proj       DEVICE bf16 [d][d] (row c, column e), 16-byte aligned.
+ *   gate         DEVICE fp32 [B][Hh].
+ *   softmax_scale  <= 0 selects 1/sqrt(d).   eps: added to the denominator.
+ *   out          DEVICE bf16 [B][N][Hh][d], 16-byte aligned; may not alias q/k/v.
+ *   workspace    DEVICE, >= salad_workspace_bytes(B, N, Hh, d), 256-byte aligned.
+ * Never synchronises.  Arithmetic: bf16 tensor-core products with fp32
+ * accumulation, fp32 softmax, one round-to-nearest-even to bf16 at the store.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA (launch failures).  A
+ * device-side time-out is reported later by salad_check_status.
+ */
+int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                       int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                       const float* gate, float softmax_scale, float eps, void* out, void* workspace,
+                       size_t workspace_bytes, salad_stream_t stream);
+
+/*
+ * The linear-branch state alone (summary section 2.1: ReLU linear attention),
+ * computed by the same kernels salad_attn_forward uses:
+ *   S_out  DEVICE fp32 [B*Hh][d][d], S[c][e] = sum_j relu(k_j[c]) v_j[e]
+ *   z_out  DEVICE fp32 [B*Hh][d],    z[c]    = sum_j relu(k_j[c])
+ *   gate   DEVICE fp32 [B][Hh] or NULL; (b, h) with gate 0 are skipped and their
+ *          S/z rows are left untouched.
+ * Same workspace rules as salad_attn_forward.  Errors as salad_attn_forward.
+ */
+int salad_linear_state(const void* k, const void* v, int B, int N, int num_heads, int d, const float* gate,
+                       float* S_out, float* z_out, void* workspace, size_t workspace_bytes,
+                       salad_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the workspace status word.
+ * Returns SALAD_ERR_DEVICE_TIMEOUT if a kernel of an earlier call gave up on a
+ * bounded wait (its output is then invalid), SALAD_ERR_CUDA if the stream
+ * reports an error, SALAD_OK otherwise.
+ */
+int salad_check_status(void* workspace, salad_stream_t stream);
+
+/*
+ * Test hook: the longest time, in nanoseconds, a kernel waits on a pipeline
+ * barrier before it records SALAD_ERR_DEVICE_TIMEOUT and returns.  The default
+ * is 2 s; 0 makes every wait that is not already satisfied fail at once.
+ * Affects launches made after the call (host-global setting).
+ */
+void salad_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * Profiling hook: caller-owned CUDA events (cudaEvent_t, passed as void*) that
+ * subsequent salad_attn_forward calls record on their stream before the
+ * linear-branch kernels, before the attention kernel and after it.  Pass NULLs
+ * to stop.  Host-global setting; it changes no result.
+ */
+void salad_set_phase_events(void* before_linear, void* before_attention, void* after_attention);
+
+const char* salad_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SALAD_H_ */

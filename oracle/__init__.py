@@ -23,9 +23,9 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (-O2, OpenMP, no fast-math)."""
+    """Compile the oracle with gcc (-O3, OpenMP, no fast-math: IEEE fp64 in source order)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
+        subprocess.check_call(["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c99",
                                "-o", _LIB, _SRC, "-lm"])
     return _LIB
 

@@ -7,13 +7,13 @@
  *   - the parallel dual-branch layer and the shared Q/K/V
  *     (SALAD technical summary, section 2.1 "Architecture design");
  *   - the sparse branch as static spatio-temporal sliding-window attention
- *     (ST-SWA, named in Figure 1 of the sciencestack SALAD page and in the
- *     summary's "Significance" section as "static sparse attention such as a
- *     sliding window");
+ *     (ST-SWA, a baseline in Figure 1 of the sciencestack SALAD page; the
+ *     summary's section 5 names sliding windows as the static kind of sparse
+ *     attention the method applies to);
  *   - the ReLU-based O(N) linear branch (summary section 2.1);
  *   - the static projection on the linear output (summary section 2.2, LWSS);
- *   - the input-dependent gate in (0,1) on the linear branch (summary section
- *     2.2, ITADS; sciencestack TL;DR "input-dependent scalar gate");
+ *   - a scalar gate in (0,1) that depends on the input and scales the linear
+ *     branch (summary section 2.2, ITADS; the sciencestack TL;DR);
  *   - dropping the linear branch when the gate is 0 (summary section 2.3).
  * The pages give no formula; the readings taken where they are silent are:
  *   token n <-> (t, y, x) with n = (t*H + y)*W + x; key/query block I holds
@@ -95,7 +95,8 @@ int64_t oracle_block_mask(int T, int H, int W, int blk, int Hh, const int32_t *w
 
 /*
  * Linear-branch state of every (b, h), over all N real tokens (global and
- * non-causal, as the summary's "global token interaction" says):
+ * non-causal: the summary's section 2.1 gives the linear branch the job of
+ * interactions between all tokens):
  *   z[c]    = sum_j relu(k_j[c])
  *   S[c][e] = sum_j relu(k_j[c]) * v_j[e]
  * q/k/v are bf16 bits [B][N][Hh][d].  S: fp64 [B*Hh][d][d], z: fp64 [B*Hh][d].
@@ -119,6 +120,7 @@ void oracle_linear_state(const uint16_t *k, const uint16_t *v, int B, int N, int
                 pv[c] = bf16_to_double(v[off + c]);
             }
             for (int c = 0; c < d; ++c) {
+                if (pk[c] == 0.0) continue; /* relu(k) = 0 adds exact zeros */
                 zb[c] += pk[c];
                 for (int e = 0; e < d; ++e) Sb[(int64_t)c * d + e] += pk[c] * pv[e];
             }

@@ -4,10 +4,10 @@ This module is shared by the tests, the benchmark and the CPU oracle's callers.
 It draws random numbers and rounds them to bf16; it holds none of the
 method's arithmetic (no attention, no mask logic).
 
-Workloads follow the video-DiT shapes the SALAD pages quote (Wan2.1-1.3B and
-Wan2.1-14B, SALAD technical summary section 4 "Results"): latent token grids
-T x H x W in raster order, 12 or 40 heads of width 128, and block sparsity near
-90% (SALAD summary section 3, "90% sparsity").  No dataset or trained weight is
+Workloads follow the video-DiT models the SALAD pages evaluate (Wan2.1-1.3B and
+Wan2.1-14B, SALAD technical summary section 4): latent token grids T x H x W in
+raster order, 12 or 40 heads of width 128, and block sparsity near the 90% the
+summary's section 3 reports.  No dataset or trained weight is
 involved: every tensor is drawn from the distributions below.
 
 Recipe (numpy PCG64 ``default_rng(seed)``, float32 draws, in this order):
@@ -136,15 +136,17 @@ def make_inputs(wl: Workload, v_mean: float = 0.0, gate: float | None = None,
                   w_proj=f32_to_bf16_bits(w), gate=g, windows=wl.windows())
 
 
-def sample_query_blocks(wl: Workload, per_bh: int = 32, seed: int = 12345) -> np.ndarray:
-    """Query blocks to check at full size: every block of the first and the last
-    (b, h), plus ``per_bh`` seeded random blocks of every (b, h) including the
-    last (possibly partial) block.  Returns int32 [n, 2] of (b*Hh + h, I)."""
+def sample_query_blocks(wl: Workload, per_bh: int = 32, full_first_last: bool = True,
+                        seed: int = 12345) -> np.ndarray:
+    """Query blocks to check at full size: (optionally) every block of the first
+    and the last (b, h), plus ``per_bh`` seeded random blocks of every (b, h)
+    and the last (possibly partial) block of each.  Returns int32 [n, 2] of
+    (b*Hh + h, I)."""
     rng = np.random.default_rng(seed)
     BH, nb = wl.B * wl.Hh, wl.nb
     pairs = set()
     for bh in range(BH):
-        if bh in (0, BH - 1):
+        if full_first_last and bh in (0, BH - 1):
             pairs.update((bh, i) for i in range(nb))
         else:
             picks = rng.choice(nb, size=min(per_bh, nb), replace=False)

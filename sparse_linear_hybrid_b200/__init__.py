@@ -1,0 +1,189 @@
+"""Python binding of libsalad, the SALAD hybrid attention layer for B200.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``libsalad.so`` (built by ``python -m sparse_linear_hybrid_b200.build``).
+PyTorch supplies device memory and streams.  There is no CPU fallback: calls
+raise if the library is missing or a tensor is not on a CUDA device.
+
+The entry points mirror ``include/salad.h``:
+    mask_num_blocks, build_block_mask, workspace_bytes, attn_forward,
+    linear_state, check_status, set_wait_limit_ns, set_phase_events, status_string
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsalad.so")
+_lib = None
+
+SALAD_OK = 0
+SALAD_ERR_INVALID_ARG = -1
+SALAD_ERR_UNSUPPORTED = -2
+SALAD_ERR_CAPACITY = -3
+SALAD_ERR_WORKSPACE = -4
+SALAD_ERR_CUDA = -5
+SALAD_ERR_DEVICE_TIMEOUT = -6
+
+
+class SaladError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsalad.so (raises when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_linear_hybrid_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i, p, f, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+        L.salad_mask_num_blocks.argtypes = [i, i, i, i, ctypes.POINTER(i)]
+        L.salad_mask_num_blocks.restype = i
+        L.salad_build_block_mask.argtypes = [i, i, i, i, i, p, p, p, ctypes.c_int64,
+                                             ctypes.POINTER(ctypes.c_int64), p]
+        L.salad_build_block_mask.restype = i
+        L.salad_workspace_bytes.argtypes = [i, i, i, i]
+        L.salad_workspace_bytes.restype = sz
+        L.salad_attn_forward.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
+        L.salad_attn_forward.restype = i
+        L.salad_linear_state.argtypes = [p, p, i, i, i, i, p, p, p, p, sz, p]
+        L.salad_linear_state.restype = i
+        L.salad_check_status.argtypes = [p, p]
+        L.salad_check_status.restype = i
+        L.salad_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.salad_set_wait_limit_ns.restype = None
+        L.salad_set_phase_events.argtypes = [p, p, p]
+        L.salad_set_phase_events.restype = None
+        L.salad_status_string.argtypes = [i]
+        L.salad_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().salad_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != SALAD_OK:
+        raise SaladError(status, what)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor, dtype, name: str) -> ctypes.c_void_p:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (libsalad has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def mask_num_blocks(T: int, H: int, W: int, block: int) -> int:
+    nb = ctypes.c_int(0)
+    _check(lib().salad_mask_num_blocks(T, H, W, block, ctypes.byref(nb)), "salad_mask_num_blocks")
+    return nb.value
+
+
+def build_block_mask(T: int, H: int, W: int, block: int, windows, device=None, stream=None):
+    """ST-SWA block mask as a per-head CSR: (row_ptr, col_idx) int32 CUDA tensors."""
+    win = np.ascontiguousarray(windows, dtype=np.int32).reshape(-1, 3)
+    heads = win.shape[0]
+    nb = mask_num_blocks(T, H, W, block)
+    device = torch.device("cuda") if device is None else torch.device(device)
+    row_ptr = torch.empty(heads * nb + 1, dtype=torch.int32, device=device)
+    nnz = ctypes.c_int64(0)
+    s = _stream(stream)
+    st = lib().salad_build_block_mask(T, H, W, block, heads, win.ctypes.data_as(ctypes.c_void_p),
+                                      _dev_ptr(row_ptr, torch.int32, "row_ptr"), None, 0,
+                                      ctypes.byref(nnz), s)
+    if st not in (SALAD_OK, SALAD_ERR_CAPACITY):
+        _check(st, "salad_build_block_mask")
+    col_idx = torch.empty(max(int(nnz.value), 1), dtype=torch.int32, device=device)
+    _check(lib().salad_build_block_mask(T, H, W, block, heads, win.ctypes.data_as(ctypes.c_void_p),
+                                        _dev_ptr(row_ptr, torch.int32, "row_ptr"),
+                                        _dev_ptr(col_idx, torch.int32, "col_idx"),
+                                        col_idx.numel(), ctypes.byref(nnz), s),
+           "salad_build_block_mask")
+    return row_ptr, col_idx[:int(nnz.value)]
+
+
+def workspace_bytes(B: int, N: int, heads: int, d: int) -> int:
+    n = lib().salad_workspace_bytes(B, N, heads, d)
+    if n == 0:
+        raise SaladError(SALAD_ERR_INVALID_ARG, "salad_workspace_bytes")
+    return int(n)
+
+
+def new_workspace(B: int, N: int, heads: int, d: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace of the size salad_attn_forward needs."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    return torch.zeros(workspace_bytes(B, N, heads, d), dtype=torch.uint8, device=device)
+
+
+def attn_forward(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_scale: float = 0.0,
+                 eps: float = 1e-6, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """out = sparse ST-SWA attention + gate * (ReLU linear attention @ w_proj).
+
+    q, k, v: bf16 CUDA [B, N, Hh, d]; w_proj bf16 [d, d]; gate fp32 [B, Hh].
+    """
+    B, N, Hh, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = new_workspace(B, N, Hh, d, q.device)
+    _check(lib().salad_attn_forward(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
+        B, N, Hh, d, block, _dev_ptr(row_ptr, torch.int32, "row_ptr"),
+        _dev_ptr(col_idx, torch.int32, "col_idx"), _dev_ptr(w_proj, torch.bfloat16, "w_proj"),
+        _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps),
+        _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream)), "salad_attn_forward")
+    return out
+
+
+def linear_state(k, v, gate=None, workspace=None, stream=None):
+    """(S fp32 [B*Hh, d, d], z fp32 [B*Hh, d]) of the ReLU linear branch."""
+    B, N, Hh, d = k.shape
+    if workspace is None:
+        workspace = new_workspace(B, N, Hh, d, k.device)
+    S = torch.zeros(B * Hh, d, d, dtype=torch.float32, device=k.device)
+    z = torch.zeros(B * Hh, d, dtype=torch.float32, device=k.device)
+    g = None if gate is None else _dev_ptr(gate, torch.float32, "gate")
+    _check(lib().salad_linear_state(
+        _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"), B, N, Hh, d, g,
+        _dev_ptr(S, torch.float32, "S"), _dev_ptr(z, torch.float32, "z"),
+        _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "salad_linear_state")
+    return S, z
+
+
+def check_status(workspace, stream=None) -> int:
+    """Synchronise and return (and clear) the workspace status; see salad.h."""
+    return int(lib().salad_check_status(_dev_ptr(workspace, torch.uint8, "workspace"), _stream(stream)))
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    lib().salad_set_wait_limit_ns(int(limit_ns))
+
+
+def set_phase_events(before_linear=None, before_attention=None, after_attention=None) -> None:
+    """Record these torch.cuda.Event objects inside later attn_forward calls
+    (before the linear-branch kernels, before and after the attention kernel)."""
+    h = [None if e is None else ctypes.c_void_p(e.cuda_event)
+         for e in (before_linear, before_attention, after_attention)]
+    lib().salad_set_phase_events(*h)

@@ -1,0 +1,273 @@
+// C ABI of libsalad: argument validation, TMA tensor maps, launches, status.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+using namespace salad;
+
+namespace {
+
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<void*> g_ev_linear{nullptr}, g_ev_attn{nullptr}, g_ev_end{nullptr};
+
+bool record(const std::atomic<void*>& ev, cudaStream_t s) {
+  void* e = ev.load();
+  return e == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(e), s) == cudaSuccess;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+              const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[3];
+  cuuint64_t st[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
+  std::memset(m, 0, sizeof(*m));
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [B][N][Hh][d] bf16 viewed as a 3-D tensor (Hh*d, N, B); box (64, rows, 1).
+bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int Hh, int d, uint32_t rows) {
+  const uint64_t dims[3] = {(uint64_t)Hh * d, (uint64_t)N, (uint64_t)B};
+  const uint64_t strides[2] = {(uint64_t)Hh * d * 2, (uint64_t)N * Hh * d * 2};
+  const uint32_t box[3] = {64, rows, 1};
+  return make_map(m, base, 3, dims, strides, box);
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Shared checks of salad_attn_forward / salad_linear_state.
+int check_common(const void* k, const void* v, int B, int N, int Hh, int d, void* workspace,
+                 size_t workspace_bytes) {
+  if (!k || !v || !workspace) return SALAD_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || Hh < 1 || d < 1) return SALAD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
+  if (Hh > 65535 || (long long)B * Hh > 65535) return SALAD_ERR_UNSUPPORTED;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(workspace, 256)) return SALAD_ERR_INVALID_ARG;
+  if (workspace_bytes < workspace_layout(B, N, Hh, d).total) return SALAD_ERR_WORKSPACE;
+  return SALAD_OK;
+}
+
+int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const float* gate, uint8_t* ws,
+               const WorkspaceLayout& L, cudaStream_t s) {
+  CUtensorMap tk, tv;
+  if (!make_bnhd_map(&tk, k, B, N, Hh, d, 64) || !make_bnhd_map(&tv, v, B, N, Hh, d, 64)) return SALAD_ERR_CUDA;
+  LinearArgs la{};
+  la.tm_k = &tk;
+  la.tm_v = &tv;
+  la.gate = gate;
+  la.partial = reinterpret_cast<float*>(ws + L.off_partial);
+  la.sz = reinterpret_cast<uint16_t*>(ws + L.off_sz);
+  la.B = B;
+  la.N = N;
+  la.heads = Hh;
+  la.d = d;
+  la.splits = L.splits;
+  la.chunks_per_split = L.chunks_per_split;
+  la.status = reinterpret_cast<uint32_t*>(ws + L.off_status);
+  la.wait_limit_ns = g_wait_limit_ns.load();
+  return launch_linear_reduce(la, s) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int salad_mask_num_blocks(int T, int H, int W, int block, int* nb) {
+  if (!nb || T < 1 || H < 1 || W < 1 || block < 1) return SALAD_ERR_INVALID_ARG;
+  const long long N = (long long)T * H * W;
+  if (N >= (1ll << 31)) return SALAD_ERR_INVALID_ARG;
+  *nb = (int)((N + block - 1) / block);
+  return SALAD_OK;
+}
+
+int salad_build_block_mask(int T, int H, int W, int block, int num_heads, const int32_t* windows,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int64_t* nnz_out,
+                           salad_stream_t stream) {
+  int nb = 0;
+  int st = salad_mask_num_blocks(T, H, W, block, &nb);
+  if (st != SALAD_OK) return st;
+  if (!windows || !row_ptr || num_heads < 1 || num_heads > kMaxHeads || col_capacity < 0)
+    return SALAD_ERR_INVALID_ARG;
+  if (col_capacity > 0 && !col_idx) return SALAD_ERR_INVALID_ARG;
+  if (!aligned(row_ptr, 4) || (col_idx && !aligned(col_idx, 4))) return SALAD_ERR_INVALID_ARG;
+  // every kept pair must be addressable by an int32 offset
+  if ((long long)num_heads * nb * nb >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
+  WindowTable win{};
+  for (int h = 0; h < num_heads; ++h)
+    for (int a = 0; a < 3; ++a) {
+      if (windows[3 * h + a] < 0) return SALAD_ERR_INVALID_ARG;
+      win.w[3 * h + a] = windows[3 * h + a];
+    }
+  MaskGrid g{T, H, W, block, nb, num_heads, (long long)T * H * W};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_mask_count(g, win, row_ptr, s) != cudaSuccess) return SALAD_ERR_CUDA;
+  if (launch_mask_scan(row_ptr, num_heads * nb, s) != cudaSuccess) return SALAD_ERR_CUDA;
+  int32_t total = 0;
+  if (cudaMemcpyAsync(&total, row_ptr + (size_t)num_heads * nb, sizeof(total), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  if (nnz_out) *nnz_out = total;
+  if (total > col_capacity) return SALAD_ERR_CAPACITY;
+  if (total > 0 && launch_mask_fill(g, win, row_ptr, col_idx, s) != cudaSuccess) return SALAD_ERR_CUDA;
+  return SALAD_OK;
+}
+
+size_t salad_workspace_bytes(int B, int N, int num_heads, int d) {
+  if (B < 1 || N < 1 || num_heads < 1 || (d != 64 && d != 128)) return 0;
+  return workspace_layout(B, N, num_heads, d).total;
+}
+
+int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                       int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                       const float* gate, float softmax_scale, float eps, void* out, void* workspace,
+                       size_t workspace_bytes, salad_stream_t stream) {
+  if (!q || !row_ptr || !col_idx || !w_proj || !gate || !out) return SALAD_ERR_INVALID_ARG;
+  int st = check_common(k, v, B, N, num_heads, d, workspace, workspace_bytes);
+  if (st != SALAD_OK) return st;
+  if (block != 64 && block != 128) return SALAD_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(w_proj, 16) || !aligned(gate, 4) ||
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4))
+    return SALAD_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(softmax_scale)) return SALAD_ERR_INVALID_ARG;
+  const size_t tensor_bytes = (size_t)B * N * num_heads * d * 2;
+  if (overlaps(out, tensor_bytes, q, tensor_bytes) || overlaps(out, tensor_bytes, k, tensor_bytes) ||
+      overlaps(out, tensor_bytes, v, tensor_bytes))
+    return SALAD_ERR_INVALID_ARG;
+  const long long qtiles = (N + 127) / 128;
+  if (qtiles * B * num_heads >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
+
+  const WorkspaceLayout L = workspace_layout(B, N, num_heads, d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  if (!record(g_ev_linear, s)) return SALAD_ERR_CUDA;
+  st = run_linear(k, v, B, N, num_heads, d, gate, ws, L, s);
+  if (st != SALAD_OK) return st;
+
+  CUtensorMap tq, tk, tv, to, tsz, tw;
+  const int BH = B * num_heads;
+  const uint64_t sz_dims[3] = {(uint64_t)2 * d, (uint64_t)d + 16, (uint64_t)BH};
+  const uint64_t sz_strides[2] = {(uint64_t)2 * d * 2, (uint64_t)(d + 16) * 2 * d * 2};
+  const uint32_t sz_box[3] = {64, (uint32_t)d + 16, 1};
+  const uint64_t w_dims[2] = {(uint64_t)d, (uint64_t)d};
+  const uint64_t w_strides[1] = {(uint64_t)d * 2};
+  const uint32_t w_box[2] = {64, (uint32_t)d};
+  if (!make_bnhd_map(&tq, q, B, N, num_heads, d, 128) || !make_bnhd_map(&tk, k, B, N, num_heads, d, block) ||
+      !make_bnhd_map(&tv, v, B, N, num_heads, d, block) || !make_bnhd_map(&to, out, B, N, num_heads, d, 128) ||
+      !make_map(&tsz, ws + L.off_sz, 3, sz_dims, sz_strides, sz_box) ||
+      !make_map(&tw, w_proj, 2, w_dims, w_strides, w_box))
+    return SALAD_ERR_CUDA;
+
+  AttnArgs aa{};
+  aa.tm_q = &tq;
+  aa.tm_k = &tk;
+  aa.tm_v = &tv;
+  aa.tm_out = &to;
+  aa.tm_sz = &tsz;
+  aa.tm_w = &tw;
+  aa.row_ptr = row_ptr;
+  aa.col_idx = col_idx;
+  aa.gate = gate;
+  aa.B = B;
+  aa.N = N;
+  aa.heads = num_heads;
+  aa.d = d;
+  aa.block = block;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)d);
+  aa.scale_log2 = scale * 1.4426950408889634f;
+  aa.eps = eps;
+  aa.status = reinterpret_cast<uint32_t*>(ws + L.off_status);
+  aa.wait_limit_ns = g_wait_limit_ns.load();
+  if (!record(g_ev_attn, s)) return SALAD_ERR_CUDA;
+  if (launch_attention(aa, s) != cudaSuccess) return SALAD_ERR_CUDA;
+  return record(g_ev_end, s) ? SALAD_OK : SALAD_ERR_CUDA;
+}
+
+int salad_linear_state(const void* k, const void* v, int B, int N, int num_heads, int d, const float* gate,
+                       float* S_out, float* z_out, void* workspace, size_t workspace_bytes,
+                       salad_stream_t stream) {
+  if (!S_out || !z_out) return SALAD_ERR_INVALID_ARG;
+  int st = check_common(k, v, B, N, num_heads, d, workspace, workspace_bytes);
+  if (st != SALAD_OK) return st;
+  if ((gate && !aligned(gate, 4)) || !aligned(S_out, 4) || !aligned(z_out, 4)) return SALAD_ERR_INVALID_ARG;
+  const WorkspaceLayout L = workspace_layout(B, N, num_heads, d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = run_linear(k, v, B, N, num_heads, d, gate, ws, L, s);
+  if (st != SALAD_OK) return st;
+  return launch_linear_export(reinterpret_cast<const uint16_t*>(ws + L.off_sz), gate, B * num_heads, d, S_out,
+                              z_out, s) == cudaSuccess
+             ? SALAD_OK
+             : SALAD_ERR_CUDA;
+}
+
+int salad_check_status(void* workspace, salad_stream_t stream) {
+  if (!workspace) return SALAD_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SALAD_ERR_CUDA;
+  uint32_t word = 0;
+  uint32_t* dev = static_cast<uint32_t*>(workspace);
+  if (cudaMemcpyAsync(&word, dev, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  if (word == 0) return SALAD_OK;
+  if (cudaMemsetAsync(dev, 0, sizeof(word), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  return (word & kStatusTimeout) ? SALAD_ERR_DEVICE_TIMEOUT : SALAD_ERR_CUDA;
+}
+
+void salad_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns.store(limit_ns); }
+
+void salad_set_phase_events(void* before_linear, void* before_attention, void* after_attention) {
+  g_ev_linear.store(before_linear);
+  g_ev_attn.store(before_attention);
+  g_ev_end.store(after_attention);
+}
+
+const char* salad_status_string(int status) {
+  switch (status) {
+    case SALAD_OK: return "ok";
+    case SALAD_ERR_INVALID_ARG: return "invalid argument";
+    case SALAD_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SALAD_ERR_CAPACITY: return "col_idx capacity too small";
+    case SALAD_ERR_WORKSPACE: return "workspace too small";
+    case SALAD_ERR_CUDA: return "CUDA error";
+    case SALAD_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,554 @@
+// SALAD hybrid attention forward: block-sparse softmax attention over the kept
+// key blocks (ST-SWA, sciencestack SALAD page Figure 1; the sparse branch of
+// SALAD summary section 2.1) fused with the epilogue of the ReLU linear branch, its
+// static projection and the per-(b, h) gate (summary sections 2.1-2.3):
+//
+//   o_sp  = softmax(scale * q K_kept^T) V_kept          (online softmax)
+//   o_lin = relu(q)^T S / (relu(q) . z + eps)           (S, z from linear.cu)
+//   out   = o_sp + g * (o_lin W);   out = o_sp when g == 0 (branch dropped)
+//
+// One CTA owns a 128-row query tile of one (b, h) (two 64-token query blocks
+// when block == 64, whose kept-key lists are merged; a key tile then carries a
+// bit per half saying which rows may see it).  Warp roles, 192 threads:
+//   warp 0     TMA producer: Q once, then K/V tiles of the kept blocks into a
+//              2-deep ring, then (when g != 0) [S|z] and W for the epilogue;
+//   warp 1     tcgen05 issuer (one thread) and TMEM owner:
+//              S_j = Q K_j^T into one of two TMEM buffers, O += P_j V_j;
+//   warps 2-5  softmax: one query row per thread, online softmax with lazy
+//              rescaling of O in TMEM, P_j written to shared memory as bf16;
+//              then the fused epilogue and one TMA store of bf16 out.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256, 256+d); the
+// epilogue reuses column 0 for U = relu(Q)[S|z] and then for Y = o_lin W.
+// The [S|z] and o_lin operands are fed as bf16 hi + lo pairs (K doubled), so the
+// epilogue products keep ~16 mantissa bits.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace salad {
+namespace {
+
+constexpr uint64_t kDrainNs = 1000000000ull;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+template <int D, int BLK>
+struct AttnCfg {
+  static constexpr int QROWS = 128;
+  static constexpr int DCH = D / 64;                // 64-column chunks of a d-wide row
+  static constexpr int Q_BYTES = QROWS * D * 2;     // DCH chunks of 16 KB
+  static constexpr int KV_BOX = BLK * 128;          // one [BLK x 64] box
+  static constexpr int KV_BYTES = DCH * KV_BOX;     // one K or V tile
+  static constexpr int RING_BYTES = 4 * KV_BYTES;   // K[2], V[2]
+  static constexpr int SZ_ROWS = D + 16;
+  static constexpr int SZ_CH = 2 * D / 64;
+  static constexpr int SZ_CH_BYTES = SZ_ROWS * 128;
+  static constexpr int SZ_BYTES = SZ_CH * SZ_CH_BYTES;
+  static constexpr int W_CH_BYTES = D * 128;
+  static constexpr int W_BYTES = DCH * W_CH_BYTES;
+  static constexpr int OVL_BYTES = RING_BYTES > SZ_BYTES + W_BYTES ? RING_BYTES : SZ_BYTES + W_BYTES;
+  static constexpr int P_CH = (BLK > D ? BLK : D) / 64;  // P in the loop, o_lo in the epilogue
+  static constexpr int P_BYTES = P_CH * 16384;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K0 = OFF_RING;
+  static constexpr int OFF_V0 = OFF_RING + 2 * KV_BYTES;
+  static constexpr int OFF_SZ = OFF_RING;
+  static constexpr int OFF_W = OFF_RING + SZ_BYTES;
+  static constexpr int OFF_P = OFF_RING + OVL_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int SMEM_USED = OFF_BAR + 512 + 1024;
+  // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
+  static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_U = 0, TM_Y = 0;
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false, false);   // Q K^T
+  static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);     // P V   (V MN-major)
+  static constexpr uint32_t IDESC_U = idesc_bf16(128, D + 16, false, false);  // relu(Q) [S|z]
+  static constexpr uint32_t IDESC_Y = idesc_bf16(128, D, false, true);      // o_lin W (W MN-major)
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct AttnShared {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, pv_done;
+  uint64_t ep_full, q_relu, u_done, a2_full, y_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+// Kept key tiles of one 128-row query tile, in ascending key-block order.
+// bits: bit s set when query half s (block == 64) or the whole tile uses it.
+struct KeyIter {
+  const int32_t* a;
+  const int32_t* b;
+  int na, nb, ia, ib;
+  __device__ __forceinline__ bool next(int& col, int& bits) {
+    if (ia < na && (ib >= nb || a[ia] <= b[ib])) {
+      col = a[ia++];
+      bits = 1;
+      if (ib < nb && b[ib] == col) {
+        bits |= 2;
+        ++ib;
+      }
+      return true;
+    }
+    if (ib < nb) {
+      col = b[ib++];
+      bits = 2;
+      return true;
+    }
+    return false;
+  }
+};
+
+template <int BLK>
+__device__ __forceinline__ KeyIter make_iter(const int32_t* row_ptr, const int32_t* col_idx, int h, int nb,
+                                             int qtile) {
+  KeyIter it{};
+  if (BLK == 128) {
+    const int r = h * nb + qtile;
+    it.a = col_idx + row_ptr[r];
+    it.na = row_ptr[r + 1] - row_ptr[r];
+    it.b = nullptr;
+    it.nb = 0;
+  } else {
+    const int I0 = 2 * qtile, I1 = 2 * qtile + 1;
+    const int r0 = h * nb + I0;
+    it.a = col_idx + row_ptr[r0];
+    it.na = row_ptr[r0 + 1] - row_ptr[r0];
+    if (I1 < nb) {
+      it.b = col_idx + row_ptr[r0 + 1];
+      it.nb = row_ptr[r0 + 2] - row_ptr[r0 + 1];
+    } else {
+      it.b = nullptr;
+      it.nb = 0;
+    }
+  }
+  it.ia = it.ib = 0;
+  return it;
+}
+
+__device__ __forceinline__ void record_timeout(AttnShared* sh, uint32_t* status) {
+  sh->abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
+}
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(192, 1)
+    salad_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                      const __grid_constant__ CUtensorMap tm_sz, const __grid_constant__ CUtensorMap tm_w,
+                      const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                      const float* __restrict__ gate, int heads, int N, int qtiles, float scale_log2, float eps,
+                      uint32_t* status, uint64_t limit_ns) {
+  using C = AttnCfg<D, BLK>;
+  const int bh = blockIdx.x / qtiles, qtile = blockIdx.x % qtiles;
+  const int b = bh / heads, h = bh % heads;
+  const int nb = (N + BLK - 1) / BLK;
+  const float g = gate[bh];
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  AttnShared* sh = reinterpret_cast<AttnShared*>(smem + C::OFF_BAR);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh->q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh->k_full[s], 1);
+      mbar_init(&sh->k_empty[s], 1);
+      mbar_init(&sh->v_full[s], 1);
+      mbar_init(&sh->v_empty[s], 1);
+      mbar_init(&sh->s_full[s], 1);
+      mbar_init(&sh->s_free[s], 4);
+    }
+    mbar_init(&sh->p_full, 4);
+    mbar_init(&sh->pv_done, 1);
+    mbar_init(&sh->ep_full, 1);
+    mbar_init(&sh->q_relu, 4);
+    mbar_init(&sh->u_done, 1);
+    mbar_init(&sh->a2_full, 4);
+    mbar_init(&sh->y_done, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ============================ TMA producer
+    if (lane == 0) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      tma_prefetch_map(&tm_out);
+      mbar_arrive_expect_tx(&sh->q_full, C::Q_BYTES);
+#pragma unroll
+      for (int ch = 0; ch < C::DCH; ++ch)
+        tma_load_3d(smem + C::OFF_Q + ch * 16384, &tm_q, &sh->q_full, h * D + ch * 64, qtile * 128, b);
+      KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
+      int col, bits, j = 0;
+      bool ok = true;
+      while (it.next(col, bits)) {
+        const int s = j & 1;
+        const uint32_t ph = ((j >> 1) & 1) ^ 1;
+        if (sh->abort_flag || !mbar_wait(&sh->k_empty[s], ph, limit_ns)) { ok = false; break; }
+        mbar_arrive_expect_tx(&sh->k_full[s], C::KV_BYTES);
+        uint8_t* kt = smem + C::OFF_K0 + s * C::KV_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch)
+          tma_load_3d(kt + ch * C::KV_BOX, &tm_k, &sh->k_full[s], h * D + ch * 64, col * BLK, b);
+        if (sh->abort_flag || !mbar_wait(&sh->v_empty[s], ph, limit_ns)) { ok = false; ++j; break; }
+        mbar_arrive_expect_tx(&sh->v_full[s], C::KV_BYTES);
+        uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch)
+          tma_load_3d(vt + ch * C::KV_BOX, &tm_v, &sh->v_full[s], h * D + ch * 64, col * BLK, b);
+        ++j;
+      }
+      const int n = j;
+      if (ok && g != 0.0f) {
+        // epilogue operands overwrite the ring: wait until the last uses of both stages are consumed
+        for (int s = 0; s < 2 && ok; ++s) {
+          const int uses = (n - s + 1) / 2;
+          if (uses > 0) {
+            const uint32_t par = (uint32_t)((uses - 1) & 1);
+            ok = mbar_wait(&sh->k_empty[s], par, limit_ns) && mbar_wait(&sh->v_empty[s], par, limit_ns);
+          }
+        }
+        if (ok) {
+          mbar_arrive_expect_tx(&sh->ep_full, C::SZ_BYTES + C::W_BYTES);
+#pragma unroll
+          for (int ch = 0; ch < C::SZ_CH; ++ch)
+            tma_load_3d(smem + C::OFF_SZ + ch * C::SZ_CH_BYTES, &tm_sz, &sh->ep_full, ch * 64, 0, bh);
+#pragma unroll
+          for (int ch = 0; ch < C::DCH; ++ch)
+            tma_load_2d(smem + C::OFF_W + ch * C::W_CH_BYTES, &tm_w, &sh->ep_full, ch * 64, 0);
+        }
+      }
+      if (!ok) {
+        record_timeout(sh, status);
+        // copies already issued must land before the CTA may exit
+        mbar_wait(&sh->q_full, 0, kDrainNs);
+        for (int i = (n > 2 ? n - 2 : 0); i < n; ++i) {
+          mbar_wait(&sh->k_full[i & 1], (i >> 1) & 1, kDrainNs);
+          mbar_wait(&sh->v_full[i & 1], (i >> 1) & 1, kDrainNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ============================ tcgen05 issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&sh->q_full, 0, limit_ns);
+      const uint32_t q_addr = sbase + C::OFF_Q;
+      const uint32_t p_addr = sbase + C::OFF_P;
+      KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
+      int col, bits, j = 0;
+      // O += P_i V_i
+      auto issue_pv = [&](int i) -> bool {
+        const int s = i & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->p_full, (uint32_t)(i & 1), limit_ns)) return false;
+        if (!mbar_wait(&sh->v_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
+        tc_fence_after();
+        const uint32_t vt = sbase + C::OFF_V0 + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BLK / 16; ++kk) {
+          const uint64_t a = sw128_desc(p_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(vt + kk * 2048, C::KV_BOX, 1024);
+          mma_bf16_ss(tmem + C::TM_O, a, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&sh->pv_done);
+        mma_commit(&sh->v_empty[s]);
+        return true;
+      };
+      while (ok && it.next(col, bits)) {
+        const int s = j & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->k_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait(&sh->s_free[s], (uint32_t)(((j - 2) >> 1) & 1), limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kt = sbase + C::OFF_K0 + s * C::KV_BYTES;
+        const uint32_t d_s = tmem + (s ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sw128_desc(q_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(kt + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
+          mma_bf16_ss(d_s, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sh->s_full[s]);
+        mma_commit(&sh->k_empty[s]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; ++j; break; }
+        ++j;
+      }
+      if (ok && j >= 1) ok = issue_pv(j - 1);
+      if (ok && g != 0.0f) {
+        // U = relu(Q) [S_hi ; S_lo | z_hi ; z_lo]   (K = 2d: relu(Q) is fed twice)
+        ok = mbar_wait(&sh->q_relu, 0, limit_ns) && mbar_wait(&sh->ep_full, 0, limit_ns);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t szb = sbase + C::OFF_SZ;
+#pragma unroll
+          for (int kk = 0; kk < 2 * D / 16; ++kk) {
+            const int qk = kk % (D / 16);
+            const uint64_t a = sw128_desc(q_addr + (qk / 4) * 16384 + (qk % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(szb + (kk / 4) * C::SZ_CH_BYTES + (kk % 4) * 32, 16, 1024);
+            mma_bf16_ss(tmem + C::TM_U, a, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sh->u_done);
+          // Y = [o_hi | o_lo] [W ; W]
+          ok = mbar_wait(&sh->a2_full, 0, limit_ns);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t wb = sbase + C::OFF_W;
+#pragma unroll
+            for (int kk = 0; kk < 2 * D / 16; ++kk) {
+              const int ch = kk / 4;  // chunk of [o_hi | o_lo]
+              const uint32_t abase = ch < C::DCH ? q_addr + ch * 16384 : p_addr + (ch - C::DCH) * 16384;
+              const uint64_t a = sw128_desc(abase + (kk % 4) * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(wb + (kk % (D / 16)) * 2048, C::W_CH_BYTES, 1024);
+              mma_bf16_ss(tmem + C::TM_Y, a, bd, C::IDESC_Y, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sh->y_done);
+          }
+        }
+      }
+      if (!ok) {
+        record_timeout(sh, status);
+        mma_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0, kDrainNs);
+      }
+    }
+  } else {
+    // ============================ softmax / epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                        // query row within the tile
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int half = BLK == 64 ? (r >> 6) : 0;
+    const uint32_t q_addr = sbase + C::OFF_Q;
+    const uint32_t p_addr = sbase + C::OFF_P;
+    float m_ref = -INFINITY;  // running reference max (raw score units)
+    float l = 0.f;
+    bool ok = true;
+    KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
+    int col, bits, j = 0;
+    while (it.next(col, bits)) {
+      const int s = j & 1;
+      const bool aborted = __shfl_sync(0xffffffffu, sh->abort_flag != 0, 0);
+      if (aborted || !mbar_wait_warp(&sh->s_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
+      tc_fence_after();
+      float sv[BLK];
+#pragma unroll
+      for (int c = 0; c < BLK / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(lane_addr + (s ? C::TM_S1 : C::TM_S0) + c * 32, rr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(rr[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->s_free[s]);
+
+      const bool use = ((bits >> half) & 1) != 0;
+      const int valid = min(BLK, N - col * BLK);  // real keys in this block
+      float alpha = 1.f;
+      bool rescale = false;
+      if (use) {
+        float mt = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < BLK; ++i)
+          if (i < valid) mt = fmaxf(mt, sv[i]);
+        if (m_ref == -INFINITY) {
+          m_ref = mt;
+        } else if ((mt - m_ref) * scale_log2 > kRescaleThreshold) {
+          alpha = ex2_approx((m_ref - mt) * scale_log2);
+          m_ref = mt;
+          rescale = true;
+        }
+        const float mb = m_ref * scale_log2;
+        float rs = 0.f;
+#pragma unroll
+        for (int i = 0; i < BLK; ++i) {
+          const float p = i < valid ? ex2_approx(fmaf(sv[i], scale_log2, -mb)) : 0.f;
+          sv[i] = p;
+          rs += p;
+        }
+        l = l * alpha + rs;
+      } else {
+#pragma unroll
+        for (int i = 0; i < BLK; ++i) sv[i] = 0.f;
+      }
+      // P_j may overwrite the P buffer and O may be rescaled only after PV_{j-1}
+      if (j >= 1) {
+        if (!mbar_wait_warp(&sh->pv_done, (uint32_t)((j - 1) & 1), limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(lane_addr + C::TM_O + c * 32, rr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+            tmem_st32(lane_addr + C::TM_O + c * 32, rr);
+          }
+          tmem_st_wait();
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < BLK / 8; ++c) {
+        const uint32_t addr = p_addr + (c / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(c % 8));
+        st_shared_v4(addr, pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
+                     pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]), pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->p_full);
+      ++j;
+    }
+    const int n = j;
+    if (ok && n >= 1) {
+      ok = mbar_wait_warp(&sh->pv_done, (uint32_t)((n - 1) & 1), limit_ns);
+      tc_fence_after();
+    }
+    if (ok) ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);  // the staging area below is the Q tile
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    const bool lin = ok && g != 0.0f;
+    if (lin) {
+      // relu(Q) in place (Q is no longer read by the S MMAs)
+#pragma unroll
+      for (int ch = 0; ch < C::DCH; ++ch)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t addr = q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)c);
+          uint32_t x0, x1, x2, x3;
+          ld_shared_v4(addr, x0, x1, x2, x3);
+          x0 &= ~(((x0 >> 15) & 0x00010001u) * 0xFFFFu);
+          x1 &= ~(((x1 >> 15) & 0x00010001u) * 0xFFFFu);
+          x2 &= ~(((x2 >> 15) & 0x00010001u) * 0xFFFFu);
+          x3 &= ~(((x3 >> 15) & 0x00010001u) * 0xFFFFu);
+          st_shared_v4(addr, x0, x1, x2, x3);
+        }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->q_relu);
+    }
+    bool lin_ok = lin && mbar_wait_warp(&sh->u_done, 0, limit_ns);
+    if (lin && !lin_ok) ok = false;
+    if (lin_ok) {
+      tc_fence_after();
+      uint32_t zr[16];
+      tmem_ld16(lane_addr + C::TM_U + D, zr);
+      tmem_ld_wait();
+      const float inv_den = 1.f / (__uint_as_float(zr[0]) + eps);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(lane_addr + C::TM_U + c * 32, rr);
+        tmem_ld_wait();
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float o0 = __uint_as_float(rr[2 * i]) * inv_den, o1 = __uint_as_float(rr[2 * i + 1]) * inv_den;
+          hi[i] = pack_bf16x2(o0, o1);
+          lo[i] = pack_bf16x2(o0 - bf16_lo_to_f32(hi[i]), o1 - bf16_hi_to_f32(hi[i]));
+        }
+        // columns [32c, 32c+32): chunk (32c)/64, 16-byte pieces ((32c)%64)/8 .. +3
+        const int ch = (c * 32) / 64, pc0 = ((c * 32) % 64) / 8;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t off = ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)(pc0 + k));
+          st_shared_v4(q_addr + off, hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
+          st_shared_v4(p_addr + off, lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->a2_full);
+      lin_ok = mbar_wait_warp(&sh->y_done, 0, limit_ns);
+      if (!lin_ok) ok = false;
+      tc_fence_after();
+    }
+    if (ok) {
+      // out = O / l + g * Y  -> bf16 staging in the Q tile -> one TMA store per 64 columns
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ro[32], ry[32];
+        if (n >= 1) {
+          tmem_ld32(lane_addr + C::TM_O + c * 32, ro);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ro[i] = 0u;
+        }
+        if (lin_ok) tmem_ld32(lane_addr + C::TM_Y + c * 32, ry);
+        tmem_ld_wait();
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float o0 = __uint_as_float(ro[2 * i]) * inv_l, o1 = __uint_as_float(ro[2 * i + 1]) * inv_l;
+          if (lin_ok) {
+            o0 = fmaf(g, __uint_as_float(ry[2 * i]), o0);
+            o1 = fmaf(g, __uint_as_float(ry[2 * i + 1]), o1);
+          }
+          packed[i] = pack_bf16x2(o0, o1);
+        }
+        const int ch = (c * 32) / 64, pc0 = ((c * 32) % 64) / 8;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          st_shared_v4(q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)(pc0 + k)), packed[4 * k],
+                       packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+      }
+      fence_proxy_async_smem();
+    } else {
+      record_timeout(sh, status);
+    }
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 64 && !sh->abort_flag) {
+#pragma unroll
+      for (int ch = 0; ch < C::DCH; ++ch)
+        tma_store_3d(&tm_out, smem + C::OFF_Q + ch * 16384, h * D + ch * 64, qtile * 128, b);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, int BLK>
+cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
+  using C = AttnCfg<D, BLK>;
+  cudaError_t e =
+      cudaFuncSetAttribute(salad_attn_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int qtiles = (a.N + 127) / 128;
+  const long long grid = (long long)qtiles * a.B * a.heads;
+  salad_attn_kernel<D, BLK><<<(unsigned)grid, 192, C::SMEM, s>>>(
+      *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_sz, *a.tm_w, a.row_ptr, a.col_idx, a.gate, a.heads, a.N, qtiles,
+      a.scale_log2, a.eps, a.status, a.wait_limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
+  if (a.d == 64) return a.block == 64 ? launch_attn_t<64, 64>(a, s) : launch_attn_t<64, 128>(a, s);
+  return a.block == 64 ? launch_attn_t<128, 64>(a, s) : launch_attn_t<128, 128>(a, s);
+}
+
+}  // namespace salad

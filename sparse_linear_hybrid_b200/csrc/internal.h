@@ -1,0 +1,76 @@
+// Internal declarations shared by the libsalad translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/salad.h"
+
+namespace salad {
+
+constexpr int kMaxHeads = 256;
+
+// Window table passed by value to the mask kernels (kMaxHeads * 12 bytes).
+struct WindowTable {
+  int32_t w[3 * kMaxHeads];
+};
+
+struct MaskGrid {
+  int T, H, W, block, nb, heads;
+  long long N;
+};
+
+cudaError_t launch_mask_count(const MaskGrid& g, const WindowTable& win, int32_t* row_ptr, cudaStream_t s);
+cudaError_t launch_mask_scan(int32_t* row_ptr, int n, cudaStream_t s);
+cudaError_t launch_mask_fill(const MaskGrid& g, const WindowTable& win, const int32_t* row_ptr, int32_t* col_idx,
+                             cudaStream_t s);
+
+// Workspace layout of the forward pass (byte offsets from the workspace base).
+struct WorkspaceLayout {
+  int splits;             // split-N factor of the linear-branch reduction
+  int chunks_per_split;   // 64-token chunks per split
+  size_t off_status;      // uint32 status word
+  size_t off_sz;          // bf16 [B*Hh][d+16][2d]: [S | z]^T split into hi and lo halves
+  size_t off_partial;     // fp32 [splits][B*Hh][d+1][d]: per-split S rows, then z
+  size_t total;
+};
+WorkspaceLayout workspace_layout(int B, int N, int heads, int d);
+
+struct LinearArgs {
+  const CUtensorMap* tm_k;  // box (64, 64 tokens, 1)
+  const CUtensorMap* tm_v;
+  const float* gate;        // nullable
+  float* partial;
+  uint16_t* sz;
+  int B, N, heads, d, splits, chunks_per_split;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_linear_reduce(const LinearArgs& a, cudaStream_t s);
+cudaError_t launch_linear_export(const uint16_t* sz, const float* gate, int BH, int d, float* S_out, float* z_out,
+                                 cudaStream_t s);
+
+struct AttnArgs {
+  const CUtensorMap* tm_q;    // box (64, 128, 1)
+  const CUtensorMap* tm_k;    // box (64, block, 1)
+  const CUtensorMap* tm_v;    // box (64, block, 1)
+  const CUtensorMap* tm_out;  // box (64, 128, 1)
+  const CUtensorMap* tm_sz;   // box (64, d+16, 1)
+  const CUtensorMap* tm_w;    // box (64, d)
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const float* gate;
+  int B, N, heads, d, block;
+  float scale_log2;  // softmax scale * log2(e)
+  float eps;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// Status word bits written by kernels.
+constexpr uint32_t kStatusTimeout = 1u;
+
+}  // namespace salad

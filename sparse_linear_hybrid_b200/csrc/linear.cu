@@ -1,0 +1,332 @@
+// Linear-branch state of SALAD's ReLU linear attention (SALAD summary section
+// 2.1: a ReLU-based linear attention of O(N) cost that carries global token
+// interactions).  Per (b, h), over all N tokens:
+//   S[c][e] = sum_j relu(k_j[c]) v_j[e]        z[c] = sum_j relu(k_j[c])
+//
+// linear_partial_kernel: grid (splits, B*Hh).  Each CTA streams its share of
+// 64-token chunks through a 3-stage TMA ring; four warps apply ReLU to the K
+// tile in shared memory (accumulating z in fp32 on the way) and one thread
+// issues tcgen05 MMAs  D[c][e] += relu(K)^T[c][tok] * V[tok][e]  with both
+// operands MN-major and the fp32 accumulator in tensor memory.  The CTA writes
+// its partial S and z in fp32.
+// linear_finalize_kernel: fixed-order sum of the partials (deterministic), then
+// [S | z] transposed and split into bf16 hi + lo halves, the B operand layout
+// the attention epilogue feeds to the tensor cores.
+#include "internal.h"
+#include "ptx.cuh"
+
+#include <cuda_bf16.h>
+
+namespace salad {
+namespace {
+
+constexpr int kTok = 64;      // tokens per chunk
+constexpr int kStages = 3;
+constexpr uint64_t kDrainNs = 1000000000ull;
+
+struct LinShared {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t relu[kStages];
+  uint64_t acc_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  float zred[256];
+};
+
+template <int D>
+struct LinCfg {
+  static constexpr int BOX_BYTES = kTok * 128;          // one [64 tokens x 64 cols] bf16 box
+  static constexpr int TILE_BYTES = (D / 64) * BOX_BYTES;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;    // K tile then V tile
+  static constexpr int OFF_BAR = kStages * STAGE_BYTES;
+  static constexpr int SMEM = OFF_BAR + (int)sizeof(LinShared) + 1024;  // + alignment slack
+  // M is padded to 128 for D = 64: the second 64-row half of A reads the V tile
+  // and lands in accumulator rows 64..127, which are never read.
+  static constexpr uint32_t IDESC = idesc_bf16(128, D, true, true);
+};
+
+
+
+__device__ __forceinline__ void record_timeout(LinShared* sh, uint32_t* status) {
+  sh->abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    linear_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const float* __restrict__ gate, float* __restrict__ partial, int heads, int N,
+                          int chunks_per_split, uint32_t* status, uint64_t limit_ns) {
+  using C = LinCfg<D>;
+  const int split = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
+  if (gate != nullptr && gate[bh] == 0.0f) return;  // branch dropped for this (b, h)
+  const int b = bh / heads, h = bh % heads;
+  const int total_chunks = (N + kTok - 1) / kTok;
+  const int c_begin = split * chunks_per_split;
+  const int n_chunks = min(total_chunks, c_begin + chunks_per_split) - c_begin;  // >= 1 by construction
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  LinShared* sh = reinterpret_cast<LinShared*>(smem + C::OFF_BAR);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 1);
+      mbar_init(&sh->relu[s], 4);
+    }
+    mbar_init(&sh->acc_done, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < n_chunks; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->empty[s], ph ^ 1, limit_ns)) {
+          record_timeout(sh, status);
+          break;
+        }
+        uint8_t* kt = smem + s * C::STAGE_BYTES;
+        uint8_t* vt = kt + C::TILE_BYTES;
+        mbar_arrive_expect_tx(&sh->full[s], C::STAGE_BYTES);
+        const int row = (c_begin + it) * kTok;
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) {
+          tma_load_3d(kt + ch * C::BOX_BYTES, &tm_k, &sh->full[s], h * D + ch * 64, row, b);
+          tma_load_3d(vt + ch * C::BOX_BYTES, &tm_v, &sh->full[s], h * D + ch * 64, row, b);
+        }
+        issued = it + 1;
+      }
+      if (sh->abort_flag) {
+        // let every copy this thread started land before the CTA can exit
+        for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
+          mbar_wait(&sh->full[it % kStages], (it / kStages) & 1, kDrainNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      for (int it = 0; it < n_chunks; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->relu[s], ph, limit_ns)) {
+          record_timeout(sh, status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kt = smem_u32(smem + s * C::STAGE_BYTES);
+        const uint32_t vt = kt + C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kTok / 16; ++kk) {
+          const uint64_t a = sw128_desc(kt + kk * 2048, C::BOX_BYTES, 1024);
+          const uint64_t bdesc = sw128_desc(vt + kk * 2048, C::BOX_BYTES, 1024);
+          mma_bf16_ss(tmem, a, bdesc, C::IDESC, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&sh->empty[s]);
+      }
+      if (sh->abort_flag) {
+        mma_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0, kDrainNs);
+      } else {
+        mma_commit(&sh->acc_done);
+      }
+    }
+  } else {
+    // ---------------- ReLU + z (warps 2..5), then the accumulator write-out
+    const int t = threadIdx.x - 64;           // 0..127
+    constexpr int PAIRS = D / 2;               // bf16 pairs per token row
+    constexpr int RSTEP = 128 / PAIRS;         // threads sharing a column pair
+    const int p = t % PAIRS, r0 = t / PAIRS;
+    const uint32_t col_off = (uint32_t)(p / 32) * C::BOX_BYTES;
+    const uint32_t piece = (uint32_t)((p % 32) / 4), word = (uint32_t)(p % 4) * 4;
+    float z0 = 0.f, z1 = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_chunks && ok; ++it) {
+      const int s = it % kStages;
+      const uint32_t ph = (it / kStages) & 1;
+      if (sh->abort_flag || !mbar_wait(&sh->full[s], ph, limit_ns)) {
+        record_timeout(sh, status);
+        ok = false;
+        break;
+      }
+      const uint32_t kt = smem_u32(smem + s * C::STAGE_BYTES) + col_off;
+#pragma unroll 8
+      for (int r = r0; r < kTok; r += RSTEP) {
+        const uint32_t addr = kt + sw128_offset((uint32_t)r, piece) + word;
+        uint32_t v;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+        const uint32_t neg = ((v >> 15) & 0x00010001u) * 0xFFFFu;  // 0xFFFF in each negative half
+        v &= ~neg;
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+        z0 += bf16_lo_to_f32(v);
+        z1 += bf16_hi_to_f32(v);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->relu[s]);
+    }
+    // z: fixed-order reduction of the threads that share a column pair
+    sh->zred[2 * t] = z0;
+    sh->zred[2 * t + 1] = z1;
+    named_bar_sync(1, 128);
+    float* dst = partial + ((size_t)split * BH + bh) * (size_t)(D + 1) * D;
+    if (t < D) {
+      float zc = 0.f;
+      for (int k = 0; k < RSTEP; ++k) zc += sh->zred[2 * ((t / 2) + k * PAIRS) + (t & 1)];
+      dst[(size_t)D * D + t] = zc;
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && mbar_wait_warp(&sh->acc_done, 0, limit_ns)) {
+      tc_fence_after();
+      const int quarter = warp & 3;
+      const int c = quarter * 32 + lane;  // accumulator row = feature c of relu(k)
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + cc * 32, r);
+        tmem_ld_wait();
+        if (c < D) {
+          float4* row = reinterpret_cast<float4*>(dst + (size_t)c * D + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            row[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                 __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        }
+      }
+    } else if (ok) {
+      record_timeout(sh, status);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// grid (B*Hh, D/16), 256 threads.  CTA (bh, g) owns features c in [16g, 16g+16).
+// sz[bh][e][c] = hi(S[c][e]), sz[bh][e][D+c] = lo(S[c][e]) for e < D; row D holds
+// z the same way; rows D+1 .. D+15 are zero.
+template <int D>
+__global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __restrict__ partial,
+                                                              const float* __restrict__ gate,
+                                                              uint16_t* __restrict__ sz, int splits) {
+  const int bh = blockIdx.x, g = blockIdx.y, BH = gridDim.x;
+  if (gate != nullptr && gate[bh] == 0.0f) return;
+  __shared__ float acc[16][D + 1];
+  __shared__ float zacc[16];
+  const size_t slab = (size_t)(D + 1) * D;
+  for (int idx = threadIdx.x; idx < 16 * D; idx += 256) {
+    const int cl = idx / D, e = idx % D, c = 16 * g + cl;
+    float s = 0.f;
+    for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * BH + bh) * slab + (size_t)c * D + e];
+    acc[cl][e] = s;
+  }
+  if (threadIdx.x < 16) {
+    const int c = 16 * g + threadIdx.x;
+    float s = 0.f;
+    for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * BH + bh) * slab + (size_t)D * D + c];
+    zacc[threadIdx.x] = s;
+  }
+  __syncthreads();
+  uint16_t* out = sz + (size_t)bh * (D + 16) * (2 * D);
+  for (int idx = threadIdx.x; idx < (D + 16) * 16; idx += 256) {
+    const int e = idx / 16, cl = idx % 16, c = 16 * g + cl;
+    const float x = e < D ? acc[cl][e] : (e == D ? zacc[cl] : 0.f);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+    out[(size_t)e * (2 * D) + c] = __bfloat16_as_ushort(hi);
+    out[(size_t)e * (2 * D) + D + c] = __bfloat16_as_ushort(lo);
+  }
+}
+
+// S_out[bh][c][e] = hi + lo, z_out[bh][c] likewise (for salad_linear_state).
+template <int D>
+__global__ void linear_export_kernel(const uint16_t* __restrict__ sz, const float* __restrict__ gate,
+                                     float* __restrict__ S_out, float* __restrict__ z_out) {
+  const int bh = blockIdx.x;
+  if (gate != nullptr && gate[bh] == 0.0f) return;
+  const uint16_t* in = sz + (size_t)bh * (D + 16) * (2 * D);
+  for (int idx = threadIdx.x; idx < (D + 1) * D; idx += blockDim.x) {
+    const int e = idx / D, c = idx % D;  // row e of sz, feature c
+    const float v = __bfloat162float(__ushort_as_bfloat16(in[(size_t)e * 2 * D + c])) +
+                    __bfloat162float(__ushort_as_bfloat16(in[(size_t)e * 2 * D + D + c]));
+    if (e < D)
+      S_out[((size_t)bh * D + c) * D + e] = v;
+    else
+      z_out[(size_t)bh * D + c] = v;
+  }
+}
+
+template <int D>
+cudaError_t launch_linear_t(const LinearArgs& a, cudaStream_t s) {
+  using C = LinCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(linear_partial_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int BH = a.B * a.heads;
+  linear_partial_kernel<D><<<dim3(a.splits, BH), 192, C::SMEM, s>>>(
+      *a.tm_k, *a.tm_v, a.gate, a.partial, a.heads, a.N, a.chunks_per_split, a.status, a.wait_limit_ns);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  linear_finalize_kernel<D><<<dim3(BH, D / 16), 256, 0, s>>>(a.partial, a.gate, a.sz, a.splits);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+WorkspaceLayout workspace_layout(int B, int N, int heads, int d) {
+  WorkspaceLayout L{};
+  const long long BH = (long long)B * heads;
+  const int total_chunks = (N + kTok - 1) / kTok;
+  // about two CTAs per SM of a 148-SM B200 in one wave
+  int splits = (int)(296 / BH);
+  if (splits < 1) splits = 1;
+  if (splits > total_chunks) splits = total_chunks;
+  const int cps = (total_chunks + splits - 1) / splits;
+  splits = (total_chunks + cps - 1) / cps;  // every split owns at least one chunk
+  L.splits = splits;
+  L.chunks_per_split = cps;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  L.off_status = 0;
+  L.off_sz = 256;
+  L.off_partial = L.off_sz + up((size_t)BH * (d + 16) * (2 * d) * 2);
+  L.total = L.off_partial + up((size_t)splits * BH * (d + 1) * d * 4);
+  return L;
+}
+
+cudaError_t launch_linear_reduce(const LinearArgs& a, cudaStream_t s) {
+  return a.d == 64 ? launch_linear_t<64>(a, s) : launch_linear_t<128>(a, s);
+}
+
+cudaError_t launch_linear_export(const uint16_t* sz, const float* gate, int BH, int d, float* S_out, float* z_out,
+                                 cudaStream_t s) {
+  if (d == 64)
+    linear_export_kernel<64><<<BH, 256, 0, s>>>(sz, gate, S_out, z_out);
+  else
+    linear_export_kernel<128><<<BH, 256, 0, s>>>(sz, gate, S_out, z_out);
+  return cudaGetLastError();
+}
+
+}  // namespace salad

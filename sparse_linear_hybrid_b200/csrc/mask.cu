@@ -1,0 +1,127 @@
+// Block-mask builder: static spatio-temporal sliding window (ST-SWA) over a
+// T x H x W token grid in raster order, reduced to a per-head CSR list of kept
+// key blocks (SALAD sparse branch; sciencestack SALAD page, Figure 1 baseline
+// "ST-SWA"; SALAD summary section 2.1).
+//
+// A block of raster-ordered tokens is a union of row segments: each (t, y) row
+// it touches contributes one contiguous x interval.  Block pair (I, J) is kept
+// iff some segment of I and some segment of J have |dt| <= wt, |dy| <= wh and
+// x intervals no more than ww apart.  This is exact for the token-pair rule
+// (some i in I, j in J inside the window) because the window is a box.
+//
+// Three launches: count (one warp per CSR row), an in-place inclusive scan of
+// the counts, fill (one warp per row; ballot compaction keeps columns sorted).
+#include "internal.h"
+
+namespace salad {
+namespace {
+
+__device__ __forceinline__ long long llmin(long long a, long long b) { return a < b ? a : b; }
+
+__device__ bool block_pair_kept(const MaskGrid& g, int wt, int wh, int ww, int I, int J) {
+  const long long a0 = (long long)I * g.block, a1 = llmin(g.N, a0 + g.block) - 1;
+  const long long c0 = (long long)J * g.block, c1 = llmin(g.N, c0 + g.block) - 1;
+  const long long ra0 = a0 / g.W, ra1 = a1 / g.W, rc0 = c0 / g.W, rc1 = c1 / g.W;
+  // frame-level rejection: the frames of I and J are more than wt apart
+  const long long ta0 = ra0 / g.H, ta1 = ra1 / g.H, tc0 = rc0 / g.H, tc1 = rc1 / g.H;
+  if (tc0 - ta1 > wt || ta0 - tc1 > wt) return false;
+  for (long long ra = ra0; ra <= ra1; ++ra) {
+    const int ta = (int)(ra / g.H), ya = (int)(ra % g.H);
+    const int xa0 = ra == ra0 ? (int)(a0 % g.W) : 0;
+    const int xa1 = ra == ra1 ? (int)(a1 % g.W) : g.W - 1;
+    for (long long rc = rc0; rc <= rc1; ++rc) {
+      const int tc = (int)(rc / g.H), yc = (int)(rc % g.H);
+      if (abs(ta - tc) > wt || abs(ya - yc) > wh) continue;
+      const int xc0 = rc == rc0 ? (int)(c0 % g.W) : 0;
+      const int xc1 = rc == rc1 ? (int)(c1 % g.W) : g.W - 1;
+      const int gap = max(0, max(xc0 - xa1, xa0 - xc1));
+      if (gap <= ww) return true;
+    }
+  }
+  return false;
+}
+
+// grid (nb, heads), 32 threads: row_ptr[1 + h*nb + I] = number of kept J.
+__global__ void __launch_bounds__(32) mask_count_kernel(MaskGrid g, WindowTable win, int32_t* row_ptr) {
+  const int I = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
+  const int wt = win.w[3 * h], wh = win.w[3 * h + 1], ww = win.w[3 * h + 2];
+  int cnt = 0;
+  for (int J = lane; J < g.nb; J += 32) cnt += block_pair_kept(g, wt, wh, ww, I, J) ? 1 : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) row_ptr[1 + (long long)h * g.nb + I] = cnt;
+}
+
+// One CTA of 1024 threads: row_ptr[0] = 0, row_ptr[1..n] = inclusive prefix sums.
+__global__ void __launch_bounds__(1024) mask_scan_kernel(int32_t* row_ptr, int n) {
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    carry = 0;
+    row_ptr[0] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < n; base += 1024) {
+    const int i = base + tid;
+    int v = i < n ? row_ptr[1 + i] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      int t = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += u;
+      }
+      warp_tot[lane] = t;
+    }
+    __syncthreads();
+    const int prefix = carry + (warp > 0 ? warp_tot[warp - 1] : 0);
+    if (i < n) row_ptr[1 + i] = prefix + v;
+    __syncthreads();
+    if (tid == 0) carry += warp_tot[31];
+    __syncthreads();
+  }
+}
+
+// grid (nb, heads), 32 threads: ascending kept columns of row (h, I).
+__global__ void __launch_bounds__(32) mask_fill_kernel(MaskGrid g, WindowTable win, const int32_t* row_ptr,
+                                                       int32_t* col_idx) {
+  const int I = blockIdx.x, h = blockIdx.y, lane = threadIdx.x;
+  const int wt = win.w[3 * h], wh = win.w[3 * h + 1], ww = win.w[3 * h + 2];
+  int out = row_ptr[(long long)h * g.nb + I];
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int J0 = 0; J0 < g.nb; J0 += 32) {
+    const int J = J0 + lane;
+    const bool kept = J < g.nb && block_pair_kept(g, wt, wh, ww, I, J);
+    const unsigned m = __ballot_sync(0xffffffffu, kept);
+    if (kept) col_idx[out + __popc(m & lt_mask)] = J;
+    out += __popc(m);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_mask_count(const MaskGrid& g, const WindowTable& win, int32_t* row_ptr, cudaStream_t s) {
+  mask_count_kernel<<<dim3(g.nb, g.heads), 32, 0, s>>>(g, win, row_ptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mask_scan(int32_t* row_ptr, int n, cudaStream_t s) {
+  mask_scan_kernel<<<1, 1024, 0, s>>>(row_ptr, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mask_fill(const MaskGrid& g, const WindowTable& win, const int32_t* row_ptr, int32_t* col_idx,
+                             cudaStream_t s) {
+  mask_fill_kernel<<<dim3(g.nb, g.heads), 32, 0, s>>>(g, win, row_ptr, col_idx);
+  return cudaGetLastError();
+}
+
+}  // namespace salad

@@ -1,0 +1,133 @@
+"""Host-only checks of the C ABI (no GPU needed).
+
+The library must load without a GPU, export every function include/salad.h
+declares, and reject bad arguments with the documented status before anything
+is launched (the pointers below are never dereferenced).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_linear_hybrid_b200 as sl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "salad.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_linear_hybrid_b200 import build
+    build.build()
+    return sl.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(salad_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["salad_build_block_mask", "salad_attn_forward", "salad_workspace_bytes",
+                     "salad_check_status", "salad_status_string", "salad_mask_num_blocks",
+                     "salad_linear_state"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+FAKE = 0x100000  # 16-byte aligned, never dereferenced by argument checks
+
+
+def p(x):
+    return ctypes.c_void_p(x)
+
+
+def forward(L, **kw):
+    a = dict(q=FAKE, k=FAKE + 0x10000000, v=FAKE + 0x20000000, B=1, N=256, H=2, d=64, block=64,
+             row_ptr=FAKE, col_idx=FAKE, w=FAKE, gate=FAKE, scale=0.0, eps=1e-6,
+             out=FAKE + 0x30000000, ws=0x40000000, ws_bytes=1 << 30)
+    a.update(kw)
+    return L.salad_attn_forward(p(a["q"]), p(a["k"]), p(a["v"]), a["B"], a["N"], a["H"], a["d"],
+                                a["block"], p(a["row_ptr"]), p(a["col_idx"]), p(a["w"]),
+                                p(a["gate"]), a["scale"], a["eps"], p(a["out"]), p(a["ws"]),
+                                a["ws_bytes"], None)
+
+
+def test_forward_argument_errors(L):
+    assert forward(L, q=0) == sl.SALAD_ERR_INVALID_ARG
+    assert forward(L, gate=0) == sl.SALAD_ERR_INVALID_ARG
+    assert forward(L, ws=0) == sl.SALAD_ERR_INVALID_ARG
+    assert forward(L, N=0) == sl.SALAD_ERR_INVALID_ARG
+    assert forward(L, B=-1) == sl.SALAD_ERR_INVALID_ARG
+    assert forward(L, d=96) == sl.SALAD_ERR_UNSUPPORTED
+    assert forward(L, d=256) == sl.SALAD_ERR_UNSUPPORTED
+    assert forward(L, block=32) == sl.SALAD_ERR_UNSUPPORTED
+    assert forward(L, q=FAKE + 8) == sl.SALAD_ERR_INVALID_ARG          # misaligned
+    assert forward(L, ws=0x40000000 + 64) == sl.SALAD_ERR_INVALID_ARG   # workspace needs 256 B
+    assert forward(L, ws_bytes=16) == sl.SALAD_ERR_WORKSPACE
+    assert forward(L, eps=-1.0) == sl.SALAD_ERR_INVALID_ARG
+    assert forward(L, eps=float("nan")) == sl.SALAD_ERR_INVALID_ARG
+    assert forward(L, out=FAKE) == sl.SALAD_ERR_INVALID_ARG             # out aliases q
+
+
+def test_workspace_bytes(L):
+    assert L.salad_workspace_bytes(1, 256, 2, 64) > 0
+    assert L.salad_workspace_bytes(1, 256, 2, 96) == 0
+    assert L.salad_workspace_bytes(0, 256, 2, 64) == 0
+    small = L.salad_workspace_bytes(1, 32760, 12, 128)
+    big = L.salad_workspace_bytes(2, 32760, 12, 128)
+    assert big > small > 0
+    assert small % 256 == 0
+
+
+def test_mask_num_blocks_and_mask_errors(L):
+    nb = ctypes.c_int(0)
+    assert L.salad_mask_num_blocks(21, 30, 52, 128, ctypes.byref(nb)) == 0 and nb.value == 256
+    assert L.salad_mask_num_blocks(21, 45, 80, 128, ctypes.byref(nb)) == 0 and nb.value == 591
+    assert L.salad_mask_num_blocks(4, 8, 8, 64, ctypes.byref(nb)) == 0 and nb.value == 4
+    assert L.salad_mask_num_blocks(0, 8, 8, 64, ctypes.byref(nb)) == sl.SALAD_ERR_INVALID_ARG
+    assert L.salad_mask_num_blocks(4, 8, 8, 64, None) == sl.SALAD_ERR_INVALID_ARG
+    assert L.salad_mask_num_blocks(2048, 2048, 2048, 64, ctypes.byref(nb)) == sl.SALAD_ERR_INVALID_ARG
+    import numpy as np
+    win = np.array([[1, 4, 4], [1, -1, 4]], dtype=np.int32)
+    nnz = ctypes.c_int64(0)
+    rc = L.salad_build_block_mask(4, 8, 8, 64, 2, win.ctypes.data_as(ctypes.c_void_p), p(FAKE), None, 0,
+                                  ctypes.byref(nnz), None)
+    assert rc == sl.SALAD_ERR_INVALID_ARG  # negative window
+    win = np.array([[1, 4, 4]], dtype=np.int32)
+    assert L.salad_build_block_mask(4, 8, 8, 64, 0, win.ctypes.data_as(ctypes.c_void_p), p(FAKE), None, 0,
+                                    None, None) == sl.SALAD_ERR_INVALID_ARG
+    assert L.salad_build_block_mask(4, 8, 8, 64, 1, None, p(FAKE), None, 0, None, None) == \
+        sl.SALAD_ERR_INVALID_ARG
+    assert L.salad_build_block_mask(4, 8, 8, 64, 1, win.ctypes.data_as(ctypes.c_void_p), p(FAKE), None, 5,
+                                    None, None) == sl.SALAD_ERR_INVALID_ARG  # capacity without buffer
+
+
+def test_linear_state_argument_errors(L):
+    rc = L.salad_linear_state(p(FAKE), p(FAKE), 1, 256, 2, 64, None, None, p(FAKE), p(0x40000000), 1 << 30, None)
+    assert rc == sl.SALAD_ERR_INVALID_ARG
+    rc = L.salad_linear_state(p(FAKE), p(FAKE), 1, 256, 2, 80, None, p(FAKE), p(FAKE), p(0x40000000), 1 << 30,
+                              None)
+    assert rc == sl.SALAD_ERR_UNSUPPORTED
+
+
+def test_status_strings(L):
+    for code in range(-6, 1):
+        assert sl.status_string(code)
+    assert sl.status_string(-6) == "device-side wait timed out"
+    assert sl.status_string(42) == "unknown status"
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        sl.attn_forward(x, x, x, torch.zeros(3, dtype=torch.int32), torch.zeros(3, dtype=torch.int32),
+                        torch.zeros(64, 64, dtype=torch.bfloat16), torch.zeros(1, 1), 64)
