@@ -44,7 +44,9 @@ FLUSH_BYTES = 256 << 20
 # dram__bytes_read.sum + dram__bytes_write.sum of one attention-kernel launch,
 # from an ncu capture (see profiles/), keyed by the kernel sources it was taken
 # on; stale entries are ignored.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "wan1.3b-32760tok-90pct": {"source": "ca03da024a89505d", "bytes": 303_307_520 + 85_044_736},
+}
 
 
 def kernel_source_hash() -> str:
@@ -144,6 +146,32 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+class DriverEvents:
+    """Raw CUDA events (driver API through ctypes) that the library records on
+    its own stream inside salad_attn_forward; torch.cuda.Event cannot time
+    events recorded outside torch."""
+
+    def __init__(self):
+        import ctypes
+        self.ct = ctypes
+        self.cu = ctypes.CDLL("libcuda.so.1")
+
+    def create(self):
+        ev = self.ct.c_void_p()
+        if self.cu.cuEventCreate(self.ct.byref(ev), 0) != 0:
+            raise RuntimeError("cuEventCreate failed")
+        return ev
+
+    def elapsed_ms(self, a, b) -> float:
+        ms = self.ct.c_float()
+        if self.cu.cuEventElapsedTime(self.ct.byref(ms), a, b) != 0:
+            raise RuntimeError("cuEventElapsedTime failed")
+        return float(ms.value)
+
+    def destroy(self, ev):
+        self.cu.cuEventDestroy_v2(ev)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -241,6 +269,34 @@ def run_reference(args, wl):
 
 
 # --------------------------------------------------------------------------- GPU leg
+def run_e2e(args, q, k, v, w, gate, out, flush, step, flops, world, max_over_ranks, barrier):
+    """Same metric end to end: every step copies its inputs from pinned host
+    memory, runs the C-ABI forward and copies the output back, all between the
+    CUDA events.  Two untimed warm-up steps first."""
+    import torch
+    pin = {n: t.cpu().pin_memory() for n, t in dict(q=q, k=k, v=v, w=w, gate=gate).items()}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    ke = max(3, min(args.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ke + 2)]
+    barrier()
+    for i in range(ke + 2):
+        flush.zero_()
+        a, b = ev[i]
+        a.record()
+        for dst, n in ((q, "q"), (k, "k"), (v, "v"), (w, "w"), (gate, "gate")):
+            dst.copy_(pin[n], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        b.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev[2:]))
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = out_h.numel() * out_h.element_size()
+    return {"value": round(world * ke * flops / (e2e_ms / 1e3) / 1e12, 3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms / ke, 3),
+            "steps": ke}
+
+
 def run_salad(args, wl):
     import torch
     import torch.distributed as dist
@@ -295,7 +351,8 @@ def run_salad(args, wl):
 
     K = args.steps
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    ev = [(E(), E(), E(), E(), E()) for _ in range(K)]
+    drv = DriverEvents()
+    ev = [(E(), drv.create(), drv.create(), drv.create(), E()) for _ in range(K)]
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -304,7 +361,7 @@ def run_salad(args, wl):
         for i in range(K):
             flush.zero_()
             e_start, e_lin, e_att, e_end, e_stop = ev[i]
-            sl.set_phase_events(e_lin, e_att, e_end)
+            sl.lib().salad_set_phase_events(e_lin, e_att, e_end)
             e_start.record()
             step()
             e_stop.record()
@@ -316,8 +373,11 @@ def run_salad(args, wl):
     if status != sl.SALAD_OK:
         raise RuntimeError(f"device status after the timed steps: {sl.status_string(status)}")
     step_ms = [a.elapsed_time(b) for a, _, _, _, b in ev]
-    lin_ms = [b.elapsed_time(c) for _, b, c, _, _ in ev]
-    att_ms = [c.elapsed_time(d) for _, _, c, d, _ in ev]
+    lin_ms = [drv.elapsed_ms(b, c) for _, b, c, _, _ in ev]
+    att_ms = [drv.elapsed_ms(c, d) for _, _, c, d, _ in ev]
+    for _, b, c, d, _ in ev:
+        for x in (b, c, d):
+            drv.destroy(x)
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / K
     value = world * K * flops / (total_ms / 1e3) / 1e12
@@ -349,31 +409,9 @@ def run_salad(args, wl):
 
     # end to end through the C ABI with host buffers: H2D of the step's inputs
     # from pinned memory, the forward, D2H of the output, all inside the events
-    pin = {n: t.cpu().pin_memory() for n, t in dict(q=q, k=k, v=v, w=w, gate=gate).items()}
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    ke = max(3, min(K, 20))
-    e2e_ev = [(E(), E()) for _ in range(ke + 2)]
-    barrier()
-    for i in range(ke + 2):
-        flush.zero_()
-        a, b = e2e_ev[i]
-        a.record()
-        q.copy_(pin["q"], non_blocking=True)
-        k.copy_(pin["k"], non_blocking=True)
-        v.copy_(pin["v"], non_blocking=True)
-        w.copy_(pin["w"], non_blocking=True)
-        gate.copy_(pin["gate"], non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
-        b.record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev[2:]))
-    h2d = sum(t.numel() * t.element_size() for t in pin.values())
-    d2h = out_h.numel() * out_h.element_size()
-    e2e = {"value": round(world * ke * flops / (e2e_ms / 1e3) / 1e12, 3), "unit": UNIT,
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-           "ms_per_step": round(e2e_ms / ke, 3)}
-    del pin, out_h
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, q, k, v, w, gate, out, flush, step, flops, world, max_over_ranks, barrier)
 
     dense = None
     if not args.no_dense:
@@ -424,6 +462,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(si.WORKLOADS))
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-window comparison run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle forward budget for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -182,8 +182,12 @@ def set_wait_limit_ns(limit_ns: int) -> None:
 
 
 def set_phase_events(before_linear=None, before_attention=None, after_attention=None) -> None:
-    """Record these torch.cuda.Event objects inside later attn_forward calls
-    (before the linear-branch kernels, before and after the attention kernel)."""
-    h = [None if e is None else ctypes.c_void_p(e.cuda_event)
-         for e in (before_linear, before_attention, after_attention)]
+    """Record these CUDA events (raw cudaEvent_t handles, or objects with a
+    ``cuda_event`` handle) inside later attn_forward calls: before the
+    linear-branch kernels, before and after the attention kernel."""
+    def handle(e):
+        if e is None or isinstance(e, ctypes.c_void_p):
+            return e
+        return ctypes.c_void_p(e.cuda_event if hasattr(e, "cuda_event") else int(e))
+    h = [handle(e) for e in (before_linear, before_attention, after_attention)]
     lib().salad_set_phase_events(*h)
