@@ -116,6 +116,42 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
                        const float* gate, float softmax_scale, float eps, void* out, void* workspace,
                        size_t workspace_bytes, salad_stream_t stream);
 
+/* Size of the static device scratch behind salad_attn_forward_static: 32 MiB.
+ * The scratch grows with B*Hh, not with N: at d = 128 it covers any N up to
+ * B*Hh = 240 (about 900 at d = 64); the 12-head 32,760-token layer needs 20 MB,
+ * the 40-head 75,600-token one 21 MB. */
+#define SALAD_STATIC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * salad_attn_forward for callers that cannot allocate device memory.  (The
+ * SALAD pages have no counterpart of this entry point; it changes how the
+ * scratch is provided, not what is computed.)
+ *
+ * Some callers cannot call cudaMalloc: a plugin inside a serving engine that
+ * reserves the device memory pool up front and forbids other allocations, or a
+ * latency-critical path that may not pay cudaMalloc's implicit device
+ * synchronisation.  This entry point takes the same arguments as
+ * salad_attn_forward minus the workspace: its scratch is a file-scope static
+ * device array of SALAD_STATIC_SCRATCH_BYTES that every GPU loading the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree or
+ * allocating library routine.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (once, cached); make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the previous call's
+ *     contents; the call clears the status word it needs at zero.  Calls that
+ *     may overlap on the GPU (other streams, other threads) race on the array:
+ *     serialise them.
+ *   - Device time-outs are recorded in the array's status word, which
+ *     salad_check_status cannot see; an output produced after a time-out is
+ *     invalid.
+ * Errors: as salad_attn_forward; WORKSPACE when salad_workspace_bytes(B, N,
+ * num_heads, d) exceeds SALAD_STATIC_SCRATCH_BYTES; CUDA when the scratch
+ * address cannot be obtained.
+ */
+int salad_attn_forward_static(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                              int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                              const float* gate, float softmax_scale, float eps, void* out, salad_stream_t stream);
+
 /*
  * The linear-branch state alone (summary section 2.1: ReLU linear attention),
  * computed by the same kernels salad_attn_forward uses:

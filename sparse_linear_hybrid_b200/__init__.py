@@ -7,7 +7,7 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, workspace_bytes, attn_forward,
-    linear_state, check_status, set_wait_limit_ns, set_phase_events, status_string
+    attn_forward_static, linear_state, check_status, set_wait_limit_ns, set_phase_events, status_string
 """
 from __future__ import annotations
 
@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
         L.salad_workspace_bytes.restype = sz
         L.salad_attn_forward.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
         L.salad_attn_forward.restype = i
+        L.salad_attn_forward_static.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p]
+        L.salad_attn_forward_static.restype = i
         L.salad_linear_state.argtypes = [p, p, i, i, i, i, p, p, p, p, sz, p]
         L.salad_linear_state.restype = i
         L.salad_check_status.argtypes = [p, p]
@@ -153,6 +155,22 @@ def attn_forward(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_sc
         _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps),
         _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream)), "salad_attn_forward")
+    return out
+
+
+def attn_forward_static(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_scale: float = 0.0,
+                        eps: float = 1e-6, out=None, stream=None) -> torch.Tensor:
+    """attn_forward for callers that cannot allocate device memory: the
+    scratch is the library's static device array (see salad.h)."""
+    B, N, Hh, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().salad_attn_forward_static(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
+        B, N, Hh, d, block, _dev_ptr(row_ptr, torch.int32, "row_ptr"),
+        _dev_ptr(col_idx, torch.int32, "col_idx"), _dev_ptr(w_proj, torch.bfloat16, "w_proj"),
+        _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps),
+        _dev_ptr(out, torch.bfloat16, "out"), _stream(stream)), "salad_attn_forward_static")
     return out
 
 
