@@ -1,7 +1,7 @@
 // SALAD hybrid attention forward: block-sparse softmax attention over the kept
 // key blocks (ST-SWA, sciencestack SALAD page Figure 1; the sparse branch of
-// SALAD summary section 2.1) fused with the epilogue of the ReLU linear branch, its
-// static projection and the per-(b, h) gate (summary sections 2.1-2.3):
+// SALAD summary section 2.1) fused with the epilogue of the ReLU linear branch,
+// its static projection and the per-(b, h) gate (summary sections 2.1-2.3):
 //
 //   o_sp  = softmax(scale * q K_kept^T) V_kept          (online softmax)
 //   o_lin = relu(q)^T S / (relu(q) . z + eps)           (S, z from linear.cu)
@@ -13,14 +13,20 @@
 //   warp 0     TMA producer: Q once, then K/V tiles of the kept blocks into a
 //              2-deep ring, then (when g != 0) [S|z] and W for the epilogue;
 //   warp 1     tcgen05 issuer (one thread) and TMEM owner:
-//              S_j = Q K_j^T into one of two TMEM buffers, O += P_j V_j;
-//   warps 2-5  softmax: one query row per thread, online softmax with lazy
-//              rescaling of O in TMEM, P_j written to shared memory as bf16;
-//              then the fused epilogue and one TMA store of bf16 out.
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256, 256+d); the
-// epilogue reuses column 0 for U = relu(Q)[S|z] and then for Y = o_lin W.
-// The [S|z] and o_lin operands are fed as bf16 hi + lo pairs (K doubled), so the
-// epilogue products keep ~16 mantissa bits.
+//              S_j = Q K_j^T (A, B in shared memory) into one of two TMEM
+//              buffers; O += P_j V_j with P_j read from TMEM;
+//   warps 2-5  softmax: one query row per thread; online softmax whose running
+//              maximum is only moved (and O rescaled in TMEM) when it grows by
+//              more than 2^8; P_j written to TMEM as bf16; then the fused
+//              epilogue and one TMA store of bf16 out.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
+// P0 [384,448), P1 [448,512) (bf16 pairs).  P is double-buffered: the
+// softmax writes P_{j+1} while PV_j still reads P_j, and waits on PV_j only
+// when it must rescale O.  Every barrier a role waits on two tiles apart is
+// split per buffer, so no wait can fall a phase behind.  The epilogue reuses [0, d+16) for
+// U = relu(Q)[S|z] and then for Y = o_lin W, and [384, 384+d) for o_lin as bf16
+// hi + lo halves (the A operand of Y).  The [S|z] and o_lin operands are fed as
+// hi + lo pairs (K doubled), so the epilogue products keep ~16 mantissa bits.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -45,32 +51,31 @@ struct AttnCfg {
   static constexpr int W_CH_BYTES = D * 128;
   static constexpr int W_BYTES = DCH * W_CH_BYTES;
   static constexpr int OVL_BYTES = RING_BYTES > SZ_BYTES + W_BYTES ? RING_BYTES : SZ_BYTES + W_BYTES;
-  static constexpr int P_CH = (BLK > D ? BLK : D) / 64;  // P in the loop, o_lo in the epilogue
-  static constexpr int P_BYTES = P_CH * 16384;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + Q_BYTES;
   static constexpr int OFF_K0 = OFF_RING;
   static constexpr int OFF_V0 = OFF_RING + 2 * KV_BYTES;
   static constexpr int OFF_SZ = OFF_RING;
   static constexpr int OFF_W = OFF_RING + SZ_BYTES;
-  static constexpr int OFF_P = OFF_RING + OVL_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + OVL_BYTES;
   static constexpr int SMEM_USED = OFF_BAR + 512 + 1024;
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
   static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_U = 0, TM_Y = 0;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P = 384, TM_U = 0, TM_Y = 0, TM_OLIN = 384;
+  static constexpr uint32_t P_COLS = BLK / 2;       // one P buffer: BLK bf16 per row
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false, false);   // Q K^T
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);     // P V   (V MN-major)
   static constexpr uint32_t IDESC_U = idesc_bf16(128, D + 16, false, false);  // relu(Q) [S|z]
   static constexpr uint32_t IDESC_Y = idesc_bf16(128, D, false, true);      // o_lin W (W MN-major)
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(TM_P + 2 * P_COLS <= 512 && TM_OLIN + D <= 512, "tensor memory budget");
 };
 
 struct AttnShared {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done;
+  uint64_t p_full[2], pv_done[2];
   uint64_t ep_full, q_relu, u_done, a2_full, y_done;
   uint64_t drain;
   uint32_t tmem_base;
@@ -134,6 +139,8 @@ __device__ __forceinline__ void record_timeout(AttnShared* sh, uint32_t* status)
   atomicOr(status, kStatusTimeout);
 }
 
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) { return x & ~(((x >> 15) & 0x00010001u) * 0xFFFFu); }
+
 template <int D, int BLK>
 __global__ void __launch_bounds__(192, 1)
     salad_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -163,9 +170,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&sh->v_empty[s], 1);
       mbar_init(&sh->s_full[s], 1);
       mbar_init(&sh->s_free[s], 4);
+      mbar_init(&sh->pv_done[s], 1);
+      mbar_init(&sh->p_full[s], 4);
     }
-    mbar_init(&sh->p_full, 4);
-    mbar_init(&sh->pv_done, 1);
     mbar_init(&sh->ep_full, 1);
     mbar_init(&sh->q_relu, 4);
     mbar_init(&sh->u_done, 1);
@@ -250,23 +257,22 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       bool ok = mbar_wait(&sh->q_full, 0, limit_ns);
       const uint32_t q_addr = sbase + C::OFF_Q;
-      const uint32_t p_addr = sbase + C::OFF_P;
       KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
       int col, bits, j = 0;
-      // O += P_i V_i
+      // O += P_i V_i, P_i from tensor memory
       auto issue_pv = [&](int i) -> bool {
         const int s = i & 1;
-        if (sh->abort_flag || !mbar_wait(&sh->p_full, (uint32_t)(i & 1), limit_ns)) return false;
+        if (sh->abort_flag || !mbar_wait(&sh->p_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
         if (!mbar_wait(&sh->v_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
         tc_fence_after();
         const uint32_t vt = sbase + C::OFF_V0 + s * C::KV_BYTES;
+        const uint32_t pt = tmem + C::TM_P + s * C::P_COLS;
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk) {
-          const uint64_t a = sw128_desc(p_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(vt + kk * 2048, C::KV_BOX, 1024);
-          mma_bf16_ss(tmem + C::TM_O, a, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::TM_O, pt + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&sh->pv_done);
+        mma_commit(&sh->pv_done[s]);
         mma_commit(&sh->v_empty[s]);
         return true;
       };
@@ -303,18 +309,15 @@ __global__ void __launch_bounds__(192, 1)
             mma_bf16_ss(tmem + C::TM_U, a, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
           }
           mma_commit(&sh->u_done);
-          // Y = [o_hi | o_lo] [W ; W]
+          // Y = [o_hi | o_lo] [W ; W], o_hi | o_lo from tensor memory
           ok = mbar_wait(&sh->a2_full, 0, limit_ns);
           if (ok) {
             tc_fence_after();
             const uint32_t wb = sbase + C::OFF_W;
 #pragma unroll
             for (int kk = 0; kk < 2 * D / 16; ++kk) {
-              const int ch = kk / 4;  // chunk of [o_hi | o_lo]
-              const uint32_t abase = ch < C::DCH ? q_addr + ch * 16384 : p_addr + (ch - C::DCH) * 16384;
-              const uint64_t a = sw128_desc(abase + (kk % 4) * 32, 16, 1024);
               const uint64_t bd = sw128_desc(wb + (kk % (D / 16)) * 2048, C::W_CH_BYTES, 1024);
-              mma_bf16_ss(tmem + C::TM_Y, a, bd, C::IDESC_Y, kk > 0 ? 1u : 0u);
+              mma_bf16_ts(tmem + C::TM_Y, tmem + C::TM_OLIN + kk * 8, bd, C::IDESC_Y, kk > 0 ? 1u : 0u);
             }
             mma_commit(&sh->y_done);
           }
@@ -331,9 +334,9 @@ __global__ void __launch_bounds__(192, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                        // query row within the tile
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int half = BLK == 64 ? (r >> 6) : 0;
+    const int half = BLK == 64 ? (r >> 6) : 0;               // uniform within a warp
     const uint32_t q_addr = sbase + C::OFF_Q;
-    const uint32_t p_addr = sbase + C::OFF_P;
+    const uint64_t c2 = f32x2_pack(scale_log2, scale_log2);
     float m_ref = -INFINITY;  // running reference max (raw score units)
     float l = 0.f;
     bool ok = true;
@@ -344,28 +347,45 @@ __global__ void __launch_bounds__(192, 1)
       const bool aborted = __shfl_sync(0xffffffffu, sh->abort_flag != 0, 0);
       if (aborted || !mbar_wait_warp(&sh->s_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
       tc_fence_after();
-      float sv[BLK];
+      uint32_t sr[BLK];
 #pragma unroll
-      for (int c = 0; c < BLK / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_addr + (s ? C::TM_S1 : C::TM_S0) + c * 32, rr);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(rr[i]);
-      }
+      for (int c = 0; c < BLK / 32; ++c)
+        tmem_ld32(lane_addr + (s ? C::TM_S1 : C::TM_S0) + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->s_free[s]);
 
-      const bool use = ((bits >> half) & 1) != 0;
-      const int valid = min(BLK, N - col * BLK);  // real keys in this block
+      const bool use = ((bits >> half) & 1) != 0;      // warp-uniform
+      const int valid = min(BLK, N - col * BLK);       // real keys in this block
+      // tile maximum: four independent 3-input max chains
+      float mt;
+      if (valid == BLK) {
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < BLK; i += 8) {
+          m0 = fmax3(m0, __uint_as_float(sr[i + 0]), __uint_as_float(sr[i + 1]));
+          m1 = fmax3(m1, __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+          m2 = fmax3(m2, __uint_as_float(sr[i + 4]), __uint_as_float(sr[i + 5]));
+          m3 = fmax3(m3, __uint_as_float(sr[i + 6]), __uint_as_float(sr[i + 7]));
+        }
+        mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      } else {
+        // partial last block: keys past N never count
+#pragma unroll
+        for (int i = 0; i < BLK; ++i)
+          if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < BLK; i += 4) {
+          m0 = fmax3(m0, __uint_as_float(sr[i + 0]), __uint_as_float(sr[i + 1]));
+          m1 = fmax3(m1, __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+        }
+        mt = fmaxf(m0, m1);
+      }
       float alpha = 1.f;
       bool rescale = false;
       if (use) {
-        float mt = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < BLK; ++i)
-          if (i < valid) mt = fmaxf(mt, sv[i]);
         if (m_ref == -INFINITY) {
           m_ref = mt;
         } else if ((mt - m_ref) * scale_log2 > kRescaleThreshold) {
@@ -373,51 +393,67 @@ __global__ void __launch_bounds__(192, 1)
           m_ref = mt;
           rescale = true;
         }
-        const float mb = m_ref * scale_log2;
-        float rs = 0.f;
-#pragma unroll
-        for (int i = 0; i < BLK; ++i) {
-          const float p = i < valid ? ex2_approx(fmaf(sv[i], scale_log2, -mb)) : 0.f;
-          sv[i] = p;
-          rs += p;
-        }
-        l = l * alpha + rs;
-      } else {
-#pragma unroll
-        for (int i = 0; i < BLK; ++i) sv[i] = 0.f;
       }
-      // P_j may overwrite the P buffer and O may be rescaled only after PV_{j-1}
-      if (j >= 1) {
-        if (!mbar_wait_warp(&sh->pv_done, (uint32_t)((j - 1) & 1), limit_ns)) { ok = false; break; }
+      // p = 2^(s * c - m_ref * c) in pairs; rows that do not use the tile write zeros
+      uint32_t pk[BLK / 2];
+      float rs;
+      {
+        const uint64_t nmb2 = f32x2_pack(-m_ref * scale_log2, -m_ref * scale_log2);
+        uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // 0.0f pairs
+#pragma unroll
+        for (int i = 0; i < BLK / 2; ++i) {
+          const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nmb2);
+          float x0, x1;
+          f32x2_unpack(x, x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          const uint64_t pp = f32x2_pack(p0, p1);
+          if ((i & 3) == 0) acc0 = f32x2_add(acc0, pp);
+          if ((i & 3) == 1) acc1 = f32x2_add(acc1, pp);
+          if ((i & 3) == 2) acc2 = f32x2_add(acc2, pp);
+          if ((i & 3) == 3) acc3 = f32x2_add(acc3, pp);
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        const uint64_t a = f32x2_add(f32x2_add(acc0, acc1), f32x2_add(acc2, acc3));
+        float a0, a1;
+        f32x2_unpack(a, a0, a1);
+        rs = a0 + a1;
+      }
+      if (!use) {
+#pragma unroll
+        for (int i = 0; i < BLK / 2; ++i) pk[i] = 0u;
+        rs = 0.f;
+      }
+      l = l * alpha + rs;
+      // P buffer s was last read by PV_{j-2}; O may be rescaled only after PV_{j-1}
+      if (j >= 2) {
+        if (!mbar_wait_warp(&sh->pv_done[s], (uint32_t)(((j - 2) >> 1) & 1), limit_ns)) { ok = false; break; }
+      }
+      if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
+        if (!mbar_wait_warp(&sh->pv_done[s ^ 1], (uint32_t)(((j - 1) >> 1) & 1), limit_ns)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t rr[32];
-            tmem_ld32(lane_addr + C::TM_O + c * 32, rr);
-            tmem_ld_wait();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(lane_addr + C::TM_O + c * 32, rr);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-            tmem_st32(lane_addr + C::TM_O + c * 32, rr);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+          tmem_st32(lane_addr + C::TM_O + c * 32, rr);
         }
       }
+      tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < BLK / 8; ++c) {
-        const uint32_t addr = p_addr + (c / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(c % 8));
-        st_shared_v4(addr, pack_bf16x2(sv[8 * c], sv[8 * c + 1]), pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]),
-                     pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]), pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]));
-      }
-      fence_proxy_async_smem();
+      for (int c = 0; c < BLK / 64; ++c)
+        tmem_st32(lane_addr + C::TM_P + s * C::P_COLS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[c * 32]));
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->p_full);
+      if (lane == 0) mbar_arrive(&sh->p_full[s]);
       ++j;
     }
     const int n = j;
     if (ok && n >= 1) {
-      ok = mbar_wait_warp(&sh->pv_done, (uint32_t)((n - 1) & 1), limit_ns);
+      ok = mbar_wait_warp(&sh->pv_done[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), limit_ns);
       tc_fence_after();
     }
     if (ok) ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);  // the staging area below is the Q tile
@@ -432,11 +468,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t addr = q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)c);
           uint32_t x0, x1, x2, x3;
           ld_shared_v4(addr, x0, x1, x2, x3);
-          x0 &= ~(((x0 >> 15) & 0x00010001u) * 0xFFFFu);
-          x1 &= ~(((x1 >> 15) & 0x00010001u) * 0xFFFFu);
-          x2 &= ~(((x2 >> 15) & 0x00010001u) * 0xFFFFu);
-          x3 &= ~(((x3 >> 15) & 0x00010001u) * 0xFFFFu);
-          st_shared_v4(addr, x0, x1, x2, x3);
+          st_shared_v4(addr, relu_bf16x2(x0), relu_bf16x2(x1), relu_bf16x2(x2), relu_bf16x2(x3));
         }
       fence_proxy_async_smem();
       __syncwarp();
@@ -450,28 +482,26 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld16(lane_addr + C::TM_U + D, zr);
       tmem_ld_wait();
       const float inv_den = 1.f / (__uint_as_float(zr[0]) + eps);
+      // o_lin as bf16 hi + lo halves into tensor memory: hi at TM_OLIN, lo at TM_OLIN + d/2
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_addr + C::TM_U + c * 32, rr);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(lane_addr + C::TM_U + c * 64, ra);
+        tmem_ld32(lane_addr + C::TM_U + c * 64 + 32, rb);
         tmem_ld_wait();
-        uint32_t hi[16], lo[16];
+        uint32_t hi[32], lo[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float o0 = __uint_as_float(rr[2 * i]) * inv_den, o1 = __uint_as_float(rr[2 * i + 1]) * inv_den;
+        for (int i = 0; i < 32; ++i) {
+          const uint32_t* src = i < 16 ? ra : rb;
+          const int k = (i % 16) * 2;
+          const float o0 = __uint_as_float(src[k]) * inv_den, o1 = __uint_as_float(src[k + 1]) * inv_den;
           hi[i] = pack_bf16x2(o0, o1);
           lo[i] = pack_bf16x2(o0 - bf16_lo_to_f32(hi[i]), o1 - bf16_hi_to_f32(hi[i]));
         }
-        // columns [32c, 32c+32): chunk (32c)/64, 16-byte pieces ((32c)%64)/8 .. +3
-        const int ch = (c * 32) / 64, pc0 = ((c * 32) % 64) / 8;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t off = ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)(pc0 + k));
-          st_shared_v4(q_addr + off, hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
-          st_shared_v4(p_addr + off, lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
-        }
+        tmem_st32(lane_addr + C::TM_OLIN + c * 32, hi);
+        tmem_st32(lane_addr + C::TM_OLIN + D / 2 + c * 32, lo);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->a2_full);

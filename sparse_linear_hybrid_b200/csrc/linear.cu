@@ -225,39 +225,71 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// grid (B*Hh, D/16), 256 threads.  CTA (bh, g) owns features c in [16g, 16g+16).
-// sz[bh][e][c] = hi(S[c][e]), sz[bh][e][D+c] = lo(S[c][e]) for e < D; row D holds
-// z the same way; rows D+1 .. D+15 are zero.
+// grid (B*Hh, D/ROWS), 256 threads.  CTA (bh, g) owns features c in
+// [ROWS*g, ROWS*g + ROWS): it sums their split partials in split order (float4
+// loads, coalesced along e), then writes them transposed as bf16 hi + lo:
+// sz[bh][e][c] = hi(S[c][e]), sz[bh][e][D+c] = lo(S[c][e]) for e < D; row D
+// holds z the same way; rows D+1 .. D+15 are zero.
 template <int D>
 __global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __restrict__ partial,
                                                               const float* __restrict__ gate,
                                                               uint16_t* __restrict__ sz, int splits) {
+  constexpr int E4 = D / 4;        // float4 per partial row
+  constexpr int ROWS = 256 / E4;   // features per CTA: 8 (d = 128) or 16 (d = 64)
   const int bh = blockIdx.x, g = blockIdx.y, BH = gridDim.x;
   if (gate != nullptr && gate[bh] == 0.0f) return;
-  __shared__ float acc[16][D + 1];
-  __shared__ float zacc[16];
-  const size_t slab = (size_t)(D + 1) * D;
-  for (int idx = threadIdx.x; idx < 16 * D; idx += 256) {
-    const int cl = idx / D, e = idx % D, c = 16 * g + cl;
-    float s = 0.f;
-    for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * BH + bh) * slab + (size_t)c * D + e];
-    acc[cl][e] = s;
+  __shared__ float acc[ROWS][D + 1];
+  __shared__ float zacc[ROWS];
+  const size_t slab = (size_t)(D + 1) * D, split_stride = (size_t)BH * slab;
+  const int t = threadIdx.x, rr = t / E4, e4 = (t % E4) * 4;
+  const float4* src = reinterpret_cast<const float4*>(partial + (size_t)bh * slab + (size_t)(ROWS * g + rr) * D + e4);
+  const size_t step4 = split_stride / 4;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  int sp = 0;
+  for (; sp + 4 <= splits; sp += 4) {
+    const float4 a0 = src[(size_t)(sp + 0) * step4], a1 = src[(size_t)(sp + 1) * step4];
+    const float4 a2 = src[(size_t)(sp + 2) * step4], a3 = src[(size_t)(sp + 3) * step4];
+    s.x = (((s.x + a0.x) + a1.x) + a2.x) + a3.x;
+    s.y = (((s.y + a0.y) + a1.y) + a2.y) + a3.y;
+    s.z = (((s.z + a0.z) + a1.z) + a2.z) + a3.z;
+    s.w = (((s.w + a0.w) + a1.w) + a2.w) + a3.w;
   }
-  if (threadIdx.x < 16) {
-    const int c = 16 * g + threadIdx.x;
-    float s = 0.f;
-    for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * BH + bh) * slab + (size_t)D * D + c];
-    zacc[threadIdx.x] = s;
+  for (; sp < splits; ++sp) {
+    const float4 a0 = src[(size_t)sp * step4];
+    s.x += a0.x;
+    s.y += a0.y;
+    s.z += a0.z;
+    s.w += a0.w;
+  }
+  acc[rr][e4 + 0] = s.x;
+  acc[rr][e4 + 1] = s.y;
+  acc[rr][e4 + 2] = s.z;
+  acc[rr][e4 + 3] = s.w;
+  if (t < ROWS) {
+    const float* zsrc = partial + (size_t)bh * slab + (size_t)D * D + ROWS * g + t;
+    float z = 0.f;
+    for (int q = 0; q < splits; ++q) z += zsrc[(size_t)q * split_stride];
+    zacc[t] = z;
   }
   __syncthreads();
   uint16_t* out = sz + (size_t)bh * (D + 16) * (2 * D);
-  for (int idx = threadIdx.x; idx < (D + 16) * 16; idx += 256) {
-    const int e = idx / 16, cl = idx % 16, c = 16 * g + cl;
-    const float x = e < D ? acc[cl][e] : (e == D ? zacc[cl] : 0.f);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-    out[(size_t)e * (2 * D) + c] = __bfloat16_as_ushort(hi);
-    out[(size_t)e * (2 * D) + D + c] = __bfloat16_as_ushort(lo);
+  for (int e = t; e < D + 16; e += 256) {
+    uint32_t hi[ROWS / 2], lo[ROWS / 2];
+#pragma unroll
+    for (int k = 0; k < ROWS; k += 2) {
+      const float x0 = e < D ? acc[k][e] : (e == D ? zacc[k] : 0.f);
+      const float x1 = e < D ? acc[k + 1][e] : (e == D ? zacc[k + 1] : 0.f);
+      const uint32_t h = pack_bf16x2(x0, x1);
+      hi[k / 2] = h;
+      lo[k / 2] = pack_bf16x2(x0 - bf16_lo_to_f32(h), x1 - bf16_hi_to_f32(h));
+    }
+    uint4* dh = reinterpret_cast<uint4*>(out + (size_t)e * (2 * D) + ROWS * g);
+    uint4* dl = reinterpret_cast<uint4*>(out + (size_t)e * (2 * D) + D + ROWS * g);
+#pragma unroll
+    for (int k = 0; k < ROWS / 8; ++k) {
+      dh[k] = make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
+      dl[k] = make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+    }
   }
 }
 
@@ -290,7 +322,7 @@ cudaError_t launch_linear_t(const LinearArgs& a, cudaStream_t s) {
       *a.tm_k, *a.tm_v, a.gate, a.partial, a.heads, a.N, a.chunks_per_split, a.status, a.wait_limit_ns);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  linear_finalize_kernel<D><<<dim3(BH, D / 16), 256, 0, s>>>(a.partial, a.gate, a.sz, a.splits);
+  linear_finalize_kernel<D><<<dim3(BH, D / (256 / (D / 4))), 256, 0, s>>>(a.partial, a.gate, a.sz, a.splits);
   return cudaGetLastError();
 }
 
