@@ -57,11 +57,12 @@ struct AttnArgs {
   const CUtensorMap* tm_k;    // box (64, block, 1)
   const CUtensorMap* tm_v;    // box (64, block, 1)
   const CUtensorMap* tm_out;  // box (64, 128, 1)
-  const CUtensorMap* tm_sz;   // box (64, d+16, 1)
+  const CUtensorMap* tm_sz;   // box (64, d, 1): the S rows of [S|z]
   const CUtensorMap* tm_w;    // box (64, d)
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const float* gate;
+  const uint16_t* sz;         // [S|z] operand in the workspace (z is read from its row d)
   int B, N, heads, d, block;
   float scale_log2;  // softmax scale * log2(e)
   float eps;
