@@ -181,7 +181,7 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
   const int BH = B * num_heads;
   const uint64_t sz_dims[3] = {(uint64_t)2 * d, (uint64_t)d + 16, (uint64_t)BH};
   const uint64_t sz_strides[2] = {(uint64_t)2 * d * 2, (uint64_t)(d + 16) * 2 * d * 2};
-  const uint32_t sz_box[3] = {64, (uint32_t)d, 1};
+  const uint32_t sz_box[3] = {64, (uint32_t)d + 16, 1};
   const uint64_t w_dims[2] = {(uint64_t)d, (uint64_t)d};
   const uint64_t w_strides[1] = {(uint64_t)d * 2};
   const uint32_t w_box[2] = {64, (uint32_t)d};

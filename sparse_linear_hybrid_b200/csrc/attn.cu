@@ -9,23 +9,26 @@
 //
 // One CTA owns a 128-row query tile of one (b, h) (two 64-token query blocks
 // when block == 64, whose kept-key lists are merged; a key tile then carries a
-// bit per half saying which rows may see it).  Two CTAs share an SM (about
-// 97 KB of shared memory and 256 tensor-memory columns each), so one CTA's
-// softmax, MMAs, loads and epilogue overlap the other's.  160 threads:
-//   warp 0, lane 0   control: TMA loads (Q once, then the K and V tile of each
-//                    kept block, single-buffered) and the tcgen05 MMAs
-//                    S_j = Q K_j^T and O += P_j V_j;  warp 0 owns the TMEM;
-//   warps 1-4        softmax, one query row per thread: online softmax whose
-//                    running maximum only moves (and O is only rescaled) when
-//                    it grows by more than 2^8; P_j is written as bf16 into the
-//                    first columns of S_j's own tensor memory; then the fused
-//                    epilogue and one TMA store of bf16 out.
-// Tensor memory: S [0, block) (P aliased on its first block/2 columns),
-// O [128, 128+d).  Epilogue (g != 0): U = relu(Q) [S_hi ; S_lo] lands on [0, d),
-// the softmax warps replace it by o' = (l g / (relu(q).z + eps)) U as bf16
-// hi + lo halves, and O += [o'_hi | o'_lo] [W ; W] accumulates the projected
-// linear branch into O, so out = O / l.  [S|z] and o' are split into hi + lo
-// bf16 pairs (K doubled), keeping ~16 mantissa bits in the epilogue products.
+// bit per half saying which rows may see it).  Warp roles, 320 threads:
+//   warp 0     TMA producer: Q once, then K/V tiles of the kept blocks into a
+//              2-deep ring, then (when g != 0) [S|z] and W for the epilogue;
+//   warp 1     tcgen05 issuer (one thread) and TMEM owner:
+//              S_j = Q K_j^T (A, B in shared memory) into one of two TMEM
+//              buffers; O += P_j V_j with P_j read from TMEM;
+//   warps 2-9  softmax, two threads per query row (each takes half of the key
+//              columns of a tile and half of the feature columns of O): online
+//              softmax whose running maximum is only moved (and O rescaled in
+//              TMEM) when it grows by more than 2^8; P_j written to TMEM as
+//              bf16; then the fused epilogue and one TMA store of bf16 out.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
+// P0 [384,448), P1 [448,512) (bf16 pairs).  P is double-buffered: the
+// softmax writes P_{j+1} while PV_j still reads P_j, and waits on PV_j only
+// when it must rescale O.  Every barrier a role waits on two tiles apart is
+// split per buffer, so no wait can fall a phase behind.  The epilogue reuses
+// [0, d+16) for U = relu(Q)[S|z] and then for Y = o_lin W, and [384, 384+d)
+// for o_lin as bf16 hi + lo halves (the A operand of Y).  The [S|z] and o_lin
+// operands are fed as hi + lo pairs (K doubled), so the epilogue products keep
+// ~16 mantissa bits.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -35,42 +38,56 @@ namespace {
 constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
-template <int D, int BLK>
-struct AttnCfg {
-  static constexpr int DCH = D / 64;               // 64-column chunks of a d-wide row
-  static constexpr int Q_BYTES = 128 * D * 2;      // DCH chunks of 16 KB
-  static constexpr int KV_BOX = BLK * 128;         // one [BLK x 64] box
-  static constexpr int KV_BYTES = DCH * KV_BOX;    // one K or V tile
-  static constexpr int SZ_CH = 2 * D / 64;         // K chunks of [S_hi ; S_lo]^T (d rows each)
-  static constexpr int SZ_CH_BYTES = D * 128;
-  static constexpr int SZ_BYTES = SZ_CH * SZ_CH_BYTES;
-  static constexpr int W_CH_BYTES = D * 128;
-  static constexpr int W_BYTES = DCH * W_CH_BYTES;
-  static constexpr int OVL_BYTES = 2 * KV_BYTES > SZ_BYTES ? 2 * KV_BYTES : SZ_BYTES;
-  static constexpr int OFF_Q = 0;                  // Q; relu(Q) in the epilogue; then W
-  static constexpr int OFF_K = Q_BYTES;            // K and V tiles; [S|z] operand; out staging
-  static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_SZ = OFF_K;
-  static constexpr int OFF_W = OFF_Q;
-  static constexpr int OFF_BAR = OFF_K + OVL_BYTES;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t TM_S = 0, TM_O = 128, TM_U = 0, TM_OL = 0;
-  static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false, false);  // Q K^T
-  static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);    // P V   (V MN-major)
-  static constexpr uint32_t IDESC_U = idesc_bf16(128, D, false, false);    // relu(Q) [S_hi ; S_lo]
-  static constexpr uint32_t IDESC_Y = idesc_bf16(128, D, false, true);     // o' W   (W MN-major)
-  static_assert(W_BYTES <= Q_BYTES, "W reuses the Q tile");
-  static_assert(SMEM <= 113 * 1024, "two CTAs per SM");
-};
-
 struct AttnShared {
-  uint64_t q_full, k_full, v_full, k_free;
-  uint64_t s_full, p_full, pv_done;
-  uint64_t sz_full, q_relu, u_done, w_full, a2_full, y_done;
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full[2], pv_done[2];
+  uint64_t ep_full, q_relu, u_done, a2_full, y_done;
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
+  uint64_t xbar[4];       // per lane quarter: the two halves of its rows meet here (64 arrivals)
+  float xmax[2][2][128];  // per tile parity, per half: partial row maxima
+  float xsum[2][128];     // per half: partial row sums
 };
+
+template <int D, int BLK>
+struct AttnCfg {
+  static constexpr int QROWS = 128;
+  static constexpr int DCH = D / 64;                // 64-column chunks of a d-wide row
+  static constexpr int Q_BYTES = QROWS * D * 2;     // DCH chunks of 16 KB
+  static constexpr int KV_BOX = BLK * 128;          // one [BLK x 64] box
+  static constexpr int KV_BYTES = DCH * KV_BOX;     // one K or V tile
+  static constexpr int RING_BYTES = 4 * KV_BYTES;   // K[2], V[2]
+  static constexpr int SZ_ROWS = D + 16;
+  static constexpr int SZ_CH = 2 * D / 64;
+  static constexpr int SZ_CH_BYTES = SZ_ROWS * 128;
+  static constexpr int SZ_BYTES = SZ_CH * SZ_CH_BYTES;
+  static constexpr int W_CH_BYTES = D * 128;
+  static constexpr int W_BYTES = DCH * W_CH_BYTES;
+  static constexpr int OVL_BYTES = RING_BYTES > SZ_BYTES + W_BYTES ? RING_BYTES : SZ_BYTES + W_BYTES;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K0 = OFF_RING;
+  static constexpr int OFF_V0 = OFF_RING + 2 * KV_BYTES;
+  static constexpr int OFF_SZ = OFF_RING;
+  static constexpr int OFF_W = OFF_RING + SZ_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + OVL_BYTES;
+  static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(AttnShared) + 1024;
+  // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
+  static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P = 384, TM_U = 0, TM_Y = 0, TM_OLIN = 384;
+  static constexpr uint32_t P_COLS = BLK / 2;       // one P buffer: BLK bf16 per row
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false, false);   // Q K^T
+  static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);     // P V   (V MN-major)
+  static constexpr uint32_t IDESC_U = idesc_bf16(128, D + 16, false, false);  // relu(Q) [S|z]
+  static constexpr uint32_t IDESC_Y = idesc_bf16(128, D, false, true);      // o_lin W (W MN-major)
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(TM_P + 2 * P_COLS <= 512 && TM_OLIN + D <= 512, "tensor memory budget");
+};
+
+
 
 // Kept key tiles of one 128-row query tile, in ascending key-block order.
 // bits: bit s set when query half s (block == 64) or the whole tile uses it.
@@ -132,13 +149,13 @@ __device__ __forceinline__ void record_timeout(AttnShared* sh, uint32_t* status)
 __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) { return x & ~(((x >> 15) & 0x00010001u) * 0xFFFFu); }
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(160, 2)
+__global__ void __launch_bounds__(320, 1)
     salad_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
                       const __grid_constant__ CUtensorMap tm_sz, const __grid_constant__ CUtensorMap tm_w,
                       const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
-                      const float* __restrict__ gate, const uint16_t* __restrict__ sz, int heads, int N,
-                      int qtiles, float scale_log2, float eps, uint32_t* status, uint64_t limit_ns) {
+                      const float* __restrict__ gate, int heads, int N, int qtiles, float scale_log2, float eps,
+                      uint32_t* status, uint64_t limit_ns) {
   using C = AttnCfg<D, BLK>;
   const int bh = blockIdx.x / qtiles, qtile = blockIdx.x % qtiles;
   const int b = bh / heads, h = bh % heads;
@@ -153,24 +170,28 @@ __global__ void __launch_bounds__(160, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
-    mbar_init(&sh->k_full, 1);
-    mbar_init(&sh->v_full, 1);
-    mbar_init(&sh->k_free, 1);
-    mbar_init(&sh->s_full, 1);
-    mbar_init(&sh->p_full, 4);
-    mbar_init(&sh->pv_done, 1);
-    mbar_init(&sh->sz_full, 1);
-    mbar_init(&sh->q_relu, 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh->k_full[s], 1);
+      mbar_init(&sh->k_empty[s], 1);
+      mbar_init(&sh->v_full[s], 1);
+      mbar_init(&sh->v_empty[s], 1);
+      mbar_init(&sh->s_full[s], 1);
+      mbar_init(&sh->s_free[s], 8);
+      mbar_init(&sh->pv_done[s], 1);
+      mbar_init(&sh->p_full[s], 8);
+    }
+    mbar_init(&sh->ep_full, 1);
+    mbar_init(&sh->q_relu, 8);
     mbar_init(&sh->u_done, 1);
-    mbar_init(&sh->w_full, 1);
-    mbar_init(&sh->a2_full, 4);
+    mbar_init(&sh->a2_full, 8);
     mbar_init(&sh->y_done, 1);
     mbar_init(&sh->drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&sh->xbar[q], 64);
     sh->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(&sh->tmem_base, 256);
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -179,118 +200,132 @@ __global__ void __launch_bounds__(160, 2)
   const uint32_t tmem = sh->tmem_base;
 
   if (warp == 0) {
-    // ============================ control: TMA + tcgen05 (one thread)
+    // ============================ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
       tma_prefetch_map(&tm_out);
-      const uint32_t q_addr = sbase + C::OFF_Q, k_addr = sbase + C::OFF_K, v_addr = sbase + C::OFF_V;
-      KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
-      int col, bits, ncol, nbits;
-      bool have = it.next(col, bits);
-      // TMA bookkeeping for the drain on time-out
-      int k_issued = 0, v_issued = 0, ep_issued = 0;
       mbar_arrive_expect_tx(&sh->q_full, C::Q_BYTES);
 #pragma unroll
       for (int ch = 0; ch < C::DCH; ++ch)
         tma_load_3d(smem + C::OFF_Q + ch * 16384, &tm_q, &sh->q_full, h * D + ch * 64, qtile * 128, b);
-      if (have) {
-        mbar_arrive_expect_tx(&sh->k_full, C::KV_BYTES);
-        mbar_arrive_expect_tx(&sh->v_full, C::KV_BYTES);
+      KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
+      int col, bits, j = 0;
+      bool ok = true;
+      while (it.next(col, bits)) {
+        const int s = j & 1;
+        const uint32_t ph = ((j >> 1) & 1) ^ 1;
+        if (sh->abort_flag || !mbar_wait(&sh->k_empty[s], ph, limit_ns)) { ok = false; break; }
+        mbar_arrive_expect_tx(&sh->k_full[s], C::KV_BYTES);
+        uint8_t* kt = smem + C::OFF_K0 + s * C::KV_BYTES;
 #pragma unroll
-        for (int ch = 0; ch < C::DCH; ++ch) {
-          tma_load_3d(smem + C::OFF_K + ch * C::KV_BOX, &tm_k, &sh->k_full, h * D + ch * 64, col * BLK, b);
-          tma_load_3d(smem + C::OFF_V + ch * C::KV_BOX, &tm_v, &sh->v_full, h * D + ch * 64, col * BLK, b);
-        }
-        k_issued = v_issued = 1;
+        for (int ch = 0; ch < C::DCH; ++ch)
+          tma_load_3d(kt + ch * C::KV_BOX, &tm_k, &sh->k_full[s], h * D + ch * 64, col * BLK, b);
+        if (sh->abort_flag || !mbar_wait(&sh->v_empty[s], ph, limit_ns)) { ok = false; ++j; break; }
+        mbar_arrive_expect_tx(&sh->v_full[s], C::KV_BYTES);
+        uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch)
+          tma_load_3d(vt + ch * C::KV_BOX, &tm_v, &sh->v_full[s], h * D + ch * 64, col * BLK, b);
+        ++j;
       }
+      const int n = j;
+      if (ok && g != 0.0f) {
+        // epilogue operands overwrite the ring: wait until the last uses of both stages are consumed
+        for (int s = 0; s < 2 && ok; ++s) {
+          const int uses = (n - s + 1) / 2;
+          if (uses > 0) {
+            const uint32_t par = (uint32_t)((uses - 1) & 1);
+            ok = mbar_wait(&sh->k_empty[s], par, limit_ns) && mbar_wait(&sh->v_empty[s], par, limit_ns);
+          }
+        }
+        if (ok) {
+          mbar_arrive_expect_tx(&sh->ep_full, C::SZ_BYTES + C::W_BYTES);
+#pragma unroll
+          for (int ch = 0; ch < C::SZ_CH; ++ch)
+            tma_load_3d(smem + C::OFF_SZ + ch * C::SZ_CH_BYTES, &tm_sz, &sh->ep_full, ch * 64, 0, bh);
+#pragma unroll
+          for (int ch = 0; ch < C::DCH; ++ch)
+            tma_load_2d(smem + C::OFF_W + ch * C::W_CH_BYTES, &tm_w, &sh->ep_full, ch * 64, 0);
+        }
+      }
+      if (!ok) {
+        record_timeout(sh, status);
+        // copies already issued must land before the CTA may exit
+        mbar_wait(&sh->q_full, 0, kDrainNs);
+        for (int i = (n > 2 ? n - 2 : 0); i < n; ++i) {
+          mbar_wait(&sh->k_full[i & 1], (i >> 1) & 1, kDrainNs);
+          mbar_wait(&sh->v_full[i & 1], (i >> 1) & 1, kDrainNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ============================ tcgen05 issuer
+    if (lane == 0) {
       bool ok = mbar_wait(&sh->q_full, 0, limit_ns);
-      int j = 0;
-      while (ok && have) {
-        const uint32_t ph = (uint32_t)(j & 1);
-        const bool more = it.next(ncol, nbits);
-        // S_j = Q K_j^T   (the S/P columns are free: PV_{j-1} was awaited below)
-        if (sh->abort_flag || !mbar_wait(&sh->k_full, ph, limit_ns)) { ok = false; break; }
+      const uint32_t q_addr = sbase + C::OFF_Q;
+      KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
+      int col, bits, j = 0;
+      // O += P_i V_i, P_i from tensor memory
+      auto issue_pv = [&](int i) -> bool {
+        const int s = i & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->p_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
+        if (!mbar_wait(&sh->v_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
         tc_fence_after();
+        const uint32_t vt = sbase + C::OFF_V0 + s * C::KV_BYTES;
+        const uint32_t pt = tmem + C::TM_P + s * C::P_COLS;
+#pragma unroll
+        for (int kk = 0; kk < BLK / 16; ++kk) {
+          const uint64_t bd = sw128_desc(vt + kk * 2048, C::KV_BOX, 1024);
+          mma_bf16_ts(tmem + C::TM_O, pt + kk * 8, bd, C::IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&sh->pv_done[s]);
+        mma_commit(&sh->v_empty[s]);
+        return true;
+      };
+      while (ok && it.next(col, bits)) {
+        const int s = j & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->k_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait(&sh->s_free[s], (uint32_t)(((j - 2) >> 1) & 1), limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kt = sbase + C::OFF_K0 + s * C::KV_BYTES;
+        const uint32_t d_s = tmem + (s ? C::TM_S1 : C::TM_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t a = sw128_desc(q_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(k_addr + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
-          mma_bf16_ss(tmem + C::TM_S, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+          const uint64_t bd = sw128_desc(kt + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
+          mma_bf16_ss(d_s, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sh->s_full);
-        mma_commit(&sh->k_free);
-        // K_{j+1} may overwrite K_j once S_j is done
-        if (!mbar_wait(&sh->k_free, ph, limit_ns)) { ok = false; break; }
-        if (more) {
-          mbar_arrive_expect_tx(&sh->k_full, C::KV_BYTES);
-#pragma unroll
-          for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_3d(smem + C::OFF_K + ch * C::KV_BOX, &tm_k, &sh->k_full, h * D + ch * 64, ncol * BLK, b);
-          ++k_issued;
-        }
-        // O += P_j V_j  (P_j from tensor memory, on S_j's columns)
-        if (sh->abort_flag || !mbar_wait(&sh->p_full, ph, limit_ns) || !mbar_wait(&sh->v_full, ph, limit_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BLK / 16; ++kk) {
-          const uint64_t bd = sw128_desc(v_addr + kk * 2048, C::KV_BOX, 1024);
-          mma_bf16_ts(tmem + C::TM_O, tmem + C::TM_S + kk * 8, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&sh->pv_done);
-        // V_{j+1} may overwrite V_j, and S_{j+1} may overwrite P_j, once PV_j is done
-        if (!mbar_wait(&sh->pv_done, ph, limit_ns)) { ok = false; break; }
-        if (more) {
-          mbar_arrive_expect_tx(&sh->v_full, C::KV_BYTES);
-#pragma unroll
-          for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_3d(smem + C::OFF_V + ch * C::KV_BOX, &tm_v, &sh->v_full, h * D + ch * 64, ncol * BLK, b);
-          ++v_issued;
-        }
-        col = ncol;
-        bits = nbits;
-        have = more;
+        mma_commit(&sh->s_full[s]);
+        mma_commit(&sh->k_empty[s]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; ++j; break; }
         ++j;
       }
+      if (ok && j >= 1) ok = issue_pv(j - 1);
       if (ok && g != 0.0f) {
-        // U = relu(Q) [S_hi ; S_lo]  (K = 2d: relu(Q) is fed twice), into S's columns
-        mbar_arrive_expect_tx(&sh->sz_full, C::SZ_BYTES);
-#pragma unroll
-        for (int ch = 0; ch < C::SZ_CH; ++ch)
-          tma_load_3d(smem + C::OFF_SZ + ch * C::SZ_CH_BYTES, &tm_sz, &sh->sz_full, ch * 64, 0, bh);
-        ep_issued = 1;
-        ok = mbar_wait(&sh->q_relu, 0, limit_ns) && mbar_wait(&sh->sz_full, 0, limit_ns);
+        // U = relu(Q) [S_hi ; S_lo | z_hi ; z_lo]   (K = 2d: relu(Q) is fed twice)
+        ok = mbar_wait(&sh->q_relu, 0, limit_ns) && mbar_wait(&sh->ep_full, 0, limit_ns);
         if (ok) {
           tc_fence_after();
+          const uint32_t szb = sbase + C::OFF_SZ;
 #pragma unroll
           for (int kk = 0; kk < 2 * D / 16; ++kk) {
             const int qk = kk % (D / 16);
             const uint64_t a = sw128_desc(q_addr + (qk / 4) * 16384 + (qk % 4) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(sbase + C::OFF_SZ + (kk / 4) * C::SZ_CH_BYTES + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(szb + (kk / 4) * C::SZ_CH_BYTES + (kk % 4) * 32, 16, 1024);
             mma_bf16_ss(tmem + C::TM_U, a, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
           }
           mma_commit(&sh->u_done);
-          // W replaces relu(Q) once U is done
-          ok = mbar_wait(&sh->u_done, 0, limit_ns);
-        }
-        if (ok) {
-          mbar_arrive_expect_tx(&sh->w_full, C::W_BYTES);
-#pragma unroll
-          for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_2d(smem + C::OFF_W + ch * C::W_CH_BYTES, &tm_w, &sh->w_full, ch * 64, 0);
-          ep_issued = 2;
-          // O += [o'_hi | o'_lo] [W ; W]   (o' from tensor memory)
-          ok = mbar_wait(&sh->a2_full, 0, limit_ns) && mbar_wait(&sh->w_full, 0, limit_ns);
+          // Y = [o_hi | o_lo] [W ; W], o_hi | o_lo from tensor memory
+          ok = mbar_wait(&sh->a2_full, 0, limit_ns);
           if (ok) {
             tc_fence_after();
+            const uint32_t wb = sbase + C::OFF_W;
 #pragma unroll
             for (int kk = 0; kk < 2 * D / 16; ++kk) {
-              const uint64_t bd = sw128_desc(sbase + C::OFF_W + (kk % (D / 16)) * 2048, C::W_CH_BYTES, 1024);
-              mma_bf16_ts(tmem + C::TM_O, tmem + C::TM_OL + kk * 8, bd, C::IDESC_Y, (j > 0 || kk > 0) ? 1u : 0u);
+              const uint64_t bd = sw128_desc(wb + (kk % (D / 16)) * 2048, C::W_CH_BYTES, 1024);
+              mma_bf16_ts(tmem + C::TM_Y, tmem + C::TM_OLIN + kk * 8, bd, C::IDESC_Y, kk > 0 ? 1u : 0u);
             }
             mma_commit(&sh->y_done);
           }
@@ -298,64 +333,79 @@ __global__ void __launch_bounds__(160, 2)
       }
       if (!ok) {
         record_timeout(sh, status);
-        // let every copy and MMA this thread started finish before the CTA can exit
         mma_commit(&sh->drain);
         mbar_wait(&sh->drain, 0, kDrainNs);
-        mbar_wait(&sh->q_full, 0, kDrainNs);
-        if (k_issued > 0) mbar_wait(&sh->k_full, (uint32_t)((k_issued - 1) & 1), kDrainNs);
-        if (v_issued > 0) mbar_wait(&sh->v_full, (uint32_t)((v_issued - 1) & 1), kDrainNs);
-        if (ep_issued >= 1) mbar_wait(&sh->sz_full, 0, kDrainNs);
-        if (ep_issued >= 2) mbar_wait(&sh->w_full, 0, kDrainNs);
       }
     }
   } else {
-    // ============================ softmax / epilogue (warps 1..4)
+    // ============================ softmax / epilogue (warps 2..9): two threads per query row
+    // Warps w and w+4 sit on the same TMEM lane quarter (w & 3) and own the same
+    // 32 query rows; hf = 0 takes key columns [0, BLK/2) and feature columns
+    // [0, D/2), hf = 1 the other halves.  The two halves exchange their partial
+    // row maxima through shared memory each tile, so both take the same
+    // (running-max, rescale) decision; partial row sums are combined once at the end.
+    constexpr int HC = BLK / 2;                               // key columns per thread
+    constexpr int HD = D / 2;                                 // feature columns per thread
+    const int sw = warp - 2;
+    const int hf = sw >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                        // query row within the tile
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int half = BLK == 64 ? (r >> 6) : 0;               // uniform within a warp
+    const int half = BLK == 64 ? (r >> 6) : 0;               // query half (block 64), warp-uniform
     const uint32_t q_addr = sbase + C::OFF_Q;
     const uint64_t c2 = f32x2_pack(scale_log2, scale_log2);
-    float m_ref = -INFINITY;  // running reference max (raw score units)
-    float l = 0.f;
+    float m_ref = -INFINITY;  // running reference max (raw score units), same in both halves
+    float l = 0.f;            // this half's share of the row sum
     bool ok = true;
     KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
     int col, bits, j = 0;
     while (it.next(col, bits)) {
-      const uint32_t ph = (uint32_t)(j & 1);
+      const int s = j & 1;
       const bool aborted = __shfl_sync(0xffffffffu, sh->abort_flag != 0, 0);
-      if (aborted || !mbar_wait_warp(&sh->s_full, ph, limit_ns)) { ok = false; break; }
+      if (aborted || !mbar_wait_warp(&sh->s_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
       tc_fence_after();
+      uint32_t sr[HC];
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c)
+        tmem_ld32(lane_addr + (s ? C::TM_S1 : C::TM_S0) + hf * HC + c * 32,
+                  *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->s_free[s]);
+
       const bool use = ((bits >> half) & 1) != 0;      // warp-uniform
-      const int valid = min(BLK, N - col * BLK);       // real keys in this block (warp-uniform)
-      const uint32_t s_addr = lane_addr + C::TM_S;
-      // pass 1: tile maximum, 64 columns at a time, independent 3-input max chains
+      const int valid = min(BLK, N - col * BLK) - hf * HC;  // real keys among this thread's columns
       float mt;
-      {
+      if (valid >= HC) {
         float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int hh = 0; hh < BLK / 64; ++hh) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(s_addr + hh * 64, ra);
-          tmem_ld32(s_addr + hh * 64 + 32, rb);
-          tmem_ld_wait();
-          if (valid < BLK) {  // partial last block: keys past N never count
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (hh * 64 + i >= valid) ra[i] = __float_as_uint(-INFINITY);
-              if (hh * 64 + 32 + i >= valid) rb[i] = __float_as_uint(-INFINITY);
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            m0 = fmax3(m0, __uint_as_float(ra[i + 0]), __uint_as_float(ra[i + 1]));
-            m1 = fmax3(m1, __uint_as_float(ra[i + 2]), __uint_as_float(ra[i + 3]));
-            m2 = fmax3(m2, __uint_as_float(rb[i + 0]), __uint_as_float(rb[i + 1]));
-            m3 = fmax3(m3, __uint_as_float(rb[i + 2]), __uint_as_float(rb[i + 3]));
-          }
+        for (int i = 0; i < HC; i += 8) {
+          m0 = fmax3(m0, __uint_as_float(sr[i + 0]), __uint_as_float(sr[i + 1]));
+          m1 = fmax3(m1, __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+          m2 = fmax3(m2, __uint_as_float(sr[i + 4]), __uint_as_float(sr[i + 5]));
+          m3 = fmax3(m3, __uint_as_float(sr[i + 6]), __uint_as_float(sr[i + 7]));
         }
         mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      } else {
+        // partial last block: keys past N never count (valid may be <= 0 here)
+#pragma unroll
+        for (int i = 0; i < HC; ++i)
+          if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < HC; i += 4) {
+          m0 = fmax3(m0, __uint_as_float(sr[i + 0]), __uint_as_float(sr[i + 1]));
+          m1 = fmax3(m1, __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+        }
+        mt = fmaxf(m0, m1);
       }
+      // both halves of the row agree on the tile maximum (one barrier phase per tile;
+      // a bounded wait, so a time-out on either side cannot hang its partner)
+      sh->xmax[j & 1][hf][r] = mt;
+      mbar_arrive(&sh->xbar[quarter]);
+      if (!mbar_wait_warp(&sh->xbar[quarter], (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+      mt = fmaxf(mt, sh->xmax[j & 1][hf ^ 1][r]);
       float alpha = 1.f;
       bool rescale = false;
       if (use) {
@@ -367,104 +417,98 @@ __global__ void __launch_bounds__(160, 2)
           rescale = true;
         }
       }
-      // pass 2: p = 2^(s * c - m_ref * c) in pairs, 64 columns at a time; P goes
-      // as bf16 pairs over S_j's first block/2 columns (this lane's row only:
-      // columns [32hh, 32hh+32) were read before they are rewritten); rows that
-      // do not use the tile write zeros
+      // p = 2^(s * c - m_ref * c) in pairs; rows that do not use the tile write zeros
+      uint32_t pk[HC / 2];
       float rs;
       {
         const uint64_t nmb2 = f32x2_pack(-m_ref * scale_log2, -m_ref * scale_log2);
         uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // 0.0f pairs
 #pragma unroll
-        for (int hh = 0; hh < BLK / 64; ++hh) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(s_addr + hh * 64, ra);
-          tmem_ld32(s_addr + hh * 64 + 32, rb);
-          tmem_ld_wait();
-          uint32_t pk[32];
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const uint32_t* src = k < 16 ? ra : rb;
-            const int e = (k % 16) * 2;
-            const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(src[e]), __uint_as_float(src[e + 1])), c2, nmb2);
+        for (int i = 0; i < HC / 2; ++i) {
+          const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nmb2);
+          float p0, p1;
+          if ((i & 3) == 3) {
+            // one pair in four on the FMA pipe, relieving the special-function unit
+            exp2_fma_x2(x, p0, p1);
+          } else {
             float x0, x1;
             f32x2_unpack(x, x0, x1);
-            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            if (valid < BLK) {
-              const int cidx = hh * 64 + 2 * k;
-              if (cidx >= valid) p0 = 0.f;
-              if (cidx + 1 >= valid) p1 = 0.f;
-            }
-            const uint64_t pp = f32x2_pack(p0, p1);
-            if ((k & 3) == 0) acc0 = f32x2_add(acc0, pp);
-            if ((k & 3) == 1) acc1 = f32x2_add(acc1, pp);
-            if ((k & 3) == 2) acc2 = f32x2_add(acc2, pp);
-            if ((k & 3) == 3) acc3 = f32x2_add(acc3, pp);
-            pk[k] = use ? pack_bf16x2(p0, p1) : 0u;
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
           }
-          tmem_st32(s_addr + hh * 32, pk);
+          const uint64_t pp = f32x2_pack(p0, p1);
+          if ((i & 3) == 0) acc0 = f32x2_add(acc0, pp);
+          if ((i & 3) == 1) acc1 = f32x2_add(acc1, pp);
+          if ((i & 3) == 2) acc2 = f32x2_add(acc2, pp);
+          if ((i & 3) == 3) acc3 = f32x2_add(acc3, pp);
+          pk[i] = pack_bf16x2(p0, p1);
         }
-        const uint64_t acc = f32x2_add(f32x2_add(acc0, acc1), f32x2_add(acc2, acc3));
+        const uint64_t a = f32x2_add(f32x2_add(acc0, acc1), f32x2_add(acc2, acc3));
         float a0, a1;
-        f32x2_unpack(acc, a0, a1);
-        rs = use ? a0 + a1 : 0.f;
+        f32x2_unpack(a, a0, a1);
+        rs = a0 + a1;
+      }
+      if (!use) {
+#pragma unroll
+        for (int i = 0; i < HC / 2; ++i) pk[i] = 0u;
+        rs = 0.f;
       }
       l = l * alpha + rs;
-      // O holds PV_0 .. PV_{j-1} (all complete: S_j was issued after PV_{j-1} finished)
+      // P buffer s was last read by PV_{j-2}; O may be rescaled only after PV_{j-1}
+      if (j >= 2) {
+        if (!mbar_wait_warp(&sh->pv_done[s], (uint32_t)(((j - 2) >> 1) & 1), limit_ns)) { ok = false; break; }
+      }
       if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
+        if (!mbar_wait_warp(&sh->pv_done[s ^ 1], (uint32_t)(((j - 1) >> 1) & 1), limit_ns)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < HD / 32; ++c) {
           uint32_t rr[32];
-          tmem_ld32(lane_addr + C::TM_O + c * 32, rr);
+          tmem_ld32(lane_addr + C::TM_O + hf * HD + c * 32, rr);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          tmem_st32(lane_addr + C::TM_O + c * 32, rr);
+          tmem_st32(lane_addr + C::TM_O + hf * HD + c * 32, rr);
         }
+      }
+      tc_fence_after();
+      if constexpr (HC / 2 == 32) {
+        tmem_st32(lane_addr + C::TM_P + s * C::P_COLS + hf * (HC / 2), *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      } else {
+        tmem_st16(lane_addr + C::TM_P + s * C::P_COLS + hf * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->p_full);
+      if (lane == 0) mbar_arrive(&sh->p_full[s]);
       ++j;
     }
     const int n = j;
     if (ok && n >= 1) {
-      ok = mbar_wait_warp(&sh->pv_done, (uint32_t)((n - 1) & 1), limit_ns);
+      ok = mbar_wait_warp(&sh->pv_done[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), limit_ns);
       tc_fence_after();
     }
-    if (ok) ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);
+    // the row sum of both halves (barrier phase n)
+    if (ok) {
+      sh->xsum[hf][r] = l;
+      mbar_arrive(&sh->xbar[quarter]);
+      ok = mbar_wait_warp(&sh->xbar[quarter], (uint32_t)(n & 1), limit_ns);
+      if (ok) l += sh->xsum[hf ^ 1][r];
+    }
+    if (ok) ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);  // the staging area below is the Q tile
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const bool lin = ok && g != 0.0f;
-    float den = 0.f;
     if (lin) {
-      // relu(Q) in place (the S MMAs are done with Q); den = relu(q) . z with
-      // z = z_hi + z_lo from row d of the [S|z] operand in global memory
-      const uint16_t* zrow = sz + ((size_t)bh * (D + 16) + D) * (2 * D);
-      float d0 = 0.f, d1 = 0.f;
+      // relu(Q) in place (Q is no longer read by the S MMAs); each half does half the pieces
 #pragma unroll
       for (int ch = 0; ch < C::DCH; ++ch)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t addr = q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)c);
-          uint32_t x[4];
-          ld_shared_v4(addr, x[0], x[1], x[2], x[3]);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) x[k] = relu_bf16x2(x[k]);
-          st_shared_v4(addr, x[0], x[1], x[2], x[3]);
-          const int f0 = ch * 64 + c * 8;  // first feature of this 16-byte piece
-          const uint4 zh = __ldg(reinterpret_cast<const uint4*>(zrow + f0));
-          const uint4 zl = __ldg(reinterpret_cast<const uint4*>(zrow + D + f0));
-          const uint32_t zhw[4] = {zh.x, zh.y, zh.z, zh.w}, zlw[4] = {zl.x, zl.y, zl.z, zl.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float z0 = bf16_lo_to_f32(zhw[k]) + bf16_lo_to_f32(zlw[k]);
-            const float z1 = bf16_hi_to_f32(zhw[k]) + bf16_hi_to_f32(zlw[k]);
-            d0 = fmaf(bf16_lo_to_f32(x[k]), z0, d0);
-            d1 = fmaf(bf16_hi_to_f32(x[k]), z1, d1);
-          }
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t addr = q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)(hf * 4 + c));
+          uint32_t x0, x1, x2, x3;
+          ld_shared_v4(addr, x0, x1, x2, x3);
+          st_shared_v4(addr, relu_bf16x2(x0), relu_bf16x2(x1), relu_bf16x2(x2), relu_bf16x2(x3));
         }
-      den = d0 + d1;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->q_relu);
@@ -473,25 +517,26 @@ __global__ void __launch_bounds__(160, 2)
     if (lin && !lin_ok) ok = false;
     if (lin_ok) {
       tc_fence_after();
-      // o' = (l g / (den + eps)) U, as bf16 hi + lo halves over U's own columns
-      // (32 columns of U at a time; each piece is read before its columns are
-      // rewritten, since o'_hi of columns [32c, 32c+32) lands on [16c, 16c+16))
-      const float sc = l * g / (den + eps);
-      uint32_t ra[D / 32][32];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_addr + C::TM_U + c * 32, ra[c]);
+      uint32_t zr[16];
+      tmem_ld16(lane_addr + C::TM_U + D, zr);
       tmem_ld_wait();
+      const float inv_den = 1.f / (__uint_as_float(zr[0]) + eps);
+      // o_lin of this half's features as bf16 hi + lo halves into tensor memory:
+      // hi of feature pair (2w, 2w+1) at TM_OLIN + w, lo at TM_OLIN + D/2 + w
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t ra[32];
+        tmem_ld32(lane_addr + C::TM_U + hf * HD + c * 32, ra);
+        tmem_ld_wait();
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float o0 = __uint_as_float(ra[c][2 * i]) * sc, o1 = __uint_as_float(ra[c][2 * i + 1]) * sc;
+          const float o0 = __uint_as_float(ra[2 * i]) * inv_den, o1 = __uint_as_float(ra[2 * i + 1]) * inv_den;
           hi[i] = pack_bf16x2(o0, o1);
           lo[i] = pack_bf16x2(o0 - bf16_lo_to_f32(hi[i]), o1 - bf16_hi_to_f32(hi[i]));
         }
-        tmem_st16(lane_addr + C::TM_OL + c * 16, hi);
-        tmem_st16(lane_addr + C::TM_OL + D / 2 + c * 16, lo);
+        tmem_st16(lane_addr + C::TM_OLIN + hf * (HD / 2) + c * 16, hi);
+        tmem_st16(lane_addr + C::TM_OLIN + D / 2 + hf * (HD / 2) + c * 16, lo);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -502,37 +547,44 @@ __global__ void __launch_bounds__(160, 2)
       tc_fence_after();
     }
     if (ok) {
-      // out = O / l  -> bf16 staging over the K/V tiles -> one TMA store per 64 columns
-      const uint32_t st_addr = sbase + C::OFF_K;
+      // out = O / l + g * Y for this half's features -> bf16 staging in the Q tile
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ro[32];
-        if (n >= 1 || lin_ok) {
-          tmem_ld32(lane_addr + C::TM_O + c * 32, ro);
-          tmem_ld_wait();
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t ro[32], ry[32];
+        if (n >= 1) {
+          tmem_ld32(lane_addr + C::TM_O + hf * HD + c * 32, ro);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ro[i] = 0u;
         }
+        if (lin_ok) tmem_ld32(lane_addr + C::TM_Y + hf * HD + c * 32, ry);
+        tmem_ld_wait();
         uint32_t packed[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          packed[i] = pack_bf16x2(__uint_as_float(ro[2 * i]) * inv_l, __uint_as_float(ro[2 * i + 1]) * inv_l);
-        const int ch = (c * 32) / 64, pc0 = ((c * 32) % 64) / 8;
+        for (int i = 0; i < 16; ++i) {
+          float o0 = __uint_as_float(ro[2 * i]) * inv_l, o1 = __uint_as_float(ro[2 * i + 1]) * inv_l;
+          if (lin_ok) {
+            o0 = fmaf(g, __uint_as_float(ry[2 * i]), o0);
+            o1 = fmaf(g, __uint_as_float(ry[2 * i + 1]), o1);
+          }
+          packed[i] = pack_bf16x2(o0, o1);
+        }
+        const int f0 = hf * HD + c * 32;  // first feature of these 32 columns
+        const int ch = f0 / 64, pc0 = (f0 % 64) / 8;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          st_shared_v4(st_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)(pc0 + k)), packed[4 * k],
+          st_shared_v4(q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)(pc0 + k)), packed[4 * k],
                        packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
       }
       fence_proxy_async_smem();
     } else {
       record_timeout(sh, status);
     }
-    named_bar_sync(1, 128);
-    if (threadIdx.x == 32 && !sh->abort_flag) {
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 64 && !sh->abort_flag) {
 #pragma unroll
       for (int ch = 0; ch < C::DCH; ++ch)
-        tma_store_3d(&tm_out, smem + C::OFF_K + ch * 16384, h * D + ch * 64, qtile * 128, b);
+        tma_store_3d(&tm_out, smem + C::OFF_Q + ch * 16384, h * D + ch * 64, qtile * 128, b);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -540,9 +592,9 @@ __global__ void __launch_bounds__(160, 2)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -552,14 +604,11 @@ cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   cudaError_t e =
       cudaFuncSetAttribute(salad_attn_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(salad_attn_kernel<D, BLK>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
   const int qtiles = (a.N + 127) / 128;
   const long long grid = (long long)qtiles * a.B * a.heads;
-  salad_attn_kernel<D, BLK><<<(unsigned)grid, 160, C::SMEM, s>>>(
-      *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_sz, *a.tm_w, a.row_ptr, a.col_idx, a.gate, a.sz, a.heads, a.N,
-      qtiles, a.scale_log2, a.eps, a.status, a.wait_limit_ns);
+  salad_attn_kernel<D, BLK><<<(unsigned)grid, 320, C::SMEM, s>>>(
+      *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_sz, *a.tm_w, a.row_ptr, a.col_idx, a.gate, a.heads, a.N, qtiles,
+      a.scale_log2, a.eps, a.status, a.wait_limit_ns);
   return cudaGetLastError();
 }
 

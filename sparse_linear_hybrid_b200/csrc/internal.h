@@ -57,7 +57,7 @@ struct AttnArgs {
   const CUtensorMap* tm_k;    // box (64, block, 1)
   const CUtensorMap* tm_v;    // box (64, block, 1)
   const CUtensorMap* tm_out;  // box (64, 128, 1)
-  const CUtensorMap* tm_sz;   // box (64, d, 1): the S rows of [S|z]
+  const CUtensorMap* tm_sz;   // box (64, d+16, 1)
   const CUtensorMap* tm_w;    // box (64, d)
   const int32_t* row_ptr;
   const int32_t* col_idx;

@@ -271,6 +271,41 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+// Two non-negative floats to a bf16 pair (round to nearest, ties away from
+// zero) with integer adds and one byte permute, keeping the conversion off the
+// special-function pipe that the exponentials saturate.
+__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the special-function unit.
+// Range reduction (Cody-Waite style, with the round-to-nearest constant
+// 1.5 * 2^23): x = j + f, j integer, |f| <= 1/2; 2^f from a cubic fitted here by
+// least squares at Chebyshev nodes on [-1/2, 1/2] (max relative error 7.5e-5);
+// 2^j applied by adding j to the exponent field.  x is clamped to >= -126:
+// then j >= -126 and the exponent field of the result stays >= 0 (the cubic is
+// in [0.707, 1.415]), so inputs down to -inf give tiny non-negative values.
+__device__ __forceinline__ void exp2_fma_x2(uint64_t x, float& p0, float& p1) {
+  float x0, x1;
+  f32x2_unpack(x, x0, x1);
+  x = f32x2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = f32x2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f32x2_add(x, magic);                                // j sits in t's low mantissa bits
+  const uint64_t jf = f32x2_add(t, f32x2_pack(-12582912.f, -12582912.f));  // j as a float (exact)
+  const uint64_t f = f32x2_fma(jf, f32x2_pack(-1.f, -1.f), x);          // x - j (exact)
+  uint64_t p = f32x2_fma(f32x2_pack(0.0551716648f, 0.0551716648f), f, f32x2_pack(0.242611125f, 0.242611125f));
+  p = f32x2_fma(p, f, f32x2_pack(0.693260968f, 0.693260968f));
+  p = f32x2_fma(p, f, f32x2_pack(0.999928057f, 0.999928057f));
+  float q0, q1, t0, t1;
+  f32x2_unpack(p, q0, q1);
+  f32x2_unpack(t, t0, t1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
