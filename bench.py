@@ -45,7 +45,7 @@ FLUSH_BYTES = 256 << 20
 # from an ncu capture (see profiles/), keyed by the kernel sources it was taken
 # on; stale entries are ignored.
 NCU_TRAFFIC = {
-    "wan1.3b-32760tok-90pct": {"source": "ca03da024a89505d", "bytes": 303_307_520 + 85_044_736},
+    "wan1.3b-32760tok-90pct": {"source": "f4d56b39c27e1f78", "bytes": 303_439_360 + 87_331_328},
 }
 
 
