@@ -118,7 +118,7 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
 
 /* Size of the static device scratch behind salad_attn_forward_static: 32 MiB.
  * The scratch grows with B*Hh, not with N: at d = 128 it covers any N up to
- * B*Hh = 240 (about 900 at d = 64); the 12-head 32,760-token layer needs 20 MB,
+ * B*Hh = 250 (about 1,000 at d = 64); the 12-head 32,760-token layer needs 20 MB,
  * the 40-head 75,600-token one 21 MB. */
 #define SALAD_STATIC_SCRATCH_BYTES (32u << 20)
 

@@ -79,8 +79,10 @@ int check_common(const void* k, const void* v, int B, int N, int Hh, int d, void
   return SALAD_OK;
 }
 
-int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const float* gate, uint8_t* ws,
-               const WorkspaceLayout& L, cudaStream_t s) {
+// The linear-branch kernels.  Forward (S_out == nullptr): z and (S W)^T into the
+// workspace.  State export: S and z into S_out / z_out.
+int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const float* gate, const void* w_proj,
+               float* S_out, float* z_out, uint8_t* ws, const WorkspaceLayout& L, cudaStream_t s) {
   CUtensorMap tk, tv;
   if (!make_bnhd_map(&tk, k, B, N, Hh, d, 64) || !make_bnhd_map(&tv, v, B, N, Hh, d, 64)) return SALAD_ERR_CUDA;
   LinearArgs la{};
@@ -88,7 +90,10 @@ int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const 
   la.tm_v = &tv;
   la.gate = gate;
   la.partial = reinterpret_cast<float*>(ws + L.off_partial);
-  la.sz = reinterpret_cast<uint16_t*>(ws + L.off_sz);
+  la.w = static_cast<const uint16_t*>(w_proj);
+  la.t_op = reinterpret_cast<uint16_t*>(ws + L.off_t);
+  la.z = S_out ? z_out : reinterpret_cast<float*>(ws + L.off_z);
+  la.S_out = S_out;
   la.B = B;
   la.N = N;
   la.heads = Hh;
@@ -174,21 +179,17 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   if (!record(g_ev_linear, s)) return SALAD_ERR_CUDA;
-  st = run_linear(k, v, B, N, num_heads, d, gate, ws, L, s);
+  st = run_linear(k, v, B, N, num_heads, d, gate, w_proj, nullptr, nullptr, ws, L, s);
   if (st != SALAD_OK) return st;
 
-  CUtensorMap tq, tk, tv, to, tsz, tw;
+  CUtensorMap tq, tk, tv, to, tt;
   const int BH = B * num_heads;
-  const uint64_t sz_dims[3] = {(uint64_t)2 * d, (uint64_t)d + 16, (uint64_t)BH};
-  const uint64_t sz_strides[2] = {(uint64_t)2 * d * 2, (uint64_t)(d + 16) * 2 * d * 2};
-  const uint32_t sz_box[3] = {64, (uint32_t)d + 16, 1};
-  const uint64_t w_dims[2] = {(uint64_t)d, (uint64_t)d};
-  const uint64_t w_strides[1] = {(uint64_t)d * 2};
-  const uint32_t w_box[2] = {64, (uint32_t)d};
+  const uint64_t t_dims[3] = {(uint64_t)2 * d, (uint64_t)d, (uint64_t)BH};
+  const uint64_t t_strides[2] = {(uint64_t)2 * d * 2, (uint64_t)d * 2 * d * 2};
+  const uint32_t t_box[3] = {64, (uint32_t)d, 1};
   if (!make_bnhd_map(&tq, q, B, N, num_heads, d, 128) || !make_bnhd_map(&tk, k, B, N, num_heads, d, block) ||
       !make_bnhd_map(&tv, v, B, N, num_heads, d, block) || !make_bnhd_map(&to, out, B, N, num_heads, d, 128) ||
-      !make_map(&tsz, ws + L.off_sz, 3, sz_dims, sz_strides, sz_box) ||
-      !make_map(&tw, w_proj, 2, w_dims, w_strides, w_box))
+      !make_map(&tt, ws + L.off_t, 3, t_dims, t_strides, t_box))
     return SALAD_ERR_CUDA;
 
   AttnArgs aa{};
@@ -196,12 +197,11 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
   aa.tm_k = &tk;
   aa.tm_v = &tv;
   aa.tm_out = &to;
-  aa.tm_sz = &tsz;
-  aa.tm_w = &tw;
+  aa.tm_t = &tt;
   aa.row_ptr = row_ptr;
   aa.col_idx = col_idx;
   aa.gate = gate;
-  aa.sz = reinterpret_cast<const uint16_t*>(ws + L.off_sz);
+  aa.z = reinterpret_cast<const float*>(ws + L.off_z);
   aa.B = B;
   aa.N = N;
   aa.heads = num_heads;
@@ -227,12 +227,7 @@ int salad_linear_state(const void* k, const void* v, int B, int N, int num_heads
   const WorkspaceLayout L = workspace_layout(B, N, num_heads, d);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = run_linear(k, v, B, N, num_heads, d, gate, ws, L, s);
-  if (st != SALAD_OK) return st;
-  return launch_linear_export(reinterpret_cast<const uint16_t*>(ws + L.off_sz), gate, B * num_heads, d, S_out,
-                              z_out, s) == cudaSuccess
-             ? SALAD_OK
-             : SALAD_ERR_CUDA;
+  return run_linear(k, v, B, N, num_heads, d, gate, nullptr, S_out, z_out, ws, L, s);
 }
 
 int salad_check_status(void* workspace, salad_stream_t stream) {

@@ -7,28 +7,35 @@
 //   o_lin = relu(q)^T S / (relu(q) . z + eps)           (S, z from linear.cu)
 //   out   = o_sp + g * (o_lin W);   out = o_sp when g == 0 (branch dropped)
 //
+// The projection is applied to the state ahead of time (linear.cu hands over
+// T = S W), so the linear branch costs one product per query tile:
+//   g * (o_lin W) = g * (relu(q) T) / (relu(q) . z + eps).
+//
 // One CTA owns a 128-row query tile of one (b, h) (two 64-token query blocks
 // when block == 64, whose kept-key lists are merged; a key tile then carries a
 // bit per half saying which rows may see it).  Warp roles, 320 threads:
 //   warp 0     TMA producer: Q once, then K/V tiles of the kept blocks into a
-//              2-deep ring, then (when g != 0) [S|z] and W for the epilogue;
+//              2-deep ring, then (when g != 0) T; once the last S product has
+//              read Q, the whole warp applies ReLU to Q in place;
 //   warp 1     tcgen05 issuer (one thread) and TMEM owner:
 //              S_j = Q K_j^T (A, B in shared memory) into one of two TMEM
-//              buffers; O += P_j V_j with P_j read from TMEM;
+//              buffers; O += P_j V_j with P_j read from TMEM; at the end
+//              U = relu(Q) T into the S buffer the last tile left free, issued
+//              as soon as its operands are in, before or after the last PV;
 //   warps 2-9  softmax, two threads per query row (each takes half of the key
-//              columns of a tile and half of the feature columns of O): online
-//              softmax whose running maximum is only moved (and O rescaled in
-//              TMEM) when it grows by more than 2^8; P_j written to TMEM as
-//              bf16; then the fused epilogue and one TMA store of bf16 out.
+//              columns of a tile and half of the feature columns of O): first
+//              relu(q) . z for their row from the Q tile (while the first S is
+//              computed), then online softmax whose running maximum is only
+//              moved (and O rescaled in TMEM) when it grows by more than 2^8;
+//              P_j written to TMEM as bf16; finally out = O / l + g U / den and
+//              one TMA store of bf16 out.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
 // P0 [384,448), P1 [448,512) (bf16 pairs).  P is double-buffered: the
 // softmax writes P_{j+1} while PV_j still reads P_j, and waits on PV_j only
 // when it must rescale O.  Every barrier a role waits on two tiles apart is
-// split per buffer, so no wait can fall a phase behind.  The epilogue reuses
-// [0, d+16) for U = relu(Q)[S|z] and then for Y = o_lin W, and [384, 384+d)
-// for o_lin as bf16 hi + lo halves (the A operand of Y).  The [S|z] and o_lin
-// operands are fed as hi + lo pairs (K doubled), so the epilogue products keep
-// ~16 mantissa bits.
+// split per buffer, so no wait can fall a phase behind.  T is fed as a hi + lo
+// pair of bf16 halves (K doubled, relu(Q) read twice), so U keeps ~16 mantissa
+// bits of T.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -43,7 +50,7 @@ struct AttnShared {
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], pv_done[2];
-  uint64_t ep_full, q_relu, u_done, a2_full, y_done;
+  uint64_t t_full, q_relu, u_done;
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
@@ -60,31 +67,29 @@ struct AttnCfg {
   static constexpr int KV_BOX = BLK * 128;          // one [BLK x 64] box
   static constexpr int KV_BYTES = DCH * KV_BOX;     // one K or V tile
   static constexpr int RING_BYTES = 4 * KV_BYTES;   // K[2], V[2]
-  static constexpr int SZ_ROWS = D + 16;
-  static constexpr int SZ_CH = 2 * D / 64;
-  static constexpr int SZ_CH_BYTES = SZ_ROWS * 128;
-  static constexpr int SZ_BYTES = SZ_CH * SZ_CH_BYTES;
-  static constexpr int W_CH_BYTES = D * 128;
-  static constexpr int W_BYTES = DCH * W_CH_BYTES;
-  static constexpr int OVL_BYTES = RING_BYTES > SZ_BYTES + W_BYTES ? RING_BYTES : SZ_BYTES + W_BYTES;
+  static constexpr int T_CH = 2 * D / 64;          // 64-column chunks of the [T_hi | T_lo] operand
+  static constexpr int T_CH_BYTES = D * 128;        // D rows (feature f) of 128 bytes
+  static constexpr int T_BYTES = T_CH * T_CH_BYTES;
+  // T goes into the K ring once the last S product has read it when it fits
+  // there (d <= block); otherwise it has a region of its own, loaded up front.
+  static constexpr bool T_IN_RING = D <= BLK;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + Q_BYTES;
   static constexpr int OFF_K0 = OFF_RING;
   static constexpr int OFF_V0 = OFF_RING + 2 * KV_BYTES;
-  static constexpr int OFF_SZ = OFF_RING;
-  static constexpr int OFF_W = OFF_RING + SZ_BYTES;
-  static constexpr int OFF_BAR = OFF_RING + OVL_BYTES;
+  static constexpr int OFF_T = T_IN_RING ? OFF_K0 : OFF_RING + RING_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + RING_BYTES + (T_IN_RING ? 0 : T_BYTES);
   static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(AttnShared) + 1024;
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
   static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P = 384, TM_U = 0, TM_Y = 0, TM_OLIN = 384;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P = 384;
   static constexpr uint32_t P_COLS = BLK / 2;       // one P buffer: BLK bf16 per row
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false, false);   // Q K^T
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);     // P V   (V MN-major)
-  static constexpr uint32_t IDESC_U = idesc_bf16(128, D + 16, false, false);  // relu(Q) [S|z]
-  static constexpr uint32_t IDESC_Y = idesc_bf16(128, D, false, true);      // o_lin W (W MN-major)
+  static constexpr uint32_t IDESC_U = idesc_bf16(128, D, false, false);     // relu(Q) [T_hi ; T_lo]
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(TM_P + 2 * P_COLS <= 512 && TM_OLIN + D <= 512, "tensor memory budget");
+  static_assert(!T_IN_RING || T_BYTES <= 2 * KV_BYTES, "T must fit the K ring");
+  static_assert(TM_P + 2 * P_COLS <= 512 && D <= 128, "tensor memory budget");
 };
 
 
@@ -146,21 +151,26 @@ __device__ __forceinline__ void record_timeout(AttnShared* sh, uint32_t* status)
   atomicOr(status, kStatusTimeout);
 }
 
-__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) { return x & ~(((x >> 15) & 0x00010001u) * 0xFFFFu); }
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0u));
+  return r;
+}
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(320, 1)
     salad_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-                      const __grid_constant__ CUtensorMap tm_sz, const __grid_constant__ CUtensorMap tm_w,
-                      const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
-                      const float* __restrict__ gate, int heads, int N, int qtiles, float scale_log2, float eps,
+                      const __grid_constant__ CUtensorMap tm_t, const int32_t* __restrict__ row_ptr,
+                      const int32_t* __restrict__ col_idx, const float* __restrict__ gate,
+                      const float* __restrict__ zvec, int heads, int N, int qtiles, float scale_log2, float eps,
                       uint32_t* status, uint64_t limit_ns) {
   using C = AttnCfg<D, BLK>;
   const int bh = blockIdx.x / qtiles, qtile = blockIdx.x % qtiles;
   const int b = bh / heads, h = bh % heads;
   const int nb = (N + BLK - 1) / BLK;
   const float g = gate[bh];
+  const bool lin = g != 0.0f;  // the linear branch is dropped for this (b, h) when its gate is 0
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -180,11 +190,9 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&sh->pv_done[s], 1);
       mbar_init(&sh->p_full[s], 8);
     }
-    mbar_init(&sh->ep_full, 1);
-    mbar_init(&sh->q_relu, 8);
+    mbar_init(&sh->t_full, 1);
+    mbar_init(&sh->q_relu, 1);
     mbar_init(&sh->u_done, 1);
-    mbar_init(&sh->a2_full, 8);
-    mbar_init(&sh->y_done, 1);
     mbar_init(&sh->drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&sh->xbar[q], 64);
     sh->abort_flag = 0;
@@ -201,6 +209,8 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ============================ TMA producer
+    int n = 0;
+    bool ok = true, t_issued = false;
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
@@ -210,9 +220,16 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int ch = 0; ch < C::DCH; ++ch)
         tma_load_3d(smem + C::OFF_Q + ch * 16384, &tm_q, &sh->q_full, h * D + ch * 64, qtile * 128, b);
+      auto load_t = [&]() {
+        mbar_arrive_expect_tx(&sh->t_full, C::T_BYTES);
+#pragma unroll
+        for (int ch = 0; ch < C::T_CH; ++ch)
+          tma_load_3d(smem + C::OFF_T + ch * C::T_CH_BYTES, &tm_t, &sh->t_full, ch * 64, 0, bh);
+        t_issued = true;
+      };
+      if (lin && !C::T_IN_RING) load_t();
       KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
       int col, bits, j = 0;
-      bool ok = true;
       while (it.next(col, bits)) {
         const int s = j & 1;
         const uint32_t ph = ((j >> 1) & 1) ^ 1;
@@ -230,35 +247,49 @@ __global__ void __launch_bounds__(320, 1)
           tma_load_3d(vt + ch * C::KV_BOX, &tm_v, &sh->v_full[s], h * D + ch * 64, col * BLK, b);
         ++j;
       }
-      const int n = j;
-      if (ok && g != 0.0f) {
-        // epilogue operands overwrite the ring: wait until the last uses of both stages are consumed
+      n = j;
+      if (ok && lin && C::T_IN_RING) {
+        // T overwrites the K ring: wait until the S products have read both stages
         for (int s = 0; s < 2 && ok; ++s) {
           const int uses = (n - s + 1) / 2;
-          if (uses > 0) {
-            const uint32_t par = (uint32_t)((uses - 1) & 1);
-            ok = mbar_wait(&sh->k_empty[s], par, limit_ns) && mbar_wait(&sh->v_empty[s], par, limit_ns);
-          }
+          if (uses > 0) ok = mbar_wait(&sh->k_empty[s], (uint32_t)((uses - 1) & 1), limit_ns);
         }
-        if (ok) {
-          mbar_arrive_expect_tx(&sh->ep_full, C::SZ_BYTES + C::W_BYTES);
-#pragma unroll
-          for (int ch = 0; ch < C::SZ_CH; ++ch)
-            tma_load_3d(smem + C::OFF_SZ + ch * C::SZ_CH_BYTES, &tm_sz, &sh->ep_full, ch * 64, 0, bh);
-#pragma unroll
-          for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_2d(smem + C::OFF_W + ch * C::W_CH_BYTES, &tm_w, &sh->ep_full, ch * 64, 0);
-        }
+        if (ok) load_t();
       }
-      if (!ok) {
-        record_timeout(sh, status);
-        // copies already issued must land before the CTA may exit
-        mbar_wait(&sh->q_full, 0, kDrainNs);
-        for (int i = (n > 2 ? n - 2 : 0); i < n; ++i) {
-          mbar_wait(&sh->k_full[i & 1], (i >> 1) & 1, kDrainNs);
-          mbar_wait(&sh->v_full[i & 1], (i >> 1) & 1, kDrainNs);
+    }
+    n = __shfl_sync(0xffffffffu, n, 0);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (ok && lin) {
+      // relu(Q) in place, once the last S product has read Q (the commit of
+      // S_{n-1} covers every earlier product as well)
+      bool ready = mbar_wait_warp(&sh->q_full, 0, limit_ns);
+      if (ready && n >= 1)
+        ready = mbar_wait_warp(&sh->k_empty[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), limit_ns);
+      if (ready) {
+        const uint32_t q_addr = sbase + C::OFF_Q;
+#pragma unroll 4
+        for (int u = lane; u < C::Q_BYTES / 16; u += 32) {
+          uint32_t x0, x1, x2, x3;
+          ld_shared_v4(q_addr + u * 16, x0, x1, x2, x3);
+          st_shared_v4(q_addr + u * 16, relu_bf16x2(x0), relu_bf16x2(x1), relu_bf16x2(x2), relu_bf16x2(x3));
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->q_relu);
+      } else {
+        ok = false;
       }
+    }
+    if (lane == 0) {
+      if (!ok) record_timeout(sh, status);
+      // every copy this thread started lands before the CTA may exit (at once
+      // unless another role gave up early)
+      mbar_wait(&sh->q_full, 0, kDrainNs);
+      for (int i = (n > 2 ? n - 2 : 0); i < n; ++i) {
+        mbar_wait(&sh->k_full[i & 1], (i >> 1) & 1, kDrainNs);
+        mbar_wait(&sh->v_full[i & 1], (i >> 1) & 1, kDrainNs);
+      }
+      if (t_issued) mbar_wait(&sh->t_full, 0, kDrainNs);
     }
   } else if (warp == 1) {
     // ============================ tcgen05 issuer
@@ -267,11 +298,9 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t q_addr = sbase + C::OFF_Q;
       KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
       int col, bits, j = 0;
-      // O += P_i V_i, P_i from tensor memory
-      auto issue_pv = [&](int i) -> bool {
+      // O += P_i V_i, P_i from tensor memory (operands already waited for)
+      auto issue_pv_now = [&](int i) {
         const int s = i & 1;
-        if (sh->abort_flag || !mbar_wait(&sh->p_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
-        if (!mbar_wait(&sh->v_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
         tc_fence_after();
         const uint32_t vt = sbase + C::OFF_V0 + s * C::KV_BYTES;
         const uint32_t pt = tmem + C::TM_P + s * C::P_COLS;
@@ -282,6 +311,12 @@ __global__ void __launch_bounds__(320, 1)
         }
         mma_commit(&sh->pv_done[s]);
         mma_commit(&sh->v_empty[s]);
+      };
+      auto issue_pv = [&](int i) -> bool {
+        const int s = i & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->p_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
+        if (!mbar_wait(&sh->v_full[s], (uint32_t)((i >> 1) & 1), limit_ns)) return false;
+        issue_pv_now(i);
         return true;
       };
       while (ok && it.next(col, bits)) {
@@ -302,33 +337,34 @@ __global__ void __launch_bounds__(320, 1)
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; ++j; break; }
         ++j;
       }
-      if (ok && j >= 1) ok = issue_pv(j - 1);
-      if (ok && g != 0.0f) {
-        // U = relu(Q) [S_hi ; S_lo | z_hi ; z_lo]   (K = 2d: relu(Q) is fed twice)
-        ok = mbar_wait(&sh->q_relu, 0, limit_ns) && mbar_wait(&sh->ep_full, 0, limit_ns);
-        if (ok) {
+      // The last PV and U = relu(Q) [T_hi ; T_lo] (K = 2d: relu(Q) is fed twice)
+      // go in whichever order their operands arrive.  U lands in the S buffer
+      // of tile n, whose previous user S_{n-2} the softmax has read by then.
+      const int n = j;
+      bool pv_left = ok && n >= 1, u_left = ok && lin;
+      const int sl = (n - 1) & 1, ub = n & 1;
+      const uint32_t ph_l = (uint32_t)(((n - 1) >> 1) & 1), ph_u = (uint32_t)(((n - 2) >> 1) & 1);
+      const uint64_t t0 = global_timer_ns();
+      while (pv_left || u_left) {
+        if (pv_left && mbar_try_wait(&sh->p_full[sl], ph_l) && mbar_try_wait(&sh->v_full[sl], ph_l)) {
+          issue_pv_now(n - 1);
+          pv_left = false;
+        } else if (u_left && mbar_try_wait(&sh->t_full, 0) && mbar_try_wait(&sh->q_relu, 0) &&
+                   (n < 2 || mbar_try_wait(&sh->s_free[ub], ph_u))) {
           tc_fence_after();
-          const uint32_t szb = sbase + C::OFF_SZ;
+          const uint32_t tb = sbase + C::OFF_T;
 #pragma unroll
           for (int kk = 0; kk < 2 * D / 16; ++kk) {
             const int qk = kk % (D / 16);
             const uint64_t a = sw128_desc(q_addr + (qk / 4) * 16384 + (qk % 4) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(szb + (kk / 4) * C::SZ_CH_BYTES + (kk % 4) * 32, 16, 1024);
-            mma_bf16_ss(tmem + C::TM_U, a, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
+            const uint64_t bd = sw128_desc(tb + (kk / 4) * C::T_CH_BYTES + (kk % 4) * 32, 16, 1024);
+            mma_bf16_ss(tmem + (ub ? C::TM_S1 : C::TM_S0), a, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
           }
           mma_commit(&sh->u_done);
-          // Y = [o_hi | o_lo] [W ; W], o_hi | o_lo from tensor memory
-          ok = mbar_wait(&sh->a2_full, 0, limit_ns);
-          if (ok) {
-            tc_fence_after();
-            const uint32_t wb = sbase + C::OFF_W;
-#pragma unroll
-            for (int kk = 0; kk < 2 * D / 16; ++kk) {
-              const uint64_t bd = sw128_desc(wb + (kk % (D / 16)) * 2048, C::W_CH_BYTES, 1024);
-              mma_bf16_ts(tmem + C::TM_Y, tmem + C::TM_OLIN + kk * 8, bd, C::IDESC_Y, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&sh->y_done);
-          }
+          u_left = false;
+        } else if (sh->abort_flag || global_timer_ns() - t0 > limit_ns) {
+          ok = false;
+          break;
         }
       }
       if (!ok) {
@@ -357,9 +393,35 @@ __global__ void __launch_bounds__(320, 1)
     float m_ref = -INFINITY;  // running reference max (raw score units), same in both halves
     float l = 0.f;            // this half's share of the row sum
     bool ok = true;
+    float gd = 0.f;           // g / (relu(q) . z + eps), the linear branch's row factor
+    if (lin) {
+      // relu(q) . z over all d features of this row (both halves compute it the
+      // same way), while the producer and the MMA warp bring in the first S
+      ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);
+      if (ok) {
+        const float4* zr = reinterpret_cast<const float4*>(zvec + (size_t)bh * D);
+        float den0 = 0.f, den1 = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch)
+#pragma unroll
+          for (int pc = 0; pc < 8; ++pc) {
+            uint32_t x[4];
+            ld_shared_v4(q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)pc), x[0], x[1], x[2], x[3]);
+            const float4 za = __ldg(zr + ch * 16 + pc * 2), zb = __ldg(zr + ch * 16 + pc * 2 + 1);
+            const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t xr = relu_bf16x2(x[i]);
+              den0 = fmaf(bf16_lo_to_f32(xr), zz[2 * i], den0);
+              den1 = fmaf(bf16_hi_to_f32(xr), zz[2 * i + 1], den1);
+            }
+          }
+        gd = g / ((den0 + den1) + eps);
+      }
+    }
     KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
     int col, bits, j = 0;
-    while (it.next(col, bits)) {
+    while (ok && it.next(col, bits)) {
       const int s = j & 1;
       const bool aborted = __shfl_sync(0xffffffffu, sh->abort_flag != 0, 0);
       if (aborted || !mbar_wait_warp(&sh->s_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
@@ -497,76 +559,33 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (ok) ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);  // the staging area below is the Q tile
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    const bool lin = ok && g != 0.0f;
-    if (lin) {
-      // relu(Q) in place (Q is no longer read by the S MMAs); each half does half the pieces
-#pragma unroll
-      for (int ch = 0; ch < C::DCH; ++ch)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t addr = q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)(hf * 4 + c));
-          uint32_t x0, x1, x2, x3;
-          ld_shared_v4(addr, x0, x1, x2, x3);
-          st_shared_v4(addr, relu_bf16x2(x0), relu_bf16x2(x1), relu_bf16x2(x2), relu_bf16x2(x3));
-        }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->q_relu);
-    }
-    bool lin_ok = lin && mbar_wait_warp(&sh->u_done, 0, limit_ns);
-    if (lin && !lin_ok) ok = false;
-    if (lin_ok) {
-      tc_fence_after();
-      uint32_t zr[16];
-      tmem_ld16(lane_addr + C::TM_U + D, zr);
-      tmem_ld_wait();
-      const float inv_den = 1.f / (__uint_as_float(zr[0]) + eps);
-      // o_lin of this half's features as bf16 hi + lo halves into tensor memory:
-      // hi of feature pair (2w, 2w+1) at TM_OLIN + w, lo at TM_OLIN + D/2 + w
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t ra[32];
-        tmem_ld32(lane_addr + C::TM_U + hf * HD + c * 32, ra);
-        tmem_ld_wait();
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float o0 = __uint_as_float(ra[2 * i]) * inv_den, o1 = __uint_as_float(ra[2 * i + 1]) * inv_den;
-          hi[i] = pack_bf16x2(o0, o1);
-          lo[i] = pack_bf16x2(o0 - bf16_lo_to_f32(hi[i]), o1 - bf16_hi_to_f32(hi[i]));
-        }
-        tmem_st16(lane_addr + C::TM_OLIN + hf * (HD / 2) + c * 16, hi);
-        tmem_st16(lane_addr + C::TM_OLIN + D / 2 + hf * (HD / 2) + c * 16, lo);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->a2_full);
-      lin_ok = mbar_wait_warp(&sh->y_done, 0, limit_ns);
-      if (!lin_ok) ok = false;
-      tc_fence_after();
-    }
+    // U has read relu(Q) once u_done completes, so the Q tile is free for staging
+    if (ok && lin) ok = mbar_wait_warp(&sh->u_done, 0, limit_ns);
     if (ok) {
-      // out = O / l + g * Y for this half's features -> bf16 staging in the Q tile
+      tc_fence_after();
+      // out = O / l + g U / den for this half's features -> bf16 staging in the Q tile
+      const uint32_t tm_u = (n & 1) ? C::TM_S1 : C::TM_S0;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
-        uint32_t ro[32], ry[32];
+        uint32_t ro[32], ru[32];
         if (n >= 1) {
           tmem_ld32(lane_addr + C::TM_O + hf * HD + c * 32, ro);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ro[i] = 0u;
         }
-        if (lin_ok) tmem_ld32(lane_addr + C::TM_Y + hf * HD + c * 32, ry);
+        if (lin) {
+          tmem_ld32(lane_addr + tm_u + hf * HD + c * 32, ru);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ru[i] = 0u;
+        }
         tmem_ld_wait();
         uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float o0 = __uint_as_float(ro[2 * i]) * inv_l, o1 = __uint_as_float(ro[2 * i + 1]) * inv_l;
-          if (lin_ok) {
-            o0 = fmaf(g, __uint_as_float(ry[2 * i]), o0);
-            o1 = fmaf(g, __uint_as_float(ry[2 * i + 1]), o1);
-          }
+          const float o0 = fmaf(gd, __uint_as_float(ru[2 * i]), __uint_as_float(ro[2 * i]) * inv_l);
+          const float o1 = fmaf(gd, __uint_as_float(ru[2 * i + 1]), __uint_as_float(ro[2 * i + 1]) * inv_l);
           packed[i] = pack_bf16x2(o0, o1);
         }
         const int f0 = hf * HD + c * 32;  // first feature of these 32 columns
@@ -607,7 +626,7 @@ cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   const int qtiles = (a.N + 127) / 128;
   const long long grid = (long long)qtiles * a.B * a.heads;
   salad_attn_kernel<D, BLK><<<(unsigned)grid, 320, C::SMEM, s>>>(
-      *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_sz, *a.tm_w, a.row_ptr, a.col_idx, a.gate, a.heads, a.N, qtiles,
+      *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_t, a.row_ptr, a.col_idx, a.gate, a.z, a.heads, a.N, qtiles,
       a.scale_log2, a.eps, a.status, a.wait_limit_ns);
   return cudaGetLastError();
 }

@@ -32,7 +32,8 @@ struct WorkspaceLayout {
   int splits;             // split-N factor of the linear-branch reduction
   int chunks_per_split;   // 64-token chunks per split
   size_t off_status;      // uint32 status word
-  size_t off_sz;          // bf16 [B*Hh][d+16][2d]: [S | z]^T split into hi and lo halves
+  size_t off_t;           // bf16 [B*Hh][d][2d]: (S W)^T split into hi and lo halves
+  size_t off_z;           // fp32 [B*Hh][d]: z
   size_t off_partial;     // fp32 [splits][B*Hh][d+1][d]: per-split S rows, then z
   size_t total;
 };
@@ -43,26 +44,26 @@ struct LinearArgs {
   const CUtensorMap* tm_v;
   const float* gate;        // nullable
   float* partial;
-  uint16_t* sz;
+  const uint16_t* w;        // forward: bf16 [d][d] projection
+  uint16_t* t_op;           // forward: (S W)^T hi | lo, bf16 [B*Hh][d][2d]
+  float* z;                 // fp32 [B*Hh][d]
+  float* S_out;             // state export: fp32 [B*Hh][d][d]; null in the forward
   int B, N, heads, d, splits, chunks_per_split;
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
 cudaError_t launch_linear_reduce(const LinearArgs& a, cudaStream_t s);
-cudaError_t launch_linear_export(const uint16_t* sz, const float* gate, int BH, int d, float* S_out, float* z_out,
-                                 cudaStream_t s);
 
 struct AttnArgs {
   const CUtensorMap* tm_q;    // box (64, 128, 1)
   const CUtensorMap* tm_k;    // box (64, block, 1)
   const CUtensorMap* tm_v;    // box (64, block, 1)
   const CUtensorMap* tm_out;  // box (64, 128, 1)
-  const CUtensorMap* tm_sz;   // box (64, d+16, 1)
-  const CUtensorMap* tm_w;    // box (64, d)
+  const CUtensorMap* tm_t;    // box (64, d, 1) over (S W)^T hi | lo
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const float* gate;
-  const uint16_t* sz;         // [S|z] operand in the workspace (z is read from its row d)
+  const float* z;             // fp32 [B*Hh][d]
   int B, N, heads, d, block;
   float scale_log2;  // softmax scale * log2(e)
   float eps;

@@ -10,8 +10,9 @@
 // operands MN-major and the fp32 accumulator in tensor memory.  The CTA writes
 // its partial S and z in fp32.
 // linear_finalize_kernel: fixed-order sum of the partials (deterministic), then
-// [S | z] transposed and split into bf16 hi + lo halves, the B operand layout
-// the attention epilogue feeds to the tensor cores.
+// either S and z in fp32 (the state export) or z in fp32 plus the projected
+// state S W as bf16 hi + lo halves in the B operand layout the attention
+// epilogue feeds to the tensor cores.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -227,32 +228,55 @@ __global__ void __launch_bounds__(192, 1)
 
 // grid (B*Hh, D/ROWS), 256 threads.  CTA (bh, g) owns features c in
 // [ROWS*g, ROWS*g + ROWS): it sums their split partials in split order (float4
-// loads, coalesced along e), then writes them transposed as bf16 hi + lo:
-// sz[bh][e][c] = hi(S[c][e]), sz[bh][e][D+c] = lo(S[c][e]) for e < D; row D
-// holds z the same way; rows D+1 .. D+15 are zero.
-template <int D>
+// loads, coalesced along e), a fixed order, so results do not vary run to run.
+//   EXPORT:  S_out[bh][c][e] and z_out[bh][c] in fp32 (salad_linear_state).
+//   forward: z_out[bh][c] in fp32 and the projected state T = S W,
+//            T[c][f] = sum_e S[c][e] W[e][f], transposed and split into bf16
+//            hi + lo halves: t_op[bh][f][c] = hi(T[c][f]), t_op[bh][f][D+c] =
+//            lo(T[c][f]).  That is the K-major B operand of the attention
+//            epilogue's U = relu(q) T, so the projection is applied to the state
+//            once per (b, h) instead of to every query row:
+//            (relu(q) S / den) W = relu(q) (S W) / den.
+template <int D, bool EXPORT>
 __global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __restrict__ partial,
                                                               const float* __restrict__ gate,
-                                                              uint16_t* __restrict__ sz, int splits) {
+                                                              const uint16_t* __restrict__ w,
+                                                              uint16_t* __restrict__ t_op, float* __restrict__ z_out,
+                                                              float* __restrict__ S_out, int splits) {
   constexpr int E4 = D / 4;        // float4 per partial row
   constexpr int ROWS = 256 / E4;   // features per CTA: 8 (d = 128) or 16 (d = 64)
+  constexpr int FG = 256 / D;      // thread groups sharing a projected column f
+  constexpr int RPT = ROWS / FG;   // rows of T per thread: 4
+  constexpr int WV = D * D / 8;    // 16-byte pieces of W
   const int bh = blockIdx.x, g = blockIdx.y, BH = gridDim.x;
   if (gate != nullptr && gate[bh] == 0.0f) return;
-  __shared__ float acc[ROWS][D + 1];
-  __shared__ float zacc[ROWS];
-  const size_t slab = (size_t)(D + 1) * D, split_stride = (size_t)BH * slab;
+  __shared__ __align__(16) float acc[ROWS][D];
+  __shared__ __align__(16) uint16_t wsm[EXPORT ? 8 : D * D];
   const int t = threadIdx.x, rr = t / E4, e4 = (t % E4) * 4;
+  if constexpr (!EXPORT) {
+    // W into shared memory first: its loads are in flight with the partials'
+    uint4 wv[WV / 256];
+#pragma unroll
+    for (int i = 0; i < WV / 256; ++i) wv[i] = __ldg(reinterpret_cast<const uint4*>(w) + i * 256 + t);
+#pragma unroll
+    for (int i = 0; i < WV / 256; ++i) reinterpret_cast<uint4*>(wsm)[i * 256 + t] = wv[i];
+  }
+  const size_t slab = (size_t)(D + 1) * D, split_stride = (size_t)BH * slab;
   const float4* src = reinterpret_cast<const float4*>(partial + (size_t)bh * slab + (size_t)(ROWS * g + rr) * D + e4);
   const size_t step4 = split_stride / 4;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
   int sp = 0;
-  for (; sp + 4 <= splits; sp += 4) {
-    const float4 a0 = src[(size_t)(sp + 0) * step4], a1 = src[(size_t)(sp + 1) * step4];
-    const float4 a2 = src[(size_t)(sp + 2) * step4], a3 = src[(size_t)(sp + 3) * step4];
-    s.x = (((s.x + a0.x) + a1.x) + a2.x) + a3.x;
-    s.y = (((s.y + a0.y) + a1.y) + a2.y) + a3.y;
-    s.z = (((s.z + a0.z) + a1.z) + a2.z) + a3.z;
-    s.w = (((s.w + a0.w) + a1.w) + a2.w) + a3.w;
+  for (; sp + 8 <= splits; sp += 8) {
+    float4 a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = src[(size_t)(sp + i) * step4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      s.x += a[i].x;
+      s.y += a[i].y;
+      s.z += a[i].z;
+      s.w += a[i].w;
+    }
   }
   for (; sp < splits; ++sp) {
     const float4 a0 = src[(size_t)sp * step4];
@@ -261,53 +285,50 @@ __global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __res
     s.z += a0.z;
     s.w += a0.w;
   }
-  acc[rr][e4 + 0] = s.x;
-  acc[rr][e4 + 1] = s.y;
-  acc[rr][e4 + 2] = s.z;
-  acc[rr][e4 + 3] = s.w;
   if (t < ROWS) {
     const float* zsrc = partial + (size_t)bh * slab + (size_t)D * D + ROWS * g + t;
     float z = 0.f;
     for (int q = 0; q < splits; ++q) z += zsrc[(size_t)q * split_stride];
-    zacc[t] = z;
+    z_out[(size_t)bh * D + ROWS * g + t] = z;
   }
-  __syncthreads();
-  uint16_t* out = sz + (size_t)bh * (D + 16) * (2 * D);
-  for (int e = t; e < D + 16; e += 256) {
-    uint32_t hi[ROWS / 2], lo[ROWS / 2];
+  if constexpr (EXPORT) {
+    float* dst = S_out + ((size_t)bh * D + ROWS * g + rr) * D + e4;  // S_out is only 4-byte aligned
+    dst[0] = s.x;
+    dst[1] = s.y;
+    dst[2] = s.z;
+    dst[3] = s.w;
+  } else {
+    *reinterpret_cast<float4*>(&acc[rr][e4]) = s;
+    __syncthreads();
+    // thread (f, fg): T rows ROWS*g + fg*RPT + k, column f
+    const int f = t % D, fg = t / D;
+    float tr[RPT];
 #pragma unroll
-    for (int k = 0; k < ROWS; k += 2) {
-      const float x0 = e < D ? acc[k][e] : (e == D ? zacc[k] : 0.f);
-      const float x1 = e < D ? acc[k + 1][e] : (e == D ? zacc[k + 1] : 0.f);
-      const uint32_t h = pack_bf16x2(x0, x1);
+    for (int k = 0; k < RPT; ++k) tr[k] = 0.f;
+#pragma unroll 4
+    for (int e = 0; e < D; e += 4) {
+      float we[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) we[i] = __uint_as_float((uint32_t)wsm[(e + i) * D + f] << 16);
+#pragma unroll
+      for (int k = 0; k < RPT; ++k) {
+        const float4 sv = *reinterpret_cast<const float4*>(&acc[fg * RPT + k][e]);
+        tr[k] = fmaf(sv.x, we[0], tr[k]);
+        tr[k] = fmaf(sv.y, we[1], tr[k]);
+        tr[k] = fmaf(sv.z, we[2], tr[k]);
+        tr[k] = fmaf(sv.w, we[3], tr[k]);
+      }
+    }
+    uint32_t hi[RPT / 2], lo[RPT / 2];
+#pragma unroll
+    for (int k = 0; k < RPT; k += 2) {
+      const uint32_t h = pack_bf16x2(tr[k], tr[k + 1]);
       hi[k / 2] = h;
-      lo[k / 2] = pack_bf16x2(x0 - bf16_lo_to_f32(h), x1 - bf16_hi_to_f32(h));
+      lo[k / 2] = pack_bf16x2(tr[k] - bf16_lo_to_f32(h), tr[k + 1] - bf16_hi_to_f32(h));
     }
-    uint4* dh = reinterpret_cast<uint4*>(out + (size_t)e * (2 * D) + ROWS * g);
-    uint4* dl = reinterpret_cast<uint4*>(out + (size_t)e * (2 * D) + D + ROWS * g);
-#pragma unroll
-    for (int k = 0; k < ROWS / 8; ++k) {
-      dh[k] = make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
-      dl[k] = make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
-    }
-  }
-}
-
-// S_out[bh][c][e] = hi + lo, z_out[bh][c] likewise (for salad_linear_state).
-template <int D>
-__global__ void linear_export_kernel(const uint16_t* __restrict__ sz, const float* __restrict__ gate,
-                                     float* __restrict__ S_out, float* __restrict__ z_out) {
-  const int bh = blockIdx.x;
-  if (gate != nullptr && gate[bh] == 0.0f) return;
-  const uint16_t* in = sz + (size_t)bh * (D + 16) * (2 * D);
-  for (int idx = threadIdx.x; idx < (D + 1) * D; idx += blockDim.x) {
-    const int e = idx / D, c = idx % D;  // row e of sz, feature c
-    const float v = __bfloat162float(__ushort_as_bfloat16(in[(size_t)e * 2 * D + c])) +
-                    __bfloat162float(__ushort_as_bfloat16(in[(size_t)e * 2 * D + D + c]));
-    if (e < D)
-      S_out[((size_t)bh * D + c) * D + e] = v;
-    else
-      z_out[(size_t)bh * D + c] = v;
+    uint16_t* row = t_op + ((size_t)bh * D + f) * (2 * D) + ROWS * g + fg * RPT;
+    *reinterpret_cast<uint2*>(row) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2*>(row + D) = make_uint2(lo[0], lo[1]);
   }
 }
 
@@ -322,7 +343,13 @@ cudaError_t launch_linear_t(const LinearArgs& a, cudaStream_t s) {
       *a.tm_k, *a.tm_v, a.gate, a.partial, a.heads, a.N, a.chunks_per_split, a.status, a.wait_limit_ns);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  linear_finalize_kernel<D><<<dim3(BH, D / (256 / (D / 4))), 256, 0, s>>>(a.partial, a.gate, a.sz, a.splits);
+  const dim3 fgrid(BH, D / (256 / (D / 4)));
+  if (a.S_out != nullptr)
+    linear_finalize_kernel<D, true><<<fgrid, 256, 0, s>>>(a.partial, a.gate, nullptr, nullptr, a.z, a.S_out,
+                                                         a.splits);
+  else
+    linear_finalize_kernel<D, false><<<fgrid, 256, 0, s>>>(a.partial, a.gate, a.w, a.t_op, a.z, nullptr,
+                                                          a.splits);
   return cudaGetLastError();
 }
 
@@ -342,23 +369,15 @@ WorkspaceLayout workspace_layout(int B, int N, int heads, int d) {
   L.chunks_per_split = cps;
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   L.off_status = 0;
-  L.off_sz = 256;
-  L.off_partial = L.off_sz + up((size_t)BH * (d + 16) * (2 * d) * 2);
+  L.off_t = 256;
+  L.off_z = L.off_t + up((size_t)BH * d * (2 * d) * 2);
+  L.off_partial = L.off_z + up((size_t)BH * d * 4);
   L.total = L.off_partial + up((size_t)splits * BH * (d + 1) * d * 4);
   return L;
 }
 
 cudaError_t launch_linear_reduce(const LinearArgs& a, cudaStream_t s) {
   return a.d == 64 ? launch_linear_t<64>(a, s) : launch_linear_t<128>(a, s);
-}
-
-cudaError_t launch_linear_export(const uint16_t* sz, const float* gate, int BH, int d, float* S_out, float* z_out,
-                                 cudaStream_t s) {
-  if (d == 64)
-    linear_export_kernel<64><<<BH, 256, 0, s>>>(sz, gate, S_out, z_out);
-  else
-    linear_export_kernel<128><<<BH, 256, 0, s>>>(sz, gate, S_out, z_out);
-  return cudaGetLastError();
 }
 
 }  // namespace salad

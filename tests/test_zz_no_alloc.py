@@ -52,7 +52,7 @@ def test_static_scratch_forward_matches_workspace_forward_on_consecutive_calls()
 
 
 def test_static_scratch_rejects_sizes_beyond_its_maximum():
-    # 8 x 40 heads at d = 128 need about 45 MB of scratch, more than the static array
+    # 8 x 40 heads at d = 128 need about 42 MB of scratch, more than the static array
     B, N, Hh, d = 8, 75600, 40, 128
     assert sl.workspace_bytes(B, N, Hh, d) > 32 << 20
     fake = ctypes.c_void_p(0x100000)
