@@ -13,10 +13,13 @@
 //
 // One CTA owns a 128-row query tile of one (b, h) (two 64-token query blocks
 // when block == 64, whose kept-key lists are merged; a key tile then carries a
-// bit per half saying which rows may see it).  Warp roles, 320 threads:
-//   warp 0     TMA producer: Q once, then K/V tiles of the kept blocks into a
+// bit per half saying which rows may see it).  Warp roles, 352 threads:
+//   warp 0     TMA producer: Q once, then K tiles of the kept blocks into a
 //              2-deep ring, then (when g != 0) T; once the last S product has
 //              read Q, the whole warp applies ReLU to Q in place;
+//   warp 10    TMA producer of the V tiles (2-deep ring).  A V stage frees up
+//              only when its PV is done; with K and V in one issue order the
+//              next K (and so the next S) would wait for that PV as well;
 //   warp 1     tcgen05 issuer (one thread) and TMEM owner:
 //              S_j = Q K_j^T (A, B in shared memory) into one of two TMEM
 //              buffers; O += P_j V_j with P_j read from TMEM; at the end
@@ -158,7 +161,7 @@ __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
 }
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     salad_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
                       const __grid_constant__ CUtensorMap tm_t, const int32_t* __restrict__ row_ptr,
@@ -214,7 +217,6 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
-      tma_prefetch_map(&tm_v);
       tma_prefetch_map(&tm_out);
       mbar_arrive_expect_tx(&sh->q_full, C::Q_BYTES);
 #pragma unroll
@@ -239,12 +241,6 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
           tma_load_3d(kt + ch * C::KV_BOX, &tm_k, &sh->k_full[s], h * D + ch * 64, col * BLK, b);
-        if (sh->abort_flag || !mbar_wait(&sh->v_empty[s], ph, limit_ns)) { ok = false; ++j; break; }
-        mbar_arrive_expect_tx(&sh->v_full[s], C::KV_BYTES);
-        uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
-#pragma unroll
-        for (int ch = 0; ch < C::DCH; ++ch)
-          tma_load_3d(vt + ch * C::KV_BOX, &tm_v, &sh->v_full[s], h * D + ch * 64, col * BLK, b);
         ++j;
       }
       n = j;
@@ -285,11 +281,28 @@ __global__ void __launch_bounds__(320, 1)
       // every copy this thread started lands before the CTA may exit (at once
       // unless another role gave up early)
       mbar_wait(&sh->q_full, 0, kDrainNs);
-      for (int i = (n > 2 ? n - 2 : 0); i < n; ++i) {
-        mbar_wait(&sh->k_full[i & 1], (i >> 1) & 1, kDrainNs);
-        mbar_wait(&sh->v_full[i & 1], (i >> 1) & 1, kDrainNs);
-      }
+      for (int i = (n > 2 ? n - 2 : 0); i < n; ++i) mbar_wait(&sh->k_full[i & 1], (i >> 1) & 1, kDrainNs);
       if (t_issued) mbar_wait(&sh->t_full, 0, kDrainNs);
+    }
+  } else if (warp == 10) {
+    // ============================ TMA producer of the V tiles
+    if (lane == 0) {
+      tma_prefetch_map(&tm_v);
+      KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
+      int col, bits, j = 0;
+      bool ok = true;
+      while (it.next(col, bits)) {
+        const int s = j & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->v_empty[s], ((j >> 1) & 1) ^ 1, limit_ns)) { ok = false; break; }
+        mbar_arrive_expect_tx(&sh->v_full[s], C::KV_BYTES);
+        uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch)
+          tma_load_3d(vt + ch * C::KV_BOX, &tm_v, &sh->v_full[s], h * D + ch * 64, col * BLK, b);
+        ++j;
+      }
+      if (!ok) record_timeout(sh, status);
+      for (int i = (j > 2 ? j - 2 : 0); i < j; ++i) mbar_wait(&sh->v_full[i & 1], (i >> 1) & 1, kDrainNs);
     }
   } else if (warp == 1) {
     // ============================ tcgen05 issuer
@@ -625,7 +638,7 @@ cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int qtiles = (a.N + 127) / 128;
   const long long grid = (long long)qtiles * a.B * a.heads;
-  salad_attn_kernel<D, BLK><<<(unsigned)grid, 320, C::SMEM, s>>>(
+  salad_attn_kernel<D, BLK><<<(unsigned)grid, 352, C::SMEM, s>>>(
       *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_t, a.row_ptr, a.col_idx, a.gate, a.z, a.heads, a.N, qtiles,
       a.scale_log2, a.eps, a.status, a.wait_limit_ns);
   return cudaGetLastError();
