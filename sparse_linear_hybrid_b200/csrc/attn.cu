@@ -15,8 +15,7 @@
 // when block == 64, whose kept-key lists are merged; a key tile then carries a
 // bit per half saying which rows may see it).  Warp roles, 352 threads:
 //   warp 0     TMA producer: Q once, then K tiles of the kept blocks into a
-//              2-deep ring, then (when g != 0) T; once the last S product has
-//              read Q, the whole warp applies ReLU to Q in place;
+//              2-deep ring, then (when g != 0) T;
 //   warp 10    TMA producer of the V tiles (2-deep ring).  A V stage frees up
 //              only when its PV is done; with K and V in one issue order the
 //              next K (and so the next S) would wait for that PV as well;
@@ -194,7 +193,7 @@ __global__ void __launch_bounds__(352, 1)
       mbar_init(&sh->p_full[s], 8);
     }
     mbar_init(&sh->t_full, 1);
-    mbar_init(&sh->q_relu, 1);
+    mbar_init(&sh->q_relu, 8);
     mbar_init(&sh->u_done, 1);
     mbar_init(&sh->drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&sh->xbar[q], 64);
@@ -251,29 +250,6 @@ __global__ void __launch_bounds__(352, 1)
           if (uses > 0) ok = mbar_wait(&sh->k_empty[s], (uint32_t)((uses - 1) & 1), limit_ns);
         }
         if (ok) load_t();
-      }
-    }
-    n = __shfl_sync(0xffffffffu, n, 0);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    if (ok && lin) {
-      // relu(Q) in place, once the last S product has read Q (the commit of
-      // S_{n-1} covers every earlier product as well)
-      bool ready = mbar_wait_warp(&sh->q_full, 0, limit_ns);
-      if (ready && n >= 1)
-        ready = mbar_wait_warp(&sh->k_empty[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), limit_ns);
-      if (ready) {
-        const uint32_t q_addr = sbase + C::OFF_Q;
-#pragma unroll 4
-        for (int u = lane; u < C::Q_BYTES / 16; u += 32) {
-          uint32_t x0, x1, x2, x3;
-          ld_shared_v4(q_addr + u * 16, x0, x1, x2, x3);
-          st_shared_v4(q_addr + u * 16, relu_bf16x2(x0), relu_bf16x2(x1), relu_bf16x2(x2), relu_bf16x2(x3));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->q_relu);
-      } else {
-        ok = false;
       }
     }
     if (lane == 0) {
@@ -559,6 +535,21 @@ __global__ void __launch_bounds__(352, 1)
       ++j;
     }
     const int n = j;
+    if (ok && lin) {
+      // relu(Q) in place for U, each thread its half of its row: the S products
+      // are done with Q (the last one completed before this thread read its S)
+#pragma unroll
+      for (int t = 0; t < C::DCH * 4; ++t) {
+        const int piece = hf * C::DCH * 4 + t;  // 16-byte piece of the row
+        const uint32_t addr = q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8));
+        uint32_t x0, x1, x2, x3;
+        ld_shared_v4(addr, x0, x1, x2, x3);
+        st_shared_v4(addr, relu_bf16x2(x0), relu_bf16x2(x1), relu_bf16x2(x2), relu_bf16x2(x3));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->q_relu);
+    }
     if (ok && n >= 1) {
       ok = mbar_wait_warp(&sh->pv_done[(n - 1) & 1], (uint32_t)(((n - 1) >> 1) & 1), limit_ns);
       tc_fence_after();
