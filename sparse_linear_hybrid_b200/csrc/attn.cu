@@ -25,12 +25,13 @@
 //              U = relu(Q) T into the S buffer the last tile left free, issued
 //              as soon as its operands are in, before or after the last PV;
 //   warps 2-9  softmax, two threads per query row (each takes half of the key
-//              columns of a tile and half of the feature columns of O): first
-//              relu(q) . z for their row from the Q tile (while the first S is
-//              computed), then online softmax whose running maximum is only
-//              moved (and O rescaled in TMEM) when it grows by more than 2^8;
-//              P_j written to TMEM as bf16; finally out = O / l + g U / den and
-//              one TMA store of bf16 out.
+//              columns of a tile and half of the feature columns of O): online
+//              softmax whose running maximum is only moved (and O rescaled in
+//              TMEM) when it grows by more than 2^8, P_j written to TMEM as
+//              bf16; after the last tile each thread applies ReLU to its half
+//              of its row of Q (the A operand of U) and sums its half of
+//              relu(q) . z; finally out = O / l + g U / den and one TMA store
+//              of bf16 out.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
 // P0 [384,448), P1 [448,512) (bf16 pairs).  P is double-buffered: the
 // softmax writes P_{j+1} while PV_j still reads P_j, and waits on PV_j only
@@ -59,6 +60,7 @@ struct AttnShared {
   uint64_t xbar[4];       // per lane quarter: the two halves of its rows meet here (64 arrivals)
   float xmax[2][2][128];  // per tile parity, per half: partial row maxima
   float xsum[2][128];     // per half: partial row sums
+  float xden[2][128];     // per half: partial relu(q) . z
 };
 
 template <int D, int BLK>
@@ -383,31 +385,6 @@ __global__ void __launch_bounds__(352, 1)
     float l = 0.f;            // this half's share of the row sum
     bool ok = true;
     float gd = 0.f;           // g / (relu(q) . z + eps), the linear branch's row factor
-    if (lin) {
-      // relu(q) . z over all d features of this row (both halves compute it the
-      // same way), while the producer and the MMA warp bring in the first S
-      ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);
-      if (ok) {
-        const float4* zr = reinterpret_cast<const float4*>(zvec + (size_t)bh * D);
-        float den0 = 0.f, den1 = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < C::DCH; ++ch)
-#pragma unroll
-          for (int pc = 0; pc < 8; ++pc) {
-            uint32_t x[4];
-            ld_shared_v4(q_addr + ch * 16384 + sw128_offset((uint32_t)r, (uint32_t)pc), x[0], x[1], x[2], x[3]);
-            const float4 za = __ldg(zr + ch * 16 + pc * 2), zb = __ldg(zr + ch * 16 + pc * 2 + 1);
-            const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint32_t xr = relu_bf16x2(x[i]);
-              den0 = fmaf(bf16_lo_to_f32(xr), zz[2 * i], den0);
-              den1 = fmaf(bf16_hi_to_f32(xr), zz[2 * i + 1], den1);
-            }
-          }
-        gd = g / ((den0 + den1) + eps);
-      }
-    }
     KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
     int col, bits, j = 0;
     while (ok && it.next(col, bits)) {
@@ -535,17 +512,32 @@ __global__ void __launch_bounds__(352, 1)
       ++j;
     }
     const int n = j;
+    float den_h = 0.f;  // relu(q) . z over this half of the row
+    if (ok && lin) ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);  // (no S product read Q when n == 0)
     if (ok && lin) {
-      // relu(Q) in place for U, each thread its half of its row: the S products
-      // are done with Q (the last one completed before this thread read its S)
+      // relu(Q) in place for U, each thread its half of its row (the S products
+      // are done with Q: the last one completed before this thread read its S),
+      // and this half's share of relu(q) . z on the way
+      const float4* zr = reinterpret_cast<const float4*>(zvec + (size_t)bh * D);
+      float d0 = 0.f, d1 = 0.f;
 #pragma unroll
       for (int t = 0; t < C::DCH * 4; ++t) {
-        const int piece = hf * C::DCH * 4 + t;  // 16-byte piece of the row
+        const int piece = hf * C::DCH * 4 + t;  // 16-byte piece of the row: features 8 * piece ...
         const uint32_t addr = q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8));
-        uint32_t x0, x1, x2, x3;
-        ld_shared_v4(addr, x0, x1, x2, x3);
-        st_shared_v4(addr, relu_bf16x2(x0), relu_bf16x2(x1), relu_bf16x2(x2), relu_bf16x2(x3));
+        uint32_t x[4];
+        ld_shared_v4(addr, x[0], x[1], x[2], x[3]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = relu_bf16x2(x[i]);
+        st_shared_v4(addr, x[0], x[1], x[2], x[3]);
+        const float4 za = __ldg(zr + piece * 2), zb = __ldg(zr + piece * 2 + 1);
+        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          d0 = fmaf(bf16_lo_to_f32(x[i]), zz[2 * i], d0);
+          d1 = fmaf(bf16_hi_to_f32(x[i]), zz[2 * i + 1], d1);
+        }
       }
+      den_h = d0 + d1;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->q_relu);
@@ -557,9 +549,13 @@ __global__ void __launch_bounds__(352, 1)
     // the row sum of both halves (barrier phase n)
     if (ok) {
       sh->xsum[hf][r] = l;
+      sh->xden[hf][r] = den_h;
       mbar_arrive(&sh->xbar[quarter]);
       ok = mbar_wait_warp(&sh->xbar[quarter], (uint32_t)(n & 1), limit_ns);
-      if (ok) l += sh->xsum[hf ^ 1][r];
+      if (ok) {
+        l += sh->xsum[hf ^ 1][r];
+        if (lin) gd = g / ((sh->xden[0][r] + sh->xden[1][r]) + eps);  // same order in both halves
+      }
     }
     if (ok) ok = mbar_wait_warp(&sh->q_full, 0, limit_ns);  // the staging area below is the Q tile
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
