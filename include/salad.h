@@ -182,6 +182,14 @@ int salad_check_status(void* workspace, salad_stream_t stream);
 void salad_set_wait_limit_ns(uint64_t limit_ns);
 
 /*
+ * Test hook: the attention kernel is persistent (one CTA per SM, each taking
+ * query tiles from a counter until none are left).  A positive value caps its
+ * grid at max_ctas CTAs, so that small inputs also run many query tiles per
+ * CTA; 0 restores one CTA per SM.  Host-global setting; it changes no result.
+ */
+void salad_set_max_ctas(int max_ctas);
+
+/*
  * Profiling hook: caller-owned CUDA events (cudaEvent_t, passed as void*) that
  * subsequent salad_attn_forward calls record on their stream before the
  * linear-branch kernels, before the attention kernel and after it.  Pass NULLs

@@ -7,7 +7,8 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, workspace_bytes, attn_forward,
-    attn_forward_static, linear_state, check_status, set_wait_limit_ns, set_phase_events, status_string
+    attn_forward_static, linear_state, check_status, set_wait_limit_ns, set_max_ctas, set_phase_events,
+    status_string
 """
 from __future__ import annotations
 
@@ -62,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.salad_check_status.restype = i
         L.salad_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.salad_set_wait_limit_ns.restype = None
+        L.salad_set_max_ctas.argtypes = [i]
+        L.salad_set_max_ctas.restype = None
         L.salad_set_phase_events.argtypes = [p, p, p]
         L.salad_set_phase_events.restype = None
         L.salad_status_string.argtypes = [i]
@@ -197,6 +200,11 @@ def check_status(workspace, stream=None) -> int:
 
 def set_wait_limit_ns(limit_ns: int) -> None:
     lib().salad_set_wait_limit_ns(int(limit_ns))
+
+
+def set_max_ctas(max_ctas: int) -> None:
+    """Test hook: cap the persistent attention grid (0: one CTA per SM)."""
+    lib().salad_set_max_ctas(int(max_ctas))
 
 
 def set_phase_events(before_linear=None, before_attention=None, after_attention=None) -> None:

@@ -13,6 +13,7 @@ using namespace salad;
 namespace {
 
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_max_ctas{0};
 std::atomic<void*> g_ev_linear{nullptr}, g_ev_attn{nullptr}, g_ev_end{nullptr};
 
 bool record(const std::atomic<void*>& ev, cudaStream_t s) {
@@ -94,6 +95,7 @@ int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const 
   la.t_op = reinterpret_cast<uint16_t*>(ws + L.off_t);
   la.z = S_out ? z_out : reinterpret_cast<float*>(ws + L.off_z);
   la.S_out = S_out;
+  la.work_ctr = reinterpret_cast<uint32_t*>(ws + L.off_status) + 1;
   la.B = B;
   la.N = N;
   la.heads = Hh;
@@ -202,6 +204,8 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
   aa.col_idx = col_idx;
   aa.gate = gate;
   aa.z = reinterpret_cast<const float*>(ws + L.off_z);
+  aa.work_ctr = reinterpret_cast<uint32_t*>(ws + L.off_status) + 1;
+  aa.max_ctas = g_max_ctas.load();
   aa.B = B;
   aa.N = N;
   aa.heads = num_heads;
@@ -246,6 +250,8 @@ int salad_check_status(void* workspace, salad_stream_t stream) {
 }
 
 void salad_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns.store(limit_ns); }
+
+void salad_set_max_ctas(int max_ctas) { g_max_ctas.store(max_ctas > 0 ? max_ctas : 0); }
 
 void salad_set_phase_events(void* before_linear, void* before_attention, void* after_attention) {
   g_ev_linear.store(before_linear);

@@ -31,7 +31,7 @@ cudaError_t launch_mask_fill(const MaskGrid& g, const WindowTable& win, const in
 struct WorkspaceLayout {
   int splits;             // split-N factor of the linear-branch reduction
   int chunks_per_split;   // 64-token chunks per split
-  size_t off_status;      // uint32 status word
+  size_t off_status;      // uint32 status word, then the uint32 work counter of the attention kernel
   size_t off_t;           // bf16 [B*Hh][d][2d]: (S W)^T split into hi and lo halves
   size_t off_z;           // fp32 [B*Hh][d]: z
   size_t off_partial;     // fp32 [splits][B*Hh][d+1][d]: per-split S rows, then z
@@ -48,6 +48,7 @@ struct LinearArgs {
   uint16_t* t_op;           // forward: (S W)^T hi | lo, bf16 [B*Hh][d][2d]
   float* z;                 // fp32 [B*Hh][d]
   float* S_out;             // state export: fp32 [B*Hh][d][d]; null in the forward
+  uint32_t* work_ctr;       // zeroed here for the attention kernel that follows
   int B, N, heads, d, splits, chunks_per_split;
   uint32_t* status;
   uint64_t wait_limit_ns;
@@ -64,6 +65,8 @@ struct AttnArgs {
   const int32_t* col_idx;
   const float* gate;
   const float* z;             // fp32 [B*Hh][d]
+  uint32_t* work_ctr;         // next work item (zeroed by the linear kernel)
+  int max_ctas;               // cap on the persistent grid (0: one CTA per SM)
   int B, N, heads, d, block;
   float scale_log2;  // softmax scale * log2(e)
   float eps;

@@ -59,9 +59,11 @@ template <int D>
 __global__ void __launch_bounds__(192, 1)
     linear_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const float* __restrict__ gate, float* __restrict__ partial, int heads, int N,
-                          int chunks_per_split, uint32_t* status, uint64_t limit_ns) {
+                          int chunks_per_split, uint32_t* work_ctr, uint32_t* status, uint64_t limit_ns) {
   using C = LinCfg<D>;
   const int split = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
+  // the attention kernel that follows in the stream hands out its work items from this counter
+  if (split == 0 && bh == 0 && threadIdx.x == 0) *work_ctr = 0u;
   if (gate != nullptr && gate[bh] == 0.0f) return;  // branch dropped for this (b, h)
   const int b = bh / heads, h = bh % heads;
   const int total_chunks = (N + kTok - 1) / kTok;
@@ -340,7 +342,8 @@ cudaError_t launch_linear_t(const LinearArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int BH = a.B * a.heads;
   linear_partial_kernel<D><<<dim3(a.splits, BH), 192, C::SMEM, s>>>(
-      *a.tm_k, *a.tm_v, a.gate, a.partial, a.heads, a.N, a.chunks_per_split, a.status, a.wait_limit_ns);
+      *a.tm_k, *a.tm_v, a.gate, a.partial, a.heads, a.N, a.chunks_per_split, a.work_ctr, a.status,
+      a.wait_limit_ns);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const dim3 fgrid(BH, D / (256 / (D / 4)));

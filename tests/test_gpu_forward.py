@@ -113,3 +113,25 @@ def test_workspace_reuse_and_status_ok():
     second = run_gpu(wl, inp, ws=ws)
     assert np.array_equal(first, second)
     assert sl.check_status(ws) == sl.SALAD_OK
+
+
+@pytest.mark.parametrize("ctas", [1, 3])
+@pytest.mark.parametrize("wl", [CASES[1], CASES[3], CASES[4], CASES[5], CASES[7]],
+                         ids=lambda w: f"{w.name}-B{w.B}H{w.Hh}d{w.d}b{w.block}N{w.N}")
+def test_persistent_grid_many_tiles_per_cta(wl, ctas):
+    """The attention kernel is persistent: with its grid capped, one CTA works
+    through many query tiles in turn (its K/V/S/P rings, Q buffers and the
+    linear-branch operand carried across tiles).  The result must match the
+    oracle and be bit-identical to the uncapped run; gates are mixed so that
+    tiles with and without the linear branch alternate."""
+    inp = si.make_inputs(wl, v_mean=0.5)
+    inp.gate.reshape(-1)[::2] = 0.0
+    ref_gpu = run_gpu(wl, inp)
+    sl.set_max_ctas(ctas)
+    try:
+        got = run_gpu(wl, inp)
+    finally:
+        sl.set_max_ctas(0)
+    ok, st = compare(got, run_oracle(wl, inp))
+    assert ok, st
+    assert np.array_equal(got, ref_gpu)
