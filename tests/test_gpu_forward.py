@@ -116,7 +116,7 @@ def test_workspace_reuse_and_status_ok():
 
 
 @pytest.mark.parametrize("ctas", [1, 3])
-@pytest.mark.parametrize("wl", [CASES[1], CASES[3], CASES[4], CASES[5], CASES[7]],
+@pytest.mark.parametrize("wl", [CASES[1], CASES[2], CASES[3], CASES[4], CASES[5], CASES[7]],
                          ids=lambda w: f"{w.name}-B{w.B}H{w.Hh}d{w.d}b{w.block}N{w.N}")
 def test_persistent_grid_many_tiles_per_cta(wl, ctas):
     """The attention kernel is persistent: with its grid capped, one CTA works
