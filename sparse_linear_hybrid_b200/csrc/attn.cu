@@ -19,18 +19,20 @@
 // item.  Every ring below keeps its protocol across items (its index counts
 // across the whole CTA).  Warp roles, 384 threads:
 //   warp 0     leader and TMA producer: takes the next item (atomic counter,
-//              handed to the other roles through a 2-slot queue), loads its Q
-//              into one of two Q buffers and its K tiles into a 2-deep ring;
-//   warp 10    TMA producer of the V tiles (2-deep ring) and of T, which goes
-//              into the V ring (as two pseudo tiles) when there is no room for
-//              it elsewhere;
+//              decoded once and handed to the other roles through a 2-slot
+//              queue), loads its Q into one of two Q buffers and its K tiles
+//              into a 2-deep ring;
+//   warp 10    TMA producer of the V tiles (2-deep ring) and of T.  Where T
+//              has no region of its own, T_hi goes through the K ring (loaded
+//              by warp 0 after the item's last K tile) and T_lo through the V
+//              ring (after the item's last V tile);
 //   warp 11    output store: one TMA store per item once the softmax warps
 //              have staged its tile, then frees that Q buffer;
 //   warp 1     tcgen05 issuer (one thread) and TMEM owner: S = Q K_j^T into one
 //              of two TMEM S buffers (A, B in shared memory); O += P_j V_j with
 //              P_j read from TMEM; U = relu(Q) [T_hi ; T_lo] of an item into the
-//              S buffer of the slot that follows its tiles, issued once the
-//              next item's first S is out;
+//              S buffer of the slot that follows its tiles, right after its
+//              last PV (the next item's first S follows U);
 //   warps 2-9  softmax, two threads per query row (each takes half of the key
 //              columns of a tile and half of the feature columns of O): online
 //              softmax whose running maximum is only moved (and O rescaled in
@@ -55,6 +57,19 @@ constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 constexpr int kThreads = 384;
 
+// A work item as the leader hands it to the other roles (through shared
+// memory, so that no other role reads the mask or the gate from global memory
+// on its way into an item).
+struct Item {
+  int w;                // work index; -1: no work left
+  int bh, qtile, b, h;
+  int n;                // kept key tiles
+  int vlast;            // real keys in the last kept tile (BLK unless it is the partial last block)
+  int ra, na, rb, nb;   // col_idx ranges of the tile's query block(s) (the second one when BLK == 64)
+  float g;              // gate of this (b, h)
+  bool lin;             // the linear branch is dropped for this (b, h) when its gate is 0
+};
+
 struct AttnShared {
   uint64_t item_full[2], item_empty[2];  // the 2-slot item queue
   uint64_t q_full[2], q_free[2], q_relu[2], staged[2];  // per Q buffer
@@ -62,14 +77,16 @@ struct AttnShared {
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], pv_done[2];
   uint64_t t_full, t_empty;
+  uint64_t z_full[2];        // per item slot: z of the item's (b, h) has landed in zs
   uint64_t drain;
   uint64_t xbar[4];          // per lane quarter: the two halves of its rows meet here (64 arrivals)
-  int item[2];
+  Item item[2];
   uint32_t tmem_base;
   volatile int abort_flag;
   float xmax[2][2][128];     // per exchange parity, per half: partial row maxima
   float xsum[2][2][128];     // per exchange parity, per half: partial row sums
   float xden[2][2][128];     // per exchange parity, per half: partial relu(q) . z
+  alignas(16) float zs[2][128];  // per item slot: z of the item's (b, h)
 };
 
 template <int D, int BLK>
@@ -83,14 +100,16 @@ struct AttnCfg {
   static constexpr int T_CH_BYTES = D * 128;        // D rows (feature f) of 128 bytes
   static constexpr int T_BYTES = T_CH * T_CH_BYTES;
   static constexpr int BASE_BYTES = 2 * Q_BYTES + 4 * KV_BYTES;  // Q[2], K[2], V[2]
-  // T has a region of its own when shared memory allows; otherwise it takes
-  // the place of both V stages, between an item's last PV and its U.
-  static constexpr bool T_IN_VRING = BASE_BYTES + T_BYTES + (int)sizeof(AttnShared) + 1024 > 232448;
+  // T has a region of its own when shared memory allows.  Otherwise its two
+  // halves travel through the rings as one extra entry each, right after the
+  // item's last K and V tiles.  Their stages free up while the item's last
+  // tile is still in the softmax, so U need not wait for the last PV.
+  static constexpr bool T_IN_RINGS = BASE_BYTES + T_BYTES + (int)sizeof(AttnShared) + 1024 > 232448;
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_K0 = 2 * Q_BYTES;
   static constexpr int OFF_V0 = OFF_K0 + 2 * KV_BYTES;
-  static constexpr int OFF_T = T_IN_VRING ? OFF_V0 : BASE_BYTES;
-  static constexpr int OFF_BAR = BASE_BYTES + (T_IN_VRING ? 0 : T_BYTES);
+  static constexpr int OFF_T = BASE_BYTES;  // dedicated T region (unused when T_IN_RINGS)
+  static constexpr int OFF_BAR = BASE_BYTES + (T_IN_RINGS ? 0 : T_BYTES);
   static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(AttnShared) + 1024;
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
   static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
@@ -100,7 +119,8 @@ struct AttnCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);     // P V   (V MN-major)
   static constexpr uint32_t IDESC_U = idesc_bf16(128, D, false, false);     // relu(Q) [T_hi ; T_lo]
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(!T_IN_VRING || T_BYTES <= 2 * KV_BYTES, "T must fit the V ring");
+  static_assert(!T_IN_RINGS || (T_BYTES == 2 * KV_BYTES && T_CH == 2 * DCH && T_CH_BYTES == KV_BOX),
+                "each half of T must have the layout of one K or V tile");
   static_assert(TM_P + 2 * P_COLS <= 512 && D <= 128, "tensor memory budget");
 };
 
@@ -156,29 +176,47 @@ __device__ __forceinline__ KeyIter make_iter(const int32_t* row_ptr, const int32
   return it;
 }
 
-// Number of kept key tiles of a query tile (what make_iter will yield).
 template <int BLK>
-__device__ __forceinline__ int count_tiles(const int32_t* row_ptr, const int32_t* col_idx, int h, int nb,
-                                           int qtile) {
-  KeyIter it = make_iter<BLK>(row_ptr, col_idx, h, nb, qtile);
-  if (BLK == 128) return it.na;
-  int col, bits, n = 0;
-  while (it.next(col, bits)) ++n;
-  return n;
+__device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, const int32_t* row_ptr,
+                                          const int32_t* col_idx, const float* gate) {
+  Item im;
+  im.w = w;
+  im.bh = w / qtiles;
+  im.qtile = w % qtiles;
+  im.b = im.bh / heads;
+  im.h = im.bh % heads;
+  im.g = gate[im.bh];
+  im.lin = im.g != 0.0f;
+  const int nb = (N + BLK - 1) / BLK;
+  KeyIter it = make_iter<BLK>(row_ptr, col_idx, im.h, nb, im.qtile);
+  im.ra = (int)(it.a - col_idx);
+  im.na = it.na;
+  im.rb = it.b ? (int)(it.b - col_idx) : 0;
+  im.nb = it.nb;
+  int last = -1;
+  if (BLK == 128) {
+    im.n = it.na;
+    if (it.na > 0) last = it.a[it.na - 1];
+  } else {
+    int col, bits, n = 0;
+    while (it.next(col, bits)) {
+      ++n;
+      last = col;
+    }
+    im.n = n;
+  }
+  im.vlast = last >= 0 ? min(BLK, N - last * BLK) : BLK;
+  return im;
 }
 
-struct Item {
-  int bh, qtile, b, h;
-  bool lin;
-};
-
-__device__ __forceinline__ Item decode_item(int w, int qtiles, int heads, const float* gate) {
-  Item it;
-  it.bh = w / qtiles;
-  it.qtile = w % qtiles;
-  it.b = it.bh / heads;
-  it.h = it.bh % heads;
-  it.lin = gate[it.bh] != 0.0f;  // the linear branch is dropped for this (b, h) when its gate is 0
+// The kept key tiles of a published item, in the order make_iter yields them.
+__device__ __forceinline__ KeyIter item_iter(const Item& im, const int32_t* col_idx) {
+  KeyIter it{};
+  it.a = col_idx + im.ra;
+  it.na = im.na;
+  it.b = im.nb > 0 ? col_idx + im.rb : nullptr;
+  it.nb = im.nb;
+  it.ia = it.ib = 0;
   return it;
 }
 
@@ -202,7 +240,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const float* __restrict__ zvec, int heads, int N, int qtiles, int num_items,
                       uint32_t* work_ctr, float scale_log2, float eps, uint32_t* status, uint64_t limit_ns) {
   using C = AttnCfg<D, BLK>;
-  const int nb = (N + BLK - 1) / BLK;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -229,6 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sh->t_full, 1);
     mbar_init(&sh->t_empty, 1);
+    mbar_init(&sh->z_full[0], 1);
+    mbar_init(&sh->z_full[1], 1);
     mbar_init(&sh->drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&sh->xbar[q], 64);
     sh->abort_flag = 0;
@@ -248,19 +287,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
+      if (C::T_IN_RINGS) tma_prefetch_map(&tm_t);
       bool ok = true;
       int seq = 0, kj = 0;
+      // next K ring entry: wait for its stage, expect its bytes
+      auto k_stage = [&]() -> uint8_t* {
+        const int s = kj & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->k_empty[s], ((kj >> 1) & 1) ^ 1, limit_ns)) return nullptr;
+        mbar_arrive_expect_tx(&sh->k_full[s], C::KV_BYTES);
+        return smem + C::OFF_K0 + s * C::KV_BYTES;
+      };
       for (;;) {
         const int slot = seq & 1;
         const uint32_t ph = (uint32_t)((seq >> 1) & 1);
         // hand the next item to the other roles
         if (sh->abort_flag || !mbar_wait(&sh->item_empty[slot], ph ^ 1, limit_ns)) { ok = false; break; }
-        int w = (int)atomicAdd(work_ctr, 1u);
-        if (w >= num_items) w = -1;
-        sh->item[slot] = w;
+        const int w = (int)atomicAdd(work_ctr, 1u);
+        Item im;
+        if (w < num_items) {
+          im = make_item<BLK>(w, qtiles, heads, N, row_ptr, col_idx, gate);
+        } else {
+          im.w = -1;
+        }
+        sh->item[slot] = im;
         mbar_arrive(&sh->item_full[slot]);
-        if (w < 0) break;
-        const Item im = decode_item(w, qtiles, heads, gate);
+        if (im.w < 0) break;
         // Q buffer `slot` is free once the output of the item two back has been stored from it
         if (!mbar_wait(&sh->q_free[slot], ph ^ 1, limit_ns)) { ok = false; break; }
         mbar_arrive_expect_tx(&sh->q_full[slot], C::Q_BYTES);
@@ -268,17 +319,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ch = 0; ch < C::DCH; ++ch)
           tma_load_3d(smem + C::OFF_Q0 + slot * C::Q_BYTES + ch * 16384, &tm_q, &sh->q_full[slot],
                       im.h * D + ch * 64, im.qtile * 128, im.b);
-        KeyIter it = make_iter<BLK>(row_ptr, col_idx, im.h, nb, im.qtile);
+        KeyIter it = item_iter(im, col_idx);
         int col, bits;
         while (it.next(col, bits)) {
-          const int s = kj & 1;
-          if (sh->abort_flag || !mbar_wait(&sh->k_empty[s], ((kj >> 1) & 1) ^ 1, limit_ns)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sh->k_full[s], C::KV_BYTES);
-          uint8_t* kt = smem + C::OFF_K0 + s * C::KV_BYTES;
+          uint8_t* kt = k_stage();
+          if (!kt) { ok = false; break; }
 #pragma unroll
           for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_3d(kt + ch * C::KV_BOX, &tm_k, &sh->k_full[s], im.h * D + ch * 64, col * BLK, im.b);
+            tma_load_3d(kt + ch * C::KV_BOX, &tm_k, &sh->k_full[kj & 1], im.h * D + ch * 64, col * BLK, im.b);
           ++kj;
+        }
+        if (ok && C::T_IN_RINGS && im.lin) {
+          // T_hi: one more K ring entry after the item's key tiles, released by U
+          uint8_t* dst = k_stage();
+          if (!dst) {
+            ok = false;
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < C::DCH; ++ch)
+              tma_load_3d(dst + ch * C::KV_BOX, &tm_t, &sh->k_full[kj & 1], ch * 64, 0, im.bh);
+            ++kj;
+          }
         }
         if (!ok) break;
         ++seq;
@@ -296,18 +357,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tm_v);
       tma_prefetch_map(&tm_t);
       bool ok = true;
-      int seq = 0, vj = 0, tl = 0;
+      int seq = 0, vj = 0, tl = 0, zc = 0;
       for (;;) {
         const int slot = seq & 1;
         if (sh->abort_flag || !mbar_wait(&sh->item_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns)) {
           ok = false;
           break;
         }
-        const int w = sh->item[slot];
+        const Item im = sh->item[slot];
         mbar_arrive(&sh->item_empty[slot]);
-        if (w < 0) break;
-        const Item im = decode_item(w, qtiles, heads, gate);
-        KeyIter it = make_iter<BLK>(row_ptr, col_idx, im.h, nb, im.qtile);
+        if (im.w < 0) break;
+        // z of this (b, h) into zs[slot], once the softmax warps are done with the
+        // z of the item two back (they arrive on q_relu after reading it)
+        if (seq >= 2 && !mbar_wait(&sh->q_relu[slot], (uint32_t)(((seq - 2) >> 1) & 1), limit_ns)) {
+          ok = false;
+          break;
+        }
+        if (im.lin) {
+          mbar_arrive_expect_tx(&sh->z_full[slot], D * 4);
+          bulk_load(sh->zs[slot], zvec + (size_t)im.bh * D, D * 4, &sh->z_full[slot]);
+        } else {
+          mbar_arrive(&sh->z_full[slot]);
+        }
+        ++zc;
+        KeyIter it = item_iter(im, col_idx);
         int col, bits;
         while (it.next(col, bits)) {
           const int s = vj & 1;
@@ -320,23 +393,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++vj;
         }
         if (!ok) break;
-        if (im.lin) {
-          if (C::T_IN_VRING) {
-            // T takes both V stages: wait until the item's last PVs have read them
-            // (two pseudo V tiles, released again by U)
-            ok = mbar_wait(&sh->v_empty[vj & 1], ((vj >> 1) & 1) ^ 1, limit_ns) &&
-                 mbar_wait(&sh->v_empty[(vj + 1) & 1], (((vj + 1) >> 1) & 1) ^ 1, limit_ns);
-            if (ok) {
-              // the pseudo tiles complete their v_full phases too, so that every
-              // stage's phase count keeps matching the V index
-              mbar_arrive(&sh->v_full[vj & 1]);
-              mbar_arrive(&sh->v_full[(vj + 1) & 1]);
-            }
-            vj += 2;
-          } else {
-            ok = mbar_wait(&sh->t_empty, (uint32_t)(tl & 1) ^ 1, limit_ns);
-          }
-          if (!ok) break;
+        if (im.lin && C::T_IN_RINGS) {
+          // T_lo: one more V ring entry, released by U
+          const int s = vj & 1;
+          if (sh->abort_flag || !mbar_wait(&sh->v_empty[s], ((vj >> 1) & 1) ^ 1, limit_ns)) { ok = false; break; }
+          mbar_arrive_expect_tx(&sh->v_full[s], C::KV_BYTES);
+          uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
+#pragma unroll
+          for (int ch = 0; ch < C::DCH; ++ch)
+            tma_load_3d(vt + ch * C::KV_BOX, &tm_t, &sh->v_full[s], (C::DCH + ch) * 64, 0, im.bh);
+          ++vj;
+        } else if (im.lin) {
+          if (!mbar_wait(&sh->t_empty, (uint32_t)(tl & 1) ^ 1, limit_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&sh->t_full, C::T_BYTES);
 #pragma unroll
           for (int ch = 0; ch < C::T_CH; ++ch)
@@ -347,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) record_timeout(sh, status);
       for (int i = (vj > 2 ? vj - 2 : 0); i < vj; ++i) mbar_wait(&sh->v_full[i & 1], (i >> 1) & 1, kDrainNs);
+      for (int i = (zc > 2 ? zc - 2 : 0); i < zc; ++i) mbar_wait(&sh->z_full[i & 1], (i >> 1) & 1, kDrainNs);
       if (tl > 0) mbar_wait(&sh->t_full, (uint32_t)((tl - 1) & 1), kDrainNs);
     }
   } else if (warp == 11) {
@@ -361,10 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = seq & 1;
         const uint32_t ph = (uint32_t)((seq >> 1) & 1);
         if (sh->abort_flag || !mbar_wait(&sh->item_full[slot], ph, limit_ns)) { ok = false; break; }
-        const int w = sh->item[slot];
+        const Item im = sh->item[slot];
         mbar_arrive(&sh->item_empty[slot]);
-        if (w < 0) break;
-        const Item im = decode_item(w, qtiles, heads, gate);
+        if (im.w < 0) break;
         if (!mbar_wait(&sh->staged[slot], ph, limit_ns)) { ok = false; break; }
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
@@ -421,36 +489,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++sj;
         return true;
       };
-      // U = relu(Q) [T_hi ; T_lo] (K = 2d: relu(Q) is fed twice) into S slot
-      // `gu`, completion on s_full like a tile; frees T's place
-      struct PendingU {
-        bool on;
-        int gu, qb, qseq, gv;  // S slot, Q buffer, item sequence number, V index of T's first pseudo tile
-      } pend{false, 0, 0, 0, 0};
-      auto issue_u = [&](const PendingU& u) -> bool {
-        const int s = u.gu & 1;
-        if (sh->abort_flag || !mbar_wait(&sh->t_full, (uint32_t)(tl & 1), limit_ns) ||
-            !mbar_wait(&sh->q_relu[u.qb], (uint32_t)((u.qseq >> 1) & 1), limit_ns))
+      // U = relu(Q) [T_hi ; T_lo] of the item in Q buffer `qb` (K = 2d: relu(Q)
+      // is fed twice) into the S slot after its tiles, completion on s_full like
+      // a tile; frees T's place.  T is in its own region, or T_hi is the K ring
+      // entry after the item's key tiles and T_lo the V ring entry after them.
+      auto issue_u = [&](int qb, int qseq) -> bool {
+        const int s = sj & 1, ks = kj & 1, vs = vj & 1;
+        const bool t_ok = C::T_IN_RINGS
+                              ? mbar_wait(&sh->k_full[ks], (uint32_t)((kj >> 1) & 1), limit_ns) &&
+                                    mbar_wait(&sh->v_full[vs], (uint32_t)((vj >> 1) & 1), limit_ns)
+                              : mbar_wait(&sh->t_full, (uint32_t)(tl & 1), limit_ns);
+        if (sh->abort_flag || !t_ok || !mbar_wait(&sh->q_relu[qb], (uint32_t)((qseq >> 1) & 1), limit_ns))
           return false;
-        if (u.gu >= 2 && !mbar_wait(&sh->s_free[s], (uint32_t)(((u.gu - 2) >> 1) & 1), limit_ns)) return false;
+        if (sj >= 2 && !mbar_wait(&sh->s_free[s], (uint32_t)(((sj - 2) >> 1) & 1), limit_ns)) return false;
         tc_fence_after();
-        const uint32_t qr = sbase + C::OFF_Q0 + u.qb * C::Q_BYTES, tb = sbase + C::OFF_T;
+        const uint32_t qr = sbase + C::OFF_Q0 + qb * C::Q_BYTES;
+        const uint32_t t_hi = C::T_IN_RINGS ? sbase + C::OFF_K0 + ks * C::KV_BYTES : sbase + C::OFF_T;
+        const uint32_t t_lo = C::T_IN_RINGS ? sbase + C::OFF_V0 + vs * C::KV_BYTES : t_hi + (C::T_CH / 2) * C::T_CH_BYTES;
         const uint32_t d_u = tmem + (s ? C::TM_S1 : C::TM_S0);
 #pragma unroll
         for (int kk = 0; kk < 2 * D / 16; ++kk) {
-          const int qk = kk % (D / 16);
+          const int qk = kk % (D / 16), ch = kk / 4;  // ch: 64-column chunk of [T_hi | T_lo]
+          const uint32_t tc = ch < C::T_CH / 2 ? t_hi + ch * C::T_CH_BYTES : t_lo + (ch - C::T_CH / 2) * C::T_CH_BYTES;
           const uint64_t a = sw128_desc(qr + (qk / 4) * 16384 + (qk % 4) * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(tb + (kk / 4) * C::T_CH_BYTES + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(tc + (kk % 4) * 32, 16, 1024);
           mma_bf16_ss(d_u, a, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
         }
         mma_commit(&sh->s_full[s]);
-        if (C::T_IN_VRING) {
-          mma_commit(&sh->v_empty[u.gv & 1]);
-          mma_commit(&sh->v_empty[(u.gv + 1) & 1]);
+        if (C::T_IN_RINGS) {
+          mma_commit(&sh->k_empty[ks]);
+          mma_commit(&sh->v_empty[vs]);
+          ++kj;
+          ++vj;
         } else {
           mma_commit(&sh->t_empty);
+          ++tl;
         }
-        ++tl;
+        ++sj;
         return true;
       };
       for (;;) {
@@ -459,20 +534,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const int w = sh->item[slot];
+        const Item im = sh->item[slot];
         mbar_arrive(&sh->item_empty[slot]);
-        if (w < 0) break;
-        const Item im = decode_item(w, qtiles, heads, gate);
+        if (im.w < 0) break;
         if (!mbar_wait(&sh->q_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns)) { ok = false; break; }
         const uint32_t q_addr = sbase + C::OFF_Q0 + slot * C::Q_BYTES;
-        const int n = count_tiles<BLK>(row_ptr, col_idx, im.h, nb, im.qtile);
+        const int n = im.n;
         const int tt0 = tt, vj0 = vj;
-        // S_0 of this item first, then the previous item's U, then S_j, PV_{j-1}, ...
+        // S_0, then S_j and PV_{j-1}, ..., PV_{n-1}, then U
         if (n >= 1 && !issue_s(q_addr)) { ok = false; break; }
-        if (pend.on) {
-          if (!issue_u(pend)) { ok = false; break; }
-          pend.on = false;
-        }
         for (int j = 1; j < n && ok; ++j) {
           if (!issue_s(q_addr) || !issue_pv(tt0 + j - 1, vj0 + j - 1, j == 1)) ok = false;
         }
@@ -480,14 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tt += n;
         vj += n;
-        if (im.lin) {
-          pend = PendingU{true, sj, slot, seq, vj};
-          ++sj;
-          if (C::T_IN_VRING) vj += 2;
-        }
+        if (im.lin && !issue_u(slot, seq)) { ok = false; break; }
         ++seq;
       }
-      if (ok && pend.on) ok = issue_u(pend);
       if (!ok) {
         record_timeout(sh, status);
         mma_commit(&sh->drain);
@@ -515,18 +580,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (;;) {
       const int slot = seq & 1;
       if (!mbar_wait_warp(&sh->item_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns)) { ok = false; break; }
-      const int w = sh->item[slot];
+      const Item im = sh->item[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->item_empty[slot]);
-      if (w < 0) break;
-      const Item im = decode_item(w, qtiles, heads, gate);
-      const float g = gate[im.bh];
+      if (im.w < 0) break;
       const uint32_t q_addr = sbase + C::OFF_Q0 + slot * C::Q_BYTES;
       float m_ref = -INFINITY;  // running reference max (raw score units), same in both halves
       float l = 0.f;            // this half's share of the row sum
-      KeyIter it = make_iter<BLK>(row_ptr, col_idx, im.h, nb, im.qtile);
-      int col, bits, j = 0;
-      while (it.next(col, bits)) {
+      KeyIter it = item_iter(im, col_idx);  // read only when BLK == 64 (which rows use a tile)
+      int j = 0;
+      for (; j < im.n; ++j) {
+        int bits = 1, vtile;
+        if (BLK == 64) {
+          int col;
+          it.next(col, bits);
+          vtile = min(BLK, N - col * BLK);
+        } else {
+          vtile = j == im.n - 1 ? im.vlast : BLK;  // only the last kept tile can be the partial block
+        }
         const int s = sj & 1, pb = tt & 1;
         const bool aborted = __shfl_sync(0xffffffffu, sh->abort_flag != 0, 0);
         if (aborted || !mbar_wait_warp(&sh->s_full[s], (uint32_t)((sj >> 1) & 1), limit_ns)) { ok = false; break; }
@@ -542,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sh->s_free[s]);
 
         const bool use = ((bits >> half) & 1) != 0;           // warp-uniform
-        const int valid = min(BLK, N - col * BLK) - hf * HC;  // real keys among this thread's columns
+        const int valid = vtile - hf * HC;  // real keys among this thread's columns
         float mt;
         if (valid >= HC) {
           float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
@@ -655,7 +726,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->p_full[pb]);
-        ++j;
         ++sj;
         ++tt;
       }
@@ -669,27 +739,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = mbar_wait_warp(&sh->q_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns);
       if (!ok) break;
       if (im.lin) {
-        const float4* zr = reinterpret_cast<const float4*>(zvec + (size_t)im.bh * D);
+        if (!mbar_wait_warp(&sh->z_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns)) {
+          ok = false;
+          break;
+        }
+        // all loads of this half-row first, then all stores: one shared-memory
+        // round trip instead of one per 16-byte piece
+        constexpr int NP = C::DCH * 4;  // 16-byte pieces in half a row
+        uint32_t x[NP][4];
+#pragma unroll
+        for (int t = 0; t < NP; ++t) {
+          const int piece = hf * NP + t;  // features 8 * piece ... 8 * piece + 7
+          ld_shared_v4(q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8)), x[t][0],
+                       x[t][1], x[t][2], x[t][3]);
+        }
+#pragma unroll
+        for (int t = 0; t < NP; ++t) {
+          const int piece = hf * NP + t;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) x[t][i] = relu_bf16x2(x[t][i]);
+          st_shared_v4(q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8)), x[t][0],
+                       x[t][1], x[t][2], x[t][3]);
+        }
+        fence_proxy_async_smem();
+        const float4* zr = reinterpret_cast<const float4*>(sh->zs[slot]) + hf * NP * 2;
         float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-        for (int t = 0; t < C::DCH * 4; ++t) {
-          const int piece = hf * C::DCH * 4 + t;  // 16-byte piece of the row: features 8 * piece ...
-          const uint32_t addr = q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8));
-          uint32_t x[4];
-          ld_shared_v4(addr, x[0], x[1], x[2], x[3]);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) x[i] = relu_bf16x2(x[i]);
-          st_shared_v4(addr, x[0], x[1], x[2], x[3]);
-          const float4 za = __ldg(zr + piece * 2), zb = __ldg(zr + piece * 2 + 1);
+        for (int t = 0; t < NP; ++t) {
+          const float4 za = zr[2 * t], zb = zr[2 * t + 1];
           const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            d0 = fmaf(bf16_lo_to_f32(x[i]), zz[2 * i], d0);
-            d1 = fmaf(bf16_hi_to_f32(x[i]), zz[2 * i + 1], d1);
+            d0 = fmaf(bf16_lo_to_f32(x[t][i]), zz[2 * i], d0);
+            d1 = fmaf(bf16_hi_to_f32(x[t][i]), zz[2 * i + 1], d1);
           }
         }
         den_h = d0 + d1;
-        fence_proxy_async_smem();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->q_relu[slot]);
@@ -706,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&sh->xbar[quarter]);
       if (!mbar_wait_warp(&sh->xbar[quarter], (uint32_t)(xc & 1), limit_ns)) { ok = false; break; }
       l += sh->xsum[xc & 1][hf ^ 1][r];
-      const float gd = im.lin ? g / ((sh->xden[xc & 1][0][r] + sh->xden[xc & 1][1][r]) + eps) : 0.f;
+      const float gd = im.lin ? im.g / ((sh->xden[xc & 1][0][r] + sh->xden[xc & 1][1][r]) + eps) : 0.f;
       ++xc;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       // U lands in the S slot after this item's tiles
