@@ -293,7 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // next K ring entry: wait for its stage, expect its bytes
       auto k_stage = [&]() -> uint8_t* {
         const int s = kj & 1;
-        if (sh->abort_flag || !mbar_wait(&sh->k_empty[s], ((kj >> 1) & 1) ^ 1, limit_ns)) return nullptr;
+        // the stage is free once the product that read entry kj - 2 is done.  With
+        // T in the rings every K entry feeds exactly one S slot use (S or U) in the
+        // same order, so that product's own completion barrier tells; otherwise
+        // the products release the stages through k_empty
+        const bool free_ok = C::T_IN_RINGS
+                                 ? (kj < 2 || mbar_wait(&sh->s_full[s], (uint32_t)(((kj - 2) >> 1) & 1), limit_ns))
+                                 : mbar_wait(&sh->k_empty[s], ((kj >> 1) & 1) ^ 1, limit_ns);
+        if (sh->abort_flag || !free_ok) return nullptr;
         mbar_arrive_expect_tx(&sh->k_full[s], C::KV_BYTES);
         return smem + C::OFF_K0 + s * C::KV_BYTES;
       };
@@ -358,6 +365,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_map(&tm_t);
       bool ok = true;
       int seq = 0, vj = 0, tl = 0, zc = 0;
+      // what last occupied each V stage: a V tile (its global tile index; its PV's
+      // pv_done frees the stage) or T_lo (U frees it through v_empty, one phase
+      // per T_lo entry of the stage)
+      // (kept in scalars: a stage number is only known at run time)
+      int gtile = 0, tile0 = -1, tile1 = -1, tlo0 = 0, tlo1 = 0;
+      bool is_tlo0 = false, is_tlo1 = false;
+      auto v_stage_free = [&](int s) -> bool {
+        if (sh->abort_flag) return false;
+        if (vj < 2) return true;
+        if (s ? is_tlo1 : is_tlo0) return mbar_wait(&sh->v_empty[s], (uint32_t)(((s ? tlo1 : tlo0) - 1) & 1), limit_ns);
+        const int g = s ? tile1 : tile0;
+        return mbar_wait(&sh->pv_done[g & 1], (uint32_t)((g >> 1) & 1), limit_ns);
+      };
       for (;;) {
         const int slot = seq & 1;
         if (sh->abort_flag || !mbar_wait(&sh->item_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns)) {
@@ -384,7 +404,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int col, bits;
         while (it.next(col, bits)) {
           const int s = vj & 1;
-          if (sh->abort_flag || !mbar_wait(&sh->v_empty[s], ((vj >> 1) & 1) ^ 1, limit_ns)) { ok = false; break; }
+          if (!v_stage_free(s)) { ok = false; break; }
+          if (s) {
+            is_tlo1 = false;
+            tile1 = gtile;
+          } else {
+            is_tlo0 = false;
+            tile0 = gtile;
+          }
+          ++gtile;
           mbar_arrive_expect_tx(&sh->v_full[s], C::KV_BYTES);
           uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
 #pragma unroll
@@ -396,7 +424,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (im.lin && C::T_IN_RINGS) {
           // T_lo: one more V ring entry, released by U
           const int s = vj & 1;
-          if (sh->abort_flag || !mbar_wait(&sh->v_empty[s], ((vj >> 1) & 1) ^ 1, limit_ns)) { ok = false; break; }
+          if (!v_stage_free(s)) { ok = false; break; }
+          if (s) {
+            is_tlo1 = true;
+            ++tlo1;
+          } else {
+            is_tlo0 = true;
+            ++tlo0;
+          }
           mbar_arrive_expect_tx(&sh->v_full[s], C::KV_BYTES);
           uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
 #pragma unroll
@@ -450,6 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int seq = 0, kj = 0, sj = 0, tt = 0, vj = 0, tl = 0;
+      // S slot reuse: the softmax frees a slot (s_free) before it signals P of the
+      // same tile (p_full), so once this thread has seen p_full of the tile that
+      // last used a slot, that slot's s_free wait is already satisfied
+      int st = 0, pf_seen = -1, slot_tile0 = -1, slot_tile1 = -1;  // S tiles issued, last p_full seen, per slot
       // O += P V for global tile `gt` of the item whose V tiles start at V index
       // `gv0` (P from tensor memory; operands waited for here)
       auto issue_pv = [&](int gt, int gv, bool first) -> bool {
@@ -457,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (sh->abort_flag || !mbar_wait(&sh->p_full[s], (uint32_t)((gt >> 1) & 1), limit_ns) ||
             !mbar_wait(&sh->v_full[vs], (uint32_t)((gv >> 1) & 1), limit_ns))
           return false;
+        pf_seen = gt;
         tc_fence_after();
         const uint32_t vt = sbase + C::OFF_V0 + vs * C::KV_BYTES;
         const uint32_t pt = tmem + C::TM_P + s * C::P_COLS;
@@ -465,15 +505,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sw128_desc(vt + kk * 2048, C::KV_BOX, 1024);
           mma_bf16_ts(tmem + C::TM_O, pt + kk * 8, bd, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&sh->pv_done[s]);
-        mma_commit(&sh->v_empty[vs]);
+        mma_commit(&sh->pv_done[s]);  // also frees the V stage
         return true;
       };
       // S = Q K^T into S slot `g` (K tile kj of the ring)
       auto issue_s = [&](uint32_t q_addr) -> bool {
         const int s = sj & 1, ks = kj & 1;
         if (sh->abort_flag || !mbar_wait(&sh->k_full[ks], (uint32_t)((kj >> 1) & 1), limit_ns)) return false;
-        if (sj >= 2 && !mbar_wait(&sh->s_free[s], (uint32_t)(((sj - 2) >> 1) & 1), limit_ns)) return false;
+        const int prev = s ? slot_tile1 : slot_tile0;
+        const bool implied = prev >= 0 && prev <= pf_seen;
+        if (sj >= 2 && !implied && !mbar_wait(&sh->s_free[s], (uint32_t)(((sj - 2) >> 1) & 1), limit_ns))
+          return false;
+        if (s) {
+          slot_tile1 = st;
+        } else {
+          slot_tile0 = st;
+        }
+        ++st;
         tc_fence_after();
         const uint32_t kt = sbase + C::OFF_K0 + ks * C::KV_BYTES;
         const uint32_t d_s = tmem + (s ? C::TM_S1 : C::TM_S0);
@@ -483,8 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sw128_desc(kt + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
           mma_bf16_ss(d_s, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sh->s_full[s]);
-        mma_commit(&sh->k_empty[ks]);
+        mma_commit(&sh->s_full[s]);  // with T in the rings this also frees the K stage
+        if (!C::T_IN_RINGS) mma_commit(&sh->k_empty[ks]);
         ++kj;
         ++sj;
         return true;
@@ -502,6 +550,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (sh->abort_flag || !t_ok || !mbar_wait(&sh->q_relu[qb], (uint32_t)((qseq >> 1) & 1), limit_ns))
           return false;
         if (sj >= 2 && !mbar_wait(&sh->s_free[s], (uint32_t)(((sj - 2) >> 1) & 1), limit_ns)) return false;
+        if (s) {
+          slot_tile1 = -1;
+        } else {
+          slot_tile0 = -1;
+        }
         tc_fence_after();
         const uint32_t qr = sbase + C::OFF_Q0 + qb * C::Q_BYTES;
         const uint32_t t_hi = C::T_IN_RINGS ? sbase + C::OFF_K0 + ks * C::KV_BYTES : sbase + C::OFF_T;
@@ -517,8 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&sh->s_full[s]);
         if (C::T_IN_RINGS) {
-          mma_commit(&sh->k_empty[ks]);
-          mma_commit(&sh->v_empty[vs]);
+          mma_commit(&sh->v_empty[vs]);  // T_lo's stage (T_hi's K stage is freed through s_full)
           ++kj;
           ++vj;
         } else {

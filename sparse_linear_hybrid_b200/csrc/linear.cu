@@ -172,16 +172,29 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       const uint32_t kt = smem_u32(smem + s * C::STAGE_BYTES) + col_off;
-#pragma unroll 8
-      for (int r = r0; r < kTok; r += RSTEP) {
-        const uint32_t addr = kt + sw128_offset((uint32_t)r, piece) + word;
-        uint32_t v;
-        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-        const uint32_t neg = ((v >> 15) & 0x00010001u) * 0xFFFFu;  // 0xFFFF in each negative half
-        v &= ~neg;
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-        z0 += bf16_lo_to_f32(v);
-        z1 += bf16_hi_to_f32(v);
+      // the rows of this column pair in batches: all loads of a batch, then its
+      // stores (one shared-memory round trip per batch, not per row)
+      constexpr int NR = kTok / RSTEP, BATCH = NR < 16 ? NR : 16;
+#pragma unroll
+      for (int r1 = 0; r1 < NR; r1 += BATCH) {
+        uint32_t v[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const uint32_t addr = kt + sw128_offset((uint32_t)(r0 + (r1 + i) * RSTEP), piece) + word;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v[i]) : "r"(addr));
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const uint32_t neg = ((v[i] >> 15) & 0x00010001u) * 0xFFFFu;  // 0xFFFF in each negative half
+          v[i] &= ~neg;
+          const uint32_t addr = kt + sw128_offset((uint32_t)(r0 + (r1 + i) * RSTEP), piece) + word;
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v[i]) : "memory");
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          z0 += bf16_lo_to_f32(v[i]);
+          z1 += bf16_hi_to_f32(v[i]);
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -289,8 +302,17 @@ __global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __res
   }
   if (t < ROWS) {
     const float* zsrc = partial + (size_t)bh * slab + (size_t)D * D + ROWS * g + t;
+    // eight independent loads at a time, added in split order
     float z = 0.f;
-    for (int q = 0; q < splits; ++q) z += zsrc[(size_t)q * split_stride];
+    int q = 0;
+    for (; q + 8 <= splits; q += 8) {
+      float a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = zsrc[(size_t)(q + i) * split_stride];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) z += a[i];
+    }
+    for (; q < splits; ++q) z += zsrc[(size_t)q * split_stride];
     z_out[(size_t)bh * D + ROWS * g + t] = z;
   }
   if constexpr (EXPORT) {
