@@ -135,3 +135,21 @@ def test_persistent_grid_many_tiles_per_cta(wl, ctas):
     ok, st = compare(got, run_oracle(wl, inp))
     assert ok, st
     assert np.array_equal(got, ref_gpu)
+
+
+@pytest.mark.parametrize("d,block", [(128, 128), (128, 64), (64, 128)])
+@pytest.mark.parametrize("factor", [5.0, 60.0])
+@pytest.mark.parametrize("where", ["first", "last"])
+def test_scores_jump_between_key_tiles(d, block, factor, where):
+    """One key block whose scores lie far above the rest.  Placed last, it moves
+    a row's maximum up in its last tiles: by ~2^17 with factor 5 (kept as large
+    p values, rescaled on the next tile) or far beyond 2^32 with factor 60, where
+    the kernel must recompute that tile against the new maximum (without that,
+    2^200 overflows).  Placed first, the maximum starts high and never moves."""
+    wl = wl_(d=d, block=block, T=4, H=8, W=16, Hh=2, window=(1, 2, 16), seed=23)  # one frame per 128 tokens
+    inp = si.make_inputs(wl)
+    k = si.bf16_bits_to_f32(inp.k).copy()
+    J = 0 if where == "first" else wl.nb - 1
+    k[:, J * block:(J + 1) * block] *= np.float32(factor)
+    inp.k = si.f32_to_bf16_bits(k)
+    check(wl, inp)
