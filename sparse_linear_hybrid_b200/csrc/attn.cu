@@ -28,22 +28,24 @@
 //              ring (after the item's last V tile);
 //   warp 11    output store: one TMA store per item once the softmax warps
 //              have staged its tile, then frees that Q buffer;
-//   warp 1     tcgen05 issuer (one thread) and TMEM owner: S = Q K_j^T into one
-//              of two TMEM S buffers (A, B in shared memory); O += P_j V_j with
+//   warp 1     tcgen05 issuer (one thread) and TMEM owner: copies the item's Q
+//              into tensor memory, S = Q K_j^T into one of two TMEM S buffers
+//              (A from tensor memory, K from shared memory); O += P_j V_j with
 //              P_j read from TMEM; U = relu(Q) [T_hi ; T_lo] of an item into the
 //              S buffer of the slot that follows its tiles, right after its
-//              last PV (the next item's first S follows U);
+//              last PV (the next item's Q copy and first S follow U);
 //   warps 2-9  softmax, two threads per query row (each takes half of the key
 //              columns of a tile and half of the feature columns of O): online
 //              softmax whose running maximum is only moved (and O rescaled in
 //              TMEM) when it grows by more than 2^8, P_j written to TMEM as
-//              bf16; after an item's last tile each thread applies ReLU to its
-//              half of its row of Q (the A operand of U) and sums its half of
-//              relu(q) . z; finally out = O / l + g U / den is staged in the
-//              item's Q buffer for the store warp.
+//              bf16; after an item's last tile each thread writes ReLU of its
+//              half of its row of Q over the Q columns (the A operand of U) and
+//              sums its half of relu(q) . z; finally out = O / l + g U / den is
+//              staged in the item's Q buffer for the store warp.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O [256,256+d),
-// P0 [384,448), P1 [448,512) (bf16 pairs).  P is double-buffered: the softmax
-// writes P_{j+1} while PV_j still reads P_j.  T is fed as a hi + lo pair of
+// P [384,384+BLK/2), Q [448,448+d/2) (bf16 pairs).  With Q in tensor memory the
+// S products read only K from shared memory.  P_{j+1} is written once PV_j has
+// completed (the softmax of tile j+1 outlasts it).  T is fed as a hi + lo pair of
 // bf16 halves (K doubled, relu(Q) read twice), so U keeps ~16 mantissa bits of
 // T.  Every barrier wait is bounded; on a time-out a role records it, stops and
 // drains what it issued.
@@ -113,15 +115,16 @@ struct AttnCfg {
   static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(AttnShared) + 1024;
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
   static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P = 384;
-  static constexpr uint32_t P_COLS = BLK / 2;       // one P buffer: BLK bf16 per row
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P = 384, TM_Q = 448;
+  static constexpr uint32_t P_COLS = BLK / 2;       // the P buffer: BLK bf16 per row
+  static constexpr uint32_t Q_COLS = D / 2;         // Q (then relu(Q)) in tensor memory: D bf16 per row
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false, false);   // Q K^T
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);     // P V   (V MN-major)
   static constexpr uint32_t IDESC_U = idesc_bf16(128, D, false, false);     // relu(Q) [T_hi ; T_lo]
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(!T_IN_RINGS || (T_BYTES == 2 * KV_BYTES && T_CH == 2 * DCH && T_CH_BYTES == KV_BOX),
                 "each half of T must have the layout of one K or V tile");
-  static_assert(TM_P + 2 * P_COLS <= 512 && D <= 128, "tensor memory budget");
+  static_assert(TM_P + P_COLS <= TM_Q && TM_Q + Q_COLS <= 512 && D <= 128, "tensor memory budget");
 };
 
 // Kept key tiles of one 128-row query tile, in ascending key-block order.
@@ -489,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // same tile (p_full), so once this thread has seen p_full of the tile that
       // last used a slot, that slot's s_free wait is already satisfied
       int st = 0, pf_seen = -1, slot_tile0 = -1, slot_tile1 = -1;  // S tiles issued, last p_full seen, per slot
+      int q_last = -1;  // S slot index of the last product that read the Q columns (S or U)
       // O += P V for global tile `gt` of the item whose V tiles start at V index
       // `gv0` (P from tensor memory; operands waited for here)
       auto issue_pv = [&](int gt, int gv, bool first) -> bool {
@@ -499,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         pf_seen = gt;
         tc_fence_after();
         const uint32_t vt = sbase + C::OFF_V0 + vs * C::KV_BYTES;
-        const uint32_t pt = tmem + C::TM_P + s * C::P_COLS;
+        const uint32_t pt = tmem + C::TM_P;
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk) {
           const uint64_t bd = sw128_desc(vt + kk * 2048, C::KV_BOX, 1024);
@@ -508,8 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&sh->pv_done[s]);  // also frees the V stage
         return true;
       };
-      // S = Q K^T into S slot `g` (K tile kj of the ring)
-      auto issue_s = [&](uint32_t q_addr) -> bool {
+      // S = Q K^T into the next S slot (K tile kj of the ring; Q from tensor memory)
+      auto issue_s = [&]() -> bool {
         const int s = sj & 1, ks = kj & 1;
         if (sh->abort_flag || !mbar_wait(&sh->k_full[ks], (uint32_t)((kj >> 1) & 1), limit_ns)) return false;
         const int prev = s ? slot_tile1 : slot_tile0;
@@ -527,12 +531,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_s = tmem + (s ? C::TM_S1 : C::TM_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sw128_desc(q_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(kt + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
-          mma_bf16_ss(d_s, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(d_s, tmem + C::TM_Q + kk * 8, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
         }
         mma_commit(&sh->s_full[s]);  // with T in the rings this also frees the K stage
         if (!C::T_IN_RINGS) mma_commit(&sh->k_empty[ks]);
+        q_last = sj;
         ++kj;
         ++sj;
         return true;
@@ -556,7 +560,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           slot_tile0 = -1;
         }
         tc_fence_after();
-        const uint32_t qr = sbase + C::OFF_Q0 + qb * C::Q_BYTES;
         const uint32_t t_hi = C::T_IN_RINGS ? sbase + C::OFF_K0 + ks * C::KV_BYTES : sbase + C::OFF_T;
         const uint32_t t_lo = C::T_IN_RINGS ? sbase + C::OFF_V0 + vs * C::KV_BYTES : t_hi + (C::T_CH / 2) * C::T_CH_BYTES;
         const uint32_t d_u = tmem + (s ? C::TM_S1 : C::TM_S0);
@@ -564,9 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 2 * D / 16; ++kk) {
           const int qk = kk % (D / 16), ch = kk / 4;  // ch: 64-column chunk of [T_hi | T_lo]
           const uint32_t tc = ch < C::T_CH / 2 ? t_hi + ch * C::T_CH_BYTES : t_lo + (ch - C::T_CH / 2) * C::T_CH_BYTES;
-          const uint64_t a = sw128_desc(qr + (qk / 4) * 16384 + (qk % 4) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(tc + (kk % 4) * 32, 16, 1024);
-          mma_bf16_ss(d_u, a, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(d_u, tmem + C::TM_Q + qk * 8, bd, C::IDESC_U, kk > 0 ? 1u : 0u);
         }
         mma_commit(&sh->s_full[s]);
         if (C::T_IN_RINGS) {
@@ -577,6 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&sh->t_empty);
           ++tl;
         }
+        q_last = sj;
         ++sj;
         return true;
       };
@@ -593,10 +596,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t q_addr = sbase + C::OFF_Q0 + slot * C::Q_BYTES;
         const int n = im.n;
         const int tt0 = tt, vj0 = vj;
-        // S_0, then S_j and PV_{j-1}, ..., PV_{n-1}, then U
-        if (n >= 1 && !issue_s(q_addr)) { ok = false; break; }
+        // Q into tensor memory (once the previous item's last S or U has read the
+        // columns), then S_0,
+        // S_j and PV_{j-1}, ..., PV_{n-1}, then U.  An item without key tiles keeps
+        // the Q columns for the relu(Q) its softmax warps write.
+        if (n >= 1) {
+          // the last product that read the Q columns has completed
+          if (q_last >= 0 && !mbar_wait(&sh->s_full[q_last & 1], (uint32_t)((q_last >> 1) & 1), limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            tmem_cp_128x256b(tmem + C::TM_Q + kk * 8, sw128_desc(q_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024));
+        }
+        if (n >= 1 && !issue_s()) { ok = false; break; }
         for (int j = 1; j < n && ok; ++j) {
-          if (!issue_s(q_addr) || !issue_pv(tt0 + j - 1, vj0 + j - 1, j == 1)) ok = false;
+          if (!issue_s() || !issue_pv(tt0 + j - 1, vj0 + j - 1, j == 1)) ok = false;
         }
         if (ok && n >= 1) ok = issue_pv(tt0 + n - 1, vj0 + n - 1, n == 1);
         if (!ok) break;
@@ -650,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           vtile = j == im.n - 1 ? im.vlast : BLK;  // only the last kept tile can be the partial block
         }
-        const int s = sj & 1, pb = tt & 1;
+        const int s = sj & 1;
         const bool aborted = __shfl_sync(0xffffffffu, sh->abort_flag != 0, 0);
         if (aborted || !mbar_wait_warp(&sh->s_full[s], (uint32_t)((sj >> 1) & 1), limit_ns)) { ok = false; break; }
         tc_fence_after();
@@ -746,18 +763,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           rs = 0.f;
         }
         l = l * alpha + rs;
-        // P buffer pb was last read by the PV of global tile tt-2; O may be rescaled
-        // only after the PV of tile tt-1 (this item's previous tile: no rescale on
-        // an item's first tile, whose reference starts at -inf)
-        if (tt >= 2) {
-          if (!mbar_wait_warp(&sh->pv_done[pb], (uint32_t)(((tt - 2) >> 1) & 1), limit_ns)) { ok = false; break; }
-        }
-        if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
-          if (!mbar_wait_warp(&sh->pv_done[pb ^ 1], (uint32_t)(((tt - 1) >> 1) & 1), limit_ns)) {
+        // the P buffer and O were last read / written by the PV of global tile tt-1
+        // (O is rescaled only within an item: an item's first tile has a reference
+        // that starts at -inf)
+        if (tt >= 1) {
+          if (!mbar_wait_warp(&sh->pv_done[(tt - 1) & 1], (uint32_t)(((tt - 1) >> 1) & 1), limit_ns)) {
             ok = false;
             break;
           }
-          tc_fence_after();
+        }
+        tc_fence_after();
+        if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
             uint32_t rr[32];
@@ -768,16 +784,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(lane_addr + C::TM_O + hf * HD + c * 32, rr);
           }
         }
-        tc_fence_after();
         if constexpr (HC / 2 == 32) {
-          tmem_st32(lane_addr + C::TM_P + pb * C::P_COLS + hf * (HC / 2), *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+          tmem_st32(lane_addr + C::TM_P + hf * (HC / 2), *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         } else {
-          tmem_st16(lane_addr + C::TM_P + pb * C::P_COLS + hf * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+          tmem_st16(lane_addr + C::TM_P + hf * (HC / 2), *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->p_full[pb]);
+        if (lane == 0) mbar_arrive(&sh->p_full[tt & 1]);
         ++sj;
         ++tt;
       }
@@ -795,8 +810,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        // all loads of this half-row first, then all stores: one shared-memory
-        // round trip instead of one per 16-byte piece
+        // this half of the row of Q from shared memory (all loads first), ReLU, into
+        // the Q columns of tensor memory (the A operand of U: the item's S products
+        // are done, the last one completed before this thread read its S)
         constexpr int NP = C::DCH * 4;  // 16-byte pieces in half a row
         uint32_t x[NP][4];
 #pragma unroll
@@ -806,14 +822,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                        x[t][1], x[t][2], x[t][3]);
         }
 #pragma unroll
-        for (int t = 0; t < NP; ++t) {
-          const int piece = hf * NP + t;
+        for (int t = 0; t < NP; ++t)
 #pragma unroll
           for (int i = 0; i < 4; ++i) x[t][i] = relu_bf16x2(x[t][i]);
-          st_shared_v4(q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8)), x[t][0],
-                       x[t][1], x[t][2], x[t][3]);
+        if constexpr (NP == 8) {
+          tmem_st32(lane_addr + C::TM_Q + hf * 4 * NP, *reinterpret_cast<uint32_t(*)[32]>(&x[0][0]));
+        } else {
+          tmem_st16(lane_addr + C::TM_Q + hf * 4 * NP, *reinterpret_cast<uint32_t(*)[16]>(&x[0][0]));
         }
-        fence_proxy_async_smem();
         const float4* zr = reinterpret_cast<const float4*>(sh->zs[slot]) + hf * NP * 2;
         float d0 = 0.f, d1 = 0.f;
 #pragma unroll
@@ -827,6 +843,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         den_h = d0 + d1;
+        tmem_st_wait();
+        tc_fence_before();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->q_relu[slot]);
