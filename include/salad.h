@@ -100,7 +100,9 @@ size_t salad_workspace_bytes(int B, int N, int num_heads, int d);
  *   q, k, v      DEVICE bf16 [B][N][Hh][d], 16-byte aligned.
  *   d            64 or 128.   block: 64 or 128.   Hh*d*2 bytes % 16 == 0.
  *   row_ptr, col_idx  DEVICE, from salad_build_block_mask with the same N
- *                (= T*H*W), block and num_heads; columns ascending.
+ *                (= T*H*W), block and num_heads; columns ascending.  (That
+ *                builder keeps every diagonal block; a row left empty by other
+ *                means gives those queries no sparse term: out = g * y.)
  *   w_proj       DEVICE bf16 [d][d] (row c, column e), 16-byte aligned.
  *   gate         DEVICE fp32 [B][Hh].
  *   softmax_scale  <= 0 selects 1/sqrt(d).   eps: added to the denominator.

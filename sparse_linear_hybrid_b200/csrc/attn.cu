@@ -798,37 +798,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       const int n = j;
-      // relu(Q) in place for U, each thread its half of its row (the S products
-      // are done with this Q buffer: the last one completed before this thread
-      // read its S), and this half's share of relu(q) . z on the way; the arrive
+      // relu(Q) over the Q columns of tensor memory for U, each thread its half of
+      // its row, and this half's share of relu(q) . z on the way; the arrive
       // happens for every item, so the barrier keeps count of items
       float den_h = 0.f;
-      ok = mbar_wait_warp(&sh->q_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns);
-      if (!ok) break;
+      // the Q buffer is overwritten by the output below: its load must be done
+      // (an item with key tiles knows it through its first S, issued after it)
+      if (n == 0 && !mbar_wait_warp(&sh->q_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns)) {
+        ok = false;
+        break;
+      }
       if (im.lin) {
         if (!mbar_wait_warp(&sh->z_full[slot], (uint32_t)((seq >> 1) & 1), limit_ns)) {
           ok = false;
           break;
         }
-        // this half of the row of Q from shared memory (all loads first), ReLU, into
-        // the Q columns of tensor memory (the A operand of U: the item's S products
-        // are done, the last one completed before this thread read its S)
-        constexpr int NP = C::DCH * 4;  // 16-byte pieces in half a row
+        // This half of the row of Q: from the Q columns of tensor memory, which hold
+        // this item's Q (its S products are done: the last one completed before
+        // this thread read its S); an item without key tiles never had its Q
+        // copied there, so it reads the Q buffer in shared memory instead.
+        constexpr int NP = C::DCH * 4;  // 16-byte pieces (8 features, 4 columns) in half a row
         uint32_t x[NP][4];
+        const uint32_t q_cols = lane_addr + C::TM_Q + hf * 4 * NP;
+        if (n >= 1) {
+          if constexpr (NP == 8) {
+            tmem_ld32(q_cols, *reinterpret_cast<uint32_t(*)[32]>(&x[0][0]));
+          } else {
+            tmem_ld16(q_cols, *reinterpret_cast<uint32_t(*)[16]>(&x[0][0]));
+          }
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-        for (int t = 0; t < NP; ++t) {
-          const int piece = hf * NP + t;  // features 8 * piece ... 8 * piece + 7
-          ld_shared_v4(q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8)), x[t][0],
-                       x[t][1], x[t][2], x[t][3]);
+          for (int t = 0; t < NP; ++t) {
+            const int piece = hf * NP + t;  // features 8 * piece ... 8 * piece + 7
+            ld_shared_v4(q_addr + (piece / 8) * 16384 + sw128_offset((uint32_t)r, (uint32_t)(piece % 8)), x[t][0],
+                         x[t][1], x[t][2], x[t][3]);
+          }
         }
 #pragma unroll
         for (int t = 0; t < NP; ++t)
 #pragma unroll
           for (int i = 0; i < 4; ++i) x[t][i] = relu_bf16x2(x[t][i]);
         if constexpr (NP == 8) {
-          tmem_st32(lane_addr + C::TM_Q + hf * 4 * NP, *reinterpret_cast<uint32_t(*)[32]>(&x[0][0]));
+          tmem_st32(q_cols, *reinterpret_cast<uint32_t(*)[32]>(&x[0][0]));
         } else {
-          tmem_st16(lane_addr + C::TM_Q + hf * 4 * NP, *reinterpret_cast<uint32_t(*)[16]>(&x[0][0]));
+          tmem_st16(q_cols, *reinterpret_cast<uint32_t(*)[16]>(&x[0][0]));
         }
         const float4* zr = reinterpret_cast<const float4*>(sh->zs[slot]) + hf * NP * 2;
         float d0 = 0.f, d1 = 0.f;

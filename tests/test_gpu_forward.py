@@ -153,3 +153,37 @@ def test_scores_jump_between_key_tiles(d, block, factor, where):
     k[:, J * block:(J + 1) * block] *= np.float32(factor)
     inp.k = si.f32_to_bf16_bits(k)
     check(wl, inp)
+
+
+@pytest.mark.parametrize("d,block", [(128, 128), (64, 128), (128, 64)])
+def test_query_block_with_no_kept_keys(d, block):
+    """A CSR row with no key blocks (the mask builder never makes one; a caller
+    may): those queries get no sparse term, out = g * (o_lin W), and the other
+    rows are unaffected.  Also runs the kernel's path for a work item without
+    key tiles."""
+    wl = wl_(d=d, block=block, B=1, Hh=2, seed=29)
+    inp = si.make_inputs(wl, v_mean=1.0)
+    rp, ci = oracle.block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)
+    nb = wl.nb
+    empty = [1, nb + nb - 1]  # row (h=0, I=1) and the last row of head 1
+    keep = np.ones(len(ci), dtype=bool)
+    for r in empty:
+        keep[rp[r]:rp[r + 1]] = False
+    counts = np.diff(rp).copy()
+    counts[empty] = 0
+    rp2 = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    ci2 = ci[keep].astype(np.int32)
+    t = upload(inp)
+    out = sl.attn_forward(t["q"], t["k"], t["v"], torch.from_numpy(rp2).cuda(), torch.from_numpy(ci2).cuda(),
+                          t["w"], t["gate"], wl.block)
+    torch.cuda.synchronize()
+    got = bf16_to_f64(out)
+    ref, _, o_lin = oracle.forward(inp.q, inp.k, inp.v, wl.block, rp2, ci2, inp.w_proj, inp.gate,
+                                   want_branches=True)
+    W = si.bf16_bits_to_f32(inp.w_proj).astype(np.float64)
+    for r in empty:
+        h, I = divmod(r, nb)
+        lo, hi = I * block, min(wl.N, (I + 1) * block)
+        ref[0, lo:hi, h] = inp.gate[0, h] * (o_lin[0, lo:hi, h] @ W)
+    ok, st = compare(got, ref)
+    assert ok, st
