@@ -203,6 +203,52 @@ def dist_env():
     return rank, world, local
 
 
+class RankGroup:
+    """The ranks of one run: one process per GPU, launched by torch.distributed.run
+    (rank, world size and local index from its environment).  With more than one
+    rank it holds the process group (NCCL on GPUs; any backend works) used for
+    the barrier around the timed region and the max of the timings; every rank
+    takes the same collective steps in the same order."""
+
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: float = 300.0):
+        self.rank, self.world, self.local = dist_env()
+        self.device = device
+        self._dist = None
+        if self.world > 1:
+            import torch.distributed as dist
+            kw = {"device_id": device} if device is not None and device.type == "cuda" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+            self._dist = dist
+
+    def barrier(self):
+        if self._dist is not None:
+            self._dist.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self._dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self._dist.all_reduce(t, op=self._dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self._dist is not None:
+            self._dist.destroy_process_group()
+            self._dist = None
+
+
+def rank_workload(wl: si.Workload, rank: int) -> si.Workload:
+    """Weak scaling: every rank runs its own batch of the workload (same shapes,
+    its own seed)."""
+    return wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def whole_job_tflops(world: int, steps: int, flops_per_step: float, total_ms: float) -> float:
+    """Throughput of the whole job: the work of all ranks over the slowest rank's time."""
+    return world * steps * flops_per_step / (total_ms / 1e3) / 1e12
+
+
 def config_of(wl: si.Workload, flops: float, nnz: int, world: int):
     return {"workload": wl.name, "B": wl.B, "heads": wl.Hh, "d": wl.d,
             "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.N, "block": wl.block,
@@ -323,28 +369,16 @@ def run_e2e(args, q, k, v, w, gate, out, flush, step, flops, world, max_over_ran
 
 def run_salad(args, wl):
     import torch
-    import torch.distributed as dist
 
     import sparse_linear_hybrid_b200 as sl
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    ranks = RankGroup("nccl", dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    my_wl = wl.with_(seed=wl.seed + 1000 * rank)
+    my_wl = rank_workload(wl, rank)
     inp = si.make_inputs(my_wl)
 
     def up(bits):
@@ -414,7 +448,7 @@ def run_salad(args, wl):
             drv.destroy(y)
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / K
-    value = world * K * flops / (total_ms / 1e3) / 1e12
+    value = whole_job_tflops(world, K, flops, total_ms)
 
     peaks = load_peaks()
     timed_s = sum(step_ms) / 1e3
@@ -484,8 +518,7 @@ def run_salad(args, wl):
                 "frac_of_bf16_peak_layer": round(value / world / peak, 4),
                 "kernel_source": src_hash}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def main():
