@@ -43,7 +43,9 @@ def _load():
         lib.oracle_forward_blocks.restype = None
         lib.oracle_forward_blocks.argtypes = ([P, P, P] + [ctypes.c_int] * 5 + [P, P, P, P]
                                               + [ctypes.c_double] * 2 + [P, P, P, ctypes.c_int]
-                                              + [P, P, P])
+                                              + [P, P, P, ctypes.c_int])
+        lib.oracle_topk_mask.restype = ctypes.c_int
+        lib.oracle_topk_mask.argtypes = [P, P] + [ctypes.c_int] * 6 + [P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -84,8 +86,9 @@ def linear_state(k, v):
 
 
 def forward_blocks(q, k, v, block, row_ptr, col_idx, w_proj, gate, pairs, tau=None,
-                   eps=1e-6, S=None, z=None, want_branches=False):
-    """Layer output for the listed (b*Hh+h, I) query blocks.
+                   eps=1e-6, S=None, z=None, want_branches=False, mask_per_bh=False):
+    """Layer output for the listed (b*Hh+h, I) query blocks.  The mask's rows are
+    (h, I), or (b*Hh+h, I) with mask_per_bh (a data-dependent mask).
 
     Returns out fp64 [npairs][block][d] (and o_sp, o_lin when want_branches).
     Rows of a partial last block past N hold NaN.
@@ -111,7 +114,7 @@ def forward_blocks(q, k, v, block, row_ptr, col_idx, w_proj, gate, pairs, tau=No
         _ptr(np.ascontiguousarray(row_ptr, dtype=np.int32)),
         _ptr(np.ascontiguousarray(col_idx, dtype=np.int32)),
         _ptr(w_proj), _ptr(gate), float(tau), float(eps),
-        _ptr(S), _ptr(z), _ptr(pairs), n, _ptr(out), _ptr(o_sp), _ptr(o_lin))
+        _ptr(S), _ptr(z), _ptr(pairs), n, _ptr(out), _ptr(o_sp), _ptr(o_lin), int(bool(mask_per_bh)))
     if want_branches:
         return out, o_sp, o_lin
     return out
@@ -123,16 +126,35 @@ def all_pairs(B, Hh, nb):
 
 
 def forward(q, k, v, block, row_ptr, col_idx, w_proj, gate, tau=None, eps=1e-6,
-            want_branches=False):
+            want_branches=False, mask_per_bh=False):
     """Full layer output fp64 [B, N, Hh, d] (every query block)."""
     B, N, Hh, d = q.shape
     nb = (N + block - 1) // block
     pairs = all_pairs(B, Hh, nb)
     res = forward_blocks(q, k, v, block, row_ptr, col_idx, w_proj, gate, pairs, tau, eps,
-                         want_branches=want_branches)
+                         want_branches=want_branches, mask_per_bh=mask_per_bh)
     outs = res if want_branches else (res,)
     full = []
     for o in outs:
         o = o.reshape(B, Hh, nb * block, d)[:, :, :N, :]
         full.append(np.ascontiguousarray(o.transpose(0, 2, 1, 3)))
     return tuple(full) if want_branches else full[0]
+
+
+def topk_mask(q, k, block, keep):
+    """Top-K dynamic block mask (see oracle_topk_mask): CSR over rows (b*Hh+h, I),
+    keep_eff = min(keep, nb) columns per row in ascending order.
+    Returns (row_ptr int32 [B*Hh*nb+1], col_idx int32 [B*Hh*nb*keep_eff])."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    B, N, Hh, d = q.shape
+    nb = (N + block - 1) // block
+    kk = min(int(keep), nb)
+    if kk < 1:
+        raise ValueError("keep must be >= 1")
+    row_ptr = np.zeros(B * Hh * nb + 1, dtype=np.int32)
+    col_idx = np.zeros(B * Hh * nb * kk, dtype=np.int32)
+    got = _load().oracle_topk_mask(_ptr(q), _ptr(k), B, N, Hh, d, int(block), int(keep), _ptr(row_ptr),
+                                   _ptr(col_idx))
+    assert got == kk
+    return row_ptr, col_idx

@@ -150,7 +150,7 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
                            int Hh, int d, int blk, const int32_t *row_ptr, const int32_t *col_idx,
                            const uint16_t *w_proj, const float *gate, double tau, double eps,
                            const double *S, const double *z, const int32_t *pairs, int npairs,
-                           double *out, double *o_sp, double *o_lin) {
+                           double *out, double *o_sp, double *o_lin, int mask_per_bh) {
     const int nb = (N + blk - 1) / blk;
     double *W = (double *)malloc(sizeof(double) * d * d);
     for (int i = 0; i < d * d; ++i) W[i] = bf16_to_double(w_proj[i]);
@@ -159,7 +159,8 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
         const int bh = pairs[2 * p], I = pairs[2 * p + 1];
         const int b = bh / Hh, h = bh % Hh;
         const double g = (double)gate[bh];
-        const int32_t r0 = row_ptr[h * nb + I], r1 = row_ptr[h * nb + I + 1];
+        const int mrow = (mask_per_bh ? bh : h) * nb + I; /* the mask has rows per head or per (b, h) */
+        const int32_t r0 = row_ptr[mrow], r1 = row_ptr[mrow + 1];
         /* gather the real key tokens of the kept key blocks, in CSR order */
         int64_t nkeys = 0;
         for (int32_t r = r0; r < r1; ++r) {
@@ -243,6 +244,95 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
 }
 
 /* Threads the OpenMP runtime will use (reported next to the CPU timings). */
+/*
+ * Top-K dynamic block mask.  The SALAD summary (section 5) names Top-K dynamic
+ * sparse attention among the kinds of sparse attention the method applies to,
+ * and gives no scoring rule.  Reading taken here: per (b, h), the mean of q
+ * over the real tokens of each block and the same for k; the score of block
+ * pair (I, J) is the dot product of the two means; row (b, h, I) keeps the
+ * `keep` highest scores (ties: the smaller J), listed in ascending J.  The
+ * arithmetic is fixed, in fp32, so that another implementation reproduces the
+ * scores bit for bit and takes the same integer decisions: each mean is the
+ * sum over the block's tokens in token order, then one division by the token
+ * count; each score is a chain of fused multiply-adds in feature order,
+ * starting from 0.
+ *
+ * q, k: bf16 [B][N][Hh][d].  kk = min(keep, nb) (keep >= 1).  row_ptr: int32
+ * [B*Hh*nb + 1] = r * kk for row r = (b*Hh + h)*nb + I; col_idx: int32
+ * [B*Hh*nb*kk].  Returns kk (0 for keep < 1).
+ */
+typedef struct {
+    float score;
+    int32_t j;
+} scored_block;
+
+static int by_score_desc_then_j(const void *a, const void *b) {
+    const scored_block *x = (const scored_block *)a, *y = (const scored_block *)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+static int by_int_asc(const void *a, const void *b) {
+    const int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+static float bf16_to_float(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+int oracle_topk_mask(const uint16_t *q, const uint16_t *k, int B, int N, int Hh, int d, int blk, int keep,
+                     int32_t *row_ptr, int32_t *col_idx) {
+    if (keep < 1) return 0;
+    const int nb = (N + blk - 1) / blk;
+    const int kk = keep < nb ? keep : nb;
+    const int64_t rows = (int64_t)B * Hh * nb;
+    for (int64_t r = 0; r <= rows; ++r) row_ptr[r] = (int32_t)(r * kk);
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < B * Hh; ++bh) {
+        const int b = bh / Hh, h = bh % Hh;
+        float *qm = (float *)malloc(sizeof(float) * nb * d);
+        float *km = (float *)malloc(sizeof(float) * nb * d);
+        scored_block *sc = (scored_block *)malloc(sizeof(scored_block) * nb);
+        int32_t *kept = (int32_t *)malloc(sizeof(int32_t) * kk);
+        for (int I = 0; I < nb; ++I) {
+            const int t0 = I * blk, t1 = (I + 1) * blk < N ? (I + 1) * blk : N;
+            for (int c = 0; c < d; ++c) {
+                float sq = 0.f, sk = 0.f;
+                for (int t = t0; t < t1; ++t) {
+                    const int64_t off = (((int64_t)b * N + t) * Hh + h) * d + c;
+                    sq += bf16_to_float(q[off]);
+                    sk += bf16_to_float(k[off]);
+                }
+                qm[(int64_t)I * d + c] = sq / (float)(t1 - t0);
+                km[(int64_t)I * d + c] = sk / (float)(t1 - t0);
+            }
+        }
+        for (int I = 0; I < nb; ++I) {
+            for (int J = 0; J < nb; ++J) {
+                float a = 0.f;
+                for (int c = 0; c < d; ++c) a = fmaf(qm[(int64_t)I * d + c], km[(int64_t)J * d + c], a);
+                sc[J].score = a;
+                sc[J].j = J;
+            }
+            qsort(sc, (size_t)nb, sizeof(scored_block), by_score_desc_then_j);
+            for (int t = 0; t < kk; ++t) kept[t] = sc[t].j;
+            qsort(kept, (size_t)kk, sizeof(int32_t), by_int_asc);
+            const int64_t r = (int64_t)bh * nb + I;
+            memcpy(col_idx + r * kk, kept, sizeof(int32_t) * kk);
+        }
+        free(qm);
+        free(km);
+        free(sc);
+        free(kept);
+    }
+    return kk;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);
