@@ -118,6 +118,45 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
                        const float* gate, float softmax_scale, float eps, void* out, void* workspace,
                        size_t workspace_bytes, salad_stream_t stream);
 
+/*
+ * Top-K dynamic block mask.  The SALAD summary (section 5) says the method also
+ * applies to Top-K dynamic sparse attention and gives no scoring rule; the rule
+ * implemented here is a reading of that sentence:
+ *   qm[b][h][I] = mean of q[b][i][h][:] over the real tokens i of block I,
+ *   km[b][h][J] likewise for k,  score(I, J) = qm[b][h][I] . km[b][h][J],
+ *   row (b, h, I) keeps the kk = min(keep, nb) key blocks J with the highest
+ *   scores (equal scores: the smaller J first), listed in ascending J.
+ * The arithmetic is fixed so that the result is reproducible bit for bit: fp32
+ * sums over the block's tokens in token order, one fp32 division by the token
+ * count, and each score a chain of fused multiply-adds over the features in
+ * order, starting from 0.
+ *
+ *   q, k       DEVICE bf16 [B][N][Hh][d], d = 64 or 128.   block >= 1, nb <= 2048.
+ *   keep       >= 1 (clamped to nb).
+ *   row_ptr    DEVICE int32 [B*Hh*nb + 1]: row r = (b*Hh + h)*nb + I holds
+ *              col_idx[r*kk .. (r+1)*kk).   col_idx: DEVICE int32 [B*Hh*nb*kk].
+ *   workspace  DEVICE, >= salad_topk_workspace_bytes(B, N, Hh, d, block), 4-byte
+ *              aligned (the block means).
+ * Rows are per (b, h): pass the mask to salad_attn_forward_bh.  Never
+ * synchronises.  Errors: INVALID_ARG, UNSUPPORTED (d, nb > 2048, sizes),
+ * WORKSPACE, CUDA.
+ */
+size_t salad_topk_workspace_bytes(int B, int N, int num_heads, int d, int block);
+int salad_build_topk_mask(const void* q, const void* k, int B, int N, int num_heads, int d, int block, int keep,
+                          int32_t* row_ptr, int32_t* col_idx, void* workspace, size_t workspace_bytes,
+                          salad_stream_t stream);
+
+/*
+ * salad_attn_forward with a mask whose rows are per (b, h) — row (b*Hh + h)*nb
+ * + I lists the key blocks of query block I of batch element b, head h (as
+ * salad_build_topk_mask writes them) — instead of per head.  Same arguments,
+ * rules and errors otherwise.
+ */
+int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                          int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                          const float* gate, float softmax_scale, float eps, void* out, void* workspace,
+                          size_t workspace_bytes, salad_stream_t stream);
+
 /* Size of the static device scratch behind salad_attn_forward_static: 32 MiB.
  * The scratch grows with B*Hh, not with N: at d = 128 it covers any N up to
  * B*Hh = 250 (about 1,000 at d = 64); the 12-head 32,760-token layer needs 20 MB,

@@ -55,6 +55,12 @@ def lib() -> ctypes.CDLL:
         L.salad_workspace_bytes.restype = sz
         L.salad_attn_forward.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
         L.salad_attn_forward.restype = i
+        L.salad_attn_forward_bh.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
+        L.salad_attn_forward_bh.restype = i
+        L.salad_topk_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.salad_topk_workspace_bytes.restype = sz
+        L.salad_build_topk_mask.argtypes = [p, p, i, i, i, i, i, i, p, p, p, sz, p]
+        L.salad_build_topk_mask.restype = i
         L.salad_attn_forward_static.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p]
         L.salad_attn_forward_static.restype = i
         L.salad_linear_state.argtypes = [p, p, i, i, i, i, p, p, p, p, sz, p]
@@ -141,17 +147,20 @@ def new_workspace(B: int, N: int, heads: int, d: int, device=None) -> torch.Tens
 
 
 def attn_forward(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_scale: float = 0.0,
-                 eps: float = 1e-6, out=None, workspace=None, stream=None) -> torch.Tensor:
-    """out = sparse ST-SWA attention + gate * (ReLU linear attention @ w_proj).
+                 eps: float = 1e-6, out=None, workspace=None, stream=None, mask_per_bh: bool = False) -> torch.Tensor:
+    """out = block-sparse attention + gate * (ReLU linear attention @ w_proj).
 
     q, k, v: bf16 CUDA [B, N, Hh, d]; w_proj bf16 [d, d]; gate fp32 [B, Hh].
+    The mask's rows are per head (build_block_mask), or per (b, h) with
+    mask_per_bh (build_topk_mask).
     """
     B, N, Hh, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = new_workspace(B, N, Hh, d, q.device)
-    _check(lib().salad_attn_forward(
+    fn = lib().salad_attn_forward_bh if mask_per_bh else lib().salad_attn_forward
+    _check(fn(
         _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
         B, N, Hh, d, block, _dev_ptr(row_ptr, torch.int32, "row_ptr"),
         _dev_ptr(col_idx, torch.int32, "col_idx"), _dev_ptr(w_proj, torch.bfloat16, "w_proj"),
@@ -159,6 +168,27 @@ def attn_forward(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_sc
         _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream)), "salad_attn_forward")
     return out
+
+
+def build_topk_mask(q, k, block: int, keep: int, workspace=None, stream=None):
+    """Top-K dynamic block mask (see salad.h) as a per-(b, h) CSR: (row_ptr,
+    col_idx) int32 CUDA tensors, min(keep, nb) ascending key blocks per row."""
+    B, N, Hh, d = q.shape
+    nb = (N + block - 1) // block
+    kk = min(int(keep), nb)
+    row_ptr = torch.empty(B * Hh * nb + 1, dtype=torch.int32, device=q.device)
+    col_idx = torch.empty(max(B * Hh * nb * kk, 1), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        n = lib().salad_topk_workspace_bytes(B, N, Hh, d, block)
+        if n == 0:
+            raise SaladError(SALAD_ERR_INVALID_ARG, "salad_topk_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    _check(lib().salad_build_topk_mask(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), B, N, Hh, d, int(block), int(keep),
+        _dev_ptr(row_ptr, torch.int32, "row_ptr"), _dev_ptr(col_idx, torch.int32, "col_idx"),
+        _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "salad_build_topk_mask")
+    return row_ptr, col_idx[:B * Hh * nb * kk]
 
 
 def attn_forward_static(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_scale: float = 0.0,

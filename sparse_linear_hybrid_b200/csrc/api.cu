@@ -157,10 +157,14 @@ size_t salad_workspace_bytes(int B, int N, int num_heads, int d) {
   return workspace_layout(B, N, num_heads, d).total;
 }
 
-int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
-                       int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
-                       const float* gate, float softmax_scale, float eps, void* out, void* workspace,
-                       size_t workspace_bytes, salad_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d, int block,
+                      const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj, const float* gate,
+                      float softmax_scale, float eps, void* out, void* workspace, size_t workspace_bytes,
+                      salad_stream_t stream, int mask_per_bh) {
   if (!q || !row_ptr || !col_idx || !w_proj || !gate || !out) return SALAD_ERR_INVALID_ARG;
   int st = check_common(k, v, B, N, num_heads, d, workspace, workspace_bytes);
   if (st != SALAD_OK) return st;
@@ -206,6 +210,7 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
   aa.z = reinterpret_cast<const float*>(ws + L.off_z);
   aa.work_ctr = reinterpret_cast<uint32_t*>(ws + L.off_status) + 1;
   aa.max_ctas = g_max_ctas.load();
+  aa.mask_per_bh = mask_per_bh;
   aa.B = B;
   aa.N = N;
   aa.heads = num_heads;
@@ -219,6 +224,62 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
   if (!record(g_ev_attn, s)) return SALAD_ERR_CUDA;
   if (launch_attention(aa, s) != cudaSuccess) return SALAD_ERR_CUDA;
   return record(g_ev_end, s) ? SALAD_OK : SALAD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                       int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                       const float* gate, float softmax_scale, float eps, void* out, void* workspace,
+                       size_t workspace_bytes, salad_stream_t stream) {
+  return attn_forward_impl(q, k, v, B, N, num_heads, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
+                           out, workspace, workspace_bytes, stream, 0);
+}
+
+int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                          int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                          const float* gate, float softmax_scale, float eps, void* out, void* workspace,
+                          size_t workspace_bytes, salad_stream_t stream) {
+  return attn_forward_impl(q, k, v, B, N, num_heads, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
+                           out, workspace, workspace_bytes, stream, 1);
+}
+
+size_t salad_topk_workspace_bytes(int B, int N, int num_heads, int d, int block) {
+  if (B < 1 || N < 1 || num_heads < 1 || (d != 64 && d != 128) || block < 1) return 0;
+  return topk_workspace_bytes(B, N, num_heads, d, block);
+}
+
+int salad_build_topk_mask(const void* q, const void* k, int B, int N, int num_heads, int d, int block, int keep,
+                          int32_t* row_ptr, int32_t* col_idx, void* workspace, size_t workspace_bytes,
+                          salad_stream_t stream) {
+  if (!q || !k || !row_ptr || !col_idx || !workspace || B < 1 || N < 1 || num_heads < 1 || block < 1 || keep < 1)
+    return SALAD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
+  const long long nb = ((long long)N + block - 1) / block;
+  if (nb > kTopkMaxBlocks) return SALAD_ERR_UNSUPPORTED;
+  const long long kk = keep < nb ? keep : nb;
+  if ((long long)B * num_heads * nb * kk >= (1ll << 31) || (long long)B * N * num_heads * d >= (1ll << 40))
+    return SALAD_ERR_UNSUPPORTED;
+  if (!aligned(q, 2) || !aligned(k, 2) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(workspace, 4))
+    return SALAD_ERR_INVALID_ARG;
+  if (workspace_bytes < topk_workspace_bytes(B, N, num_heads, d, block)) return SALAD_ERR_WORKSPACE;
+  TopkArgs ta{};
+  ta.q = static_cast<const uint16_t*>(q);
+  ta.k = static_cast<const uint16_t*>(k);
+  ta.B = B;
+  ta.N = N;
+  ta.heads = num_heads;
+  ta.d = d;
+  ta.block = block;
+  ta.nb = (int)nb;
+  ta.kk = (int)kk;
+  ta.qm = static_cast<float*>(workspace);
+  ta.km = ta.qm + (size_t)B * num_heads * nb * d;
+  ta.row_ptr = row_ptr;
+  ta.col_idx = col_idx;
+  return launch_topk_mask(ta, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
 }
 
 int salad_linear_state(const void* k, const void* v, int B, int N, int num_heads, int d, const float* gate,

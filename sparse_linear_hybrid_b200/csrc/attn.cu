@@ -181,7 +181,7 @@ __device__ __forceinline__ KeyIter make_iter(const int32_t* row_ptr, const int32
 
 template <int BLK>
 __device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, const int32_t* row_ptr,
-                                          const int32_t* col_idx, const float* gate) {
+                                          const int32_t* col_idx, const float* gate, int mask_per_bh) {
   Item im;
   im.w = w;
   im.bh = w / qtiles;
@@ -191,7 +191,8 @@ __device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, c
   im.g = gate[im.bh];
   im.lin = im.g != 0.0f;
   const int nb = (N + BLK - 1) / BLK;
-  KeyIter it = make_iter<BLK>(row_ptr, col_idx, im.h, nb, im.qtile);
+  // the mask's rows are per head, or per (b, h) for a data-dependent mask
+  KeyIter it = make_iter<BLK>(row_ptr, col_idx, mask_per_bh ? im.bh : im.h, nb, im.qtile);
   im.ra = (int)(it.a - col_idx);
   im.na = it.na;
   im.rb = it.b ? (int)(it.b - col_idx) : 0;
@@ -241,7 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_t, const int32_t* __restrict__ row_ptr,
                       const int32_t* __restrict__ col_idx, const float* __restrict__ gate,
                       const float* __restrict__ zvec, int heads, int N, int qtiles, int num_items,
-                      uint32_t* work_ctr, float scale_log2, float eps, uint32_t* status, uint64_t limit_ns) {
+                      uint32_t* work_ctr, float scale_log2, float eps, uint32_t* status, uint64_t limit_ns,
+                      int mask_per_bh) {
   using C = AttnCfg<D, BLK>;
 
   extern __shared__ uint8_t smem_raw[];
@@ -315,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int w = (int)atomicAdd(work_ctr, 1u);
         Item im;
         if (w < num_items) {
-          im = make_item<BLK>(w, qtiles, heads, N, row_ptr, col_idx, gate);
+          im = make_item<BLK>(w, qtiles, heads, N, row_ptr, col_idx, gate, mask_per_bh);
         } else {
           im.w = -1;
         }
@@ -963,7 +965,7 @@ cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   const int grid = (int)(items < ctas ? items : ctas);
   salad_attn_kernel<D, BLK><<<grid, kThreads, C::SMEM, s>>>(
       *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_t, a.row_ptr, a.col_idx, a.gate, a.z, a.heads, a.N, qtiles,
-      (int)items, a.work_ctr, a.scale_log2, a.eps, a.status, a.wait_limit_ns);
+      (int)items, a.work_ctr, a.scale_log2, a.eps, a.status, a.wait_limit_ns, a.mask_per_bh);
   return cudaGetLastError();
 }
 

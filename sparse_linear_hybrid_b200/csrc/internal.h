@@ -67,6 +67,7 @@ struct AttnArgs {
   const float* z;             // fp32 [B*Hh][d]
   uint32_t* work_ctr;         // next work item (zeroed by the linear kernel)
   int max_ctas;               // cap on the persistent grid (0: one CTA per SM)
+  int mask_per_bh;            // mask rows are (b*Hh + h, I) instead of (h, I)
   int B, N, heads, d, block;
   float scale_log2;  // softmax scale * log2(e)
   float eps;
@@ -74,6 +75,20 @@ struct AttnArgs {
   uint64_t wait_limit_ns;
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+// Top-K dynamic block mask (topk.cu).
+struct TopkArgs {
+  const uint16_t* q;  // bf16 [B][N][Hh][d]
+  const uint16_t* k;
+  int B, N, heads, d, block, nb, kk;  // kk = min(keep, nb) blocks kept per row
+  float* qm;                          // fp32 [B*Hh][nb][d] block means of q (workspace)
+  float* km;                          // and of k
+  int32_t* row_ptr;                   // [B*Hh*nb + 1]
+  int32_t* col_idx;                   // [B*Hh*nb*kk]
+};
+size_t topk_workspace_bytes(int B, int N, int heads, int d, int block);
+cudaError_t launch_topk_mask(const TopkArgs& a, cudaStream_t s);
+constexpr int kTopkMaxBlocks = 2048;  // the selection keeps one row of scores per query block in shared memory
 
 // Status word bits written by kernels.
 constexpr uint32_t kStatusTimeout = 1u;

@@ -131,3 +131,37 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(TypeError):
         sl.attn_forward(x, x, x, torch.zeros(3, dtype=torch.int32), torch.zeros(3, dtype=torch.int32),
                         torch.zeros(64, 64, dtype=torch.bfloat16), torch.zeros(1, 1), 64)
+
+
+def topk(L, **kw):
+    a = dict(q=FAKE, k=FAKE + 0x10000000, B=1, N=1000, H=2, d=64, block=64, keep=4, row_ptr=FAKE,
+             col_idx=FAKE, ws=0x40000000, ws_bytes=1 << 30)
+    a.update(kw)
+    return L.salad_build_topk_mask(p(a["q"]), p(a["k"]), a["B"], a["N"], a["H"], a["d"], a["block"], a["keep"],
+                                   p(a["row_ptr"]), p(a["col_idx"]), p(a["ws"]), a["ws_bytes"], None)
+
+
+def test_topk_mask_argument_errors(L):
+    assert topk(L, q=0) == sl.SALAD_ERR_INVALID_ARG
+    assert topk(L, col_idx=0) == sl.SALAD_ERR_INVALID_ARG
+    assert topk(L, ws=0) == sl.SALAD_ERR_INVALID_ARG
+    assert topk(L, keep=0) == sl.SALAD_ERR_INVALID_ARG
+    assert topk(L, block=0) == sl.SALAD_ERR_INVALID_ARG
+    assert topk(L, N=0) == sl.SALAD_ERR_INVALID_ARG
+    assert topk(L, d=96) == sl.SALAD_ERR_UNSUPPORTED
+    assert topk(L, N=2049 * 64) == sl.SALAD_ERR_UNSUPPORTED          # more than 2048 blocks per row
+    assert topk(L, row_ptr=FAKE + 2) == sl.SALAD_ERR_INVALID_ARG     # misaligned
+    assert topk(L, ws_bytes=16) == sl.SALAD_ERR_WORKSPACE
+    # two fp32 block means per (b, h, block, feature)
+    assert L.salad_topk_workspace_bytes(2, 1000, 3, 64, 64) == 2 * 2 * 3 * 16 * 64 * 4
+    assert L.salad_topk_workspace_bytes(1, 1000, 3, 80, 64) == 0
+
+
+def test_forward_bh_argument_errors(L):
+    def fwd(**kw):
+        a = dict(q=FAKE, k=FAKE + 0x10000000, v=FAKE + 0x20000000, out=FAKE + 0x30000000)
+        a.update(kw)
+        return L.salad_attn_forward_bh(p(a["q"]), p(a["k"]), p(a["v"]), 1, 256, 2, 64, 64, p(FAKE), p(FAKE),
+                                       p(FAKE), p(FAKE), 0.0, 1e-6, p(a["out"]), p(0x40000000), 1 << 30, None)
+    assert fwd(q=0) == sl.SALAD_ERR_INVALID_ARG
+    assert fwd(out=FAKE) == sl.SALAD_ERR_INVALID_ARG
