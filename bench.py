@@ -67,22 +67,27 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def mask_per_bh(wl: si.Workload) -> bool:
+    """True for a mask with rows per (b, h) (the Top-K mask), False for rows per head."""
+    return wl.topk > 0
+
+
 def kept_pairs_flops(row_ptr: np.ndarray, col_idx: np.ndarray, wl: si.Workload) -> float:
-    """4 * d * sum over kept (I, J) of |I| * |J| (real tokens), times B."""
+    """4 * d * sum over kept (I, J) of |I| * |J| (real tokens) over every (b, h)."""
     nb, blk, N = wl.nb, wl.block, wl.N
     sizes = np.minimum(blk, N - np.arange(nb) * blk).astype(np.float64)
-    rows = np.repeat(np.arange(wl.Hh * nb) % nb, np.diff(row_ptr))
+    rows = np.repeat(np.arange(len(row_ptr) - 1) % nb, np.diff(row_ptr))
     pairs = float(np.sum(sizes[rows] * sizes[col_idx]))
-    return 4.0 * wl.d * pairs * wl.B
+    return 4.0 * wl.d * pairs * (1 if mask_per_bh(wl) else wl.B)
 
 
 def block_flops(row_ptr, col_idx, wl, pairs):
     nb, blk, N = wl.nb, wl.block, wl.N
     sizes = np.minimum(blk, N - np.arange(nb) * blk).astype(np.float64)
+    per_bh = mask_per_bh(wl)
     tot = 0.0
     for bh, I in pairs:
-        h = int(bh) % wl.Hh
-        r = h * nb + int(I)
+        r = (int(bh) if per_bh else int(bh) % wl.Hh) * nb + int(I)
         tot += sizes[I] * float(np.sum(sizes[col_idx[row_ptr[r]:row_ptr[r + 1]]]))
     return 4.0 * wl.d * tot
 
@@ -196,6 +201,43 @@ def time_block_mask(wl, windows, row_ptr, col_idx, reps=5):
     return a.elapsed_time(b) / reps
 
 
+class TopkStep:
+    """The Top-K dynamic mask of one step through the C ABI, into fixed buffers
+    (the binding's helper allocates its outputs on every call)."""
+
+    def __init__(self, sl, wl, q, k):
+        import torch
+        self.sl, self.wl, self.q, self.k = sl, wl, q, k
+        kk = min(wl.topk, wl.nb)
+        self.row_ptr = torch.empty(wl.B * wl.Hh * wl.nb + 1, dtype=torch.int32, device=q.device)
+        self.col_idx = torch.empty(wl.B * wl.Hh * wl.nb * kk, dtype=torch.int32, device=q.device)
+        n = sl.lib().salad_topk_workspace_bytes(wl.B, wl.N, wl.Hh, wl.d, wl.block)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=q.device)
+
+    def run(self):
+        import ctypes
+
+        import torch
+        sl, wl = self.sl, self.wl
+        P = ctypes.c_void_p
+        st = sl.lib().salad_build_topk_mask(P(self.q.data_ptr()), P(self.k.data_ptr()), wl.B, wl.N, wl.Hh, wl.d,
+                                            wl.block, wl.topk, P(self.row_ptr.data_ptr()),
+                                            P(self.col_idx.data_ptr()), P(self.ws.data_ptr()), self.ws.numel(),
+                                            P(torch.cuda.current_stream().cuda_stream))
+        if st != sl.SALAD_OK:
+            raise RuntimeError(f"salad_build_topk_mask: {sl.status_string(st)}")
+
+    def device_ms(self, reps=5):
+        import torch
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            self.run()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -250,9 +292,11 @@ def whole_job_tflops(world: int, steps: int, flops_per_step: float, total_ms: fl
 
 
 def config_of(wl: si.Workload, flops: float, nnz: int, world: int):
+    rows = wl.B * wl.Hh * wl.nb if wl.topk else wl.Hh * wl.nb
+    mask = {"topk_keep": wl.topk} if wl.topk else {"window_thw": list(wl.window)}
     return {"workload": wl.name, "B": wl.B, "heads": wl.Hh, "d": wl.d,
             "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.N, "block": wl.block,
-            "window_thw": list(wl.window), "block_sparsity": round(1 - nnz / (wl.Hh * wl.nb ** 2), 5),
+            **mask, "block_sparsity": round(1 - nnz / (rows * wl.nb), 5),
             "kept_gflop_per_step": round(flops / 1e9, 3), "parallelism": f"replicas{world}",
             "l2": "flushed between steps (256 MB write outside the timed events)"}
 
@@ -264,6 +308,8 @@ def oracle_sample_rate(wl, inp, row_ptr, col_idx, budget_s, seed=0):
     (TFLOP/s, cores, sample description, seconds charged per sample)."""
     import oracle
     t0 = time.perf_counter()
+    if wl.topk:
+        oracle.topk_mask(inp.q, inp.k, wl.block, wl.topk)  # a dynamic mask is built every step
     S, z = oracle.linear_state(inp.k, inp.v)
     t_lin = time.perf_counter() - t0
     total = kept_pairs_flops(row_ptr, col_idx, wl)
@@ -275,13 +321,14 @@ def oracle_sample_rate(wl, inp, row_ptr, col_idx, budget_s, seed=0):
         batch = order[done:done + max(cores, 4)].astype(np.int32)
         t1 = time.perf_counter()
         oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate, batch,
-                              S=S, z=z)
+                              S=S, z=z, mask_per_bh=bool(wl.topk))
         t_fwd += time.perf_counter() - t1
         flops += block_flops(row_ptr, col_idx, wl, batch)
         done += len(batch)
     frac = flops / total
     charged = t_fwd + t_lin * frac
-    desc = (f"{done} of {len(order)} query blocks ({100 * frac:.2f}% of kept FLOPs) + the linear-branch state "
+    what = "the Top-K mask and the linear-branch state" if wl.topk else "the linear-branch state"
+    desc = (f"{done} of {len(order)} query blocks ({100 * frac:.2f}% of kept FLOPs) + {what} "
             f"of all heads ({t_lin:.2f}s, charged pro rata)")
     return flops / charged / 1e12, cores, desc, charged, done
 
@@ -292,12 +339,17 @@ def run_reference(args, wl):
         return
     import oracle
     inp = si.make_inputs(wl)
-    row_ptr, col_idx = oracle.block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)
-    flops_step = kept_pairs_flops(row_ptr, col_idx, wl)
     _t = time
     t0 = _t.perf_counter()
+    if wl.topk:  # a dynamic mask is built every step: charged with the linear state
+        row_ptr, col_idx = oracle.topk_mask(inp.q, inp.k, wl.block, wl.topk)
+    else:
+        row_ptr, col_idx = oracle.block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)
+    t_mask = _t.perf_counter() - t0 if wl.topk else 0.0
+    flops_step = kept_pairs_flops(row_ptr, col_idx, wl)
+    t0 = _t.perf_counter()
     S, z = oracle.linear_state(inp.k, inp.v)
-    t_lin = _t.perf_counter() - t0
+    t_lin = _t.perf_counter() - t0 + t_mask
     rng = np.random.default_rng(0)
     order = np.stack(np.unravel_index(rng.permutation(wl.B * wl.Hh * wl.nb), (wl.B * wl.Hh, wl.nb)), 1)
     cores = oracle.num_threads()
@@ -306,7 +358,7 @@ def run_reference(args, wl):
     per = max(cores, 4)
     t1 = _t.perf_counter()
     oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate,
-                          order[:per].astype(np.int32), S=S, z=z)
+                          order[:per].astype(np.int32), S=S, z=z, mask_per_bh=bool(wl.topk))
     per_block = (_t.perf_counter() - t1) / per
     m = int(max(1, min(len(order), step_budget / max(per_block, 1e-6))))
     times, flops_list = [], []
@@ -318,14 +370,15 @@ def run_reference(args, wl):
         pos += m
         t1 = _t.perf_counter()
         oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate, batch,
-                              S=S, z=z)
+                              S=S, z=z, mask_per_bh=bool(wl.topk))
         dt = _t.perf_counter() - t1
         fl = block_flops(row_ptr, col_idx, wl, batch)
         if i >= args.warmup:
             times.append(dt + t_lin * fl / flops_step)
             flops_list.append(fl)
     value = sum(flops_list) / sum(times) / 1e12
-    desc = (f"{m} query blocks per step (seeded, cycling over all {len(order)}) with the linear-branch state of "
+    what = "the Top-K mask and the linear-branch state" if wl.topk else "the linear-branch state"
+    desc = (f"{m} query blocks per step (seeded, cycling over all {len(order)}) with {what} of "
             f"all heads ({t_lin:.2f}s) charged pro rata to their kept FLOPs")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -387,10 +440,18 @@ def run_salad(args, wl):
     q, k, v, w = up(inp.q), up(inp.k), up(inp.v), up(inp.w_proj)
     gate = torch.from_numpy(inp.gate).to(dev)
     torch.cuda.synchronize()
-    row_ptr, col_idx = sl.build_block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows, device=dev)
-    # the mask build once more into the same buffers, on the device clock (the
-    # first call above also sizes col_idx and loads the kernels)
-    mask_ms = time_block_mask(wl, inp.windows, row_ptr, col_idx)
+    topk = None
+    if wl.topk:
+        # a dynamic mask: built from q and k in every step, into fixed buffers
+        topk = TopkStep(sl, wl, q, k)
+        row_ptr, col_idx = topk.row_ptr, topk.col_idx
+        topk.run()
+        mask_ms = topk.device_ms()
+    else:
+        row_ptr, col_idx = sl.build_block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows, device=dev)
+        # the mask build once more into the same buffers, on the device clock (the
+        # first call above also sizes col_idx and loads the kernels)
+        mask_ms = time_block_mask(wl, inp.windows, row_ptr, col_idx)
     rp_h, ci_h = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
     flops = kept_pairs_flops(rp_h, ci_h, wl)
     nnz = int(rp_h[-1])
@@ -399,7 +460,10 @@ def run_salad(args, wl):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step():
-        sl.attn_forward(q, k, v, row_ptr, col_idx, w, gate, wl.block, out=out, workspace=ws)
+        if topk is not None:
+            topk.run()
+        sl.attn_forward(q, k, v, row_ptr, col_idx, w, gate, wl.block, out=out, workspace=ws,
+                        mask_per_bh=topk is not None)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -472,7 +536,7 @@ def run_salad(args, wl):
                           "peak_gbs": peaks["hbm_gbs"],
                           "frac": round(kv_bytes / (lin_avg_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                           "algorithmic": "K and V read once: 4*d bytes per token per (b,h)"},
-        "mask_build_ms_once": round(mask_ms, 3),
+        ("topk_mask_ms_per_step" if wl.topk else "mask_build_ms_once"): round(mask_ms, 4),
         "attention_ms_p10_p50_p90": [round(float(np.percentile(att_ms, p)), 4) for p in (10, 50, 90)],
     }
 
@@ -484,7 +548,7 @@ def run_salad(args, wl):
 
     dense = None
     if not args.no_dense:
-        dwl = wl.with_(window=(wl.T, wl.H, wl.W))
+        dwl = wl.with_(window=(wl.T, wl.H, wl.W), topk=0)
         drp, dci = sl.build_block_mask(dwl.T, dwl.H, dwl.W, dwl.block, dwl.windows(), device=dev)
         zero_gate = torch.zeros_like(gate)
         dflops = kept_pairs_flops(drp.cpu().numpy(), dci.cpu().numpy(), dwl)
@@ -512,7 +576,7 @@ def run_salad(args, wl):
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": config_of(wl, flops, nnz, world),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * K,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (5 if wl.topk else 3) * K,
                 "clocks": clocks.summary(), "kernels": kernels, "dense": dense,
                 "wall_ms_per_step_incl_flush": round(1e3 * wall / K, 4),
                 "frac_of_bf16_peak_layer": round(value / world / peak, 4),

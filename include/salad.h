@@ -131,7 +131,8 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
  * count, and each score a chain of fused multiply-adds over the features in
  * order, starting from 0.
  *
- *   q, k       DEVICE bf16 [B][N][Hh][d], d = 64 or 128.   block >= 1, nb <= 2048.
+ *   q, k       DEVICE bf16 [B][N][Hh][d], 4-byte aligned, d = 64 or 128.   block >= 1,
+ *              nb <= 2048.
  *   keep       >= 1 (clamped to nb).
  *   row_ptr    DEVICE int32 [B*Hh*nb + 1]: row r = (b*Hh + h)*nb + I holds
  *              col_idx[r*kk .. (r+1)*kk).   col_idx: DEVICE int32 [B*Hh*nb*kk].

@@ -40,6 +40,7 @@ class Workload:
     head_scale: bool = False
     gate_lo: float = 0.0
     gate_hi: float = 1.0
+    topk: int = 0  # > 0: Top-K dynamic block mask keeping this many key blocks per query block (window unused)
 
     @property
     def N(self) -> int:
@@ -77,7 +78,11 @@ def sweep(pct: int) -> Workload:
                            window=SWEEP_WINDOWS[pct], seed=4)
 
 
-WORKLOADS = {w.name: w for w in [TINY, WAN13B_90, WAN13B_75_CFG, WAN14B_720P]
+# The 1.3B layer with a Top-K dynamic mask at the same ~90 % block sparsity
+# (26 of 256 key blocks per query block).
+WAN13B_TOPK = WAN13B_90.with_(name="wan1.3b-32760tok-topk26", topk=26, seed=5)
+
+WORKLOADS = {w.name: w for w in [TINY, WAN13B_90, WAN13B_75_CFG, WAN14B_720P, WAN13B_TOPK]
              + [sweep(p) for p in SWEEP_WINDOWS]}
 
 
