@@ -43,7 +43,9 @@ def _load():
         lib.oracle_forward_blocks.restype = None
         lib.oracle_forward_blocks.argtypes = ([P, P, P] + [ctypes.c_int] * 5 + [P, P, P, P]
                                               + [ctypes.c_double] * 2 + [P, P, P, ctypes.c_int]
-                                              + [P, P, P, ctypes.c_int])
+                                              + [P, P, P, ctypes.c_int, P])
+        lib.oracle_tile_mask.restype = ctypes.c_int64
+        lib.oracle_tile_mask.argtypes = [P, ctypes.c_int, P, P, P, ctypes.c_int64]
         lib.oracle_topk_mask.restype = ctypes.c_int
         lib.oracle_topk_mask.argtypes = [P, P] + [ctypes.c_int] * 6 + [P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -86,9 +88,11 @@ def linear_state(k, v):
 
 
 def forward_blocks(q, k, v, block, row_ptr, col_idx, w_proj, gate, pairs, tau=None,
-                   eps=1e-6, S=None, z=None, want_branches=False, mask_per_bh=False):
+                   eps=1e-6, S=None, z=None, want_branches=False, mask_per_bh=False, geom=None):
     """Layer output for the listed (b*Hh+h, I) query blocks.  The mask's rows are
-    (h, I), or (b*Hh+h, I) with mask_per_bh (a data-dependent mask).
+    (h, I), or (b*Hh+h, I) with mask_per_bh (a data-dependent mask).  With geom =
+    (T, H, W, bt, bh, bw) the blocks are 3-D tiles (block = bt*bh*bw slots; the
+    rows of `out` are the tile's slots, NaN where a slot holds no token).
 
     Returns out fp64 [npairs][block][d] (and o_sp, o_lin when want_branches).
     Rows of a partial last block past N hold NaN.
@@ -114,7 +118,8 @@ def forward_blocks(q, k, v, block, row_ptr, col_idx, w_proj, gate, pairs, tau=No
         _ptr(np.ascontiguousarray(row_ptr, dtype=np.int32)),
         _ptr(np.ascontiguousarray(col_idx, dtype=np.int32)),
         _ptr(w_proj), _ptr(gate), float(tau), float(eps),
-        _ptr(S), _ptr(z), _ptr(pairs), n, _ptr(out), _ptr(o_sp), _ptr(o_lin), int(bool(mask_per_bh)))
+        _ptr(S), _ptr(z), _ptr(pairs), n, _ptr(out), _ptr(o_sp), _ptr(o_lin), int(bool(mask_per_bh)),
+        _ptr(None if geom is None else np.ascontiguousarray(geom, dtype=np.int32)))
     if want_branches:
         return out, o_sp, o_lin
     return out
@@ -158,3 +163,58 @@ def topk_mask(q, k, block, keep):
                                    _ptr(col_idx))
     assert got == kk
     return row_ptr, col_idx
+
+
+def tile_geom(T, H, W, tile):
+    bt, bh, bw = tile
+    if T % bt:
+        raise ValueError("bt must divide T")
+    return np.array([T, H, W, bt, bh, bw], dtype=np.int32)
+
+
+def tile_slots(T, H, W, tile):
+    """Token of every slot of every tile, int64 [nb][bt*bh*bw] (-1: no token)."""
+    bt, bh, bw = tile
+    nt, nh, nw = T // bt, -(-H // bh), -(-W // bw)
+    out = np.full((nt * nh * nw, bt * bh * bw), -1, dtype=np.int64)
+    for I in range(nt * nh * nw):
+        ti, yi, xi = I // (nh * nw), (I // nw) % nh, I % nw
+        s = 0
+        for tt in range(bt):
+            for yy in range(bh):
+                for xx in range(bw):
+                    t, y, x = ti * bt + tt, yi * bh + yy, xi * bw + xx
+                    if t < T and y < H and x < W:
+                        out[I, s] = (t * H + y) * W + x
+                    s += 1
+    return out
+
+
+def tile_mask(T, H, W, tile, windows):
+    """Window mask over 3-D tile blocks: per-head CSR (row_ptr, col_idx) int32."""
+    windows = np.ascontiguousarray(windows, dtype=np.int32).reshape(-1, 3)
+    Hh = windows.shape[0]
+    geom = tile_geom(T, H, W, tile)
+    nb = (T // tile[0]) * (-(-H // tile[1])) * (-(-W // tile[2]))
+    row_ptr = np.zeros(Hh * nb + 1, dtype=np.int32)
+    total = _load().oracle_tile_mask(_ptr(geom), Hh, _ptr(windows), _ptr(row_ptr), None, 0)
+    col_idx = np.zeros(max(total, 1), dtype=np.int32)
+    _load().oracle_tile_mask(_ptr(geom), Hh, _ptr(windows), _ptr(row_ptr), _ptr(col_idx), total)
+    return row_ptr, col_idx[:total]
+
+
+def forward_tiles(q, k, v, T, H, W, tile, row_ptr, col_idx, w_proj, gate, tau=None, eps=1e-6):
+    """Full layer output fp64 [B, N, Hh, d] with 3-D tile blocks."""
+    B, N, Hh, d = q.shape
+    slots = tile_slots(T, H, W, tile)
+    nb, blk = slots.shape
+    pairs = all_pairs(B, Hh, nb)
+    res = forward_blocks(q, k, v, blk, row_ptr, col_idx, w_proj, gate, pairs, tau, eps,
+                         geom=tile_geom(T, H, W, tile))
+    res = res.reshape(B, Hh, nb, blk, d)
+    out = np.full((B, N, Hh, d), np.nan)
+    real = slots >= 0
+    for b in range(B):
+        for h in range(Hh):
+            out[b, slots[real], h] = res[b, h][real]
+    return out

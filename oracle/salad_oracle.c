@@ -94,6 +94,88 @@ int64_t oracle_block_mask(int T, int H, int W, int blk, int Hh, const int32_t *w
 }
 
 /*
+ * 3-D tile blocks (the SPADE explainer, section 1, puts attention on a 3-D grid
+ * of video blocks).  Reading taken: the T x H x W grid is cut into bt x bh x bw
+ * boxes (bt divides T; boxes at the H and W edges may stick out of the grid),
+ * numbered in raster order over (box t, box y, box x).  Box I has bt*bh*bw
+ * slots, slot s = (tt*bh + yy)*bw + xx for the point (t0 + tt, y0 + yy, x0 + xx);
+ * a slot outside the grid holds no token.  geom = {T, H, W, bt, bh, bw}.
+ * Writes the token of every slot of block I (-1 for a slot without one) and
+ * returns the slot count; without geom a block is `blk` raster tokens.
+ */
+static int block_tokens(const int32_t *geom, int64_t N, int blk, int64_t I, int64_t *tok) {
+    if (!geom) {
+        for (int s = 0; s < blk; ++s) tok[s] = I * blk + s < N ? I * blk + s : -1;
+        return blk;
+    }
+    const int T = geom[0], H = geom[1], W = geom[2], bt = geom[3], bh = geom[4], bw = geom[5];
+    const int nh = (H + bh - 1) / bh, nw = (W + bw - 1) / bw;
+    const int ti = (int)(I / ((int64_t)nh * nw)), yi = (int)((I / nw) % nh), xi = (int)(I % nw);
+    int s = 0;
+    for (int tt = 0; tt < bt; ++tt)
+        for (int yy = 0; yy < bh; ++yy)
+            for (int xx = 0; xx < bw; ++xx, ++s) {
+                const int t = ti * bt + tt, y = yi * bh + yy, x = xi * bw + xx;
+                tok[s] = (t < T && y < H && x < W) ? ((int64_t)t * H + y) * W + x : -1;
+            }
+    return s;
+}
+
+/*
+ * Window mask over 3-D tile blocks (geometry as for block_tokens): box pair
+ * (I, J) is kept when some real token of I and some real token of J lie within
+ * the window, found by brute force over the token pairs.  row_ptr: int32
+ * [Hh*nb + 1], col_idx as for oracle_block_mask; returns the kept pair count.
+ */
+int64_t oracle_tile_mask(const int32_t *geom, int Hh, const int32_t *windows, int32_t *row_ptr, int32_t *col_idx,
+                         int64_t cap) {
+    const int T = geom[0], H = geom[1], W = geom[2], bt = geom[3], bh = geom[4], bw = geom[5];
+    const int nb = (T / bt) * ((H + bh - 1) / bh) * ((W + bw - 1) / bw), slots = bt * bh * bw;
+    const int64_t N = (int64_t)T * H * W;
+    unsigned char *mark = (unsigned char *)calloc((size_t)nb * nb, 1);
+    int64_t total = 0;
+    for (int h = 0; h < Hh; ++h) {
+        const int wt = windows[3 * h + 0], wh = windows[3 * h + 1], ww = windows[3 * h + 2];
+        memset(mark, 0, (size_t)nb * nb);
+#pragma omp parallel for schedule(dynamic)
+        for (int I = 0; I < nb; ++I) {
+            int64_t *ti = (int64_t *)malloc(sizeof(int64_t) * slots), *tj = (int64_t *)malloc(sizeof(int64_t) * slots);
+            block_tokens(geom, N, 0, I, ti);
+            for (int J = 0; J < nb; ++J) {
+                block_tokens(geom, N, 0, J, tj);
+                int kept = 0;
+                for (int a = 0; a < slots && !kept; ++a) {
+                    if (ti[a] < 0) continue;
+                    const int64_t x = ti[a] % W, y = (ti[a] / W) % H, t = ti[a] / ((int64_t)W * H);
+                    for (int c = 0; c < slots; ++c) {
+                        if (tj[c] < 0) continue;
+                        const int64_t x2 = tj[c] % W, y2 = (tj[c] / W) % H, t2 = tj[c] / ((int64_t)W * H);
+                        if (llabs(t - t2) <= wt && llabs(y - y2) <= wh && llabs(x - x2) <= ww) {
+                            kept = 1;
+                            break;
+                        }
+                    }
+                }
+                mark[(int64_t)I * nb + J] = (unsigned char)kept;
+            }
+            free(ti);
+            free(tj);
+        }
+        for (int I = 0; I < nb; ++I) {
+            row_ptr[h * nb + I] = (int32_t)total;
+            for (int J = 0; J < nb; ++J)
+                if (mark[(int64_t)I * nb + J]) {
+                    if (col_idx && total < cap) col_idx[total] = J;
+                    ++total;
+                }
+        }
+    }
+    row_ptr[Hh * nb] = (int32_t)total;
+    free(mark);
+    return total;
+}
+
+/*
  * Linear-branch state of every (b, h), over all N real tokens (global and
  * non-causal: the summary's section 2.1 gives the linear branch the job of
  * interactions between all tokens):
@@ -150,8 +232,11 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
                            int Hh, int d, int blk, const int32_t *row_ptr, const int32_t *col_idx,
                            const uint16_t *w_proj, const float *gate, double tau, double eps,
                            const double *S, const double *z, const int32_t *pairs, int npairs,
-                           double *out, double *o_sp, double *o_lin, int mask_per_bh) {
-    const int nb = (N + blk - 1) / blk;
+                           double *out, double *o_sp, double *o_lin, int mask_per_bh, const int32_t *geom) {
+    /* geom: 3-D tile blocks (see block_tokens; then blk = bt*bh*bw), or NULL */
+    const int nb = geom ? (geom[0] / geom[3]) * ((geom[1] + geom[4] - 1) / geom[4]) *
+                              ((geom[2] + geom[5] - 1) / geom[5])
+                        : (N + blk - 1) / blk;
     double *W = (double *)malloc(sizeof(double) * d * d);
     for (int i = 0; i < d * d; ++i) W[i] = bf16_to_double(w_proj[i]);
 #pragma omp parallel for schedule(dynamic)
@@ -162,12 +247,8 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
         const int mrow = (mask_per_bh ? bh : h) * nb + I; /* the mask has rows per head or per (b, h) */
         const int32_t r0 = row_ptr[mrow], r1 = row_ptr[mrow + 1];
         /* gather the real key tokens of the kept key blocks, in CSR order */
-        int64_t nkeys = 0;
-        for (int32_t r = r0; r < r1; ++r) {
-            const int64_t J = col_idx[r];
-            const int64_t j_end = (J + 1) * blk < N ? (J + 1) * blk : N;
-            nkeys += j_end - J * blk;
-        }
+        int64_t *slot_tok = (int64_t *)malloc(sizeof(int64_t) * blk);
+        const int64_t nkeys = (int64_t)(r1 - r0) * blk;
         int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (nkeys > 0 ? nkeys : 1));
         double *s = (double *)malloc(sizeof(double) * (nkeys > 0 ? nkeys : 1));
         double *qi = (double *)malloc(sizeof(double) * d);
@@ -175,12 +256,15 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
         double *lin = (double *)malloc(sizeof(double) * d);
         int64_t nk = 0;
         for (int32_t r = r0; r < r1; ++r) {
-            const int64_t J = col_idx[r];
-            const int64_t j_end = (J + 1) * blk < N ? (J + 1) * blk : N;
-            for (int64_t j = J * blk; j < j_end; ++j) keys[nk++] = j;
+            block_tokens(geom, N, blk, col_idx[r], slot_tok);
+            for (int sl = 0; sl < blk; ++sl)
+                if (slot_tok[sl] >= 0) keys[nk++] = slot_tok[sl];
         }
-        const int64_t i_end = (int64_t)(I + 1) * blk < N ? (int64_t)(I + 1) * blk : N;
-        for (int64_t i = (int64_t)I * blk; i < i_end; ++i) {
+        int64_t *qtok = (int64_t *)malloc(sizeof(int64_t) * blk);
+        block_tokens(geom, N, blk, I, qtok);
+        for (int qs = 0; qs < blk; ++qs) {
+            if (qtok[qs] < 0) continue;
+            const int64_t i = qtok[qs];
             const int64_t qoff = (((int64_t)b * N + i) * Hh + h) * d;
             for (int c = 0; c < d; ++c) qi[c] = bf16_to_double(q[qoff + c]);
             /* sparse branch: exact softmax over the kept keys */
@@ -200,7 +284,7 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
                 den += pexp;
                 for (int c = 0; c < d; ++c) acc[c] += pexp * bf16_to_double(v[voff + c]);
             }
-            const int64_t ooff = ((int64_t)p * blk + (i - (int64_t)I * blk)) * d;
+            const int64_t ooff = ((int64_t)p * blk + qs) * d;
             for (int c = 0; c < d; ++c) {
                 acc[c] /= den;
                 if (o_sp) o_sp[ooff + c] = acc[c];
@@ -235,6 +319,8 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
             }
         }
         free(keys);
+        free(slot_tok);
+        free(qtok);
         free(s);
         free(qi);
         free(acc);
