@@ -78,6 +78,35 @@ int salad_build_block_mask(int T, int H, int W, int block, int num_heads, const 
                            salad_stream_t stream);
 
 /*
+ * 3-D tile blocks (the SPADE page's 3-D grid of video blocks; the SALAD
+ * summary's block structure over the T x H x W latent): block I is the box of
+ * bt x bh x bw grid points
+ *   t in [ti*bt, ti*bt+bt),  y in [yi*bh, yi*bh+bh),  x in [xi*bw, xi*bw+bw)
+ * with boxes numbered in raster order, I = (ti*nh + yi)*nw + xi, nh =
+ * ceil(H/bh), nw = ceil(W/bw).  bt must divide T; boxes at the bottom and right
+ * edges may stick out of the grid, and their slots outside it hold no token.
+ * Slot s = (tt*bh + yy)*bw + xx of box I holds token (t*H + y)*W + x of the
+ * flat [T][H][W] sequence.
+ * salad_tile_num_blocks: nb = (T/bt) * nh * nw.  Host only.  Errors:
+ * INVALID_ARG (non-positive sizes, T*H*W >= 2^31, nb == NULL); UNSUPPORTED
+ * when bt does not divide T.
+ */
+int salad_tile_num_blocks(int T, int H, int W, int bt, int bh, int bw, int* nb);
+
+/*
+ * The ST-SWA window mask over 3-D tile blocks: row (h, I) lists, in ascending
+ * order, the boxes J holding SOME token pair i in I, j in J within the head's
+ * windows (|t_i - t_j| <= wt, |y_i - y_j| <= wh, |x_i - x_j| <= ww).  Since each
+ * box covers a product of ranges (clipped to the grid), that is: on every axis
+ * the gap between the two boxes' ranges is within that axis' window.
+ * Arguments, layouts, synchronisation and errors as salad_build_block_mask
+ * (nb from salad_tile_num_blocks; UNSUPPORTED when bt does not divide T).
+ */
+int salad_build_tile_mask(int T, int H, int W, int bt, int bh, int bw, int num_heads, const int32_t* windows,
+                          int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int64_t* nnz_out,
+                          salad_stream_t stream);
+
+/*
  * Bytes of device workspace salad_attn_forward needs for these sizes (0 on bad
  * arguments).  The workspace holds a status word, the linear-branch state
  * [S | z] of every (b, h) and the split-N partial sums.  It must be zero-filled
@@ -142,6 +171,24 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
  * synchronises.  Errors: INVALID_ARG, UNSUPPORTED (d, nb > 2048, sizes),
  * WORKSPACE, CUDA.
  */
+/*
+ * The SALAD layer forward over 3-D tile blocks (salad_tile_num_blocks): the
+ * same output as salad_attn_forward, token by token, with the sparse branch's
+ * key set K(i) = every real token of the boxes kept for the box holding i.
+ *   q, k, v, out  DEVICE bf16 [B][T][H][W][Hh][d] (the [B][N][Hh][d] layout
+ *                 with N = T*H*W in raster order), 16-byte aligned.
+ *   bt*bh*bw      must be 128 (one box fills one 128-row query tile); T % bt == 0.
+ *   row_ptr, col_idx  DEVICE, from salad_build_tile_mask with the same grid,
+ *                 tile and num_heads.
+ *   Other arguments, workspace (salad_workspace_bytes(B, T*H*W, Hh, d)),
+ *   arithmetic and errors as salad_attn_forward; UNSUPPORTED when
+ *   bt*bh*bw != 128 or bt does not divide T.
+ */
+int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B, int T, int H, int W, int bt,
+                             int bh, int bw, int num_heads, int d, const int32_t* row_ptr, const int32_t* col_idx,
+                             const void* w_proj, const float* gate, float softmax_scale, float eps, void* out,
+                             void* workspace, size_t workspace_bytes, salad_stream_t stream);
+
 size_t salad_topk_workspace_bytes(int B, int N, int num_heads, int d, int block);
 int salad_build_topk_mask(const void* q, const void* k, int B, int N, int num_heads, int d, int block, int keep,
                           int32_t* row_ptr, int32_t* col_idx, void* workspace, size_t workspace_bytes,

@@ -41,6 +41,7 @@ class Workload:
     gate_lo: float = 0.0
     gate_hi: float = 1.0
     topk: int = 0  # > 0: Top-K dynamic block mask keeping this many key blocks per query block (window unused)
+    tile: tuple = ()  # (bt, bh, bw): 3-D tile blocks of bt*bh*bw = block grid points; (): raster blocks
 
     @property
     def N(self) -> int:
@@ -48,6 +49,9 @@ class Workload:
 
     @property
     def nb(self) -> int:
+        if self.tile:
+            bt, bh, bw = self.tile
+            return (self.T // bt) * (-(-self.H // bh)) * (-(-self.W // bw))
         return (self.N + self.block - 1) // self.block
 
     def windows(self) -> np.ndarray:
@@ -82,7 +86,12 @@ def sweep(pct: int) -> Workload:
 # (26 of 256 key blocks per query block).
 WAN13B_TOPK = WAN13B_90.with_(name="wan1.3b-32760tok-topk26", topk=26, seed=5)
 
-WORKLOADS = {w.name: w for w in [TINY, WAN13B_90, WAN13B_75_CFG, WAN14B_720P, WAN13B_TOPK]
+# The 1.3B layer with the same token window over 3-D tile blocks of 1 x 16 x 8
+# grid points (294 boxes per head, 12.9 % of their slots off the grid; 8.2 % of
+# the box pairs kept).
+WAN13B_TILES = WAN13B_90.with_(name="wan1.3b-32760tok-tiles1x16x8", tile=(1, 16, 8), seed=6)
+
+WORKLOADS = {w.name: w for w in [TINY, WAN13B_90, WAN13B_75_CFG, WAN14B_720P, WAN13B_TOPK, WAN13B_TILES]
              + [sweep(p) for p in SWEEP_WINDOWS]}
 
 

@@ -6,8 +6,9 @@ PyTorch supplies device memory and streams.  There is no CPU fallback: calls
 raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
-    mask_num_blocks, build_block_mask, workspace_bytes, attn_forward,
-    attn_forward_static, linear_state, check_status, set_wait_limit_ns, set_max_ctas, set_phase_events,
+    mask_num_blocks, build_block_mask, tile_num_blocks, build_tile_mask, workspace_bytes, attn_forward,
+    attn_forward_tiles, attn_forward_static, linear_state, check_status, set_wait_limit_ns, set_max_ctas,
+    set_phase_events,
     status_string
 """
 from __future__ import annotations
@@ -51,12 +52,20 @@ def lib() -> ctypes.CDLL:
         L.salad_build_block_mask.argtypes = [i, i, i, i, i, p, p, p, ctypes.c_int64,
                                              ctypes.POINTER(ctypes.c_int64), p]
         L.salad_build_block_mask.restype = i
+        L.salad_tile_num_blocks.argtypes = [i, i, i, i, i, i, ctypes.POINTER(i)]
+        L.salad_tile_num_blocks.restype = i
+        L.salad_build_tile_mask.argtypes = [i, i, i, i, i, i, i, p, p, p, ctypes.c_int64,
+                                            ctypes.POINTER(ctypes.c_int64), p]
+        L.salad_build_tile_mask.restype = i
         L.salad_workspace_bytes.argtypes = [i, i, i, i]
         L.salad_workspace_bytes.restype = sz
         L.salad_attn_forward.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
         L.salad_attn_forward.restype = i
         L.salad_attn_forward_bh.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
         L.salad_attn_forward_bh.restype = i
+        L.salad_attn_forward_tiles.argtypes = [p, p, p, i, i, i, i, i, i, i, i, i, p, p, p, p, f, f, p, p, sz,
+                                               p]
+        L.salad_attn_forward_tiles.restype = i
         L.salad_topk_workspace_bytes.argtypes = [i, i, i, i, i]
         L.salad_topk_workspace_bytes.restype = sz
         L.salad_build_topk_mask.argtypes = [p, p, i, i, i, i, i, i, p, p, p, sz, p]
@@ -110,27 +119,49 @@ def mask_num_blocks(T: int, H: int, W: int, block: int) -> int:
     return nb.value
 
 
-def build_block_mask(T: int, H: int, W: int, block: int, windows, device=None, stream=None):
-    """ST-SWA block mask as a per-head CSR: (row_ptr, col_idx) int32 CUDA tensors."""
-    win = np.ascontiguousarray(windows, dtype=np.int32).reshape(-1, 3)
-    heads = win.shape[0]
-    nb = mask_num_blocks(T, H, W, block)
+def _build_csr(name, nb, heads, call, device):
+    """Size-then-fill of a window mask CSR through `call(row_ptr, col_idx, cap, nnz)`."""
     device = torch.device("cuda") if device is None else torch.device(device)
     row_ptr = torch.empty(heads * nb + 1, dtype=torch.int32, device=device)
     nnz = ctypes.c_int64(0)
-    s = _stream(stream)
-    st = lib().salad_build_block_mask(T, H, W, block, heads, win.ctypes.data_as(ctypes.c_void_p),
-                                      _dev_ptr(row_ptr, torch.int32, "row_ptr"), None, 0,
-                                      ctypes.byref(nnz), s)
+    st = call(_dev_ptr(row_ptr, torch.int32, "row_ptr"), None, 0, nnz)
     if st not in (SALAD_OK, SALAD_ERR_CAPACITY):
-        _check(st, "salad_build_block_mask")
+        _check(st, name)
     col_idx = torch.empty(max(int(nnz.value), 1), dtype=torch.int32, device=device)
-    _check(lib().salad_build_block_mask(T, H, W, block, heads, win.ctypes.data_as(ctypes.c_void_p),
-                                        _dev_ptr(row_ptr, torch.int32, "row_ptr"),
-                                        _dev_ptr(col_idx, torch.int32, "col_idx"),
-                                        col_idx.numel(), ctypes.byref(nnz), s),
-           "salad_build_block_mask")
+    _check(call(_dev_ptr(row_ptr, torch.int32, "row_ptr"), _dev_ptr(col_idx, torch.int32, "col_idx"),
+                col_idx.numel(), nnz), name)
     return row_ptr, col_idx[:int(nnz.value)]
+
+
+def build_block_mask(T: int, H: int, W: int, block: int, windows, device=None, stream=None):
+    """ST-SWA block mask as a per-head CSR: (row_ptr, col_idx) int32 CUDA tensors."""
+    win = np.ascontiguousarray(windows, dtype=np.int32).reshape(-1, 3)
+    s = _stream(stream)
+
+    def call(rp, ci, cap, nnz):
+        return lib().salad_build_block_mask(T, H, W, block, win.shape[0], win.ctypes.data_as(ctypes.c_void_p),
+                                            rp, ci, cap, ctypes.byref(nnz), s)
+    return _build_csr("salad_build_block_mask", mask_num_blocks(T, H, W, block), win.shape[0], call, device)
+
+
+def tile_num_blocks(T: int, H: int, W: int, tile) -> int:
+    bt, bh, bw = tile
+    nb = ctypes.c_int(0)
+    _check(lib().salad_tile_num_blocks(T, H, W, bt, bh, bw, ctypes.byref(nb)), "salad_tile_num_blocks")
+    return nb.value
+
+
+def build_tile_mask(T: int, H: int, W: int, tile, windows, device=None, stream=None):
+    """ST-SWA mask over bt x bh x bw boxes of the grid: per-head CSR (row_ptr, col_idx)."""
+    bt, bh, bw = tile
+    win = np.ascontiguousarray(windows, dtype=np.int32).reshape(-1, 3)
+    s = _stream(stream)
+
+    def call(rp, ci, cap, nnz):
+        return lib().salad_build_tile_mask(T, H, W, bt, bh, bw, win.shape[0],
+                                           win.ctypes.data_as(ctypes.c_void_p), rp, ci, cap,
+                                           ctypes.byref(nnz), s)
+    return _build_csr("salad_build_tile_mask", tile_num_blocks(T, H, W, tile), win.shape[0], call, device)
 
 
 def workspace_bytes(B: int, N: int, heads: int, d: int) -> int:
@@ -167,6 +198,29 @@ def attn_forward(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_sc
         _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps),
         _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream)), "salad_attn_forward")
+    return out
+
+
+def attn_forward_tiles(q, k, v, grid, tile, row_ptr, col_idx, w_proj, gate, softmax_scale: float = 0.0,
+                       eps: float = 1e-6, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """attn_forward with 3-D tile blocks: grid = (T, H, W), tile = (bt, bh, bw)
+    with bt * bh * bw == 128; the mask from build_tile_mask."""
+    B, N, Hh, d = q.shape
+    T, H, W = grid
+    bt, bh, bw = tile
+    if N != T * H * W:
+        raise ValueError(f"q has {N} tokens, the grid {T * H * W}")
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = new_workspace(B, N, Hh, d, q.device)
+    _check(lib().salad_attn_forward_tiles(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
+        B, T, H, W, bt, bh, bw, Hh, d, _dev_ptr(row_ptr, torch.int32, "row_ptr"),
+        _dev_ptr(col_idx, torch.int32, "col_idx"), _dev_ptr(w_proj, torch.bfloat16, "w_proj"),
+        _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps),
+        _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream)), "salad_attn_forward_tiles")
     return out
 
 

@@ -39,9 +39,10 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
               const uint32_t* box) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t d[3];
-  cuuint64_t st[2];
-  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  if (rank < 1 || rank > 4) return false;
+  cuuint64_t d[4];
+  cuuint64_t st[3];
+  cuuint32_t bx[4], es[4] = {1, 1, 1, 1};
   for (int i = 0; i < rank; ++i) {
     d[i] = dims[i];
     bx[i] = box[i];
@@ -59,6 +60,16 @@ bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int Hh, int d
   const uint64_t strides[2] = {(uint64_t)Hh * d * 2, (uint64_t)N * Hh * d * 2};
   const uint32_t box[3] = {64, rows, 1};
   return make_map(m, base, 3, dims, strides, box);
+}
+
+// [B][T][H][W][Hh][d] bf16 viewed as a 4-D tensor (Hh*d, W, H, B*T); box
+// (64, bw, bh, bt), one 3-D tile block of one head's 64-feature chunk.
+bool make_tile_map(CUtensorMap* m, const void* base, int B, const TileGeom& g, int Hh, int d) {
+  const uint64_t row = (uint64_t)Hh * d * 2;
+  const uint64_t dims[4] = {(uint64_t)Hh * d, (uint64_t)g.W, (uint64_t)g.H, (uint64_t)B * g.T};
+  const uint64_t strides[3] = {row, row * g.W, row * g.W * g.H};
+  const uint32_t box[4] = {64, (uint32_t)g.bw, (uint32_t)g.bh, (uint32_t)g.bt};
+  return make_map(m, base, 4, dims, strides, box);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -119,11 +130,42 @@ int salad_mask_num_blocks(int T, int H, int W, int block, int* nb) {
   return SALAD_OK;
 }
 
+namespace {
+int build_mask_impl(int T, int H, int W, int block, int bt, int bh, int bw, int num_heads, const int32_t* windows,
+                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int64_t* nnz_out,
+                    salad_stream_t stream);
+}
+
 int salad_build_block_mask(int T, int H, int W, int block, int num_heads, const int32_t* windows,
                            int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int64_t* nnz_out,
                            salad_stream_t stream) {
+  return build_mask_impl(T, H, W, block, 0, 0, 0, num_heads, windows, row_ptr, col_idx, col_capacity, nnz_out,
+                         stream);
+}
+
+int salad_tile_num_blocks(int T, int H, int W, int bt, int bh, int bw, int* nb) {
+  if (!nb || T < 1 || H < 1 || W < 1 || bt < 1 || bh < 1 || bw < 1) return SALAD_ERR_INVALID_ARG;
+  if ((long long)T * H * W >= (1ll << 31)) return SALAD_ERR_INVALID_ARG;
+  if (T % bt != 0) return SALAD_ERR_UNSUPPORTED;
+  *nb = (T / bt) * ((H + bh - 1) / bh) * ((W + bw - 1) / bw);
+  return SALAD_OK;
+}
+
+int salad_build_tile_mask(int T, int H, int W, int bt, int bh, int bw, int num_heads, const int32_t* windows,
+                          int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int64_t* nnz_out,
+                          salad_stream_t stream) {
+  return build_mask_impl(T, H, W, 0, bt, bh, bw, num_heads, windows, row_ptr, col_idx, col_capacity, nnz_out,
+                         stream);
+}
+
+}  // extern "C"
+
+namespace {
+int build_mask_impl(int T, int H, int W, int block, int bt, int bh, int bw, int num_heads, const int32_t* windows,
+                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int64_t* nnz_out,
+                    salad_stream_t stream) {
   int nb = 0;
-  int st = salad_mask_num_blocks(T, H, W, block, &nb);
+  int st = bt > 0 ? salad_tile_num_blocks(T, H, W, bt, bh, bw, &nb) : salad_mask_num_blocks(T, H, W, block, &nb);
   if (st != SALAD_OK) return st;
   if (!windows || !row_ptr || num_heads < 1 || num_heads > kMaxHeads || col_capacity < 0)
     return SALAD_ERR_INVALID_ARG;
@@ -137,7 +179,10 @@ int salad_build_block_mask(int T, int H, int W, int block, int num_heads, const 
       if (windows[3 * h + a] < 0) return SALAD_ERR_INVALID_ARG;
       win.w[3 * h + a] = windows[3 * h + a];
     }
-  MaskGrid g{T, H, W, block, nb, num_heads, (long long)T * H * W};
+  MaskGrid g{T, H, W, bt > 0 ? bt * bh * bw : block, nb, num_heads, (long long)T * H * W};
+  g.bt = bt;
+  g.bh = bh;
+  g.bw = bw;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (launch_mask_count(g, win, row_ptr, s) != cudaSuccess) return SALAD_ERR_CUDA;
   if (launch_mask_scan(row_ptr, num_heads * nb, s) != cudaSuccess) return SALAD_ERR_CUDA;
@@ -151,6 +196,9 @@ int salad_build_block_mask(int T, int H, int W, int block, int num_heads, const 
   if (total > 0 && launch_mask_fill(g, win, row_ptr, col_idx, s) != cudaSuccess) return SALAD_ERR_CUDA;
   return SALAD_OK;
 }
+}  // namespace
+
+extern "C" {
 
 size_t salad_workspace_bytes(int B, int N, int num_heads, int d) {
   if (B < 1 || N < 1 || num_heads < 1 || (d != 64 && d != 128)) return 0;
@@ -164,7 +212,7 @@ namespace {
 int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d, int block,
                       const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj, const float* gate,
                       float softmax_scale, float eps, void* out, void* workspace, size_t workspace_bytes,
-                      salad_stream_t stream, int mask_per_bh) {
+                      salad_stream_t stream, int mask_per_bh, const TileGeom* tiles = nullptr) {
   if (!q || !row_ptr || !col_idx || !w_proj || !gate || !out) return SALAD_ERR_INVALID_ARG;
   int st = check_common(k, v, B, N, num_heads, d, workspace, workspace_bytes);
   if (st != SALAD_OK) return st;
@@ -177,7 +225,7 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
   if (overlaps(out, tensor_bytes, q, tensor_bytes) || overlaps(out, tensor_bytes, k, tensor_bytes) ||
       overlaps(out, tensor_bytes, v, tensor_bytes))
     return SALAD_ERR_INVALID_ARG;
-  const long long qtiles = (N + 127) / 128;
+  const long long qtiles = tiles ? (long long)(tiles->T / tiles->bt) * tiles->nh * tiles->nw : (N + 127) / 128;
   if (qtiles * B * num_heads >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
 
   const WorkspaceLayout L = workspace_layout(B, N, num_heads, d);
@@ -193,10 +241,13 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
   const uint64_t t_dims[3] = {(uint64_t)2 * d, (uint64_t)d, (uint64_t)BH};
   const uint64_t t_strides[2] = {(uint64_t)2 * d * 2, (uint64_t)d * 2 * d * 2};
   const uint32_t t_box[3] = {64, (uint32_t)d, 1};
-  if (!make_bnhd_map(&tq, q, B, N, num_heads, d, 128) || !make_bnhd_map(&tk, k, B, N, num_heads, d, block) ||
-      !make_bnhd_map(&tv, v, B, N, num_heads, d, block) || !make_bnhd_map(&to, out, B, N, num_heads, d, 128) ||
-      !make_map(&tt, ws + L.off_t, 3, t_dims, t_strides, t_box))
-    return SALAD_ERR_CUDA;
+  const bool maps_ok =
+      tiles ? make_tile_map(&tq, q, B, *tiles, num_heads, d) && make_tile_map(&tk, k, B, *tiles, num_heads, d) &&
+                  make_tile_map(&tv, v, B, *tiles, num_heads, d) && make_tile_map(&to, out, B, *tiles, num_heads, d)
+            : make_bnhd_map(&tq, q, B, N, num_heads, d, 128) && make_bnhd_map(&tk, k, B, N, num_heads, d, block) &&
+                  make_bnhd_map(&tv, v, B, N, num_heads, d, block) &&
+                  make_bnhd_map(&to, out, B, N, num_heads, d, 128);
+  if (!maps_ok || !make_map(&tt, ws + L.off_t, 3, t_dims, t_strides, t_box)) return SALAD_ERR_CUDA;
 
   AttnArgs aa{};
   aa.tm_q = &tq;
@@ -211,6 +262,7 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
   aa.work_ctr = reinterpret_cast<uint32_t*>(ws + L.off_status) + 1;
   aa.max_ctas = g_max_ctas.load();
   aa.mask_per_bh = mask_per_bh;
+  aa.tiles = tiles ? *tiles : TileGeom{};
   aa.B = B;
   aa.N = N;
   aa.heads = num_heads;
@@ -244,6 +296,19 @@ int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, in
                           size_t workspace_bytes, salad_stream_t stream) {
   return attn_forward_impl(q, k, v, B, N, num_heads, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
                            out, workspace, workspace_bytes, stream, 1);
+}
+
+int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B, int T, int H, int W, int bt,
+                             int bh, int bw, int num_heads, int d, const int32_t* row_ptr, const int32_t* col_idx,
+                             const void* w_proj, const float* gate, float softmax_scale, float eps, void* out,
+                             void* workspace, size_t workspace_bytes, salad_stream_t stream) {
+  int nb = 0;
+  const int st = salad_tile_num_blocks(T, H, W, bt, bh, bw, &nb);
+  if (st != SALAD_OK) return st;
+  if (bt * bh * bw != 128) return SALAD_ERR_UNSUPPORTED;
+  TileGeom g{T, H, W, bt, bh, bw, (H + bh - 1) / bh, (W + bw - 1) / bw};
+  return attn_forward_impl(q, k, v, B, T * H * W, num_heads, d, 128, row_ptr, col_idx, w_proj, gate, softmax_scale,
+                           eps, out, workspace, workspace_bytes, stream, 0, &g);
 }
 
 size_t salad_topk_workspace_bytes(int B, int N, int num_heads, int d, int block) {

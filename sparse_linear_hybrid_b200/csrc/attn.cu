@@ -179,8 +179,8 @@ __device__ __forceinline__ KeyIter make_iter(const int32_t* row_ptr, const int32
   return it;
 }
 
-template <int BLK>
-__device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, const int32_t* row_ptr,
+template <int BLK, bool TILES>
+__device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, int nb, const int32_t* row_ptr,
                                           const int32_t* col_idx, const float* gate, int mask_per_bh) {
   Item im;
   im.w = w;
@@ -190,7 +190,6 @@ __device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, c
   im.h = im.bh % heads;
   im.g = gate[im.bh];
   im.lin = im.g != 0.0f;
-  const int nb = (N + BLK - 1) / BLK;
   // the mask's rows are per head, or per (b, h) for a data-dependent mask
   KeyIter it = make_iter<BLK>(row_ptr, col_idx, mask_per_bh ? im.bh : im.h, nb, im.qtile);
   im.ra = (int)(it.a - col_idx);
@@ -209,7 +208,9 @@ __device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, c
     }
     im.n = n;
   }
-  im.vlast = last >= 0 ? min(BLK, N - last * BLK) : BLK;
+  // (a tile block is never cut short along t; its columns outside the grid are
+  // masked by position instead)
+  im.vlast = (last >= 0 && !TILES) ? min(BLK, N - last * BLK) : BLK;
   return im;
 }
 
@@ -229,13 +230,39 @@ __device__ __forceinline__ void record_timeout(AttnShared* sh, uint32_t* status)
   atomicOr(status, kStatusTimeout);
 }
 
+// TMA copies of one block of rows.  Raster blocks: rows [row0, row0 + rows)
+// of the (Hh*d, N, B) view.  Tile blocks: box I of the (Hh*d, W, H, B*T) view,
+// whose rows in shared memory follow the slot order (tt*bh + yy)*bw + xx; the
+// box's points outside the grid read as zeros and are not written back.
+template <bool TILES>
+__device__ __forceinline__ void load_block(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int row0,
+                                           int I, int b, const TileGeom& g) {
+  if constexpr (TILES) {
+    const int yt = I / g.nw;
+    tma_load_4d(dst, map, bar, c0, (I - yt * g.nw) * g.bw, (yt % g.nh) * g.bh, b * g.T + (yt / g.nh) * g.bt);
+  } else {
+    tma_load_3d(dst, map, bar, c0, row0, b);
+  }
+}
+
+template <bool TILES>
+__device__ __forceinline__ void store_block(const CUtensorMap* map, const void* src, int c0, int row0, int I, int b,
+                                            const TileGeom& g) {
+  if constexpr (TILES) {
+    const int yt = I / g.nw;
+    tma_store_4d(map, src, c0, (I - yt * g.nw) * g.bw, (yt % g.nh) * g.bh, b * g.T + (yt / g.nh) * g.bt);
+  } else {
+    tma_store_3d(map, src, c0, row0, b);
+  }
+}
+
 __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
   uint32_t r;
   asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0u));
   return r;
 }
 
-template <int D, int BLK>
+template <int D, int BLK, bool TILES>
 __global__ void __launch_bounds__(kThreads, 1)
     salad_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
@@ -243,8 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const int32_t* __restrict__ col_idx, const float* __restrict__ gate,
                       const float* __restrict__ zvec, int heads, int N, int qtiles, int num_items,
                       uint32_t* work_ctr, float scale_log2, float eps, uint32_t* status, uint64_t limit_ns,
-                      int mask_per_bh) {
+                      int mask_per_bh, const TileGeom tg) {
   using C = AttnCfg<D, BLK>;
+  static_assert(!TILES || BLK == 128, "a tile block fills one 128-row query tile");
+  const int nblocks = TILES ? qtiles : (N + BLK - 1) / BLK;  // key blocks per mask row
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -317,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int w = (int)atomicAdd(work_ctr, 1u);
         Item im;
         if (w < num_items) {
-          im = make_item<BLK>(w, qtiles, heads, N, row_ptr, col_idx, gate, mask_per_bh);
+          im = make_item<BLK, TILES>(w, qtiles, heads, N, nblocks, row_ptr, col_idx, gate, mask_per_bh);
         } else {
           im.w = -1;
         }
@@ -329,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sh->q_full[slot], C::Q_BYTES);
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
-          tma_load_3d(smem + C::OFF_Q0 + slot * C::Q_BYTES + ch * 16384, &tm_q, &sh->q_full[slot],
-                      im.h * D + ch * 64, im.qtile * 128, im.b);
+          load_block<TILES>(smem + C::OFF_Q0 + slot * C::Q_BYTES + ch * 16384, &tm_q, &sh->q_full[slot],
+                            im.h * D + ch * 64, im.qtile * 128, im.qtile, im.b, tg);
         KeyIter it = item_iter(im, col_idx);
         int col, bits;
         while (it.next(col, bits)) {
@@ -338,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!kt) { ok = false; break; }
 #pragma unroll
           for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_3d(kt + ch * C::KV_BOX, &tm_k, &sh->k_full[kj & 1], im.h * D + ch * 64, col * BLK, im.b);
+            load_block<TILES>(kt + ch * C::KV_BOX, &tm_k, &sh->k_full[kj & 1], im.h * D + ch * 64, col * BLK, col,
+                              im.b, tg);
           ++kj;
         }
         if (ok && C::T_IN_RINGS && im.lin) {
@@ -422,7 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* vt = smem + C::OFF_V0 + s * C::KV_BYTES;
 #pragma unroll
           for (int ch = 0; ch < C::DCH; ++ch)
-            tma_load_3d(vt + ch * C::KV_BOX, &tm_v, &sh->v_full[s], im.h * D + ch * 64, col * BLK, im.b);
+            load_block<TILES>(vt + ch * C::KV_BOX, &tm_v, &sh->v_full[s], im.h * D + ch * 64, col * BLK, col, im.b,
+                              tg);
           ++vj;
         }
         if (!ok) break;
@@ -476,8 +507,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&sh->staged[slot], ph, limit_ns)) { ok = false; break; }
 #pragma unroll
         for (int ch = 0; ch < C::DCH; ++ch)
-          tma_store_3d(&tm_out, smem + C::OFF_Q0 + slot * C::Q_BYTES + ch * 16384, im.h * D + ch * 64,
-                       im.qtile * 128, im.b);
+          store_block<TILES>(&tm_out, smem + C::OFF_Q0 + slot * C::Q_BYTES + ch * 16384, im.h * D + ch * 64,
+                             im.qtile * 128, im.qtile, im.b, tg);
         bulk_commit_group();
         bulk_wait_group_read0();
         mbar_arrive(&sh->q_free[slot]);
@@ -658,12 +689,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_addr = sbase + C::OFF_Q0 + slot * C::Q_BYTES;
       float m_ref = -INFINITY;  // running reference max (raw score units), same in both halves
       float l = 0.f;            // this half's share of the row sum
-      KeyIter it = item_iter(im, col_idx);  // read only when BLK == 64 (which rows use a tile)
+      // read only when BLK == 64 (which rows use a tile) or for tile blocks (where the box sits)
+      KeyIter it = item_iter(im, col_idx);
       int j = 0;
       for (; j < im.n; ++j) {
-        int bits = 1, vtile;
-        if (BLK == 64) {
-          int col;
+        int bits = 1, vtile, col = 0;
+        if (BLK == 64 || TILES) {
           it.next(col, bits);
           vtile = min(BLK, N - col * BLK);
         } else {
@@ -684,9 +715,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sh->s_free[s]);
 
         const bool use = ((bits >> half) & 1) != 0;           // warp-uniform
-        const int valid = vtile - hf * HC;  // real keys among this thread's columns
+        const int valid = vtile - hf * HC;  // real keys among this thread's columns (raster blocks)
+        // tile blocks: the part of the box inside the grid (a box at the bottom or
+        // right edge sticks out; its slots there hold no key)
+        int wr = 0, hr = 0;
+        bool full = valid >= HC;
+        if constexpr (TILES) {
+          const int yt = col / tg.nw;
+          wr = tg.W - (col - yt * tg.nw) * tg.bw;
+          hr = tg.H - (yt % tg.nh) * tg.bh;
+          full = wr >= tg.bw && hr >= tg.bh;
+        }
         float mt;
-        if (valid >= HC) {
+        if (full) {
           float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
           for (int i = 0; i < HC; i += 8) {
@@ -697,10 +738,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         } else {
-          // partial last block: keys past N never count (valid may be <= 0 here)
+          if constexpr (TILES) {
+            // slot hf * HC + i sits at (yy, xx) of its frame of the box
+            int xx = (hf * HC) % tg.bw, yy = ((hf * HC) / tg.bw) % tg.bh;
 #pragma unroll
-          for (int i = 0; i < HC; ++i)
-            if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+            for (int i = 0; i < HC; ++i) {
+              if (xx >= wr || yy >= hr) sr[i] = __float_as_uint(-INFINITY);
+              if (++xx == tg.bw) {
+                xx = 0;
+                if (++yy == tg.bh) yy = 0;
+              }
+            }
+          } else {
+            // partial last block: keys past N never count (valid may be <= 0 here)
+#pragma unroll
+            for (int i = 0; i < HC; ++i)
+              if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
+          }
           float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
           for (int i = 0; i < HC; i += 4) {
@@ -952,28 +1006,30 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int D, int BLK>
+template <int D, int BLK, bool TILES>
 cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   using C = AttnCfg<D, BLK>;
   cudaError_t e =
-      cudaFuncSetAttribute(salad_attn_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+      cudaFuncSetAttribute(salad_attn_kernel<D, BLK, TILES>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const int qtiles = (a.N + 127) / 128;
+  // a query tile is one raster tile of 128 rows, or one box
+  const int qtiles = TILES ? (a.tiles.T / a.tiles.bt) * a.tiles.nh * a.tiles.nw : (a.N + 127) / 128;
   const long long items = (long long)qtiles * a.B * a.heads;
   int ctas = sm_count();
   if (a.max_ctas > 0 && a.max_ctas < ctas) ctas = a.max_ctas;
   const int grid = (int)(items < ctas ? items : ctas);
-  salad_attn_kernel<D, BLK><<<grid, kThreads, C::SMEM, s>>>(
+  salad_attn_kernel<D, BLK, TILES><<<grid, kThreads, C::SMEM, s>>>(
       *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_t, a.row_ptr, a.col_idx, a.gate, a.z, a.heads, a.N, qtiles,
-      (int)items, a.work_ctr, a.scale_log2, a.eps, a.status, a.wait_limit_ns, a.mask_per_bh);
+      (int)items, a.work_ctr, a.scale_log2, a.eps, a.status, a.wait_limit_ns, a.mask_per_bh, a.tiles);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
-  if (a.d == 64) return a.block == 64 ? launch_attn_t<64, 64>(a, s) : launch_attn_t<64, 128>(a, s);
-  return a.block == 64 ? launch_attn_t<128, 64>(a, s) : launch_attn_t<128, 128>(a, s);
+  if (a.tiles.bt > 0) return a.d == 64 ? launch_attn_t<64, 128, true>(a, s) : launch_attn_t<128, 128, true>(a, s);
+  if (a.d == 64) return a.block == 64 ? launch_attn_t<64, 64, false>(a, s) : launch_attn_t<64, 128, false>(a, s);
+  return a.block == 64 ? launch_attn_t<128, 64, false>(a, s) : launch_attn_t<128, 128, false>(a, s);
 }
 
 }  // namespace salad

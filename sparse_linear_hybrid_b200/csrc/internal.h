@@ -20,6 +20,7 @@ struct WindowTable {
 struct MaskGrid {
   int T, H, W, block, nb, heads;
   long long N;
+  int bt = 0, bh = 0, bw = 0;  // 3-D tile blocks of bt x bh x bw points (bt = 0: raster blocks of `block` tokens)
 };
 
 cudaError_t launch_mask_count(const MaskGrid& g, const WindowTable& win, int32_t* row_ptr, cudaStream_t s);
@@ -55,8 +56,15 @@ struct LinearArgs {
 };
 cudaError_t launch_linear_reduce(const LinearArgs& a, cudaStream_t s);
 
+// 3-D tile blocks: box I = (ti*nh + yi)*nw + xi holds the points
+// [ti*bt, +bt) x [yi*bh, +bh) x [xi*bw, +bw) of the T x H x W grid, slot
+// (tt*bh + yy)*bw + xx.  bt == 0: raster blocks of consecutive tokens.
+struct TileGeom {
+  int T, H, W, bt, bh, bw, nh, nw;
+};
+
 struct AttnArgs {
-  const CUtensorMap* tm_q;    // box (64, 128, 1)
+  const CUtensorMap* tm_q;    // box (64, 128, 1); with tile blocks (Hh*d, W, H, B*T), box (64, bw, bh, bt)
   const CUtensorMap* tm_k;    // box (64, block, 1)
   const CUtensorMap* tm_v;    // box (64, block, 1)
   const CUtensorMap* tm_out;  // box (64, 128, 1)
@@ -68,6 +76,7 @@ struct AttnArgs {
   uint32_t* work_ctr;         // next work item (zeroed by the linear kernel)
   int max_ctas;               // cap on the persistent grid (0: one CTA per SM)
   int mask_per_bh;            // mask rows are (b*Hh + h, I) instead of (h, I)
+  TileGeom tiles;             // tiles.bt > 0: blocks are 3-D boxes (block == 128), maps are 4-D
   int B, N, heads, d, block;
   float scale_log2;  // softmax scale * log2(e)
   float eps;

@@ -11,6 +11,8 @@
 //
 // Three launches: count (one warp per CSR row), an in-place inclusive scan of
 // the counts, fill (one warp per row; ballot compaction keeps columns sorted).
+// The same kernels build the mask over 3-D tile blocks (bt x bh x bw boxes of
+// the grid, numbered in raster order over the boxes).
 #include "internal.h"
 
 namespace salad {
@@ -18,7 +20,25 @@ namespace {
 
 __device__ __forceinline__ long long llmin(long long a, long long b) { return a < b ? a : b; }
 
+// 3-D tile blocks: box I covers [t0, t0+bt) x [y0, min(H, y0+bh)) x
+// [x0, min(W, x0+bw)); two boxes hold a token pair inside the window exactly
+// when, on every axis, the gap between their extents is within the window.
+__device__ __forceinline__ int axis_gap(int a0, int a1, int b0, int b1) {  // inclusive ranges
+  return max(0, max(b0 - a1, a0 - b1));
+}
+
+__device__ bool tile_pair_kept(const MaskGrid& g, int wt, int wh, int ww, int I, int J) {
+  const int nh = (g.H + g.bh - 1) / g.bh, nw = (g.W + g.bw - 1) / g.bw;
+  const int ti = I / (nh * nw), yi = (I / nw) % nh, xi = I % nw;
+  const int tj = J / (nh * nw), yj = (J / nw) % nh, xj = J % nw;
+  const int ty = axis_gap(ti * g.bt, ti * g.bt + g.bt - 1, tj * g.bt, tj * g.bt + g.bt - 1);
+  const int gy = axis_gap(yi * g.bh, min(g.H, yi * g.bh + g.bh) - 1, yj * g.bh, min(g.H, yj * g.bh + g.bh) - 1);
+  const int gx = axis_gap(xi * g.bw, min(g.W, xi * g.bw + g.bw) - 1, xj * g.bw, min(g.W, xj * g.bw + g.bw) - 1);
+  return ty <= wt && gy <= wh && gx <= ww;
+}
+
 __device__ bool block_pair_kept(const MaskGrid& g, int wt, int wh, int ww, int I, int J) {
+  if (g.bt > 0) return tile_pair_kept(g, wt, wh, ww, I, J);
   const long long a0 = (long long)I * g.block, a1 = llmin(g.N, a0 + g.block) - 1;
   const long long c0 = (long long)J * g.block, c1 = llmin(g.N, c0 + g.block) - 1;
   const long long ra0 = a0 / g.W, ra1 = a1 / g.W, rc0 = c0 / g.W, rc1 = c1 / g.W;
