@@ -72,18 +72,30 @@ def mask_per_bh(wl: si.Workload) -> bool:
     return wl.topk > 0
 
 
+def block_sizes(wl: si.Workload) -> np.ndarray:
+    """Real tokens of every block: a raster block (the last one may be short), or
+    a 3-D tile block clipped to the grid."""
+    if wl.tile:
+        bt, bh, bw = wl.tile
+        nh, nw = -(-wl.H // bh), -(-wl.W // bw)
+        I = np.arange(wl.nb)
+        yi, xi = (I // nw) % nh, I % nw
+        return (bt * np.minimum(bh, wl.H - yi * bh) * np.minimum(bw, wl.W - xi * bw)).astype(np.float64)
+    return np.minimum(wl.block, wl.N - np.arange(wl.nb) * wl.block).astype(np.float64)
+
+
 def kept_pairs_flops(row_ptr: np.ndarray, col_idx: np.ndarray, wl: si.Workload) -> float:
     """4 * d * sum over kept (I, J) of |I| * |J| (real tokens) over every (b, h)."""
-    nb, blk, N = wl.nb, wl.block, wl.N
-    sizes = np.minimum(blk, N - np.arange(nb) * blk).astype(np.float64)
+    nb = wl.nb
+    sizes = block_sizes(wl)
     rows = np.repeat(np.arange(len(row_ptr) - 1) % nb, np.diff(row_ptr))
     pairs = float(np.sum(sizes[rows] * sizes[col_idx]))
     return 4.0 * wl.d * pairs * (1 if mask_per_bh(wl) else wl.B)
 
 
 def block_flops(row_ptr, col_idx, wl, pairs):
-    nb, blk, N = wl.nb, wl.block, wl.N
-    sizes = np.minimum(blk, N - np.arange(nb) * blk).astype(np.float64)
+    nb = wl.nb
+    sizes = block_sizes(wl)
     per_bh = mask_per_bh(wl)
     tot = 0.0
     for bh, I in pairs:
@@ -179,7 +191,8 @@ class DriverEvents:
 
 def time_block_mask(wl, windows, row_ptr, col_idx, reps=5):
     """Device time of one mask build (count, scan, fill) into existing buffers,
-    mean of `reps` builds on the current stream, CUDA events."""
+    mean of `reps` builds on the current stream, CUDA events (raster or tile
+    blocks, as the workload has them)."""
     import ctypes
 
     import torch
@@ -190,12 +203,14 @@ def time_block_mask(wl, windows, row_ptr, col_idx, reps=5):
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(reps):
-        st = sl.lib().salad_build_block_mask(wl.T, wl.H, wl.W, wl.block, win.shape[0],
-                                             win.ctypes.data_as(ctypes.c_void_p), ctypes.c_void_p(row_ptr.data_ptr()),
-                                             ctypes.c_void_p(col_idx.data_ptr()), col_idx.numel(), None,
-                                             ctypes.c_void_p(s))
+        bufs = (win.shape[0], win.ctypes.data_as(ctypes.c_void_p), ctypes.c_void_p(row_ptr.data_ptr()),
+                ctypes.c_void_p(col_idx.data_ptr()), col_idx.numel(), None, ctypes.c_void_p(s))
+        if wl.tile:
+            st = sl.lib().salad_build_tile_mask(wl.T, wl.H, wl.W, *wl.tile, *bufs)
+        else:
+            st = sl.lib().salad_build_block_mask(wl.T, wl.H, wl.W, wl.block, *bufs)
         if st != sl.SALAD_OK:
-            raise RuntimeError(f"salad_build_block_mask: {sl.status_string(st)}")
+            raise RuntimeError(f"mask build: {sl.status_string(st)}")
     b.record()
     torch.cuda.synchronize()
     return a.elapsed_time(b) / reps
@@ -294,14 +309,29 @@ def whole_job_tflops(world: int, steps: int, flops_per_step: float, total_ms: fl
 def config_of(wl: si.Workload, flops: float, nnz: int, world: int):
     rows = wl.B * wl.Hh * wl.nb if wl.topk else wl.Hh * wl.nb
     mask = {"topk_keep": wl.topk} if wl.topk else {"window_thw": list(wl.window)}
+    blocks = {"tile_thw": list(wl.tile), "blocks_per_head": wl.nb} if wl.tile else {}
     return {"workload": wl.name, "B": wl.B, "heads": wl.Hh, "d": wl.d,
-            "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.N, "block": wl.block,
+            "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.N, "block": wl.block, **blocks,
             **mask, "block_sparsity": round(1 - nnz / (rows * wl.nb), 5),
             "kept_gflop_per_step": round(flops / 1e9, 3), "parallelism": f"replicas{world}",
             "l2": "flushed between steps (256 MB write outside the timed events)"}
 
 
 # --------------------------------------------------------------------------- oracle legs
+def oracle_geom(wl):
+    import oracle
+    return oracle.tile_geom(wl.T, wl.H, wl.W, wl.tile) if wl.tile else None
+
+
+def oracle_mask(wl, inp):
+    import oracle
+    if wl.topk:
+        return oracle.topk_mask(inp.q, inp.k, wl.block, wl.topk)
+    if wl.tile:
+        return oracle.tile_mask(wl.T, wl.H, wl.W, wl.tile, inp.windows)
+    return oracle.block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)
+
+
 def oracle_sample_rate(wl, inp, row_ptr, col_idx, budget_s, seed=0):
     """The CPU oracle on a bounded sample: S and z of every (b, h) once, then
     seeded query blocks until `budget_s` of forward time.  Returns
@@ -321,7 +351,7 @@ def oracle_sample_rate(wl, inp, row_ptr, col_idx, budget_s, seed=0):
         batch = order[done:done + max(cores, 4)].astype(np.int32)
         t1 = time.perf_counter()
         oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate, batch,
-                              S=S, z=z, mask_per_bh=bool(wl.topk))
+                              S=S, z=z, mask_per_bh=bool(wl.topk), geom=oracle_geom(wl))
         t_fwd += time.perf_counter() - t1
         flops += block_flops(row_ptr, col_idx, wl, batch)
         done += len(batch)
@@ -341,10 +371,8 @@ def run_reference(args, wl):
     inp = si.make_inputs(wl)
     _t = time
     t0 = _t.perf_counter()
-    if wl.topk:  # a dynamic mask is built every step: charged with the linear state
-        row_ptr, col_idx = oracle.topk_mask(inp.q, inp.k, wl.block, wl.topk)
-    else:
-        row_ptr, col_idx = oracle.block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)
+    # a dynamic mask is built every step: charged with the linear state
+    row_ptr, col_idx = oracle_mask(wl, inp)
     t_mask = _t.perf_counter() - t0 if wl.topk else 0.0
     flops_step = kept_pairs_flops(row_ptr, col_idx, wl)
     t0 = _t.perf_counter()
@@ -358,7 +386,7 @@ def run_reference(args, wl):
     per = max(cores, 4)
     t1 = _t.perf_counter()
     oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate,
-                          order[:per].astype(np.int32), S=S, z=z, mask_per_bh=bool(wl.topk))
+                          order[:per].astype(np.int32), S=S, z=z, mask_per_bh=bool(wl.topk), geom=oracle_geom(wl))
     per_block = (_t.perf_counter() - t1) / per
     m = int(max(1, min(len(order), step_budget / max(per_block, 1e-6))))
     times, flops_list = [], []
@@ -370,7 +398,7 @@ def run_reference(args, wl):
         pos += m
         t1 = _t.perf_counter()
         oracle.forward_blocks(inp.q, inp.k, inp.v, wl.block, row_ptr, col_idx, inp.w_proj, inp.gate, batch,
-                              S=S, z=z, mask_per_bh=bool(wl.topk))
+                              S=S, z=z, mask_per_bh=bool(wl.topk), geom=oracle_geom(wl))
         dt = _t.perf_counter() - t1
         fl = block_flops(row_ptr, col_idx, wl, batch)
         if i >= args.warmup:
@@ -420,6 +448,12 @@ def run_e2e(args, q, k, v, w, gate, out, flush, step, flops, world, max_over_ran
             "steps": ke}
 
 
+def build_window_mask(sl, wl, windows, dev):
+    if wl.tile:
+        return sl.build_tile_mask(wl.T, wl.H, wl.W, wl.tile, windows, device=dev)
+    return sl.build_block_mask(wl.T, wl.H, wl.W, wl.block, windows, device=dev)
+
+
 def run_salad(args, wl):
     import torch
 
@@ -448,7 +482,7 @@ def run_salad(args, wl):
         topk.run()
         mask_ms = topk.device_ms()
     else:
-        row_ptr, col_idx = sl.build_block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows, device=dev)
+        row_ptr, col_idx = build_window_mask(sl, wl, inp.windows, dev)
         # the mask build once more into the same buffers, on the device clock (the
         # first call above also sizes col_idx and loads the kernels)
         mask_ms = time_block_mask(wl, inp.windows, row_ptr, col_idx)
@@ -459,11 +493,16 @@ def run_salad(args, wl):
     out = torch.empty_like(q)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
+    def forward(rp, ci, g):
+        if wl.tile:
+            sl.attn_forward_tiles(q, k, v, (wl.T, wl.H, wl.W), wl.tile, rp, ci, w, g, out=out, workspace=ws)
+        else:
+            sl.attn_forward(q, k, v, rp, ci, w, g, wl.block, out=out, workspace=ws, mask_per_bh=topk is not None)
+
     def step():
         if topk is not None:
             topk.run()
-        sl.attn_forward(q, k, v, row_ptr, col_idx, w, gate, wl.block, out=out, workspace=ws,
-                        mask_per_bh=topk is not None)
+        forward(row_ptr, col_idx, gate)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -549,7 +588,7 @@ def run_salad(args, wl):
     dense = None
     if not args.no_dense:
         dwl = wl.with_(window=(wl.T, wl.H, wl.W), topk=0)
-        drp, dci = sl.build_block_mask(dwl.T, dwl.H, dwl.W, dwl.block, dwl.windows(), device=dev)
+        drp, dci = build_window_mask(sl, dwl, dwl.windows(), dev)
         zero_gate = torch.zeros_like(gate)
         dflops = kept_pairs_flops(drp.cpu().numpy(), dci.cpu().numpy(), dwl)
         dev_ev = [(E(), E()) for _ in range(5)]
@@ -557,7 +596,7 @@ def run_salad(args, wl):
             flush.zero_()
             if i > 0:
                 dev_ev[i - 1][0].record()
-            sl.attn_forward(q, k, v, drp, dci, w, zero_gate, wl.block, out=out, workspace=ws)
+            forward(drp, dci, zero_gate)
             if i > 0:
                 dev_ev[i - 1][1].record()
         torch.cuda.synchronize()

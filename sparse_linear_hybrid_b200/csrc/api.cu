@@ -306,7 +306,12 @@ int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B,
   const int st = salad_tile_num_blocks(T, H, W, bt, bh, bw, &nb);
   if (st != SALAD_OK) return st;
   if (bt * bh * bw != 128) return SALAD_ERR_UNSUPPORTED;
-  TileGeom g{T, H, W, bt, bh, bw, (H + bh - 1) / bh, (W + bw - 1) / bw};
+  TileGeom g{T, H, W, bt, bh, bw, (H + bh - 1) / bh, (W + bw - 1) / bw, {}, {}};
+  // the kernel divides box indices (< nb) by nw and row indices (< nb / nw) by
+  // nh with multiply-high divisors, exact while n * divisor < 2^32
+  if ((uint64_t)nb * g.nw >= (1ull << 32) || (uint64_t)nb * g.nh >= (1ull << 32)) return SALAD_ERR_UNSUPPORTED;
+  g.div_nw = make_fastdiv((uint32_t)g.nw);
+  g.div_nh = make_fastdiv((uint32_t)g.nh);
   return attn_forward_impl(q, k, v, B, T * H * W, num_heads, d, 128, row_ptr, col_idx, w_proj, gate, softmax_scale,
                            eps, out, workspace, workspace_bytes, stream, 0, &g);
 }

@@ -89,6 +89,7 @@ struct AttnShared {
   float xsum[2][2][128];     // per exchange parity, per half: partial row sums
   float xden[2][2][128];     // per exchange parity, per half: partial relu(q) . z
   alignas(16) float zs[2][128];  // per item slot: z of the item's (b, h)
+  int k_edge[2];             // tile blocks: per K ring stage, which grid edges its box sticks out of
 };
 
 template <int D, int BLK>
@@ -115,6 +116,13 @@ struct AttnCfg {
   static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(AttnShared) + 1024;
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
   static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
+  // tile blocks: four 128 x 16 bf16 operands in the 32-byte-swizzled K-major
+  // layout (4 KB each) -- a tile of ones and the key-padding bias of a box at
+  // the right edge, the bottom edge and both -- after the barriers
+  static constexpr int MASK_OP_BYTES = 128 * 32;
+  static constexpr int OFF_MASK = (OFF_BAR + (int)sizeof(AttnShared) + 1023) / 1024 * 1024;
+  static constexpr int SMEM_TILES = OFF_MASK + 4 * MASK_OP_BYTES + 1024;
+  static_assert(SMEM_TILES <= 232448, "shared memory budget (tile blocks)");
   static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P = 384, TM_Q = 448;
   static constexpr uint32_t P_COLS = BLK / 2;       // the P buffer: BLK bf16 per row
   static constexpr uint32_t Q_COLS = D / 2;         // Q (then relu(Q)) in tensor memory: D bf16 per row
@@ -238,8 +246,8 @@ template <bool TILES>
 __device__ __forceinline__ void load_block(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int row0,
                                            int I, int b, const TileGeom& g) {
   if constexpr (TILES) {
-    const int yt = I / g.nw;
-    tma_load_4d(dst, map, bar, c0, (I - yt * g.nw) * g.bw, (yt % g.nh) * g.bh, b * g.T + (yt / g.nh) * g.bt);
+    const int yt = (int)fastdiv((uint32_t)I, g.div_nw), t = (int)fastdiv((uint32_t)yt, g.div_nh);
+    tma_load_4d(dst, map, bar, c0, (I - yt * g.nw) * g.bw, (yt - t * g.nh) * g.bh, b * g.T + t * g.bt);
   } else {
     tma_load_3d(dst, map, bar, c0, row0, b);
   }
@@ -249,8 +257,8 @@ template <bool TILES>
 __device__ __forceinline__ void store_block(const CUtensorMap* map, const void* src, int c0, int row0, int I, int b,
                                             const TileGeom& g) {
   if constexpr (TILES) {
-    const int yt = I / g.nw;
-    tma_store_4d(map, src, c0, (I - yt * g.nw) * g.bw, (yt % g.nh) * g.bh, b * g.T + (yt / g.nh) * g.bt);
+    const int yt = (int)fastdiv((uint32_t)I, g.div_nw), t = (int)fastdiv((uint32_t)yt, g.div_nh);
+    tma_store_4d(map, src, c0, (I - yt * g.nw) * g.bw, (yt - t * g.nh) * g.bh, b * g.T + t * g.bt);
   } else {
     tma_store_3d(map, src, c0, row0, b);
   }
@@ -311,6 +319,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sh->tmem_base, 512);
     tmem_relinquish();
   }
+  if constexpr (TILES) {
+    // Keys of a box outside the grid are masked by the tensor cores: S of a box
+    // at an edge gets one more K = 16 product, ones (128 x 16) times the box's
+    // bias (128 x 16: row n all 0 when slot n holds a key, all -inf when it lies
+    // past the edge), which adds -inf to exactly the padded columns and 0 to the
+    // rest.  Rows are uniform, so the swizzle does not move any value.
+    uint32_t* mo = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
+    const int wr = tg.W - (tg.nw - 1) * tg.bw, hr = tg.H - (tg.nh - 1) * tg.bh;  // keys of an edge box
+    for (int x = threadIdx.x; x < 4 * C::MASK_OP_BYTES / 4; x += kThreads) {
+      const int op = x / (C::MASK_OP_BYTES / 4), row = (x % (C::MASK_OP_BYTES / 4)) / 8;
+      uint32_t val = 0x3F803F80u;  // bf16 pair (1, 1)
+      if (op > 0) {
+        const bool past = ((op & 1) && row % tg.bw >= wr) || ((op & 2) && (row / tg.bw) % tg.bh >= hr);
+        val = past ? 0xFF80FF80u : 0u;  // (-inf, -inf) or (0, 0)
+      }
+      mo[x] = val;
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -325,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int seq = 0, kj = 0;
       // next K ring entry: wait for its stage, expect its bytes
-      auto k_stage = [&]() -> uint8_t* {
+      auto k_stage = [&](int edge) -> uint8_t* {
         const int s = kj & 1;
         // the stage is free once the product that read entry kj - 2 is done.  With
         // T in the rings every K entry feeds exactly one S slot use (S or U) in the
@@ -335,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  ? (kj < 2 || mbar_wait(&sh->s_full[s], (uint32_t)(((kj - 2) >> 1) & 1), limit_ns))
                                  : mbar_wait(&sh->k_empty[s], ((kj >> 1) & 1) ^ 1, limit_ns);
         if (sh->abort_flag || !free_ok) return nullptr;
+        if constexpr (TILES) sh->k_edge[s] = edge;  // read by the MMA thread after k_full
         mbar_arrive_expect_tx(&sh->k_full[s], C::KV_BYTES);
         return smem + C::OFF_K0 + s * C::KV_BYTES;
       };
@@ -363,7 +391,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         KeyIter it = item_iter(im, col_idx);
         int col, bits;
         while (it.next(col, bits)) {
-          uint8_t* kt = k_stage();
+          int edge = 0;
+          if constexpr (TILES) {
+            // bit 0: the box reaches past W; bit 1: past H
+            const int yt = (int)fastdiv((uint32_t)col, tg.div_nw);
+            const int xi = col - yt * tg.nw, yi = yt - (int)fastdiv((uint32_t)yt, tg.div_nh) * tg.nh;
+            edge = ((xi + 1) * tg.bw > tg.W ? 1 : 0) | ((yi + 1) * tg.bh > tg.H ? 2 : 0);
+          }
+          uint8_t* kt = k_stage(edge);
           if (!kt) { ok = false; break; }
 #pragma unroll
           for (int ch = 0; ch < C::DCH; ++ch)
@@ -373,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok && C::T_IN_RINGS && im.lin) {
           // T_hi: one more K ring entry after the item's key tiles, released by U
-          uint8_t* dst = k_stage();
+          uint8_t* dst = k_stage(0);
           if (!dst) {
             ok = false;
           } else {
@@ -567,6 +602,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sw128_desc(kt + (kk / 4) * C::KV_BOX + (kk % 4) * 32, 16, 1024);
           mma_bf16_ts(d_s, tmem + C::TM_Q + kk * 8, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
         }
+        if constexpr (TILES) {
+          const int edge = sh->k_edge[ks];
+          if (edge != 0)
+            mma_bf16_ss(d_s, sw32_desc(sbase + C::OFF_MASK),
+                        sw32_desc(sbase + C::OFF_MASK + edge * C::MASK_OP_BYTES), C::IDESC_S, 1u);
+        }
         mma_commit(&sh->s_full[s]);  // with T in the rings this also frees the K stage
         if (!C::T_IN_RINGS) mma_commit(&sh->k_empty[ks]);
         q_last = sj;
@@ -689,12 +730,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_addr = sbase + C::OFF_Q0 + slot * C::Q_BYTES;
       float m_ref = -INFINITY;  // running reference max (raw score units), same in both halves
       float l = 0.f;            // this half's share of the row sum
-      // read only when BLK == 64 (which rows use a tile) or for tile blocks (where the box sits)
-      KeyIter it = item_iter(im, col_idx);
+      KeyIter it = item_iter(im, col_idx);  // read only when BLK == 64 (which rows use a tile)
       int j = 0;
       for (; j < im.n; ++j) {
-        int bits = 1, vtile, col = 0;
-        if (BLK == 64 || TILES) {
+        int bits = 1, vtile;
+        if (BLK == 64) {
+          int col;
           it.next(col, bits);
           vtile = min(BLK, N - col * BLK);
         } else {
@@ -716,18 +757,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         const bool use = ((bits >> half) & 1) != 0;           // warp-uniform
         const int valid = vtile - hf * HC;  // real keys among this thread's columns (raster blocks)
-        // tile blocks: the part of the box inside the grid (a box at the bottom or
-        // right edge sticks out; its slots there hold no key)
-        int wr = 0, hr = 0;
-        bool full = valid >= HC;
-        if constexpr (TILES) {
-          const int yt = col / tg.nw;
-          wr = tg.W - (col - yt * tg.nw) * tg.bw;
-          hr = tg.H - (yt % tg.nh) * tg.bh;
-          full = wr >= tg.bw && hr >= tg.bh;
-        }
+        // (tile blocks: the tensor cores already put -inf on the slots past the grid)
         float mt;
-        if (full) {
+        if (TILES || valid >= HC) {
           float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
           for (int i = 0; i < HC; i += 8) {
@@ -738,23 +770,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         } else {
-          if constexpr (TILES) {
-            // slot hf * HC + i sits at (yy, xx) of its frame of the box
-            int xx = (hf * HC) % tg.bw, yy = ((hf * HC) / tg.bw) % tg.bh;
+          // partial last block: keys past N never count (valid may be <= 0 here)
 #pragma unroll
-            for (int i = 0; i < HC; ++i) {
-              if (xx >= wr || yy >= hr) sr[i] = __float_as_uint(-INFINITY);
-              if (++xx == tg.bw) {
-                xx = 0;
-                if (++yy == tg.bh) yy = 0;
-              }
-            }
-          } else {
-            // partial last block: keys past N never count (valid may be <= 0 here)
-#pragma unroll
-            for (int i = 0; i < HC; ++i)
-              if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
-          }
+          for (int i = 0; i < HC; ++i)
+            if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
           float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
           for (int i = 0; i < HC; i += 4) {
@@ -1009,8 +1028,9 @@ int sm_count() {
 template <int D, int BLK, bool TILES>
 cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   using C = AttnCfg<D, BLK>;
+  const int smem = TILES ? C::SMEM_TILES : C::SMEM;
   cudaError_t e =
-      cudaFuncSetAttribute(salad_attn_kernel<D, BLK, TILES>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+      cudaFuncSetAttribute(salad_attn_kernel<D, BLK, TILES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // a query tile is one raster tile of 128 rows, or one box
   const int qtiles = TILES ? (a.tiles.T / a.tiles.bt) * a.tiles.nh * a.tiles.nw : (a.N + 127) / 128;
@@ -1018,7 +1038,7 @@ cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   int ctas = sm_count();
   if (a.max_ctas > 0 && a.max_ctas < ctas) ctas = a.max_ctas;
   const int grid = (int)(items < ctas ? items : ctas);
-  salad_attn_kernel<D, BLK, TILES><<<grid, kThreads, C::SMEM, s>>>(
+  salad_attn_kernel<D, BLK, TILES><<<grid, kThreads, smem, s>>>(
       *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_t, a.row_ptr, a.col_idx, a.gate, a.z, a.heads, a.N, qtiles,
       (int)items, a.work_ctr, a.scale_log2, a.eps, a.status, a.wait_limit_ns, a.mask_per_bh, a.tiles);
   return cudaGetLastError();

@@ -59,8 +59,23 @@ cudaError_t launch_linear_reduce(const LinearArgs& a, cudaStream_t s);
 // 3-D tile blocks: box I = (ti*nh + yi)*nw + xi holds the points
 // [ti*bt, +bt) x [yi*bh, +bh) x [xi*bw, +bw) of the T x H x W grid, slot
 // (tt*bh + yy)*bw + xx.  bt == 0: raster blocks of consecutive tokens.
+// Division by a fixed d >= 1 without the divide sequence: for n * d < 2^32,
+// n / d == umulhi(n, m) with m = floor(2^32 / d) + 1 (d >= 2; the error term
+// n * (m - 2^32 / d) / 2^32 stays below 1 / d), and n itself when d == 1
+// (m = 0, one = all ones).
+struct FastDiv {
+  uint32_t m, one;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  return d <= 1 ? FastDiv{0u, 0xFFFFFFFFu} : FastDiv{(uint32_t)((1ull << 32) / d + 1), 0u};
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, FastDiv f) { return __umulhi(n, f.m) + (n & f.one); }
+#endif
+
 struct TileGeom {
   int T, H, W, bt, bh, bw, nh, nw;
+  FastDiv div_nw, div_nh;  // box index -> (t*nh + y, x) -> (t, y)
 };
 
 struct AttnArgs {

@@ -37,9 +37,9 @@ def test_tile_mask_random_sweep():
         np.testing.assert_array_equal(ci, oci)
 
 
-@pytest.mark.parametrize("tile", [(1, 16, 8), (1, 8, 16), (3, 8, 4)])
+@pytest.mark.parametrize("tile", [(1, 32, 4), (1, 16, 8), (3, 8, 4)])
 def test_tile_mask_full_size(tile):
-    wl = si.WORKLOADS["wan1.3b-32760tok-tiles1x16x8"]
+    wl = si.WORKLOADS["wan1.3b-32760tok-tiles1x32x4"]
     rp, ci = gpu_tile_mask(wl.T, wl.H, wl.W, tile, wl.windows())
     orp, oci = oracle.tile_mask(wl.T, wl.H, wl.W, tile, wl.windows())
     np.testing.assert_array_equal(rp, orp)
@@ -58,6 +58,7 @@ def test_tile_mask_rejects_a_tile_that_does_not_divide_t():
     (1, 8, 8, 8, 2, 64, (8, 4, 4), (2, 3, 3)),        # deep boxes, no padding
     (1, 2, 6, 70, 2, 128, (1, 2, 64), (0, 1, 30)),    # wide boxes
     (1, 1, 1, 5, 1, 64, (1, 1, 128), (0, 0, 1)),      # one box, five real keys
+    (1, 2, 30, 14, 2, 128, (1, 32, 4), (1, 6, 5)),    # every box past the bottom edge, some past the right
 ])
 def test_tile_forward_matches_oracle(B, T, H, W, Hh, d, tile, window):
     wl = si.Workload("tf", B=B, Hh=Hh, d=d, T=T, H=H, W=W, block=128, window=window, seed=57, tile=tile)
@@ -76,7 +77,7 @@ def test_tile_forward_matches_oracle(B, T, H, W, Hh, d, tile, window):
 
 
 def test_tile_forward_full_size_sampled():
-    wl = si.WORKLOADS["wan1.3b-32760tok-tiles1x16x8"]
+    wl = si.WORKLOADS["wan1.3b-32760tok-tiles1x32x4"]
     inp = si.make_inputs(wl)
     t = upload(inp)
     rp, ci = sl.build_tile_mask(wl.T, wl.H, wl.W, wl.tile, inp.windows)
