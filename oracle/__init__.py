@@ -48,6 +48,8 @@ def _load():
         lib.oracle_tile_mask.argtypes = [P, ctypes.c_int, P, P, P, ctypes.c_int64]
         lib.oracle_topk_mask.restype = ctypes.c_int
         lib.oracle_topk_mask.argtypes = [P, P] + [ctypes.c_int] * 6 + [P, P]
+        lib.oracle_gate.restype = None
+        lib.oracle_gate.argtypes = [P] + [ctypes.c_int] * 4 + [P, ctypes.c_int, P, P, P, ctypes.c_double, P, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -218,3 +220,20 @@ def forward_tiles(q, k, v, T, H, W, tile, row_ptr, col_idx, w_proj, gate, tau=No
         for h in range(Hh):
             out[b, slots[real], h] = res[b, h][real]
     return out
+
+
+def gate(q, t_emb, w_t, w_x, beta, threshold):
+    """Dynamic gate (see oracle_gate): returns (s, gate), fp64 [B][Hh]; gate = 0
+    where s < threshold (the linear branch dropped)."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    B, N, Hh, d = q.shape
+    t_emb = np.ascontiguousarray(t_emb, dtype=np.float64).reshape(B, -1)
+    E = t_emb.shape[1]
+    w_t = np.ascontiguousarray(w_t, dtype=np.float64).reshape(Hh, E)
+    w_x = np.ascontiguousarray(w_x, dtype=np.float64).reshape(Hh, d)
+    beta = np.ascontiguousarray(beta, dtype=np.float64).reshape(Hh)
+    s = np.zeros((B, Hh))
+    g = np.zeros((B, Hh))
+    _load().oracle_gate(_ptr(q), B, N, Hh, d, _ptr(t_emb), E, _ptr(w_t), _ptr(w_x), _ptr(beta),
+                        float(threshold), _ptr(s), _ptr(g))
+    return s, g

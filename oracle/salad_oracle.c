@@ -419,6 +419,38 @@ int oracle_topk_mask(const uint16_t *q, const uint16_t *k, int B, int N, int Hh,
     return kk;
 }
 
+/*
+ * The dynamic gate and branch dropping (SALAD technical summary, section 2.2
+ * ITADS: a lightweight module maps the denoising timestep and the hidden state
+ * to a global factor squashed by a sigmoid into (0, 1); section 2.3: at
+ * inference the linear branch is dropped where that factor is very low).  The
+ * pages give neither the module nor the threshold; the reading taken: per
+ * (b, h), with the layer's queries as the hidden state,
+ *   pooled[f] = (1/N) sum_n q[b][n][h][f]
+ *   s         = sigmoid(sum_e w_t[h][e] t_emb[b][e] + sum_f w_x[h][f] pooled[f] + beta[h])
+ *   gate      = 0 where s < threshold (the branch is dropped), s otherwise.
+ * In fp64; writes s (before dropping) and the gate, both [B][Hh].
+ */
+void oracle_gate(const uint16_t *q, int B, int N, int Hh, int d, const double *t_emb, int E,
+                 const double *w_t, const double *w_x, const double *beta, double threshold,
+                 double *s_out, double *gate_out) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < Hh; ++h) {
+            double logit = beta[h];
+            for (int e = 0; e < E; ++e) logit += w_t[(size_t)h * E + e] * t_emb[(size_t)b * E + e];
+            for (int f = 0; f < d; ++f) {
+                double sum = 0.0;
+                for (int n = 0; n < N; ++n) sum += bf16_to_double(q[(((size_t)b * N + n) * Hh + h) * d + f]);
+                logit += w_x[(size_t)h * d + f] * (sum / N);
+            }
+            const double sv = 1.0 / (1.0 + exp(-logit));
+            s_out[b * Hh + h] = sv;
+            gate_out[b * Hh + h] = sv < threshold ? 0.0 : sv;
+        }
+    }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);
