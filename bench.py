@@ -19,6 +19,7 @@ of the same workload; rank 0 alone runs it.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -324,6 +325,14 @@ def oracle_geom(wl):
     return oracle.tile_geom(wl.T, wl.H, wl.W, wl.tile) if wl.tile else None
 
 
+def oracle_itads_gate(wl, inp):
+    """The oracle's dynamic gate (with dropping) for the workload, fp32 [B][Hh]."""
+    import oracle
+    gi = si.make_gate_inputs(wl)
+    _, g = oracle.gate(inp.q, gi.t_emb, gi.w_t, gi.w_x, gi.beta, gi.threshold)
+    return g.astype(np.float32)
+
+
 def oracle_mask(wl, inp):
     import oracle
     if wl.topk:
@@ -341,6 +350,9 @@ def oracle_sample_rate(wl, inp, row_ptr, col_idx, budget_s, seed=0):
     t0 = time.perf_counter()
     if wl.topk:
         oracle.topk_mask(inp.q, inp.k, wl.block, wl.topk)  # a dynamic mask is built every step
+    if wl.itads:
+        gate_in = oracle_itads_gate(wl, inp)               # a dynamic gate is produced every step
+        inp = dataclasses.replace(inp, gate=gate_in)
     S, z = oracle.linear_state(inp.k, inp.v)
     t_lin = time.perf_counter() - t0
     total = kept_pairs_flops(row_ptr, col_idx, wl)
@@ -358,7 +370,8 @@ def oracle_sample_rate(wl, inp, row_ptr, col_idx, budget_s, seed=0):
         done += len(batch)
     frac = flops / total
     charged = t_fwd + t_lin * frac
-    what = "the Top-K mask and the linear-branch state" if wl.topk else "the linear-branch state"
+    what = ("the Top-K mask and " if wl.topk else "the dynamic gate and " if wl.itads else "") + \
+        "the linear-branch state"
     desc = (f"{done} of {len(order)} query blocks ({100 * frac:.2f}% of kept FLOPs) + {what} "
             f"of all heads ({t_lin:.2f}s, charged pro rata)")
     return flops / charged / 1e12, cores, desc, charged, done
@@ -372,9 +385,11 @@ def run_reference(args, wl):
     inp = si.make_inputs(wl)
     _t = time
     t0 = _t.perf_counter()
-    # a dynamic mask is built every step: charged with the linear state
+    # a dynamic mask or gate is built every step: charged with the linear state
     row_ptr, col_idx = oracle_mask(wl, inp)
-    t_mask = _t.perf_counter() - t0 if wl.topk else 0.0
+    if wl.itads:
+        inp = dataclasses.replace(inp, gate=oracle_itads_gate(wl, inp))
+    t_mask = _t.perf_counter() - t0 if (wl.topk or wl.itads) else 0.0
     flops_step = kept_pairs_flops(row_ptr, col_idx, wl)
     t0 = _t.perf_counter()
     S, z = oracle.linear_state(inp.k, inp.v)
@@ -406,7 +421,8 @@ def run_reference(args, wl):
             times.append(dt + t_lin * fl / flops_step)
             flops_list.append(fl)
     value = sum(flops_list) / sum(times) / 1e12
-    what = "the Top-K mask and the linear-branch state" if wl.topk else "the linear-branch state"
+    what = ("the Top-K mask and " if wl.topk else "the dynamic gate and " if wl.itads else "") + \
+        "the linear-branch state"
     desc = (f"{m} query blocks per step (seeded, cycling over all {len(order)}) with {what} of "
             f"all heads ({t_lin:.2f}s) charged pro rata to their kept FLOPs")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
@@ -421,12 +437,13 @@ def run_reference(args, wl):
 
 
 # --------------------------------------------------------------------------- GPU leg
-def run_e2e(args, q, k, v, w, gate, out, flush, step, flops, world, max_over_ranks, barrier):
-    """Same metric end to end: every step copies its inputs from pinned host
-    memory, runs the C-ABI forward and copies the output back, all between the
-    CUDA events.  Two untimed warm-up steps first."""
+def run_e2e(args, inputs, out, flush, step, flops, world, max_over_ranks, barrier):
+    """Same metric end to end: every step copies its inputs (`inputs`: name ->
+    device tensor) from pinned host memory, runs the C-ABI forward and copies
+    the output back, all between the CUDA events.  Two untimed warm-up steps
+    first."""
     import torch
-    pin = {n: t.cpu().pin_memory() for n, t in dict(q=q, k=k, v=v, w=w, gate=gate).items()}
+    pin = {n: t.cpu().pin_memory() for n, t in inputs.items()}
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     ke = max(3, min(args.steps, 20))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ke + 2)]
@@ -435,7 +452,7 @@ def run_e2e(args, q, k, v, w, gate, out, flush, step, flops, world, max_over_ran
         flush.zero_()
         a, b = ev[i]
         a.record()
-        for dst, n in ((q, "q"), (k, "k"), (v, "v"), (w, "w"), (gate, "gate")):
+        for n, dst in inputs.items():
             dst.copy_(pin[n], non_blocking=True)
         step()
         out_h.copy_(out, non_blocking=True)
@@ -494,6 +511,27 @@ def run_salad(args, wl):
     out = torch.empty_like(q)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
+    # the dynamic gate module: the gate is produced from q and the timestep
+    # embedding in every step (two launches), into the gate buffer
+    gate_step, gate_desc = None, None
+    e2e_inputs = dict(q=q, k=k, v=v, w=w, gate=gate)
+    if wl.itads:
+        gi = si.make_gate_inputs(my_wl)
+        gdev = {n: torch.from_numpy(getattr(gi, n)).to(dev) for n in ("t_emb", "w_t", "w_x", "beta")}
+        gws = torch.empty(sl.lib().salad_gate_workspace_bytes(wl.B, wl.N, wl.Hh, wl.d), dtype=torch.uint8,
+                          device=dev)
+
+        def gate_step():
+            sl.gate_forward(q, gdev["t_emb"], gdev["w_t"], gdev["w_x"], gdev["beta"], gi.threshold,
+                            gate_out=gate, workspace=gws)
+        gate_step()
+        torch.cuda.synchronize()
+        dropped = int((gate == 0).sum())
+        gate_desc = {"gate": "dynamic: sigmoid of an affine map of the timestep embedding (E = 256) and the "
+                             "token mean of q, every step", "threshold": gi.threshold,
+                     "dropped_branches": f"{dropped} of {wl.B * wl.Hh}"}
+        e2e_inputs = dict(q=q, k=k, v=v, w=w, **gdev)
+
     def forward(rp, ci, g):
         if wl.tile:
             sl.attn_forward_tiles(q, k, v, (wl.T, wl.H, wl.W), wl.tile, rp, ci, w, g, out=out, workspace=ws)
@@ -503,6 +541,8 @@ def run_salad(args, wl):
     def step():
         if topk is not None:
             topk.run()
+        if gate_step is not None:
+            gate_step()
         forward(row_ptr, col_idx, gate)
 
     for _ in range(args.warmup):
@@ -584,7 +624,7 @@ def run_salad(args, wl):
     # from pinned memory, the forward, D2H of the output, all inside the events
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, q, k, v, w, gate, out, flush, step, flops, world, max_over_ranks, barrier)
+        e2e = run_e2e(args, e2e_inputs, out, flush, step, flops, world, max_over_ranks, barrier)
 
     dense = None
     if not args.no_dense:
@@ -615,8 +655,8 @@ def run_salad(args, wl):
         line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": config_of(wl, flops, nnz, world),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (5 if wl.topk else 3) * K,
+                "config": {**config_of(wl, flops, nnz, world), **(gate_desc or {})},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (3 + (2 if wl.topk else 0) + (2 if wl.itads else 0)) * K,
                 "clocks": clocks.summary(), "kernels": kernels, "dense": dense,
                 "wall_ms_per_step_incl_flush": round(1e3 * wall / K, 4),
                 "frac_of_bf16_peak_layer": round(value / world / peak, 4),

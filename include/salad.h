@@ -189,6 +189,38 @@ int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B,
                              const void* w_proj, const float* gate, float softmax_scale, float eps, void* out,
                              void* workspace, size_t workspace_bytes, salad_stream_t stream);
 
+/*
+ * The dynamic gate of the linear branch and branch dropping.  The SALAD
+ * summary (section 2.2, ITADS) has a lightweight module turn the denoising
+ * timestep and the hidden state into a global factor s in (0, 1) through a
+ * sigmoid, and (section 2.3) drops the linear branch at inference where s is
+ * very low.  The module is not given; the one implemented here is the plainest
+ * reading, one affine map per head over the timestep embedding and the token
+ * mean of the layer's queries (the hidden state the layer sees):
+ *   s[b][h]    = sigmoid(w_t[h] . t_emb[b] + w_x[h] . (1/N) sum_n q[b][n][h][:] + beta[h])
+ *   gate[b][h] = 0 if s[b][h] < threshold (salad_attn_forward then skips the
+ *                linear branch of (b, h) entirely), s[b][h] otherwise.
+ * fp32 arithmetic in a fixed order (per feature: within a run of tokens, four
+ * interleaved token streams summed in token order and added in stream order;
+ * the runs' sums in eight interleaved groups added in order; fixed tree sums
+ * for the dot products), so repeated calls give the same bits.
+ *
+ *   q          DEVICE bf16 [B][N][Hh][d], 16-byte aligned; d = 64 or 128.
+ *   t_emb      DEVICE fp32 [B][E];  w_t DEVICE fp32 [Hh][E] (both may be NULL
+ *              when E == 0).   w_x DEVICE fp32 [Hh][d].   beta DEVICE fp32 [Hh].
+ *   threshold  finite; <= 0 drops nothing, > 1 drops every branch.
+ *   s_out      DEVICE fp32 [B][Hh] or NULL: s before dropping.
+ *   gate_out   DEVICE fp32 [B][Hh]: the gate salad_attn_forward takes.
+ *   workspace  DEVICE, >= salad_gate_workspace_bytes(B, N, Hh, d), 16-byte
+ *              aligned; no initialisation needed.
+ * Never synchronises.  Errors: INVALID_ARG, UNSUPPORTED (d, B > 65535),
+ * WORKSPACE, CUDA.
+ */
+size_t salad_gate_workspace_bytes(int B, int N, int num_heads, int d);
+int salad_gate_forward(const void* q, int B, int N, int num_heads, int d, const float* t_emb, int E,
+                       const float* w_t, const float* w_x, const float* beta, float threshold, float* s_out,
+                       float* gate_out, void* workspace, size_t workspace_bytes, salad_stream_t stream);
+
 size_t salad_topk_workspace_bytes(int B, int N, int num_heads, int d, int block);
 int salad_build_topk_mask(const void* q, const void* k, int B, int N, int num_heads, int d, int block, int keep,
                           int32_t* row_ptr, int32_t* col_idx, void* workspace, size_t workspace_bytes,

@@ -227,7 +227,7 @@ def gate(q, t_emb, w_t, w_x, beta, threshold):
     where s < threshold (the linear branch dropped)."""
     q = np.ascontiguousarray(q, dtype=np.uint16)
     B, N, Hh, d = q.shape
-    t_emb = np.ascontiguousarray(t_emb, dtype=np.float64).reshape(B, -1)
+    t_emb = np.ascontiguousarray(t_emb, dtype=np.float64)
     E = t_emb.shape[1]
     w_t = np.ascontiguousarray(w_t, dtype=np.float64).reshape(Hh, E)
     w_x = np.ascontiguousarray(w_x, dtype=np.float64).reshape(Hh, d)

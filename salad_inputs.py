@@ -42,6 +42,7 @@ class Workload:
     gate_hi: float = 1.0
     topk: int = 0  # > 0: Top-K dynamic block mask keeping this many key blocks per query block (window unused)
     tile: tuple = ()  # (bt, bh, bw): 3-D tile blocks of bt*bh*bw = block grid points; (): raster blocks
+    itads: bool = False  # the gate comes from the dynamic gate module every step (inputs: make_gate_inputs)
 
     @property
     def N(self) -> int:
@@ -92,7 +93,12 @@ WAN13B_TOPK = WAN13B_90.with_(name="wan1.3b-32760tok-topk26", topk=26, seed=5)
 # 6,582 raster block pairs for the same window.
 WAN13B_TILES = WAN13B_90.with_(name="wan1.3b-32760tok-tiles1x32x4", tile=(1, 32, 4), seed=6)
 
-WORKLOADS = {w.name: w for w in [TINY, WAN13B_90, WAN13B_75_CFG, WAN14B_720P, WAN13B_TOPK, WAN13B_TILES]
+# The 1.3B layer whose gate comes from the dynamic gate module every step, with
+# branch dropping: 3 of its 12 heads fall below the threshold.
+WAN13B_ITADS = WAN13B_90.with_(name="wan1.3b-32760tok-90pct-itads", itads=True, seed=7)
+
+WORKLOADS = {w.name: w for w in [TINY, WAN13B_90, WAN13B_75_CFG, WAN14B_720P, WAN13B_TOPK, WAN13B_TILES,
+                                 WAN13B_ITADS]
              + [sweep(p) for p in SWEEP_WINDOWS]}
 
 
@@ -168,3 +174,24 @@ def sample_query_blocks(wl: Workload, per_bh: int = 32, full_first_last: bool = 
             pairs.update((bh, int(i)) for i in picks)
             pairs.add((bh, nb - 1))
     return np.asarray(sorted(pairs), dtype=np.int32).reshape(-1, 2)
+
+
+@dataclasses.dataclass
+class GateInputs:
+    t_emb: np.ndarray   # fp32 [B][E]
+    w_t: np.ndarray     # fp32 [Hh][E]
+    w_x: np.ndarray     # fp32 [Hh][d]
+    beta: np.ndarray    # fp32 [Hh]
+    threshold: float
+
+
+def make_gate_inputs(wl: Workload, E: int = 256, threshold: float = 0.35) -> GateInputs:
+    """Seeded inputs of the dynamic gate module (its own stream, so the layer's
+    inputs do not change): t_emb ~ N(0,1), w_t ~ N(0,1/E), w_x ~ N(0, 4/d) (the
+    pooled queries are small), beta ~ N(-0.5, 1)."""
+    rng = np.random.default_rng(wl.seed + 7777)
+    t_emb = rng.standard_normal((wl.B, E), dtype=np.float32)
+    w_t = rng.standard_normal((wl.Hh, E), dtype=np.float32) / np.float32(math.sqrt(E))
+    w_x = rng.standard_normal((wl.Hh, wl.d), dtype=np.float32) * np.float32(2.0 / math.sqrt(wl.d))
+    beta = rng.standard_normal(wl.Hh, dtype=np.float32) - np.float32(0.5)
+    return GateInputs(t_emb, w_t, w_x, beta, float(threshold))

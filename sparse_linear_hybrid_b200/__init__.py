@@ -7,9 +7,8 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, tile_num_blocks, build_tile_mask, workspace_bytes, attn_forward,
-    attn_forward_tiles, attn_forward_static, linear_state, check_status, set_wait_limit_ns, set_max_ctas,
-    set_phase_events,
-    status_string
+    attn_forward_tiles, attn_forward_static, gate_forward, linear_state, check_status, set_wait_limit_ns,
+    set_max_ctas, set_phase_events, status_string
 """
 from __future__ import annotations
 
@@ -66,6 +65,10 @@ def lib() -> ctypes.CDLL:
         L.salad_attn_forward_tiles.argtypes = [p, p, p, i, i, i, i, i, i, i, i, i, p, p, p, p, f, f, p, p, sz,
                                                p]
         L.salad_attn_forward_tiles.restype = i
+        L.salad_gate_workspace_bytes.argtypes = [i, i, i, i]
+        L.salad_gate_workspace_bytes.restype = sz
+        L.salad_gate_forward.argtypes = [p, i, i, i, i, p, i, p, p, p, f, p, p, p, sz, p]
+        L.salad_gate_forward.restype = i
         L.salad_topk_workspace_bytes.argtypes = [i, i, i, i, i]
         L.salad_topk_workspace_bytes.restype = sz
         L.salad_build_topk_mask.argtypes = [p, p, i, i, i, i, i, i, p, p, p, sz, p]
@@ -222,6 +225,29 @@ def attn_forward_tiles(q, k, v, grid, tile, row_ptr, col_idx, w_proj, gate, soft
         _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream)), "salad_attn_forward_tiles")
     return out
+
+
+def gate_forward(q, t_emb, w_t, w_x, beta, threshold: float, gate_out=None, s_out=None, workspace=None,
+                 stream=None) -> torch.Tensor:
+    """Dynamic gate with branch dropping (see salad.h): fp32 [B, Hh] CUDA tensor,
+    0 where the sigmoid gate falls below `threshold`.  t_emb fp32 [B, E], w_t
+    [Hh, E], w_x [Hh, d], beta [Hh]."""
+    B, N, Hh, d = q.shape
+    E = t_emb.shape[1] if t_emb is not None else 0
+    if gate_out is None:
+        gate_out = torch.empty(B, Hh, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = lib().salad_gate_workspace_bytes(B, N, Hh, d)
+        if n == 0:
+            raise SaladError(SALAD_ERR_INVALID_ARG, "salad_gate_workspace_bytes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    opt = lambda t, name: None if t is None else _dev_ptr(t, torch.float32, name)  # noqa: E731
+    _check(lib().salad_gate_forward(
+        _dev_ptr(q, torch.bfloat16, "q"), B, N, Hh, d, opt(t_emb, "t_emb"), E, opt(w_t, "w_t"),
+        _dev_ptr(w_x, torch.float32, "w_x"), _dev_ptr(beta, torch.float32, "beta"), float(threshold),
+        opt(s_out, "s_out"), _dev_ptr(gate_out, torch.float32, "gate_out"),
+        _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "salad_gate_forward")
+    return gate_out
 
 
 def build_topk_mask(q, k, block: int, keep: int, workspace=None, stream=None):

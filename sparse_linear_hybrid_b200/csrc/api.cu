@@ -316,6 +316,41 @@ int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B,
                            eps, out, workspace, workspace_bytes, stream, 0, &g);
 }
 
+size_t salad_gate_workspace_bytes(int B, int N, int num_heads, int d) {
+  if (B < 1 || N < 1 || num_heads < 1 || (d != 64 && d != 128)) return 0;
+  return gate_workspace_bytes(B, N, num_heads, d);
+}
+
+int salad_gate_forward(const void* q, int B, int N, int num_heads, int d, const float* t_emb, int E,
+                       const float* w_t, const float* w_x, const float* beta, float threshold, float* s_out,
+                       float* gate_out, void* workspace, size_t workspace_bytes, salad_stream_t stream) {
+  if (!q || !w_x || !beta || !gate_out || !workspace || B < 1 || N < 1 || num_heads < 1 || E < 0)
+    return SALAD_ERR_INVALID_ARG;
+  if (E > 0 && (!t_emb || !w_t)) return SALAD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
+  if (B > 65535 || (long long)B * num_heads >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(workspace, 16) || !aligned(gate_out, 4) || (s_out && !aligned(s_out, 4)))
+    return SALAD_ERR_INVALID_ARG;
+  if (!std::isfinite(threshold)) return SALAD_ERR_INVALID_ARG;
+  if (workspace_bytes < gate_workspace_bytes(B, N, num_heads, d)) return SALAD_ERR_WORKSPACE;
+  GateArgs ga{};
+  ga.q = static_cast<const uint16_t*>(q);
+  ga.B = B;
+  ga.N = N;
+  ga.heads = num_heads;
+  ga.d = d;
+  ga.E = E;
+  ga.t_emb = t_emb;
+  ga.w_t = w_t;
+  ga.w_x = w_x;
+  ga.beta = beta;
+  ga.threshold = threshold;
+  ga.partial = static_cast<float*>(workspace);
+  ga.s_out = s_out;
+  ga.gate_out = gate_out;
+  return launch_gate(ga, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
+}
+
 size_t salad_topk_workspace_bytes(int B, int N, int num_heads, int d, int block) {
   if (B < 1 || N < 1 || num_heads < 1 || (d != 64 && d != 128) || block < 1) return 0;
   return topk_workspace_bytes(B, N, num_heads, d, block);

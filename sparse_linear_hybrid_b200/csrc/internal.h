@@ -100,6 +100,23 @@ struct AttnArgs {
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
 
+// Dynamic gate and branch dropping (gate.cu).
+struct GateArgs {
+  const uint16_t* q;  // bf16 [B][N][Hh][d], 16-byte aligned
+  int B, N, heads, d, E;
+  const float* t_emb;  // [B][E]
+  const float* w_t;    // [Hh][E]
+  const float* w_x;    // [Hh][d]
+  const float* beta;   // [Hh]
+  float threshold;
+  float* partial;      // workspace: [splits][B][Hh*d]
+  float* s_out;        // [B][Hh] or nullptr
+  float* gate_out;     // [B][Hh]
+};
+int gate_splits(int B, int N, int* chunk);
+size_t gate_workspace_bytes(int B, int N, int heads, int d);
+cudaError_t launch_gate(const GateArgs& a, cudaStream_t s);
+
 // Top-K dynamic block mask (topk.cu).
 struct TopkArgs {
   const uint16_t* q;  // bf16 [B][N][Hh][d]
