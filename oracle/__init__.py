@@ -50,6 +50,9 @@ def _load():
         lib.oracle_topk_mask.argtypes = [P, P] + [ctypes.c_int] * 6 + [P, P]
         lib.oracle_gate.restype = None
         lib.oracle_gate.argtypes = [P] + [ctypes.c_int] * 4 + [P, ctypes.c_int, P, P, P, ctypes.c_double, P, P]
+        lib.oracle_backward.restype = None
+        lib.oracle_backward.argtypes = ([P, P, P] + [ctypes.c_int] * 5 + [P, P, P, P] + [ctypes.c_double] * 2
+                                        + [P, ctypes.c_int, P, P, P, P, P])
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -237,3 +240,25 @@ def gate(q, t_emb, w_t, w_x, beta, threshold):
     _load().oracle_gate(_ptr(q), B, N, Hh, d, _ptr(t_emb), E, _ptr(w_t), _ptr(w_x), _ptr(beta),
                         float(threshold), _ptr(s), _ptr(g))
     return s, g
+
+
+def backward(q, k, v, block, row_ptr, col_idx, w_proj, gate, dout, tau=None, eps=1e-6, mask_per_bh=False):
+    """Gradients of the layer (raster blocks) for dL/dout = dout (fp64 [B, N, Hh, d]):
+    dict of fp64 dq, dk, dv [B, N, Hh, d], dw [d, d], dgate [B, Hh]."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    B, N, Hh, d = q.shape
+    tau = 1.0 / np.sqrt(d) if tau is None else tau
+    w_proj = np.ascontiguousarray(w_proj, dtype=np.uint16)
+    gate = np.ascontiguousarray(gate, dtype=np.float32).reshape(B, Hh)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    row_ptr = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    col_idx = np.ascontiguousarray(col_idx, dtype=np.int32)
+    res = {n: np.zeros((B, N, Hh, d)) for n in ("dq", "dk", "dv")}
+    res["dw"] = np.zeros((d, d))
+    res["dgate"] = np.zeros((B, Hh))
+    _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), B, N, Hh, d, int(block), _ptr(row_ptr), _ptr(col_idx),
+                            _ptr(w_proj), _ptr(gate), float(tau), float(eps), _ptr(dout), int(bool(mask_per_bh)),
+                            _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dw"]), _ptr(res["dgate"]))
+    return res

@@ -329,6 +329,259 @@ void oracle_forward_blocks(const uint16_t *q, const uint16_t *k, const uint16_t 
     free(W);
 }
 
+/*
+ * Backward pass of the layer (the gradients the fine-tuning of the SALAD summary,
+ * section 3, needs: the sparse branch, the linear branch, the static projection
+ * and the gate), for raster blocks, given dout = dL/dout fp64 [B][N][Hh][d].
+ * Written from the forward above by the chain rule, in the forward's notation:
+ *   sparse:  p_ij = softmax_j(s_ij), s_ij = tau q_i.k_j over the kept keys;
+ *            dp_ij = dout_i.v_j, D_i = sum_j p_ij dp_ij, ds_ij = p_ij (dp_ij - D_i);
+ *            dq_i += tau sum_j ds_ij k_j, dk_j += tau sum_i ds_ij q_i,
+ *            dv_j += sum_i p_ij dout_i
+ *   linear:  a_i = relu(q_i), den_i = a_i.z + eps, u_i = a_i^T S,
+ *            o_i = u_i / den_i, y_i = o_i W;
+ *            dgate[b][h] = sum_i dout_i.y_i   (also where g = 0);
+ *            dy_i = g dout_i, dW += sum_i o_i^T dy_i (over every (b, h));
+ *            do_i = dy_i W^T, du_i = do_i / den_i, dden_i = -(do_i.o_i) / den_i;
+ *            dS = sum_i a_i du_i^T, dz = sum_i dden_i a_i;
+ *            dq_i += [q_i > 0] (S du_i + dden_i z);
+ *            dk_j += [k_j > 0] (dS v_j + dz), dv_j += dS^T relu(k_j)
+ * (the derivative of relu at 0 is taken as 0).  Outputs fp64: dq, dk, dv
+ * [B][N][Hh][d], dw [d][d], dgate [B][Hh].  mask_per_bh as in the forward.
+ */
+static int row_has(const int32_t *cols, int32_t n, int32_t J) {
+    int32_t lo = 0, hi = n; /* columns ascending */
+    while (lo < hi) {
+        const int32_t mid = (lo + hi) / 2;
+        if (cols[mid] < J) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo < n && cols[lo] == J;
+}
+
+void oracle_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int N, int Hh, int d,
+                     int blk, const int32_t *row_ptr, const int32_t *col_idx, const uint16_t *w_proj,
+                     const float *gate, double tau, double eps, const double *dout, int mask_per_bh, double *dq,
+                     double *dk, double *dv, double *dw, double *dgate) {
+    const int nb = (N + blk - 1) / blk;
+    const int BH = B * Hh;
+    const int64_t rows = (int64_t)BH * N; /* per-row scratch, indexed (bh * N + i) */
+    double *W = (double *)malloc(sizeof(double) * d * d);
+    double *S = (double *)malloc(sizeof(double) * BH * d * d);
+    double *z = (double *)malloc(sizeof(double) * BH * d);
+    double *dS = (double *)calloc((size_t)BH * d * d, sizeof(double));
+    double *dz = (double *)calloc((size_t)BH * d, sizeof(double));
+    double *dWbh = (double *)calloc((size_t)BH * d * d, sizeof(double));
+    double *lse = (double *)malloc(sizeof(double) * rows);
+    double *Dr = (double *)malloc(sizeof(double) * rows);
+    double *du = (double *)malloc(sizeof(double) * rows * d);
+    double *dden = (double *)malloc(sizeof(double) * rows);
+    double *orow = (double *)malloc(sizeof(double) * rows * d);
+    double *yg = (double *)malloc(sizeof(double) * rows);
+    for (int i = 0; i < d * d; ++i) W[i] = bf16_to_double(w_proj[i]);
+    oracle_linear_state(k, v, B, N, Hh, d, S, z);
+
+    /* queries: softmax statistics, D_i, dq_i and the linear branch's per-row terms */
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t task = 0; task < (int64_t)BH * nb; ++task) {
+        const int bh = (int)(task / nb), I = (int)(task % nb), b = bh / Hh, h = bh % Hh;
+        const double g = (double)gate[bh];
+        const int mrow = (mask_per_bh ? bh : h) * nb + I;
+        const int32_t r0 = row_ptr[mrow], r1 = row_ptr[mrow + 1];
+        const int64_t nkeys = (int64_t)(r1 - r0) * blk;
+        int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (nkeys > 0 ? nkeys : 1));
+        double *sc = (double *)malloc(sizeof(double) * (nkeys > 0 ? nkeys : 1));
+        double *qi = (double *)malloc(sizeof(double) * d);
+        double *gi = (double *)malloc(sizeof(double) * d);
+        double *acc = (double *)malloc(sizeof(double) * d);
+        double *y = (double *)malloc(sizeof(double) * d);
+        double *dov = (double *)malloc(sizeof(double) * d);
+        int64_t nk = 0;
+        for (int32_t r = r0; r < r1; ++r)
+            for (int64_t j = (int64_t)col_idx[r] * blk; j < (int64_t)(col_idx[r] + 1) * blk && j < N; ++j)
+                keys[nk++] = j;
+        for (int64_t i = (int64_t)I * blk; i < (int64_t)(I + 1) * blk && i < N; ++i) {
+            const int64_t off = (((int64_t)b * N + i) * Hh + h) * d;
+            const int64_t ri = (int64_t)bh * N + i;
+            for (int c = 0; c < d; ++c) {
+                qi[c] = bf16_to_double(q[off + c]);
+                gi[c] = dout[off + c];
+                acc[c] = 0.0;
+            }
+            /* sparse branch: the probabilities, then D_i and dq_i */
+            double m = -INFINITY, l = 0.0;
+            for (int64_t t = 0; t < nk; ++t) {
+                const int64_t koff = (((int64_t)b * N + keys[t]) * Hh + h) * d;
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += qi[c] * bf16_to_double(k[koff + c]);
+                sc[t] = tau * dot;
+                if (sc[t] > m) m = sc[t];
+            }
+            for (int64_t t = 0; t < nk; ++t) l += exp(sc[t] - m);
+            lse[ri] = m + log(l);
+            double D = 0.0;
+            for (int64_t t = 0; t < nk; ++t) {
+                const int64_t voff = (((int64_t)b * N + keys[t]) * Hh + h) * d;
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c) dp += gi[c] * bf16_to_double(v[voff + c]);
+                sc[t] = exp(sc[t] - lse[ri]); /* p_ij */
+                D += sc[t] * dp;
+            }
+            Dr[ri] = D;
+            for (int64_t t = 0; t < nk; ++t) {
+                const int64_t kvoff = (((int64_t)b * N + keys[t]) * Hh + h) * d;
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c) dp += gi[c] * bf16_to_double(v[kvoff + c]);
+                const double ds = sc[t] * (dp - D);
+                for (int c = 0; c < d; ++c) acc[c] += tau * ds * bf16_to_double(k[kvoff + c]);
+            }
+            /* linear branch */
+            const double *Sb = S + (int64_t)bh * d * d;
+            const double *zb = z + (int64_t)bh * d;
+            double den = eps;
+            for (int c = 0; c < d; ++c) den += (qi[c] > 0.0 ? qi[c] : 0.0) * zb[c];
+            double *o = orow + ri * d;
+            for (int e = 0; e < d; ++e) {
+                double u = 0.0;
+                for (int c = 0; c < d; ++c) u += (qi[c] > 0.0 ? qi[c] : 0.0) * Sb[(int64_t)c * d + e];
+                o[e] = u / den;
+            }
+            double ygi = 0.0;
+            for (int f = 0; f < d; ++f) {
+                y[f] = 0.0;
+                for (int e = 0; e < d; ++e) y[f] += o[e] * W[e * d + f];
+                ygi += gi[f] * y[f];
+            }
+            yg[ri] = ygi;
+            double od = 0.0;
+            for (int e = 0; e < d; ++e) {
+                dov[e] = 0.0;
+                for (int f = 0; f < d; ++f) dov[e] += W[e * d + f] * g * gi[f]; /* do = (g dout) W^T */
+                od += dov[e] * o[e];
+            }
+            dden[ri] = -od / den;
+            for (int e = 0; e < d; ++e) du[ri * d + e] = dov[e] / den;
+            for (int c = 0; c < d; ++c) {
+                if (!(qi[c] > 0.0)) continue;
+                double da = dden[ri] * zb[c];
+                for (int e = 0; e < d; ++e) da += Sb[(int64_t)c * d + e] * du[ri * d + e];
+                acc[c] += da;
+            }
+            for (int c = 0; c < d; ++c) dq[off + c] = acc[c];
+        }
+        free(keys);
+        free(sc);
+        free(qi);
+        free(gi);
+        free(acc);
+        free(y);
+        free(dov);
+    }
+
+    /* per (b, h): dS, dz, the gate's gradient and this (b, h)'s share of dW */
+#pragma omp parallel for schedule(static)
+    for (int bh = 0; bh < BH; ++bh) {
+        const int b = bh / Hh, h = bh % Hh;
+        const double g = (double)gate[bh];
+        double dg = 0.0;
+        for (int64_t i = 0; i < N; ++i) {
+            const int64_t off = (((int64_t)b * N + i) * Hh + h) * d;
+            const int64_t ri = (int64_t)bh * N + i;
+            dg += yg[ri];
+            for (int c = 0; c < d; ++c) {
+                const double a = bf16_to_double(q[off + c]);
+                if (a > 0.0) {
+                    dz[(int64_t)bh * d + c] += dden[ri] * a;
+                    for (int e = 0; e < d; ++e) dS[((int64_t)bh * d + c) * d + e] += a * du[ri * d + e];
+                }
+            }
+            for (int e = 0; e < d; ++e)
+                for (int f = 0; f < d; ++f)
+                    dWbh[((int64_t)bh * d + e) * d + f] += orow[ri * d + e] * g * dout[off + f];
+        }
+        dgate[bh] = dg;
+    }
+    for (int i = 0; i < d * d; ++i) {
+        double sum = 0.0;
+        for (int bh = 0; bh < BH; ++bh) sum += dWbh[(int64_t)bh * d * d + i];
+        dw[i] = sum;
+    }
+
+    /* keys: every query of every query block whose row keeps the key's block */
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t task = 0; task < (int64_t)BH * nb; ++task) {
+        const int bh = (int)(task / nb), J = (int)(task % nb), b = bh / Hh, h = bh % Hh;
+        const double *dSb = dS + (int64_t)bh * d * d;
+        const double *dzb = dz + (int64_t)bh * d;
+        double *kj = (double *)malloc(sizeof(double) * d);
+        double *vj = (double *)malloc(sizeof(double) * d);
+        double *ak = (double *)malloc(sizeof(double) * d);
+        double *av = (double *)malloc(sizeof(double) * d);
+        for (int64_t j = (int64_t)J * blk; j < (int64_t)(J + 1) * blk && j < N; ++j) {
+            const int64_t off = (((int64_t)b * N + j) * Hh + h) * d;
+            for (int c = 0; c < d; ++c) {
+                kj[c] = bf16_to_double(k[off + c]);
+                vj[c] = bf16_to_double(v[off + c]);
+                ak[c] = 0.0;
+                av[c] = 0.0;
+            }
+            for (int I = 0; I < nb; ++I) {
+                const int mrow = (mask_per_bh ? bh : h) * nb + I;
+                if (!row_has(col_idx + row_ptr[mrow], row_ptr[mrow + 1] - row_ptr[mrow], J)) continue;
+                for (int64_t i = (int64_t)I * blk; i < (int64_t)(I + 1) * blk && i < N; ++i) {
+                    const int64_t qoff = (((int64_t)b * N + i) * Hh + h) * d;
+                    const int64_t ri = (int64_t)bh * N + i;
+                    double dot = 0.0, dp = 0.0;
+                    for (int c = 0; c < d; ++c) {
+                        dot += bf16_to_double(q[qoff + c]) * kj[c];
+                        dp += dout[qoff + c] * vj[c];
+                    }
+                    const double p = exp(tau * dot - lse[ri]);
+                    const double ds = p * (dp - Dr[ri]);
+                    for (int c = 0; c < d; ++c) {
+                        ak[c] += tau * ds * bf16_to_double(q[qoff + c]);
+                        av[c] += p * dout[qoff + c];
+                    }
+                }
+            }
+            /* linear branch through S and z */
+            for (int c = 0; c < d; ++c) {
+                if (kj[c] > 0.0) {
+                    double t = dzb[c];
+                    for (int e = 0; e < d; ++e) t += dSb[(int64_t)c * d + e] * vj[e];
+                    ak[c] += t;
+                }
+            }
+            for (int e = 0; e < d; ++e) {
+                double t = 0.0;
+                for (int c = 0; c < d; ++c)
+                    if (kj[c] > 0.0) t += dSb[(int64_t)c * d + e] * kj[c];
+                av[e] += t;
+            }
+            for (int c = 0; c < d; ++c) {
+                dk[off + c] = ak[c];
+                dv[off + c] = av[c];
+            }
+        }
+        free(kj);
+        free(vj);
+        free(ak);
+        free(av);
+    }
+    free(W);
+    free(S);
+    free(z);
+    free(dS);
+    free(dz);
+    free(dWbh);
+    free(lse);
+    free(Dr);
+    free(du);
+    free(dden);
+    free(orow);
+    free(yg);
+}
+
 /* Threads the OpenMP runtime will use (reported next to the CPU timings). */
 /*
  * Top-K dynamic block mask.  The SALAD summary (section 5) names Top-K dynamic
