@@ -48,6 +48,8 @@ FLUSH_BYTES = 256 << 20
 NCU_TRAFFIC = {
     "wan1.3b-32760tok-90pct": {"source": "008b196b7ef807a2", "bytes": 303_186_176 + 84_460_544},
     "wan1.3b-32760tok-tiles1x32x4": {"source": "008b196b7ef807a2", "bytes": 303_293_952 + 85_079_296},
+    "wan1.3b-32760tok-topk26": {"source": "008b196b7ef807a2", "bytes": 304_376_320 + 84_819_200},
+    "wan1.3b-32760tok-90pct-itads": {"source": "008b196b7ef807a2", "bytes": 303_038_976 + 83_953_408},
 }
 
 
