@@ -148,6 +148,20 @@ int salad_attn_forward(const void* q, const void* k, const void* v, int B, int N
                        size_t workspace_bytes, salad_stream_t stream);
 
 /*
+ * salad_attn_forward (mask rows per head, or per (b, h) when mask_per_bh != 0)
+ * that also writes what a training forward keeps for the backward pass:
+ *   lse[b][h][i] = log sum_{j in K(i)} exp(scale * q_i . k_j)   (natural log;
+ *                  -inf for a row whose blocks keep no key)
+ *   lse   DEVICE fp32 [B][Hh][N], 4-byte aligned.
+ * Everything else as salad_attn_forward.  fp32: the row maximum the kernel
+ * keeps plus log2 of its fp32 row sum, times ln 2.
+ */
+int salad_attn_forward_lse(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                           int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                           const float* gate, float softmax_scale, float eps, int mask_per_bh, void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, salad_stream_t stream);
+
+/*
  * Top-K dynamic block mask.  The SALAD summary (section 5) says the method also
  * applies to Top-K dynamic sparse attention and gives no scoring rule; the rule
  * implemented here is a reading of that sentence:

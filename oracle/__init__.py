@@ -53,6 +53,8 @@ def _load():
         lib.oracle_backward.restype = None
         lib.oracle_backward.argtypes = ([P, P, P] + [ctypes.c_int] * 5 + [P, P, P, P] + [ctypes.c_double] * 2
                                         + [P, ctypes.c_int, P, P, P, P, P])
+        lib.oracle_lse.restype = None
+        lib.oracle_lse.argtypes = [P, P] + [ctypes.c_int] * 5 + [P, P, ctypes.c_double, ctypes.c_int, P]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -262,3 +264,16 @@ def backward(q, k, v, block, row_ptr, col_idx, w_proj, gate, dout, tau=None, eps
                             _ptr(w_proj), _ptr(gate), float(tau), float(eps), _ptr(dout), int(bool(mask_per_bh)),
                             _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dw"]), _ptr(res["dgate"]))
     return res
+
+
+def lse(q, k, block, row_ptr, col_idx, tau=None, mask_per_bh=False):
+    """Log-sum-exp (natural log) of the sparse softmax of every query row, fp64
+    [B, Hh, N]; -inf for a row without keys."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    B, N, Hh, d = q.shape
+    tau = 1.0 / np.sqrt(d) if tau is None else tau
+    out = np.zeros((B, Hh, N))
+    _load().oracle_lse(_ptr(q), _ptr(k), B, N, Hh, d, int(block), _ptr(np.ascontiguousarray(row_ptr, np.int32)),
+                       _ptr(np.ascontiguousarray(col_idx, np.int32)), float(tau), int(bool(mask_per_bh)), _ptr(out))
+    return out

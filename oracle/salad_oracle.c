@@ -582,6 +582,45 @@ void oracle_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, in
     free(yg);
 }
 
+/*
+ * Log-sum-exp of the sparse branch's softmax for every query row (the quantity
+ * a training forward keeps for the backward pass):
+ *   lse[b][h][i] = log sum_j exp(tau q_i . k_j) over the real tokens j of the
+ *   key blocks kept for i's block (raster blocks); -inf for a row with no keys.
+ * fp64, natural log; lse is [B][Hh][N].  mask_per_bh as in the forward.
+ */
+void oracle_lse(const uint16_t *q, const uint16_t *k, int B, int N, int Hh, int d, int blk,
+                const int32_t *row_ptr, const int32_t *col_idx, double tau, int mask_per_bh, double *lse) {
+    const int nb = (N + blk - 1) / blk;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int bh = 0; bh < B * Hh; ++bh) {
+        for (int I = 0; I < nb; ++I) {
+            const int b = bh / Hh, h = bh % Hh;
+            const int mrow = (mask_per_bh ? bh : h) * nb + I;
+            for (int64_t i = (int64_t)I * blk; i < (int64_t)(I + 1) * blk && i < N; ++i) {
+                const int64_t qoff = (((int64_t)b * N + i) * Hh + h) * d;
+                double m = -INFINITY;
+                for (int pass = 0; pass < 2; ++pass) {
+                    double l = 0.0;
+                    for (int32_t r = row_ptr[mrow]; r < row_ptr[mrow + 1]; ++r) {
+                        for (int64_t j = (int64_t)col_idx[r] * blk; j < (int64_t)(col_idx[r] + 1) * blk && j < N; ++j) {
+                            const int64_t koff = (((int64_t)b * N + j) * Hh + h) * d;
+                            double dot = 0.0;
+                            for (int c = 0; c < d; ++c) dot += bf16_to_double(q[qoff + c]) * bf16_to_double(k[koff + c]);
+                            if (pass == 0) {
+                                if (tau * dot > m) m = tau * dot;
+                            } else {
+                                l += exp(tau * dot - m);
+                            }
+                        }
+                    }
+                    if (pass == 1) lse[(int64_t)bh * N + i] = l > 0.0 ? m + log(l) : -INFINITY;
+                }
+            }
+        }
+    }
+}
+
 /* Threads the OpenMP runtime will use (reported next to the CPU timings). */
 /*
  * Top-K dynamic block mask.  The SALAD summary (section 5) names Top-K dynamic

@@ -7,7 +7,7 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, tile_num_blocks, build_tile_mask, workspace_bytes, attn_forward,
-    attn_forward_tiles, attn_forward_static, gate_forward, linear_state, check_status, set_wait_limit_ns,
+    attn_forward_lse, attn_forward_tiles, attn_forward_static, gate_forward, linear_state, check_status, set_wait_limit_ns,
     set_max_ctas, set_phase_events, status_string
 """
 from __future__ import annotations
@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.salad_attn_forward.restype = i
         L.salad_attn_forward_bh.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
         L.salad_attn_forward_bh.restype = i
+        L.salad_attn_forward_lse.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, i, p, p, p, sz, p]
+        L.salad_attn_forward_lse.restype = i
         L.salad_attn_forward_tiles.argtypes = [p, p, p, i, i, i, i, i, i, i, i, i, p, p, p, p, f, f, p, p, sz,
                                                p]
         L.salad_attn_forward_tiles.restype = i
@@ -202,6 +204,27 @@ def attn_forward(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_sc
         _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream)), "salad_attn_forward")
     return out
+
+
+def attn_forward_lse(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softmax_scale: float = 0.0,
+                     eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None, mask_per_bh: bool = False):
+    """attn_forward that also returns each row's log-sum-exp of the sparse softmax
+    (natural log, fp32 [B, Hh, N]): (out, lse)."""
+    B, N, Hh, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hh, N, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(B, N, Hh, d, q.device)
+    _check(lib().salad_attn_forward_lse(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
+        B, N, Hh, d, block, _dev_ptr(row_ptr, torch.int32, "row_ptr"),
+        _dev_ptr(col_idx, torch.int32, "col_idx"), _dev_ptr(w_proj, torch.bfloat16, "w_proj"),
+        _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps), int(bool(mask_per_bh)),
+        _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(lse, torch.float32, "lse"),
+        _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "salad_attn_forward_lse")
+    return out, lse
 
 
 def attn_forward_tiles(q, k, v, grid, tile, row_ptr, col_idx, w_proj, gate, softmax_scale: float = 0.0,

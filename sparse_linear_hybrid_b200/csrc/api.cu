@@ -212,7 +212,8 @@ namespace {
 int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d, int block,
                       const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj, const float* gate,
                       float softmax_scale, float eps, void* out, void* workspace, size_t workspace_bytes,
-                      salad_stream_t stream, int mask_per_bh, const TileGeom* tiles = nullptr) {
+                      salad_stream_t stream, int mask_per_bh, const TileGeom* tiles = nullptr,
+                      float* lse = nullptr) {
   if (!q || !row_ptr || !col_idx || !w_proj || !gate || !out) return SALAD_ERR_INVALID_ARG;
   int st = check_common(k, v, B, N, num_heads, d, workspace, workspace_bytes);
   if (st != SALAD_OK) return st;
@@ -263,6 +264,7 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
   aa.max_ctas = g_max_ctas.load();
   aa.mask_per_bh = mask_per_bh;
   aa.tiles = tiles ? *tiles : TileGeom{};
+  aa.lse = lse;
   aa.B = B;
   aa.N = N;
   aa.heads = num_heads;
@@ -296,6 +298,15 @@ int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, in
                           size_t workspace_bytes, salad_stream_t stream) {
   return attn_forward_impl(q, k, v, B, N, num_heads, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
                            out, workspace, workspace_bytes, stream, 1);
+}
+
+int salad_attn_forward_lse(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
+                           int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
+                           const float* gate, float softmax_scale, float eps, int mask_per_bh, void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, salad_stream_t stream) {
+  if (!lse || !aligned(lse, 4)) return SALAD_ERR_INVALID_ARG;
+  return attn_forward_impl(q, k, v, B, N, num_heads, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
+                           out, workspace, workspace_bytes, stream, mask_per_bh ? 1 : 0, nullptr, lse);
 }
 
 int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B, int T, int H, int W, int bt,

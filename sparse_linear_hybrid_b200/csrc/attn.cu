@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const int32_t* __restrict__ col_idx, const float* __restrict__ gate,
                       const float* __restrict__ zvec, int heads, int N, int qtiles, int num_items,
                       uint32_t* work_ctr, float scale_log2, float eps, uint32_t* status, uint64_t limit_ns,
-                      int mask_per_bh, const TileGeom tg) {
+                      int mask_per_bh, const TileGeom tg, float* __restrict__ lse_out) {
   using C = AttnCfg<D, BLK>;
   static_assert(!TILES || BLK == 128, "a tile block fills one 128-row query tile");
   const int nblocks = TILES ? qtiles : (N + BLK - 1) / BLK;  // key blocks per mask row
@@ -953,6 +953,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float gd = im.lin ? im.g / ((sh->xden[xc & 1][0][r] + sh->xden[xc & 1][1][r]) + eps) : 0.f;
       ++xc;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      if constexpr (!TILES) {
+        // the row's log-sum-exp (natural log) of the sparse softmax, for training:
+        // sum_j exp(scale s_j) = 2^(m_ref * scale * log2 e) * l
+        if (lse_out != nullptr && hf == 0 && im.qtile * 128 + r < N)
+          lse_out[(size_t)im.bh * N + im.qtile * 128 + r] =
+              l > 0.f ? (m_ref * scale_log2 + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      }
       // U lands in the S slot after this item's tiles
       const int su = sj & 1;
       if (im.lin) {
@@ -1040,7 +1047,7 @@ cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
   const int grid = (int)(items < ctas ? items : ctas);
   salad_attn_kernel<D, BLK, TILES><<<grid, kThreads, smem, s>>>(
       *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_out, *a.tm_t, a.row_ptr, a.col_idx, a.gate, a.z, a.heads, a.N, qtiles,
-      (int)items, a.work_ctr, a.scale_log2, a.eps, a.status, a.wait_limit_ns, a.mask_per_bh, a.tiles);
+      (int)items, a.work_ctr, a.scale_log2, a.eps, a.status, a.wait_limit_ns, a.mask_per_bh, a.tiles, a.lse);
   return cudaGetLastError();
 }
 

@@ -92,6 +92,7 @@ struct AttnArgs {
   int max_ctas;               // cap on the persistent grid (0: one CTA per SM)
   int mask_per_bh;            // mask rows are (b*Hh + h, I) instead of (h, I)
   TileGeom tiles;             // tiles.bt > 0: blocks are 3-D boxes (block == 128), maps are 4-D
+  float* lse;                 // fp32 [B*Hh][N]: each row's log-sum-exp of the sparse softmax, or nullptr
   int B, N, heads, d, block;
   float scale_log2;  // softmax scale * log2(e)
   float eps;

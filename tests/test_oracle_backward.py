@@ -113,3 +113,18 @@ def test_gate_zero_invariants():
     np.testing.assert_allclose(got["dv"].sum(axis=1), dout.sum(axis=1), rtol=0, atol=1e-10)
     # the gate's gradient is the derivative at g = 0, which the branch still has
     assert np.all(np.abs(got["dgate"]) > 0)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(d=32, block=16, window=(1, 2, 3), seed=12), dict(window=(2, 3, 7), seed=14)])
+def test_lse_is_the_masked_logsumexp(kw):
+    from scipy.special import logsumexp
+    wl = wl_(**kw)
+    inp = si.make_inputs(wl)
+    rp, ci = oracle.block_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)
+    got = oracle.lse(inp.q, inp.k, wl.block, rp, ci)
+    q = si.bf16_bits_to_f32(inp.q).astype(np.float64)
+    k = si.bf16_bits_to_f32(inp.k).astype(np.float64)
+    s = np.einsum("bihd,bjhd->bhij", q, k) / np.sqrt(wl.d)
+    mask = brute_token_mask(wl.T, wl.H, wl.W, wl.block, inp.windows)[None]
+    ref = logsumexp(np.where(mask, s, -np.inf), axis=-1)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
