@@ -165,3 +165,62 @@ def test_forward_bh_argument_errors(L):
                                        p(FAKE), p(FAKE), 0.0, 1e-6, p(a["out"]), p(0x40000000), 1 << 30, None)
     assert fwd(q=0) == sl.SALAD_ERR_INVALID_ARG
     assert fwd(out=FAKE) == sl.SALAD_ERR_INVALID_ARG
+
+
+def test_tile_blocks_argument_errors(L):
+    import numpy as np
+    nb = ctypes.c_int(0)
+    assert L.salad_tile_num_blocks(21, 30, 52, 1, 32, 4, ctypes.byref(nb)) == 0 and nb.value == 273
+    assert L.salad_tile_num_blocks(21, 30, 52, 1, 16, 8, ctypes.byref(nb)) == 0 and nb.value == 294
+    # bt = 2 does not divide T = 21
+    assert L.salad_tile_num_blocks(21, 30, 52, 2, 8, 8, ctypes.byref(nb)) == sl.SALAD_ERR_UNSUPPORTED
+    assert L.salad_tile_num_blocks(0, 30, 52, 1, 8, 16, ctypes.byref(nb)) == sl.SALAD_ERR_INVALID_ARG
+    assert L.salad_tile_num_blocks(21, 30, 52, 1, 0, 16, ctypes.byref(nb)) == sl.SALAD_ERR_INVALID_ARG
+    assert L.salad_tile_num_blocks(21, 30, 52, 1, 8, 16, None) == sl.SALAD_ERR_INVALID_ARG
+    win = np.array([[1, -2, 4]], dtype=np.int32)
+    assert L.salad_build_tile_mask(4, 8, 8, 1, 8, 16, 1, win.ctypes.data_as(ctypes.c_void_p), p(FAKE), None, 0,
+                                   None, None) == sl.SALAD_ERR_INVALID_ARG  # negative window
+    win = np.array([[1, 2, 4]], dtype=np.int32)
+    assert L.salad_build_tile_mask(5, 8, 8, 2, 8, 8, 1, win.ctypes.data_as(ctypes.c_void_p), p(FAKE), None, 0,
+                                   None, None) == sl.SALAD_ERR_UNSUPPORTED
+
+    def fwd(T=4, H=16, W=16, bt=1, bh=8, bw=16, q=FAKE):
+        return L.salad_attn_forward_tiles(p(q), p(FAKE + 0x10000000), p(FAKE + 0x20000000), 1, T, H, W, bt, bh,
+                                          bw, 2, 64, p(FAKE), p(FAKE), p(FAKE), p(FAKE), 0.0, 1e-6,
+                                          p(FAKE + 0x30000000), p(0x40000000), 1 << 30, None)
+    assert fwd(bw=8) == sl.SALAD_ERR_UNSUPPORTED            # 64 slots: a box must fill one 128-row tile
+    assert fwd(T=3, bt=2, bh=8, bw=8) == sl.SALAD_ERR_UNSUPPORTED   # bt does not divide T
+    assert fwd(q=0) == sl.SALAD_ERR_INVALID_ARG
+    assert fwd(q=FAKE + 8) == sl.SALAD_ERR_INVALID_ARG      # misaligned
+
+
+def test_gate_argument_errors(L):
+    def gate(**kw):
+        a = dict(q=FAKE, B=1, N=1000, H=2, d=64, t_emb=FAKE, E=4, w_t=FAKE, w_x=FAKE, beta=FAKE, thr=0.3,
+                 s_out=0, gate_out=FAKE, ws=0x40000000, ws_bytes=1 << 30)
+        a.update(kw)
+        return L.salad_gate_forward(p(a["q"]), a["B"], a["N"], a["H"], a["d"], p(a["t_emb"]), a["E"],
+                                    p(a["w_t"]), p(a["w_x"]), p(a["beta"]), a["thr"], p(a["s_out"]),
+                                    p(a["gate_out"]), p(a["ws"]), a["ws_bytes"], None)
+    assert gate(q=0) == sl.SALAD_ERR_INVALID_ARG
+    assert gate(w_x=0) == sl.SALAD_ERR_INVALID_ARG
+    assert gate(gate_out=0) == sl.SALAD_ERR_INVALID_ARG
+    assert gate(t_emb=0) == sl.SALAD_ERR_INVALID_ARG        # E > 0 needs the embedding and its weights
+    assert gate(E=-1) == sl.SALAD_ERR_INVALID_ARG
+    assert gate(d=96) == sl.SALAD_ERR_UNSUPPORTED
+    assert gate(B=70000) == sl.SALAD_ERR_UNSUPPORTED
+    assert gate(thr=float("nan")) == sl.SALAD_ERR_INVALID_ARG
+    assert gate(q=FAKE + 4) == sl.SALAD_ERR_INVALID_ARG     # q needs 16 bytes
+    assert gate(ws_bytes=16) == sl.SALAD_ERR_WORKSPACE
+    assert L.salad_gate_workspace_bytes(1, 1000, 2, 64) > 0
+    assert L.salad_gate_workspace_bytes(1, 1000, 2, 96) == 0
+
+
+def test_forward_lse_argument_errors(L):
+    def fwd(lse=FAKE + 0x50000000, q=FAKE):
+        return L.salad_attn_forward_lse(p(q), p(FAKE + 0x10000000), p(FAKE + 0x20000000), 1, 256, 2, 64, 64,
+                                        p(FAKE), p(FAKE), p(FAKE), p(FAKE), 0.0, 1e-6, 0, p(FAKE + 0x30000000),
+                                        p(lse), p(0x40000000), 1 << 30, None)
+    assert fwd(lse=0) == sl.SALAD_ERR_INVALID_ARG
+    assert fwd(lse=FAKE + 0x50000002) == sl.SALAD_ERR_INVALID_ARG   # misaligned
+    assert fwd(q=0) == sl.SALAD_ERR_INVALID_ARG
