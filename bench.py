@@ -658,7 +658,8 @@ def run_salad(args, wl):
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {**config_of(wl, flops, nnz, world), **(gate_desc or {})},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (3 + (2 if wl.topk else 0) + (2 if wl.itads else 0)) * K,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": (3 + (2 if wl.topk else 0) + (2 if wl.itads else 0)) * K,
                 "clocks": clocks.summary(), "kernels": kernels, "dense": dense,
                 "wall_ms_per_step_incl_flush": round(1e3 * wall / K, 4),
                 "frac_of_bf16_peak_layer": round(value / world / peak, 4),

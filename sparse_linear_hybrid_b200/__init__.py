@@ -7,8 +7,8 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, tile_num_blocks, build_tile_mask, workspace_bytes, attn_forward,
-    attn_forward_lse, attn_forward_tiles, attn_forward_static, gate_forward, linear_state, check_status, set_wait_limit_ns,
-    set_max_ctas, set_phase_events, status_string
+    attn_forward_lse, attn_forward_tiles, attn_forward_static, gate_forward, build_topk_mask, linear_state,
+    check_status, set_wait_limit_ns, set_max_ctas, set_phase_events, status_string
 """
 from __future__ import annotations
 

@@ -115,7 +115,8 @@ def test_gate_zero_invariants():
     assert np.all(np.abs(got["dgate"]) > 0)
 
 
-@pytest.mark.parametrize("kw", [dict(), dict(d=32, block=16, window=(1, 2, 3), seed=12), dict(window=(2, 3, 7), seed=14)])
+@pytest.mark.parametrize("kw", [dict(), dict(d=32, block=16, window=(1, 2, 3), seed=12),
+                                dict(window=(2, 3, 7), seed=14)])
 def test_lse_is_the_masked_logsumexp(kw):
     from scipy.special import logsumexp
     wl = wl_(**kw)
