@@ -46,10 +46,10 @@ FLUSH_BYTES = 256 << 20
 # from an ncu capture (see profiles/), keyed by the kernel sources it was taken
 # on; stale entries are ignored.
 NCU_TRAFFIC = {
-    "wan1.3b-32760tok-90pct": {"source": "008b196b7ef807a2", "bytes": 303_186_176 + 84_460_544},
-    "wan1.3b-32760tok-tiles1x32x4": {"source": "008b196b7ef807a2", "bytes": 303_293_952 + 85_079_296},
-    "wan1.3b-32760tok-topk26": {"source": "008b196b7ef807a2", "bytes": 304_376_320 + 84_819_200},
-    "wan1.3b-32760tok-90pct-itads": {"source": "008b196b7ef807a2", "bytes": 303_038_976 + 83_953_408},
+    "wan1.3b-32760tok-90pct": {"source": "613b0b110525a10e", "bytes": 303_341_568 + 84_111_616},
+    "wan1.3b-32760tok-tiles1x32x4": {"source": "613b0b110525a10e", "bytes": 303_325_440 + 83_893_248},
+    "wan1.3b-32760tok-topk26": {"source": "613b0b110525a10e", "bytes": 303_766_528 + 85_206_528},
+    "wan1.3b-32760tok-90pct-itads": {"source": "613b0b110525a10e", "bytes": 303_142_144 + 84_182_272},
 }
 
 
