@@ -162,6 +162,40 @@ int salad_attn_forward_lse(const void* q, const void* k, const void* v, int B, i
                            void* workspace, size_t workspace_bytes, salad_stream_t stream);
 
 /*
+ * Backward pass of the sparse branch (block-sparse softmax attention over the
+ * kept key blocks), for training through the layer (the SALAD summary,
+ * section 3, fine-tunes the model with the layer in place).  With
+ * p_ij = exp(scale q_i.k_j - lse_i) over the kept keys of i and o_i the branch
+ * output (out of salad_attn_forward_lse when every gate is 0):
+ *   D_i = dout_i . o_i,   ds_ij = p_ij (dout_i . v_j - D_i)
+ *   dq_i = scale sum_j ds_ij k_j,  dk_j = scale sum_i ds_ij q_i,  dv_j = sum_i p_ij dout_i
+ *   q, k, v, o, dout  DEVICE bf16 [B][N][Hh][d], 16-byte aligned; d = 64 or 128.
+ *   lse        DEVICE fp32 [B][Hh][N] from salad_attn_forward_lse (natural log).
+ *   block      128 (raster blocks).
+ *   row_ptr, col_idx      the mask the forward used (rows per head, or per
+ *                         (b, h) when mask_per_bh != 0).
+ *   t_row_ptr, t_col_idx  its transpose with the same row numbering: row
+ *                         (h or b*Hh+h, J) lists, ascending, the query blocks
+ *                         whose rows keep key block J.  The window masks of
+ *                         salad_build_block_mask are symmetric: pass the same
+ *                         arrays.
+ *   softmax_scale  <= 0 selects 1/sqrt(d) (as in the forward).
+ *   dq, dk, dv DEVICE fp32 [B][N][Hh][d], 16-byte aligned.
+ *   workspace  DEVICE, >= salad_backward_workspace_bytes(B, N, Hh), 256-byte
+ *              aligned; its first word is a status word like the forward's
+ *              (zero it once after allocation; read it with salad_check_status).
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation (P and dS are
+ * rounded to bf16 as operands), fp32 elsewhere.  Never synchronises.
+ * Errors: INVALID_ARG, UNSUPPORTED (d, block), WORKSPACE, CUDA.
+ */
+size_t salad_backward_workspace_bytes(int B, int N, int num_heads);
+int salad_attn_backward_sparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                               const float* lse, int B, int N, int num_heads, int d, int block,
+                               const int32_t* row_ptr, const int32_t* col_idx, const int32_t* t_row_ptr,
+                               const int32_t* t_col_idx, int mask_per_bh, float softmax_scale, float* dq, float* dk,
+                               float* dv, void* workspace, size_t workspace_bytes, salad_stream_t stream);
+
+/*
  * Top-K dynamic block mask.  The SALAD summary (section 5) says the method also
  * applies to Top-K dynamic sparse attention and gives no scoring rule; the rule
  * implemented here is a reading of that sentence:

@@ -7,7 +7,7 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, tile_num_blocks, build_tile_mask, workspace_bytes, attn_forward,
-    attn_forward_lse, attn_forward_tiles, attn_forward_static, gate_forward, build_topk_mask, linear_state,
+    attn_forward_lse, attn_backward_sparse, attn_forward_tiles, attn_forward_static, gate_forward, build_topk_mask, linear_state,
     check_status, set_wait_limit_ns, set_max_ctas, set_phase_events, status_string
 """
 from __future__ import annotations
@@ -64,6 +64,11 @@ def lib() -> ctypes.CDLL:
         L.salad_attn_forward_bh.restype = i
         L.salad_attn_forward_lse.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, i, p, p, p, sz, p]
         L.salad_attn_forward_lse.restype = i
+        L.salad_backward_workspace_bytes.argtypes = [i, i, i]
+        L.salad_backward_workspace_bytes.restype = sz
+        L.salad_attn_backward_sparse.argtypes = [p, p, p, p, p, p, i, i, i, i, i, p, p, p, p, i, f, p, p, p, p, sz,
+                                                 p]
+        L.salad_attn_backward_sparse.restype = i
         L.salad_attn_forward_tiles.argtypes = [p, p, p, i, i, i, i, i, i, i, i, i, p, p, p, p, f, f, p, p, sz,
                                                p]
         L.salad_attn_forward_tiles.restype = i
@@ -225,6 +230,30 @@ def attn_forward_lse(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softma
         _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(lse, torch.float32, "lse"),
         _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "salad_attn_forward_lse")
     return out, lse
+
+
+def attn_backward_sparse(q, k, v, o, dout, lse, row_ptr, col_idx, block: int = 128, t_row_ptr=None,
+                         t_col_idx=None, softmax_scale: float = 0.0, mask_per_bh: bool = False, workspace=None,
+                         stream=None):
+    """Gradients of the sparse branch (see salad.h): (dq, dk, dv) fp32 [B, N, Hh, d].
+    o is the branch output and lse the forward's log-sum-exp (attn_forward_lse);
+    the transposed mask defaults to the mask itself (window masks are symmetric)."""
+    B, N, Hh, d = q.shape
+    t_row_ptr = row_ptr if t_row_ptr is None else t_row_ptr
+    t_col_idx = col_idx if t_col_idx is None else t_col_idx
+    grads = [torch.empty(B, N, Hh, d, dtype=torch.float32, device=q.device) for _ in range(3)]
+    if workspace is None:
+        workspace = torch.zeros(lib().salad_backward_workspace_bytes(B, N, Hh), dtype=torch.uint8, device=q.device)
+    i32 = lambda t, name: _dev_ptr(t, torch.int32, name)  # noqa: E731
+    _check(lib().salad_attn_backward_sparse(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
+        _dev_ptr(o, torch.bfloat16, "o"), _dev_ptr(dout, torch.bfloat16, "dout"), _dev_ptr(lse, torch.float32, "lse"),
+        B, N, Hh, d, int(block), i32(row_ptr, "row_ptr"), i32(col_idx, "col_idx"), i32(t_row_ptr, "t_row_ptr"),
+        i32(t_col_idx, "t_col_idx"), int(bool(mask_per_bh)), float(softmax_scale),
+        *[_dev_ptr(g, torch.float32, n) for g, n in zip(grads, ("dq", "dk", "dv"))],
+        _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "salad_attn_backward_sparse")
+    return tuple(grads)
 
 
 def attn_forward_tiles(q, k, v, grid, tile, row_ptr, col_idx, w_proj, gate, softmax_scale: float = 0.0,

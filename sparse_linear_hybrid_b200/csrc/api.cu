@@ -309,6 +309,68 @@ int salad_attn_forward_lse(const void* q, const void* k, const void* v, int B, i
                            out, workspace, workspace_bytes, stream, mask_per_bh ? 1 : 0, nullptr, lse);
 }
 
+size_t salad_backward_workspace_bytes(int B, int N, int num_heads) {
+  if (B < 1 || N < 1 || num_heads < 1) return 0;
+  const size_t npad = ((size_t)N + 127) / 128 * 128;
+  return 256 + 2 * (size_t)B * num_heads * npad * sizeof(float);
+}
+
+int salad_attn_backward_sparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                               const float* lse, int B, int N, int num_heads, int d, int block,
+                               const int32_t* row_ptr, const int32_t* col_idx, const int32_t* t_row_ptr,
+                               const int32_t* t_col_idx, int mask_per_bh, float softmax_scale, float* dq, float* dk,
+                               float* dv, void* workspace, size_t workspace_bytes, salad_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !t_row_ptr || !t_col_idx || !dq || !dk ||
+      !dv || !workspace)
+    return SALAD_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || num_heads < 1) return SALAD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
+  if (block != 128) return SALAD_ERR_UNSUPPORTED;
+  if (num_heads > 65535 || (long long)B * num_heads * ((N + 127) / 128) >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
+  const void* p16[] = {q, k, v, o, dout, dq, dk, dv, workspace};
+  for (const void* ptr : p16)
+    if (!aligned(ptr, 16)) return SALAD_ERR_INVALID_ARG;
+  if (!aligned(lse, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(t_row_ptr, 4) ||
+      !aligned(t_col_idx, 4))
+    return SALAD_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return SALAD_ERR_INVALID_ARG;
+  if (workspace_bytes < salad_backward_workspace_bytes(B, N, num_heads)) return SALAD_ERR_WORKSPACE;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_bnhd_map(&tq, q, B, N, num_heads, d, 128) || !make_bnhd_map(&tk, k, B, N, num_heads, d, 128) ||
+      !make_bnhd_map(&tv, v, B, N, num_heads, d, 128) || !make_bnhd_map(&tdo, dout, B, N, num_heads, d, 128))
+    return SALAD_ERR_CUDA;
+  BwdArgs ba{};
+  ba.tm_q = &tq;
+  ba.tm_k = &tk;
+  ba.tm_v = &tv;
+  ba.tm_do = &tdo;
+  ba.o = static_cast<const uint16_t*>(o);
+  ba.dout = static_cast<const uint16_t*>(dout);
+  ba.lse = lse;
+  ba.row_ptr = row_ptr;
+  ba.col_idx = col_idx;
+  ba.t_row_ptr = t_row_ptr;
+  ba.t_col_idx = t_col_idx;
+  ba.B = B;
+  ba.N = N;
+  ba.heads = num_heads;
+  ba.d = d;
+  ba.nb = (N + 127) / 128;
+  ba.npad = ba.nb * 128;
+  ba.mask_per_bh = mask_per_bh ? 1 : 0;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  ba.status = reinterpret_cast<uint32_t*>(ws);
+  ba.lse2 = reinterpret_cast<float*>(ws + 256);
+  ba.dvec = ba.lse2 + (size_t)B * num_heads * ba.npad;
+  ba.dq = dq;
+  ba.dk = dk;
+  ba.dv = dv;
+  ba.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)d);
+  ba.scale_log2 = ba.scale * 1.4426950408889634f;
+  ba.wait_limit_ns = g_wait_limit_ns.load();
+  return launch_backward(ba, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
+}
+
 int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B, int T, int H, int W, int bt,
                              int bh, int bw, int num_heads, int d, const int32_t* row_ptr, const int32_t* col_idx,
                              const void* w_proj, const float* gate, float softmax_scale, float eps, void* out,

@@ -1,0 +1,519 @@
+// Backward pass of the sparse branch (block-sparse softmax attention over the
+// kept key blocks; the fine-tuning of the SALAD summary, section 3, trains
+// through it).  With p_ij = exp(scale q_i.k_j - lse_i) over the kept keys,
+// the row log-sum-exp lse_i kept by the forward, and o_i the branch output:
+//   D_i   = dout_i . o_i
+//   dp_ij = dout_i . v_j,      ds_ij = p_ij (dp_ij - D_i)
+//   dq_i  = scale sum_j ds_ij k_j
+//   dk_j  = scale sum_i ds_ij q_i,      dv_j = sum_i p_ij dout_i
+// Three kernels (raster blocks of 128 tokens):
+//   bwd_prep_kernel  D_i and lse_i in base 2 (lse * log2 e) into the workspace,
+//                    rows padded to whole 128-row tiles (pad rows: p = 0, D = 0)
+//   bwd_dq_kernel    one CTA per (query tile, b, h), over its kept key tiles:
+//                    S = Q K^T and dP = dO V^T on the tensor cores (SS form),
+//                    one thread per row forms dS = P (dP - D) into tensor
+//                    memory as bf16, and dQ += dS K (A from tensor memory, K
+//                    as an MN-major B operand)
+//   bwd_dkdv_kernel  one CTA per (key tile, b, h), over the query tiles whose
+//                    rows keep it (the transposed mask): S^T = K Q^T and
+//                    dP^T = V dO^T, one thread per key row forms P^T and dS^T
+//                    (bf16, written over the columns of S^T and dP^T it has
+//                    read), dV += P^T dO and dK += dS^T Q
+// Warp roles, 192 threads: warp 0 lane 0 issues the TMA loads and the MMAs in
+// program order (K/V or Q/dO tiles in a 2-deep ring), warp 1 owns the tensor
+// memory, warps 2-5 take one row each (TMEM lane quarter = warp % 4).  Every
+// barrier wait is bounded; on a time-out the kernel records it and drains.
+// Gradients are written in fp32.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace salad {
+namespace {
+
+constexpr int kBwdThreads = 192;
+constexpr uint64_t kBwdDrainNs = 1000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdShared {
+  uint64_t fixed_full;    // the CTA's fixed tiles (Q and dO, or K and V)
+  uint64_t ring_full[2];  // the streamed tiles (K and V, or Q, dO and the row vectors)
+  uint64_t sdp_full;      // S and dP of the current tile are in tensor memory
+  uint64_t ds_full;       // the four row warps have written dS (and P^T) of the tile
+  uint64_t mm_done;       // the gradient products of the tile have completed
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int DCH = D / 64;
+  static constexpr int TILE = 128 * D * 2;  // one 128-row tile of q, k, v or dout (DCH boxes of 16 KB)
+  static constexpr int VEC = 2 * 128 * 4;   // lse2 and D of 128 rows
+  static constexpr int OFF_FIX = 0;         // two fixed tiles
+  static constexpr int OFF_RING = 2 * TILE; // two stages of two tiles
+  static constexpr int OFF_VEC = 6 * TILE;  // two stages of row vectors (dK/dV kernel)
+  static constexpr int OFF_BAR = OFF_VEC + 2 * VEC;
+  static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(BwdShared) + 1024;
+  // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
+  static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
+  static constexpr uint32_t IDESC_SS = idesc_bf16(128, 128, false, false);  // X Y^T, both K-major
+  static constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);      // A (tmem) x B (MN-major)
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// 128 x 128 product X Y^T of two K-major 128 x D tiles in shared memory.
+template <int D>
+__device__ __forceinline__ void mma_xyt(uint32_t d_tmem, uint32_t x, uint32_t y) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+    mma_bf16_ss(d_tmem, sw128_desc(x + off, 16, 1024), sw128_desc(y + off, 16, 1024), BwdCfg<D>::IDESC_SS,
+                kk > 0 ? 1u : 0u);
+  }
+}
+
+// D += A B with A = 128 x 128 bf16 in tensor memory (columns a_tmem ...), B a
+// 128 x D tile in shared memory read as an MN-major operand.
+template <int D>
+__device__ __forceinline__ void mma_grad(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b + kk * 2048, 16384, 1024), BwdCfg<D>::IDESC_G,
+                (accumulate || kk > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ void bwd_timeout(BwdShared* sh, uint32_t* status) {
+  sh->abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
+}
+
+// D_i and lse_i * log2 e per row, into [B*Hh][Npad] (pad rows: lse2 = +inf, D = 0).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                                                       const float* __restrict__ lse, int B, int N, int heads,
+                                                       int npad, float* __restrict__ lse2, float* __restrict__ dvec) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (long long)B * heads * npad) return;
+  const int bh = (int)(t / npad), n = (int)(t % npad), b = bh / heads, h = bh % heads;
+  if (n >= N) {
+    lse2[t] = INFINITY;
+    dvec[t] = 0.f;
+    return;
+  }
+  const uint4* po = reinterpret_cast<const uint4*>(o + (((size_t)b * N + n) * heads + h) * D);
+  const uint4* pd = reinterpret_cast<const uint4*>(dout + (((size_t)b * N + n) * heads + h) * D);
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 x = po[c], y = pd[c];
+    const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(bf16_lo_to_f32(xa[i]), bf16_lo_to_f32(ya[i]), acc);
+      acc = fmaf(bf16_hi_to_f32(xa[i]), bf16_hi_to_f32(ya[i]), acc);
+    }
+  }
+  dvec[t] = acc;
+  lse2[t] = lse[(size_t)bh * N + n] * kLog2e;
+}
+
+// ------------------------------------------------------------------ dQ
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                  const float* __restrict__ lse2, const float* __restrict__ dvec, float* __restrict__ dq, int N,
+                  int heads, int nb, int npad, int mask_per_bh, float scale, float scale_log2, uint32_t* status,
+                  uint64_t limit_ns) {
+  using C = BwdCfg<D>;
+  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 384;
+  extern __shared__ uint8_t bwd_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~uintptr_t(1023));
+  BwdShared* sh = reinterpret_cast<BwdShared*>(smem + C::OFF_BAR);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x % nb, bh = blockIdx.x / nb, b = bh / heads, h = bh % heads;
+  const int mrow = (mask_per_bh ? bh : h) * nb + qt;
+  const int c0 = row_ptr[mrow], n = row_ptr[mrow + 1] - c0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh->fixed_full, 1);
+    mbar_init(&sh->ring_full[0], 1);
+    mbar_init(&sh->ring_full[1], 1);
+    mbar_init(&sh->sdp_full, 1);
+    mbar_init(&sh->ds_full, 4);
+    mbar_init(&sh->mm_done, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const uint32_t q_s = sbase + C::OFF_FIX, do_s = q_s + C::TILE;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int loads = 0;  // ring loads issued
+      auto load_kv = [&](int j) {
+        const int s = j & 1, col = col_idx[c0 + j];
+        uint8_t* dst = smem + C::OFF_RING + s * 2 * C::TILE;
+        mbar_arrive_expect_tx(&sh->ring_full[s], 2 * C::TILE);
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch) {
+          tma_load_3d(dst + ch * 16384, &tm_k, &sh->ring_full[s], h * D + ch * 64, col * 128, b);
+          tma_load_3d(dst + C::TILE + ch * 16384, &tm_v, &sh->ring_full[s], h * D + ch * 64, col * 128, b);
+        }
+        ++loads;
+      };
+      mbar_arrive_expect_tx(&sh->fixed_full, 2 * C::TILE);
+#pragma unroll
+      for (int ch = 0; ch < C::DCH; ++ch) {
+        tma_load_3d(smem + C::OFF_FIX + ch * 16384, &tm_q, &sh->fixed_full, h * D + ch * 64, qt * 128, b);
+        tma_load_3d(smem + C::OFF_FIX + C::TILE + ch * 16384, &tm_do, &sh->fixed_full, h * D + ch * 64, qt * 128,
+                    b);
+      }
+      for (int j = 0; j < n && j < 2; ++j) load_kv(j);
+      ok = mbar_wait(&sh->fixed_full, 0, limit_ns);
+      if (ok && n >= 1) {
+        ok = mbar_wait(&sh->ring_full[0], 0, limit_ns);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t kt = sbase + C::OFF_RING;
+          mma_xyt<D>(tmem + TM_S, q_s, kt);
+          mma_xyt<D>(tmem + TM_DP, do_s, kt + C::TILE);
+          mma_commit(&sh->sdp_full);
+        }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int s = j & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->ds_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        mma_grad<D>(tmem + TM_DQ, tmem + TM_DS, sbase + C::OFF_RING + s * 2 * C::TILE, j > 0);
+        mma_commit(&sh->mm_done);
+        if (j + 1 < n) {
+          const int s1 = (j + 1) & 1;
+          if (!mbar_wait(&sh->ring_full[s1], (uint32_t)(((j + 1) >> 1) & 1), limit_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kt = sbase + C::OFF_RING + s1 * 2 * C::TILE;
+          mma_xyt<D>(tmem + TM_S, q_s, kt);
+          mma_xyt<D>(tmem + TM_DP, do_s, kt + C::TILE);
+          mma_commit(&sh->sdp_full);
+        }
+        if (j + 2 < n) {
+          // stage s is free once the dQ product of tile j has read its K
+          if (!mbar_wait(&sh->mm_done, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+          load_kv(j + 2);
+        }
+      }
+      if (!ok) {
+        bwd_timeout(sh, status);
+        mma_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0, kBwdDrainNs);
+      }
+      // every copy this thread started lands before the CTA exits
+      mbar_wait(&sh->fixed_full, 0, kBwdDrainNs);
+      for (int i = (loads > 2 ? loads - 2 : 0); i < loads; ++i)
+        mbar_wait(&sh->ring_full[i & 1], (uint32_t)((i >> 1) & 1), kBwdDrainNs);
+    }
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------- one thread per query row
+    const int quarter = warp & 3, r = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float l2 = lse2[(size_t)bh * npad + qt * 128 + r];
+    const float Dr = dvec[(size_t)bh * npad + qt * 128 + r];
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int valid = min(128, N - col_idx[c0 + j] * 128);  // real keys of the tile
+      if (!mbar_wait_warp(&sh->sdp_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+      // (S and dP of tile j were committed after the dQ product of tile j - 1, so
+      // that product, the last reader of the dS columns, has completed too)
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32], pr[32], dsp[16];
+        tmem_ld32(lane_addr + TM_S + c * 32, sr);
+        tmem_ld32(lane_addr + TM_DP + c * 32, pr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k0 = c * 32 + 2 * i;
+          const float p0 = k0 < valid ? ex2_approx(__uint_as_float(sr[2 * i]) * scale_log2 - l2) : 0.f;
+          const float p1 = k0 + 1 < valid ? ex2_approx(__uint_as_float(sr[2 * i + 1]) * scale_log2 - l2) : 0.f;
+          dsp[i] = pack_bf16x2(p0 * (__uint_as_float(pr[2 * i]) - Dr), p1 * (__uint_as_float(pr[2 * i + 1]) - Dr));
+        }
+        tmem_st16(lane_addr + TM_DS + c * 16, dsp);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->ds_full);
+    }
+    if (ok && n >= 1) ok = mbar_wait_warp(&sh->mm_done, (uint32_t)((n - 1) & 1), limit_ns);
+    if (!ok) {
+      bwd_timeout(sh, status);
+    } else {
+      tc_fence_after();
+      const int row = qt * 128 + r;
+      float* dst = dq + (((size_t)b * N + row) * heads + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t g[32];
+        if (n >= 1) {
+          tmem_ld32(lane_addr + TM_DQ + c * 32, g);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) g[i] = 0u;
+        }
+        if (row < N) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + c * 32 + i) =
+                make_float4(__uint_as_float(g[i]) * scale, __uint_as_float(g[i + 1]) * scale,
+                            __uint_as_float(g[i + 2]) * scale, __uint_as_float(g[i + 3]) * scale);
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ dK, dV
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const int32_t* __restrict__ t_row_ptr, const int32_t* __restrict__ t_col_idx,
+                    const float* __restrict__ lse2, const float* __restrict__ dvec, float* __restrict__ dk,
+                    float* __restrict__ dv, int N, int heads, int nb, int npad, int mask_per_bh, float scale,
+                    float scale_log2, uint32_t* status, uint64_t limit_ns) {
+  using C = BwdCfg<D>;
+  // S^T [0,128) (P^T as bf16 over its first 64 columns), dP^T [128,256) (dS^T
+  // over its first 64), dV [256,256+D), dK [384,384+D)
+  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 384;
+  extern __shared__ uint8_t bwd_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~uintptr_t(1023));
+  BwdShared* sh = reinterpret_cast<BwdShared*>(smem + C::OFF_BAR);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x % nb, bh = blockIdx.x / nb, b = bh / heads, h = bh % heads;
+  const int mrow = (mask_per_bh ? bh : h) * nb + kt;
+  const int c0 = t_row_ptr[mrow], n = t_row_ptr[mrow + 1] - c0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh->fixed_full, 1);
+    mbar_init(&sh->ring_full[0], 1);
+    mbar_init(&sh->ring_full[1], 1);
+    mbar_init(&sh->sdp_full, 1);
+    mbar_init(&sh->ds_full, 4);
+    mbar_init(&sh->mm_done, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const uint32_t k_s = sbase + C::OFF_FIX, v_s = k_s + C::TILE;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int loads = 0;
+      auto load_q = [&](int j) {
+        const int s = j & 1, qi = t_col_idx[c0 + j];
+        uint8_t* dst = smem + C::OFF_RING + s * 2 * C::TILE;
+        float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC + s * C::VEC);
+        mbar_arrive_expect_tx(&sh->ring_full[s], 2 * C::TILE + C::VEC);
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch) {
+          tma_load_3d(dst + ch * 16384, &tm_q, &sh->ring_full[s], h * D + ch * 64, qi * 128, b);
+          tma_load_3d(dst + C::TILE + ch * 16384, &tm_do, &sh->ring_full[s], h * D + ch * 64, qi * 128, b);
+        }
+        bulk_load(vec, lse2 + (size_t)bh * npad + qi * 128, 512, &sh->ring_full[s]);
+        bulk_load(vec + 128, dvec + (size_t)bh * npad + qi * 128, 512, &sh->ring_full[s]);
+        ++loads;
+      };
+      mbar_arrive_expect_tx(&sh->fixed_full, 2 * C::TILE);
+#pragma unroll
+      for (int ch = 0; ch < C::DCH; ++ch) {
+        tma_load_3d(smem + C::OFF_FIX + ch * 16384, &tm_k, &sh->fixed_full, h * D + ch * 64, kt * 128, b);
+        tma_load_3d(smem + C::OFF_FIX + C::TILE + ch * 16384, &tm_v, &sh->fixed_full, h * D + ch * 64, kt * 128, b);
+      }
+      for (int j = 0; j < n && j < 2; ++j) load_q(j);
+      ok = mbar_wait(&sh->fixed_full, 0, limit_ns);
+      if (ok && n >= 1) {
+        ok = mbar_wait(&sh->ring_full[0], 0, limit_ns);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t qs = sbase + C::OFF_RING;
+          mma_xyt<D>(tmem + TM_S, k_s, qs);
+          mma_xyt<D>(tmem + TM_DP, v_s, qs + C::TILE);
+          mma_commit(&sh->sdp_full);
+        }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int s = j & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->ds_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qs = sbase + C::OFF_RING + s * 2 * C::TILE;
+        mma_grad<D>(tmem + TM_DV, tmem + TM_S, qs + C::TILE, j > 0);  // dV += P^T dO
+        mma_grad<D>(tmem + TM_DK, tmem + TM_DP, qs, j > 0);          // dK += dS^T Q
+        mma_commit(&sh->mm_done);
+        if (j + 1 < n) {
+          // S^T and dP^T of the next tile overwrite P^T and dS^T: issued after
+          // the products that read them, which the tensor cores run in order
+          const int s1 = (j + 1) & 1;
+          if (!mbar_wait(&sh->ring_full[s1], (uint32_t)(((j + 1) >> 1) & 1), limit_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qn = sbase + C::OFF_RING + s1 * 2 * C::TILE;
+          mma_xyt<D>(tmem + TM_S, k_s, qn);
+          mma_xyt<D>(tmem + TM_DP, v_s, qn + C::TILE);
+          mma_commit(&sh->sdp_full);
+        }
+        if (j + 2 < n) {
+          if (!mbar_wait(&sh->mm_done, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+          load_q(j + 2);
+        }
+      }
+      if (!ok) {
+        bwd_timeout(sh, status);
+        mma_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0, kBwdDrainNs);
+      }
+      mbar_wait(&sh->fixed_full, 0, kBwdDrainNs);
+      for (int i = (loads > 2 ? loads - 2 : 0); i < loads; ++i)
+        mbar_wait(&sh->ring_full[i & 1], (uint32_t)((i >> 1) & 1), kBwdDrainNs);
+    }
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------- one thread per key row
+    const int quarter = warp & 3, r = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait_warp(&sh->sdp_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+      // the row vectors of this query tile landed with its tiles (ring_full of stage s)
+      if (!mbar_wait_warp(&sh->ring_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
+      tc_fence_after();
+      const float* l2v = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * C::VEC);
+      const float* dvv = l2v + 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32], pr[32];
+        tmem_ld32(lane_addr + TM_S + c * 32, sr);
+        tmem_ld32(lane_addr + TM_DP + c * 32, pr);
+        tmem_ld_wait();
+        uint32_t pp[16], dsp[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int q0 = c * 32 + 2 * i;
+          const float p0 = ex2_approx(__uint_as_float(sr[2 * i]) * scale_log2 - l2v[q0]);
+          const float p1 = ex2_approx(__uint_as_float(sr[2 * i + 1]) * scale_log2 - l2v[q0 + 1]);
+          pp[i] = pack_bf16x2(p0, p1);
+          dsp[i] = pack_bf16x2(p0 * (__uint_as_float(pr[2 * i]) - dvv[q0]),
+                               p1 * (__uint_as_float(pr[2 * i + 1]) - dvv[q0 + 1]));
+        }
+        // columns [16c, 16c + 16) of each region: already read by this thread
+        tmem_st16(lane_addr + TM_S + c * 16, pp);
+        tmem_st16(lane_addr + TM_DP + c * 16, dsp);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->ds_full);
+    }
+    if (ok && n >= 1) ok = mbar_wait_warp(&sh->mm_done, (uint32_t)((n - 1) & 1), limit_ns);
+    if (!ok) {
+      bwd_timeout(sh, status);
+    } else {
+      tc_fence_after();
+      const int row = kt * 128 + r;
+      const size_t off = (((size_t)b * N + row) * heads + h) * D;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float* dst = (part == 0 ? dv : dk) + off;
+        const float mul = part == 0 ? 1.f : scale;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t g[32];
+          if (n >= 1) {
+            tmem_ld32(lane_addr + (part == 0 ? TM_DV : TM_DK) + c * 32, g);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) g[i] = 0u;
+          }
+          if (row < N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + c * 32 + i) =
+                  make_float4(__uint_as_float(g[i]) * mul, __uint_as_float(g[i + 1]) * mul,
+                              __uint_as_float(g[i + 2]) * mul, __uint_as_float(g[i + 3]) * mul);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t s) {
+  using C = BwdCfg<D>;
+  const long long rows = (long long)a.B * a.heads * a.npad;
+  bwd_prep_kernel<D><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(a.o, a.dout, a.lse, a.B, a.N, a.heads, a.npad,
+                                                                   a.lse2, a.dvec);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int grid = a.B * a.heads * a.nb;
+  e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<D><<<grid, kBwdThreads, C::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.row_ptr, a.col_idx,
+                                                      a.lse2, a.dvec, a.dq, a.N, a.heads, a.nb, a.npad,
+                                                      a.mask_per_bh, a.scale, a.scale_log2, a.status,
+                                                      a.wait_limit_ns);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  bwd_dkdv_kernel<D><<<grid, kBwdThreads, C::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.t_row_ptr,
+                                                        a.t_col_idx, a.lse2, a.dvec, a.dk, a.dv, a.N, a.heads, a.nb,
+                                                        a.npad, a.mask_per_bh, a.scale, a.scale_log2, a.status,
+                                                        a.wait_limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s) {
+  return a.d == 64 ? launch_bwd_t<64>(a, s) : launch_bwd_t<128>(a, s);
+}
+
+}  // namespace salad

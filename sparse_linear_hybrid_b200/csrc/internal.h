@@ -101,6 +101,23 @@ struct AttnArgs {
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
 
+// Backward pass of the sparse branch (bwd.cu); raster blocks of 128 tokens.
+struct BwdArgs {
+  const CUtensorMap *tm_q, *tm_k, *tm_v, *tm_do;  // box (64, 128, 1)
+  const uint16_t* o;     // bf16 [B][N][Hh][d]: the branch output
+  const uint16_t* dout;  // bf16 [B][N][Hh][d]
+  const float* lse;      // fp32 [B*Hh][N], natural log
+  const int32_t *row_ptr, *col_idx;      // mask rows (query block -> kept key blocks)
+  const int32_t *t_row_ptr, *t_col_idx;  // its transpose (key block -> query blocks that keep it)
+  float *lse2, *dvec;    // workspace: fp32 [B*Hh][npad] each
+  float *dq, *dk, *dv;   // fp32 [B][N][Hh][d]
+  int B, N, heads, d, nb, npad, mask_per_bh;
+  float scale, scale_log2;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s);
+
 // Dynamic gate and branch dropping (gate.cu).
 struct GateArgs {
   const uint16_t* q;  // bf16 [B][N][Hh][d], 16-byte aligned

@@ -1,0 +1,48 @@
+"""The backward pass of the sparse branch on the GPU (salad_attn_backward_sparse)
+against the oracle's backward with every gate 0 (then the layer is the sparse
+branch alone and out is its output): dq, dk and dv within rel-L2 1e-2 and a
+max-abs error of 3e-2 of the largest reference value (bf16 operands P and dS,
+fp32 accumulation; D_i from the bf16 output), at ragged shapes, both head
+widths, a full window and a 9,360-token grid."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import salad_inputs as si
+import sparse_linear_hybrid_b200 as sl
+from parity import upload
+
+pytestmark = pytest.mark.gpu
+
+
+def check(got, ref, name):
+    err = np.abs(got - ref)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert np.all(np.isfinite(got)), name
+    assert rel <= 1e-2 and err.max() <= 3e-2 * np.abs(ref).max(), (name, rel, err.max(), np.abs(ref).max())
+
+
+@pytest.mark.parametrize("B,T,H,W,Hh,d,window", [
+    (1, 2, 8, 16, 2, 64, (1, 2, 3)),        # 256 tokens
+    (2, 3, 9, 13, 2, 128, (1, 3, 4)),       # 351 tokens: ragged last block
+    (1, 3, 9, 13, 1, 64, (2, 8, 12)),       # full window
+    (1, 6, 30, 52, 1, 128, (1, 10, 13)),    # 9,360 tokens
+])
+def test_backward_matches_oracle(B, T, H, W, Hh, d, window):
+    wl = si.Workload("bw", B=B, Hh=Hh, d=d, T=T, H=H, W=W, block=128, window=window, seed=71)
+    inp = si.make_inputs(wl, v_mean=0.5, gate=0.0)
+    t = upload(inp)
+    rng = np.random.default_rng(72)
+    dout_bits = si.f32_to_bf16_bits(rng.standard_normal((B, wl.N, Hh, d), dtype=np.float32))
+    dout = torch.from_numpy(dout_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    rp, ci = sl.build_block_mask(T, H, W, 128, inp.windows)
+    out, lse = sl.attn_forward_lse(t["q"], t["k"], t["v"], rp, ci, t["w"], t["gate"], 128)
+    ws = torch.zeros(sl.lib().salad_backward_workspace_bytes(B, wl.N, Hh), dtype=torch.uint8, device="cuda")
+    dq, dk, dv = sl.attn_backward_sparse(t["q"], t["k"], t["v"], out, dout, lse, rp, ci, workspace=ws)
+    assert sl.check_status(ws) == sl.SALAD_OK
+    orp, oci = oracle.block_mask(T, H, W, 128, inp.windows)
+    ref = oracle.backward(inp.q, inp.k, inp.v, 128, orp, oci, inp.w_proj, inp.gate,
+                          si.bf16_bits_to_f32(dout_bits).astype(np.float64))
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        check(g.cpu().numpy().astype(np.float64), ref[name], name)
