@@ -648,6 +648,38 @@ def run_salad(args, wl):
                  "tflops": round(dflops / (dms / 1e3) / 1e12, 2),
                  "sparse_speedup_vs_dense": round(dms / ms_per_step, 3)}
 
+    # the backward pass of the sparse branch (dq, dk, dv) on this workload's q, k, v:
+    # its output and log-sum-exp from a gate-0 forward, a seeded dout, K timed
+    # steps with the L2 flush between them (not part of the headline step)
+    backward = None
+    if not args.no_backward and not wl.tile and not wl.topk and wl.block == 128:
+        zero_gate = torch.zeros_like(gate)
+        o_sp, lse = sl.attn_forward_lse(q, k, v, row_ptr, col_idx, w, zero_gate, wl.block, workspace=ws)
+        g_bits = si.f32_to_bf16_bits(np.random.default_rng(my_wl.seed + 99).standard_normal(
+            (wl.B, wl.N, wl.Hh, wl.d), dtype=np.float32))
+        dout = up(g_bits)
+        bws = torch.zeros(sl.lib().salad_backward_workspace_bytes(wl.B, wl.N, wl.Hh), dtype=torch.uint8, device=dev)
+        kb = max(3, min(K, 20))
+        bev = [(E(), E()) for _ in range(kb)]
+        for i in range(3 + kb):
+            flush.zero_()
+            if i >= 3:
+                bev[i - 3][0].record()
+            sl.attn_backward_sparse(q, k, v, o_sp, dout, lse, row_ptr, col_idx, workspace=bws)
+            if i >= 3:
+                bev[i - 3][1].record()
+        torch.cuda.synchronize()
+        if sl.check_status(bws) != sl.SALAD_OK:
+            raise RuntimeError("device status after the backward steps")
+        bms = statistics.median(a.elapsed_time(b) for a, b in bev)
+        bflops = 2.5 * flops
+        backward = {"branch": "sparse: dq, dk, dv (salad_attn_backward_sparse, 3 launches)",
+                    "ms_per_step_p50": round(bms, 4), "tflops": round(bflops / (bms / 1e3) / 1e12, 2),
+                    "frac": round(bflops / (bms / 1e3) / 1e12 / peak, 4),
+                    "algorithmic": "2.5 x the forward's kept FLOPs (the S, dP, dV, dK and dQ products; the two "
+                                   "kernels each recompute S and dP, so 3.5 x is executed)", "steps": kb}
+        del o_sp, lse, dout, bws
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, desc, _, _ = oracle_sample_rate(wl, inp, rp_h, ci_h, budget_s=args.cpu_seconds)
@@ -660,7 +692,7 @@ def run_salad(args, wl):
                 "config": {**config_of(wl, flops, nnz, world), **(gate_desc or {})},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": (3 + (2 if wl.topk else 0) + (2 if wl.itads else 0)) * K,
-                "clocks": clocks.summary(), "kernels": kernels, "dense": dense,
+                "clocks": clocks.summary(), "kernels": kernels, "dense": dense, "backward": backward,
                 "wall_ms_per_step_incl_flush": round(1e3 * wall / K, 4),
                 "frac_of_bf16_peak_layer": round(value / world / peak, 4),
                 "kernel_source": src_hash}
@@ -678,6 +710,7 @@ def main():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-window comparison run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle forward budget for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
