@@ -196,6 +196,35 @@ int salad_attn_backward_sparse(const void* q, const void* k, const void* v, cons
                                float* dv, void* workspace, size_t workspace_bytes, salad_stream_t stream);
 
 /*
+ * Backward pass of the whole layer: the sparse branch as above plus the linear
+ * branch, its projection and the gate (the gradients the fine-tuning needs).
+ * With a_i = relu(q_i), S and z the branch's state, den_i = a_i.z + eps,
+ * o_i = a_i^T S / den_i, y_i = o_i W, out_i = o_sp_i + g y_i:
+ *   dgate[b][h] = sum_i dout_i.y_i;   dW = sum over (b, h, i) of o_i^T (g dout_i)
+ *   du_i = (g dout_i W^T) / den_i,  dden_i = -(g dout_i W^T).o_i / den_i,
+ *   dS = sum_i a_i du_i^T,  dz = sum_i dden_i a_i
+ *   dq_i += [q_i > 0] (S du_i + dden_i z),  dk_j += [k_j > 0] (dS v_j + dz),
+ *   dv_j += dS^T relu(k_j)
+ * and the sparse branch's gradients with o_sp_i = out_i - g y_i in D_i.
+ *   out, lse   from salad_attn_forward_lse with the same inputs.
+ *   w_proj     DEVICE bf16 [d][d], 16-byte aligned;  gate DEVICE fp32 [B][Hh].
+ *   dq, dk, dv DEVICE fp32 [B][N][Hh][d], 16-byte aligned (written).
+ *   dw         DEVICE fp32 [d][d];  dgate DEVICE fp32 [B][Hh] (written).
+ *   workspace  DEVICE, >= salad_layer_backward_workspace_bytes(B, N, Hh, d),
+ *              256-byte aligned, status word first (zero it once).
+ * Other arguments as salad_attn_backward_sparse.  The linear branch's terms are
+ * fp32 CUDA-core arithmetic in a fixed order (deterministic).  Errors:
+ * INVALID_ARG, UNSUPPORTED (d, block != 128, B*Hh > 65535), WORKSPACE, CUDA.
+ */
+size_t salad_layer_backward_workspace_bytes(int B, int N, int num_heads, int d);
+int salad_attn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                        const float* lse, int B, int N, int num_heads, int d, int block, const int32_t* row_ptr,
+                        const int32_t* col_idx, const int32_t* t_row_ptr, const int32_t* t_col_idx, int mask_per_bh,
+                        const void* w_proj, const float* gate, float softmax_scale, float eps, float* dq, float* dk,
+                        float* dv, float* dw, float* dgate, void* workspace, size_t workspace_bytes,
+                        salad_stream_t stream);
+
+/*
  * Top-K dynamic block mask.  The SALAD summary (section 5) says the method also
  * applies to Top-K dynamic sparse attention and gives no scoring rule; the rule
  * implemented here is a reading of that sentence:

@@ -7,7 +7,7 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, tile_num_blocks, build_tile_mask, workspace_bytes, attn_forward,
-    attn_forward_lse, attn_backward_sparse, attn_forward_tiles, attn_forward_static, gate_forward, build_topk_mask, linear_state,
+    attn_forward_lse, attn_backward_sparse, attn_backward, attn_forward_tiles, attn_forward_static, gate_forward, build_topk_mask, linear_state,
     check_status, set_wait_limit_ns, set_max_ctas, set_phase_events, status_string
 """
 from __future__ import annotations
@@ -69,6 +69,11 @@ def lib() -> ctypes.CDLL:
         L.salad_attn_backward_sparse.argtypes = [p, p, p, p, p, p, i, i, i, i, i, p, p, p, p, i, f, p, p, p, p, sz,
                                                  p]
         L.salad_attn_backward_sparse.restype = i
+        L.salad_layer_backward_workspace_bytes.argtypes = [i, i, i, i]
+        L.salad_layer_backward_workspace_bytes.restype = sz
+        L.salad_attn_backward.argtypes = [p, p, p, p, p, p, i, i, i, i, i, p, p, p, p, i, p, p, f, f, p, p, p, p, p,
+                                          p, sz, p]
+        L.salad_attn_backward.restype = i
         L.salad_attn_forward_tiles.argtypes = [p, p, p, i, i, i, i, i, i, i, i, i, p, p, p, p, f, f, p, p, sz,
                                                p]
         L.salad_attn_forward_tiles.restype = i
@@ -254,6 +259,36 @@ def attn_backward_sparse(q, k, v, o, dout, lse, row_ptr, col_idx, block: int = 1
         _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "salad_attn_backward_sparse")
     return tuple(grads)
+
+
+def attn_backward(q, k, v, out, dout, lse, row_ptr, col_idx, w_proj, gate, block: int = 128, t_row_ptr=None,
+                  t_col_idx=None, softmax_scale: float = 0.0, eps: float = 1e-6, mask_per_bh: bool = False,
+                  workspace=None, stream=None):
+    """Gradients of the whole layer (see salad.h): dict of fp32 CUDA tensors dq, dk,
+    dv [B, N, Hh, d], dw [d, d] and dgate [B, Hh].  out and lse come from
+    attn_forward_lse on the same inputs."""
+    B, N, Hh, d = q.shape
+    t_row_ptr = row_ptr if t_row_ptr is None else t_row_ptr
+    t_col_idx = col_idx if t_col_idx is None else t_col_idx
+    res = {n: torch.empty(B, N, Hh, d, dtype=torch.float32, device=q.device) for n in ("dq", "dk", "dv")}
+    res["dw"] = torch.empty(d, d, dtype=torch.float32, device=q.device)
+    res["dgate"] = torch.empty(B, Hh, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = lib().salad_layer_backward_workspace_bytes(B, N, Hh, d)
+        if n == 0:
+            raise SaladError(SALAD_ERR_INVALID_ARG, "salad_layer_backward_workspace_bytes")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    i32 = lambda t, name: _dev_ptr(t, torch.int32, name)  # noqa: E731
+    f32 = lambda name: _dev_ptr(res[name], torch.float32, name)  # noqa: E731
+    _check(lib().salad_attn_backward(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
+        _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(dout, torch.bfloat16, "dout"),
+        _dev_ptr(lse, torch.float32, "lse"), B, N, Hh, d, int(block), i32(row_ptr, "row_ptr"),
+        i32(col_idx, "col_idx"), i32(t_row_ptr, "t_row_ptr"), i32(t_col_idx, "t_col_idx"), int(bool(mask_per_bh)),
+        _dev_ptr(w_proj, torch.bfloat16, "w_proj"), _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale),
+        float(eps), f32("dq"), f32("dk"), f32("dv"), f32("dw"), f32("dgate"),
+        _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "salad_attn_backward")
+    return res
 
 
 def attn_forward_tiles(q, k, v, grid, tile, row_ptr, col_idx, w_proj, gate, softmax_scale: float = 0.0,

@@ -20,7 +20,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libsalad.so")
-SOURCES = ["api.cu", "mask.cu", "linear.cu", "attn.cu", "noalloc.cu", "topk.cu", "gate.cu", "bwd.cu"]
+SOURCES = ["api.cu", "mask.cu", "linear.cu", "attn.cu", "noalloc.cu", "topk.cu", "gate.cu", "bwd.cu", "bwd_linear.cu"]
 HEADERS = ["ptx.cuh", "internal.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

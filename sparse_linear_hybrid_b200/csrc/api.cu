@@ -371,6 +371,151 @@ int salad_attn_backward_sparse(const void* q, const void* k, const void* v, cons
   return launch_backward(ba, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+// Workspace of the layer backward (byte offsets; every region 256-byte aligned).
+struct LayerBwdLayout {
+  WorkspaceLayout fwd;  // the forward's workspace (status word at 0, the state export's partials)
+  size_t off_S, off_z, off_lse2, off_dvec, off_o, off_dy, off_du, off_dden, off_yg, off_partial, off_dS, off_dz, total;
+  int splits, npad;
+};
+LayerBwdLayout layer_bwd_layout(int B, int N, int heads, int d) {
+  LayerBwdLayout L{};
+  L.fwd = workspace_layout(B, N, heads, d);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t BH = (size_t)B * heads, rows = (size_t)B * N * heads;
+  L.npad = (N + 127) / 128 * 128;
+  L.splits = 8;
+  size_t o = up(L.fwd.total);
+  L.off_S = o;       o += up(BH * d * d * 4);
+  L.off_z = o;       o += up(BH * d * 4);
+  L.off_lse2 = o;    o += up(BH * L.npad * 4);
+  L.off_dvec = o;    o += up(BH * L.npad * 4);
+  L.off_o = o;       o += up(rows * d * 4);
+  L.off_dy = o;      o += up(rows * d * 4);
+  L.off_du = o;      o += up(rows * d * 4);
+  L.off_dden = o;    o += up(BH * N * 4);
+  L.off_yg = o;      o += up(BH * N * 4);
+  L.off_partial = o; o += up((size_t)2 * L.splits * BH * d * d * 4);
+  L.off_dS = o;      o += up(BH * d * d * 4);
+  L.off_dz = o;      o += up(BH * d * 4);
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+extern "C" {
+
+size_t salad_layer_backward_workspace_bytes(int B, int N, int num_heads, int d) {
+  if (B < 1 || N < 1 || num_heads < 1 || (d != 64 && d != 128)) return 0;
+  return layer_bwd_layout(B, N, num_heads, d).total;
+}
+
+int salad_attn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                        const float* lse, int B, int N, int num_heads, int d, int block, const int32_t* row_ptr,
+                        const int32_t* col_idx, const int32_t* t_row_ptr, const int32_t* t_col_idx, int mask_per_bh,
+                        const void* w_proj, const float* gate, float softmax_scale, float eps, float* dq, float* dk,
+                        float* dv, float* dw, float* dgate, void* workspace, size_t workspace_bytes,
+                        salad_stream_t stream) {
+  if (!q || !k || !v || !out || !dout || !lse || !row_ptr || !col_idx || !t_row_ptr || !t_col_idx || !w_proj ||
+      !gate || !dq || !dk || !dv || !dw || !dgate || !workspace)
+    return SALAD_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || num_heads < 1) return SALAD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
+  if (block != 128) return SALAD_ERR_UNSUPPORTED;
+  if (num_heads > 65535 || (long long)B * num_heads > 65535 ||
+      (long long)B * num_heads * ((N + 127) / 128) >= (1ll << 31))
+    return SALAD_ERR_UNSUPPORTED;
+  const void* p16[] = {q, k, v, out, dout, w_proj, dq, dk, dv};
+  for (const void* ptr : p16)
+    if (!aligned(ptr, 16)) return SALAD_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(lse, 4) || !aligned(gate, 4) || !aligned(dw, 4) || !aligned(dgate, 4) ||
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(t_row_ptr, 4) || !aligned(t_col_idx, 4))
+    return SALAD_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale) || !std::isfinite(eps) || eps < 0.f) return SALAD_ERR_INVALID_ARG;
+  const LayerBwdLayout L = layer_bwd_layout(B, N, num_heads, d);
+  if (workspace_bytes < L.total) return SALAD_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  // 1. the linear branch's state S, z (fp32)
+  int st = run_linear(k, v, B, N, num_heads, d, nullptr, w_proj, F(L.off_S), F(L.off_z), ws, L.fwd, s);
+  if (st != SALAD_OK) return st;
+  LinBwdArgs la{};
+  la.q = static_cast<const uint16_t*>(q);
+  la.k = static_cast<const uint16_t*>(k);
+  la.v = static_cast<const uint16_t*>(v);
+  la.out = static_cast<const uint16_t*>(out);
+  la.dout = static_cast<const uint16_t*>(dout);
+  la.w = static_cast<const uint16_t*>(w_proj);
+  la.lse = lse;
+  la.gate = gate;
+  la.S = F(L.off_S);
+  la.z = F(L.off_z);
+  la.dq = dq;
+  la.dk = dk;
+  la.dv = dv;
+  la.dw = dw;
+  la.dgate = dgate;
+  la.lse2 = F(L.off_lse2);
+  la.dvec = F(L.off_dvec);
+  la.o_s = F(L.off_o);
+  la.dy_s = F(L.off_dy);
+  la.du_s = F(L.off_du);
+  la.dden_s = F(L.off_dden);
+  la.yg_s = F(L.off_yg);
+  la.partial = F(L.off_partial);
+  la.dS = F(L.off_dS);
+  la.dz = F(L.off_dz);
+  la.B = B;
+  la.N = N;
+  la.heads = num_heads;
+  la.d = d;
+  la.npad = L.npad;
+  la.splits = L.splits;
+  la.eps = eps;
+  // 2. per-row terms of the linear branch, D_i and lse2; dq starts as the linear branch's part
+  if (launch_linear_backward_rows(la, s) != cudaSuccess) return SALAD_ERR_CUDA;
+  // 3. the sparse branch: dq += ..., dk and dv written
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_bnhd_map(&tq, q, B, N, num_heads, d, 128) || !make_bnhd_map(&tk, k, B, N, num_heads, d, 128) ||
+      !make_bnhd_map(&tv, v, B, N, num_heads, d, 128) || !make_bnhd_map(&tdo, dout, B, N, num_heads, d, 128))
+    return SALAD_ERR_CUDA;
+  BwdArgs ba{};
+  ba.tm_q = &tq;
+  ba.tm_k = &tk;
+  ba.tm_v = &tv;
+  ba.tm_do = &tdo;
+  ba.o = static_cast<const uint16_t*>(out);
+  ba.dout = static_cast<const uint16_t*>(dout);
+  ba.lse = lse;
+  ba.row_ptr = row_ptr;
+  ba.col_idx = col_idx;
+  ba.t_row_ptr = t_row_ptr;
+  ba.t_col_idx = t_col_idx;
+  ba.lse2 = la.lse2;
+  ba.dvec = la.dvec;
+  ba.dq = dq;
+  ba.dk = dk;
+  ba.dv = dv;
+  ba.B = B;
+  ba.N = N;
+  ba.heads = num_heads;
+  ba.d = d;
+  ba.nb = L.npad / 128;
+  ba.npad = L.npad;
+  ba.mask_per_bh = mask_per_bh ? 1 : 0;
+  ba.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)d);
+  ba.scale_log2 = ba.scale * 1.4426950408889634f;
+  ba.status = reinterpret_cast<uint32_t*>(ws + L.fwd.off_status);
+  ba.wait_limit_ns = g_wait_limit_ns.load();
+  ba.full = 1;
+  if (launch_backward(ba, s) != cudaSuccess) return SALAD_ERR_CUDA;
+  // 4. dS, dz, dW, dgate, then the linear parts of dk and dv
+  return launch_linear_backward_tail(la, s) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
+}
+
 int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B, int T, int H, int W, int bt,
                              int bh, int bw, int num_heads, int d, const int32_t* row_ptr, const int32_t* col_idx,
                              const void* w_proj, const float* gate, float softmax_scale, float eps, void* out,

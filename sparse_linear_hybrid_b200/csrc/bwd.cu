@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                   const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
                   const float* __restrict__ lse2, const float* __restrict__ dvec, float* __restrict__ dq, int N,
                   int heads, int nb, int npad, int mask_per_bh, float scale, float scale_log2, uint32_t* status,
-                  uint64_t limit_ns) {
+                  uint64_t limit_ns, int accumulate) {
   using C = BwdCfg<D>;
   constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 384;
   extern __shared__ uint8_t bwd_smem_raw[];
@@ -276,10 +276,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (row < N) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + c * 32 + i) =
-                make_float4(__uint_as_float(g[i]) * scale, __uint_as_float(g[i + 1]) * scale,
-                            __uint_as_float(g[i + 2]) * scale, __uint_as_float(g[i + 3]) * scale);
+          for (int i = 0; i < 32; i += 4) {
+            float4 val = make_float4(__uint_as_float(g[i]) * scale, __uint_as_float(g[i + 1]) * scale,
+                                     __uint_as_float(g[i + 2]) * scale, __uint_as_float(g[i + 3]) * scale);
+            float4* p4 = reinterpret_cast<float4*>(dst + c * 32 + i);
+            if (accumulate) {  // the linear branch's part is already there
+              const float4 prev = *p4;
+              val.x += prev.x;
+              val.y += prev.y;
+              val.z += prev.z;
+              val.w += prev.w;
+            }
+            *p4 = val;
+          }
         }
       }
     }
@@ -488,17 +497,20 @@ template <int D>
 cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t s) {
   using C = BwdCfg<D>;
   const long long rows = (long long)a.B * a.heads * a.npad;
-  bwd_prep_kernel<D><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(a.o, a.dout, a.lse, a.B, a.N, a.heads, a.npad,
-                                                                   a.lse2, a.dvec);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!a.full) {  // with the linear branch the row kernel has written lse2 and D
+    bwd_prep_kernel<D><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(a.o, a.dout, a.lse, a.B, a.N, a.heads, a.npad,
+                                                                     a.lse2, a.dvec);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int grid = a.B * a.heads * a.nb;
   e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   bwd_dq_kernel<D><<<grid, kBwdThreads, C::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.row_ptr, a.col_idx,
                                                       a.lse2, a.dvec, a.dq, a.N, a.heads, a.nb, a.npad,
                                                       a.mask_per_bh, a.scale, a.scale_log2, a.status,
-                                                      a.wait_limit_ns);
+                                                      a.wait_limit_ns, a.full);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);

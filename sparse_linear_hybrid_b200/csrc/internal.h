@@ -115,8 +115,24 @@ struct BwdArgs {
   float scale, scale_log2;
   uint32_t* status;
   uint64_t wait_limit_ns;
+  int full = 0;  // with the linear branch: D_i and lse2 come from the row kernel, dq is added to
 };
 cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s);
+
+// Backward pass of the linear branch, projection and gate (bwd_linear.cu).
+struct LinBwdArgs {
+  const uint16_t *q, *k, *v, *out, *dout, *w;  // bf16
+  const float *lse, *gate, *S, *z;             // S fp32 [B*Hh][d][d], z [B*Hh][d]
+  float *dq, *dk, *dv, *dw, *dgate;
+  float *lse2, *dvec;                          // [B*Hh][npad], read by the sparse backward
+  float *o_s, *dy_s, *du_s;                    // fp32 [B][N][Hh][d] scratch
+  float *dden_s, *yg_s;                        // fp32 [B*Hh][N] scratch
+  float *partial, *dS, *dz;                    // [2][splits][B*Hh][d][d], [B*Hh][d][d], [B*Hh][d]
+  int B, N, heads, d, npad, splits;
+  float eps;
+};
+cudaError_t launch_linear_backward_rows(const LinBwdArgs& a, cudaStream_t s);
+cudaError_t launch_linear_backward_tail(const LinBwdArgs& a, cudaStream_t s);
 
 // Dynamic gate and branch dropping (gate.cu).
 struct GateArgs {

@@ -46,3 +46,37 @@ def test_backward_matches_oracle(B, T, H, W, Hh, d, window):
                           si.bf16_bits_to_f32(dout_bits).astype(np.float64))
     for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
         check(g.cpu().numpy().astype(np.float64), ref[name], name)
+
+
+@pytest.mark.parametrize("B,T,H,W,Hh,d,window", [
+    (2, 3, 9, 13, 2, 128, (1, 3, 4)),       # 351 tokens, ragged
+    (1, 2, 8, 16, 3, 64, (1, 2, 3)),        # 256 tokens, d = 64
+    (1, 6, 30, 52, 1, 128, (1, 10, 13)),    # 9,360 tokens
+])
+def test_layer_backward_matches_oracle(B, T, H, W, Hh, d, window):
+    """The whole layer's gradients (salad_attn_backward) with gates in (0, 1) and,
+    where there are several branches, one gate 0, against the oracle: dq, dk, dv
+    as above; dW and dgate within rel-L2 1e-2."""
+    wl = si.Workload("lbw", B=B, Hh=Hh, d=d, T=T, H=H, W=W, block=128, window=window, seed=73)
+    inp = si.make_inputs(wl, v_mean=0.5)
+    if B * Hh > 1:
+        inp.gate[0, 0] = 0.0                                # one dropped branch
+    t = upload(inp)
+    rng = np.random.default_rng(74)
+    dout_bits = si.f32_to_bf16_bits(rng.standard_normal((B, wl.N, Hh, d), dtype=np.float32))
+    dout = torch.from_numpy(dout_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    rp, ci = sl.build_block_mask(T, H, W, 128, inp.windows)
+    out, lse = sl.attn_forward_lse(t["q"], t["k"], t["v"], rp, ci, t["w"], t["gate"], 128)
+    ws = torch.zeros(sl.lib().salad_layer_backward_workspace_bytes(B, wl.N, Hh, d), dtype=torch.uint8,
+                     device="cuda")
+    got = sl.attn_backward(t["q"], t["k"], t["v"], out, dout, lse, rp, ci, t["w"], t["gate"], workspace=ws)
+    assert sl.check_status(ws) == sl.SALAD_OK
+    orp, oci = oracle.block_mask(T, H, W, 128, inp.windows)
+    ref = oracle.backward(inp.q, inp.k, inp.v, 128, orp, oci, inp.w_proj, inp.gate,
+                          si.bf16_bits_to_f32(dout_bits).astype(np.float64))
+    for name in ("dq", "dk", "dv"):
+        check(got[name].cpu().numpy().astype(np.float64), ref[name], name)
+    for name in ("dw", "dgate"):
+        g = got[name].cpu().numpy().astype(np.float64)
+        diff = np.linalg.norm(g - ref[name])
+        assert np.all(np.isfinite(g)) and diff <= 1e-2 * np.linalg.norm(ref[name]), (name, diff)
