@@ -224,3 +224,43 @@ def test_forward_lse_argument_errors(L):
     assert fwd(lse=0) == sl.SALAD_ERR_INVALID_ARG
     assert fwd(lse=FAKE + 0x50000002) == sl.SALAD_ERR_INVALID_ARG   # misaligned
     assert fwd(q=0) == sl.SALAD_ERR_INVALID_ARG
+
+
+def test_backward_argument_errors(L):
+    def sparse(**kw):
+        a = dict(q=FAKE, o=FAKE + 0x30000000, lse=FAKE + 0x50000000, block=128, d=64, dq=FAKE + 0x60000000,
+                 ws=0x40000000, ws_bytes=1 << 30, scale=0.0)
+        a.update(kw)
+        return L.salad_attn_backward_sparse(p(a["q"]), p(FAKE + 0x10000000), p(FAKE + 0x20000000), p(a["o"]),
+                                            p(FAKE + 0x70000000), p(a["lse"]), 1, 256, 2, a["d"], a["block"],
+                                            p(FAKE), p(FAKE), p(FAKE), p(FAKE), 0, a["scale"], p(a["dq"]),
+                                            p(FAKE + 0x80000000), p(FAKE + 0x90000000), p(a["ws"]), a["ws_bytes"],
+                                            None)
+    assert sparse(q=0) == sl.SALAD_ERR_INVALID_ARG
+    assert sparse(lse=0) == sl.SALAD_ERR_INVALID_ARG
+    assert sparse(d=96) == sl.SALAD_ERR_UNSUPPORTED
+    assert sparse(block=64) == sl.SALAD_ERR_UNSUPPORTED        # raster blocks of 128 only
+    assert sparse(dq=FAKE + 0x60000004) == sl.SALAD_ERR_INVALID_ARG   # gradients need 16 bytes
+    assert sparse(scale=float("nan")) == sl.SALAD_ERR_INVALID_ARG
+    assert sparse(ws_bytes=64) == sl.SALAD_ERR_WORKSPACE
+    # a status word, then lse2 and D for every padded row
+    assert L.salad_backward_workspace_bytes(1, 256, 2) == 256 + 2 * 2 * 256 * 4
+    assert L.salad_backward_workspace_bytes(0, 256, 2) == 0
+
+    def layer(**kw):
+        a = dict(w=FAKE + 0xA0000000, eps=1e-6, block=128, B=1, ws=0x40000000, ws_bytes=1 << 34)
+        a.update(kw)
+        return L.salad_attn_backward(p(FAKE), p(FAKE + 0x10000000), p(FAKE + 0x20000000), p(FAKE + 0x30000000),
+                                     p(FAKE + 0x70000000), p(FAKE + 0x50000000), a["B"], 256, 2, 64, a["block"],
+                                     p(FAKE), p(FAKE), p(FAKE), p(FAKE), 0, p(a["w"]), p(FAKE), 0.0, a["eps"],
+                                     p(FAKE + 0x60000000), p(FAKE + 0x80000000), p(FAKE + 0x90000000), p(FAKE),
+                                     p(FAKE), p(a["ws"]), a["ws_bytes"], None)
+    assert layer(w=0) == sl.SALAD_ERR_INVALID_ARG
+    assert layer(eps=-1.0) == sl.SALAD_ERR_INVALID_ARG
+    assert layer(block=64) == sl.SALAD_ERR_UNSUPPORTED
+    assert layer(B=40000) == sl.SALAD_ERR_UNSUPPORTED          # B * Hh above 65535
+    assert layer(ws=0x40000000 + 16) == sl.SALAD_ERR_INVALID_ARG
+    assert layer(ws_bytes=1024) == sl.SALAD_ERR_WORKSPACE
+    small = L.salad_layer_backward_workspace_bytes(1, 256, 2, 64)
+    assert small > L.salad_workspace_bytes(1, 256, 2, 64) and small % 256 == 0
+    assert L.salad_layer_backward_workspace_bytes(1, 256, 2, 96) == 0
