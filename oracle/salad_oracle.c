@@ -606,7 +606,8 @@ void oracle_lse(const uint16_t *q, const uint16_t *k, int B, int N, int Hh, int 
                         for (int64_t j = (int64_t)col_idx[r] * blk; j < (int64_t)(col_idx[r] + 1) * blk && j < N; ++j) {
                             const int64_t koff = (((int64_t)b * N + j) * Hh + h) * d;
                             double dot = 0.0;
-                            for (int c = 0; c < d; ++c) dot += bf16_to_double(q[qoff + c]) * bf16_to_double(k[koff + c]);
+                            for (int c = 0; c < d; ++c)
+                                dot += bf16_to_double(q[qoff + c]) * bf16_to_double(k[koff + c]);
                             if (pass == 0) {
                                 if (tau * dot > m) m = tau * dot;
                             } else {

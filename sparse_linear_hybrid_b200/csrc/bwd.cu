@@ -90,9 +90,9 @@ __device__ __forceinline__ void bwd_timeout(BwdShared* sh, uint32_t* status) {
 
 // D_i and lse_i * log2 e per row, into [B*Hh][Npad] (pad rows: lse2 = +inf, D = 0).
 template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
-                                                       const float* __restrict__ lse, int B, int N, int heads,
-                                                       int npad, float* __restrict__ lse2, float* __restrict__ dvec) {
+__global__ void __launch_bounds__(256)
+    bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout, const float* __restrict__ lse,
+                    int B, int N, int heads, int npad, float* __restrict__ lse2, float* __restrict__ dvec) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= (long long)B * heads * npad) return;
   const int bh = (int)(t / npad), n = (int)(t % npad), b = bh / heads, h = bh % heads;

@@ -140,8 +140,8 @@ cudaError_t launch_gate(const GateArgs& a, cudaStream_t s) {
   int chunk = 0;
   const int splits = gate_splits(a.B, a.N, &chunk);
   const int C8 = a.heads * a.d / 8;
-  gate_pool_kernel<<<dim3(splits, a.B), dim3(kPoolThreads, kPoolRows), 0, s>>>(reinterpret_cast<const uint4*>(a.q), a.N, C8, chunk,
-                                                              a.partial);
+  gate_pool_kernel<<<dim3(splits, a.B), dim3(kPoolThreads, kPoolRows), 0, s>>>(
+      reinterpret_cast<const uint4*>(a.q), a.N, C8, chunk, a.partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   gate_finalize_kernel<<<a.B * a.heads, kFinThreads * kFinGroups, 0, s>>>(
