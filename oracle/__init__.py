@@ -33,8 +33,12 @@ def build(force: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB)
+        # SALAD_ORACLE_LIB: load another build of this source instead (the
+        # mutation tests point it at copies with a planted mistake)
+        other = os.environ.get("SALAD_ORACLE_LIB")
+        if not other:
+            build()
+        lib = ctypes.CDLL(other or _LIB)
         P = ctypes.c_void_p
         lib.oracle_block_mask.restype = ctypes.c_int64
         lib.oracle_block_mask.argtypes = [ctypes.c_int] * 5 + [P, P, P, ctypes.c_int64]
