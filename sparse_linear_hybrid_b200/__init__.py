@@ -237,15 +237,28 @@ def attn_forward_lse(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softma
     return out, lse
 
 
+def _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh):
+    """The transposed mask the backward walks for dk and dv: given, or the mask
+    itself for the symmetric window masks (rows per head).  A mask with rows
+    per (b, h) (Top-K) is not symmetric, so its transpose must be given."""
+    if (t_row_ptr is None) != (t_col_idx is None):
+        raise ValueError("give both t_row_ptr and t_col_idx, or neither")
+    if t_row_ptr is None:
+        if mask_per_bh:
+            raise ValueError("a mask with rows per (b, h) needs its transpose (t_row_ptr, t_col_idx)")
+        return row_ptr, col_idx
+    return t_row_ptr, t_col_idx
+
+
 def attn_backward_sparse(q, k, v, o, dout, lse, row_ptr, col_idx, block: int = 128, t_row_ptr=None,
                          t_col_idx=None, softmax_scale: float = 0.0, mask_per_bh: bool = False, workspace=None,
                          stream=None):
     """Gradients of the sparse branch (see salad.h): (dq, dk, dv) fp32 [B, N, Hh, d].
     o is the branch output and lse the forward's log-sum-exp (attn_forward_lse);
-    the transposed mask defaults to the mask itself (window masks are symmetric)."""
+    the transposed mask defaults to the mask itself, which is right for the
+    symmetric window masks; a mask with rows per (b, h) needs its transpose."""
     B, N, Hh, d = q.shape
-    t_row_ptr = row_ptr if t_row_ptr is None else t_row_ptr
-    t_col_idx = col_idx if t_col_idx is None else t_col_idx
+    t_row_ptr, t_col_idx = _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh)
     grads = [torch.empty(B, N, Hh, d, dtype=torch.float32, device=q.device) for _ in range(3)]
     if workspace is None:
         workspace = torch.zeros(lib().salad_backward_workspace_bytes(B, N, Hh), dtype=torch.uint8, device=q.device)
@@ -268,8 +281,7 @@ def attn_backward(q, k, v, out, dout, lse, row_ptr, col_idx, w_proj, gate, block
     dv [B, N, Hh, d], dw [d, d] and dgate [B, Hh].  out and lse come from
     attn_forward_lse on the same inputs."""
     B, N, Hh, d = q.shape
-    t_row_ptr = row_ptr if t_row_ptr is None else t_row_ptr
-    t_col_idx = col_idx if t_col_idx is None else t_col_idx
+    t_row_ptr, t_col_idx = _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh)
     res = {n: torch.empty(B, N, Hh, d, dtype=torch.float32, device=q.device) for n in ("dq", "dk", "dv")}
     res["dw"] = torch.empty(d, d, dtype=torch.float32, device=q.device)
     res["dgate"] = torch.empty(B, Hh, dtype=torch.float32, device=q.device)

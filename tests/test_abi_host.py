@@ -264,3 +264,13 @@ def test_backward_argument_errors(L):
     small = L.salad_layer_backward_workspace_bytes(1, 256, 2, 64)
     assert small > L.salad_workspace_bytes(1, 256, 2, 64) and small % 256 == 0
     assert L.salad_layer_backward_workspace_bytes(1, 256, 2, 96) == 0
+
+
+def test_backward_binding_needs_the_transpose_of_a_per_bh_mask():
+    import torch
+    x = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
+    idx = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        sl.attn_backward_sparse(x, x, x, x, x, torch.zeros(1, 1, 128), idx, idx, mask_per_bh=True)
+    with pytest.raises(ValueError):
+        sl.attn_backward(x, x, x, x, x, torch.zeros(1, 1, 128), idx, idx, x, torch.zeros(1, 1), t_row_ptr=idx)
