@@ -274,3 +274,13 @@ def test_backward_binding_needs_the_transpose_of_a_per_bh_mask():
         sl.attn_backward_sparse(x, x, x, x, x, torch.zeros(1, 1, 128), idx, idx, mask_per_bh=True)
     with pytest.raises(ValueError):
         sl.attn_backward(x, x, x, x, x, torch.zeros(1, 1, 128), idx, idx, x, torch.zeros(1, 1), t_row_ptr=idx)
+
+
+@pytest.mark.parametrize("compiler,std,ext", [("gcc", "-std=c99", "c"), ("g++", "-std=c++17", "cpp")])
+def test_header_compiles_standalone(tmp_path, compiler, std, ext):
+    """include/salad.h is a plain C header: it compiles on its own as C99 and as C++."""
+    import subprocess
+    src = tmp_path / f"use.{ext}"
+    src.write_text('#include "salad.h"\nint main(void) { return salad_status_string(0) == 0; }\n')
+    subprocess.check_call([compiler, std, "-Wall", "-Wextra", "-Werror", f"-I{os.path.join(ROOT, 'include')}", "-c",
+                           str(src), "-o", str(tmp_path / "use.o")])
