@@ -107,6 +107,18 @@ int salad_build_tile_mask(int T, int H, int W, int bt, int bh, int bw, int num_h
                           salad_stream_t stream);
 
 /*
+ * Host-side check of a block mask in the CSR layout the layer takes (for masks
+ * a caller builds or transposes itself): row_ptr[0] == 0, row_ptr
+ * non-decreasing with at most nb entries a row, every column in [0, nb) and the
+ * columns of a row strictly ascending.
+ *   row_ptr  HOST int32 [rows + 1];  col_idx HOST int32 [row_ptr[rows]] (may be
+ *            NULL when every row is empty).
+ *   bad_row  HOST, nullable: the first offending row (-1 when the mask is valid).
+ * Returns SALAD_OK or SALAD_ERR_INVALID_ARG.  Reads host memory only.
+ */
+int salad_validate_mask(const int32_t* row_ptr, const int32_t* col_idx, int64_t rows, int nb, int64_t* bad_row);
+
+/*
  * Bytes of device workspace salad_attn_forward needs for these sizes (0 on bad
  * arguments).  The workspace holds a status word, the linear-branch state
  * [S | z] of every (b, h) and the split-N partial sums.  It must be zero-filled

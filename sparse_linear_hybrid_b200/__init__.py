@@ -6,9 +6,10 @@ PyTorch supplies device memory and streams.  There is no CPU fallback: calls
 raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
-    mask_num_blocks, build_block_mask, tile_num_blocks, build_tile_mask, workspace_bytes, attn_forward,
-    attn_forward_lse, attn_backward_sparse, attn_backward, attn_forward_tiles, attn_forward_static, gate_forward, build_topk_mask, linear_state,
-    check_status, set_wait_limit_ns, set_max_ctas, set_phase_events, status_string
+    mask_num_blocks, build_block_mask, validate_mask, tile_num_blocks, build_tile_mask, build_topk_mask,
+    workspace_bytes, attn_forward, attn_forward_lse, attn_forward_tiles, attn_forward_static, attn_backward_sparse,
+    attn_backward, gate_forward, linear_state, check_status, set_wait_limit_ns, set_max_ctas, set_phase_events,
+    status_string
 """
 from __future__ import annotations
 
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.salad_build_tile_mask.argtypes = [i, i, i, i, i, i, i, p, p, p, ctypes.c_int64,
                                             ctypes.POINTER(ctypes.c_int64), p]
         L.salad_build_tile_mask.restype = i
+        L.salad_validate_mask.argtypes = [p, p, ctypes.c_int64, i, ctypes.POINTER(ctypes.c_int64)]
+        L.salad_validate_mask.restype = i
         L.salad_workspace_bytes.argtypes = [i, i, i, i]
         L.salad_workspace_bytes.restype = sz
         L.salad_attn_forward.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
@@ -157,6 +160,17 @@ def build_block_mask(T: int, H: int, W: int, block: int, windows, device=None, s
         return lib().salad_build_block_mask(T, H, W, block, win.shape[0], win.ctypes.data_as(ctypes.c_void_p),
                                             rp, ci, cap, ctypes.byref(nnz), s)
     return _build_csr("salad_build_block_mask", mask_num_blocks(T, H, W, block), win.shape[0], call, device)
+
+
+def validate_mask(row_ptr, col_idx, nb: int) -> int:
+    """Host check of a CSR mask (see salad.h): returns -1 when valid, else the
+    first offending row.  Accepts numpy arrays or tensors (copied to the host)."""
+    rp = np.ascontiguousarray(row_ptr.cpu().numpy() if hasattr(row_ptr, "cpu") else row_ptr, dtype=np.int32)
+    ci = np.ascontiguousarray(col_idx.cpu().numpy() if hasattr(col_idx, "cpu") else col_idx, dtype=np.int32)
+    bad = ctypes.c_int64(-1)
+    cols = ci.ctypes.data_as(ctypes.c_void_p) if ci.size else None
+    lib().salad_validate_mask(rp.ctypes.data_as(ctypes.c_void_p), cols, len(rp) - 1, int(nb), ctypes.byref(bad))
+    return int(bad.value)
 
 
 def tile_num_blocks(T: int, H: int, W: int, tile) -> int:

@@ -534,6 +534,26 @@ int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B,
                            eps, out, workspace, workspace_bytes, stream, 0, &g);
 }
 
+int salad_validate_mask(const int32_t* row_ptr, const int32_t* col_idx, int64_t rows, int nb, int64_t* bad_row) {
+  if (bad_row) *bad_row = -1;
+  if (!row_ptr || rows < 0 || nb < 1) return SALAD_ERR_INVALID_ARG;
+  if (row_ptr[0] != 0) {
+    if (bad_row) *bad_row = 0;
+    return SALAD_ERR_INVALID_ARG;
+  }
+  for (int64_t r = 0; r < rows; ++r) {
+    const int32_t a = row_ptr[r], e = row_ptr[r + 1];
+    bool ok = e >= a && e - a <= nb && (e == a || col_idx != nullptr);
+    for (int32_t i = a; ok && i < e; ++i)
+      ok = col_idx[i] >= 0 && col_idx[i] < nb && (i == a || col_idx[i] > col_idx[i - 1]);
+    if (!ok) {
+      if (bad_row) *bad_row = r;
+      return SALAD_ERR_INVALID_ARG;
+    }
+  }
+  return SALAD_OK;
+}
+
 size_t salad_gate_workspace_bytes(int B, int N, int num_heads, int d) {
   if (B < 1 || N < 1 || num_heads < 1 || (d != 64 && d != 128)) return 0;
   return gate_workspace_bytes(B, N, num_heads, d);

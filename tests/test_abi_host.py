@@ -284,3 +284,24 @@ def test_header_compiles_standalone(tmp_path, compiler, std, ext):
     src.write_text('#include "salad.h"\nint main(void) { return salad_status_string(0) == 0; }\n')
     subprocess.check_call([compiler, std, "-Wall", "-Wextra", "-Werror", f"-I{os.path.join(ROOT, 'include')}", "-c",
                            str(src), "-o", str(tmp_path / "use.o")])
+
+
+def test_validate_mask():
+    import numpy as np
+
+    import oracle
+    rp, ci = oracle.block_mask(4, 8, 8, 64, np.array([[1, 4, 4], [0, 0, 0]], dtype=np.int32))
+    assert sl.validate_mask(rp, ci, 4) == -1                      # the builders' masks are valid
+    trp, tci = oracle.tile_mask(2, 5, 7, (1, 2, 3), np.array([[1, 1, 2]], dtype=np.int32))
+    assert sl.validate_mask(trp, tci, len(trp) - 1) == -1
+    bad = ci.copy()
+    bad[rp[2]] = 4                                                # out of range in row 2
+    assert sl.validate_mask(rp, bad, 4) == 2
+    bad = ci.copy()
+    r = int(np.argmax(np.diff(rp) >= 2))                          # a row with two columns
+    bad[rp[r]], bad[rp[r] + 1] = bad[rp[r] + 1], bad[rp[r]]       # not ascending
+    assert sl.validate_mask(rp, bad, 4) == r
+    badp = rp.copy()
+    badp[3] = badp[2] - 1                                         # row_ptr decreasing
+    assert sl.validate_mask(badp, ci, 4) in (2, 3)
+    assert sl.validate_mask(np.array([0, 0, 0], dtype=np.int32), np.zeros(0, dtype=np.int32), 4) == -1
