@@ -226,7 +226,7 @@ int salad_attn_backward_sparse(const void* q, const void* k, const void* v, cons
  *              256-byte aligned, status word first (zero it once).
  * Other arguments as salad_attn_backward_sparse.  The linear branch's terms are
  * fp32 CUDA-core arithmetic in a fixed order (deterministic).  Errors:
- * INVALID_ARG, UNSUPPORTED (d, block != 128, B*Hh > 65535), WORKSPACE, CUDA.
+ * INVALID_ARG, UNSUPPORTED (d, block != 128, B*Hh > 65534), WORKSPACE, CUDA.
  */
 size_t salad_layer_backward_workspace_bytes(int B, int N, int num_heads, int d);
 int salad_attn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,

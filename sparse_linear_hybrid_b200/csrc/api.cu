@@ -424,8 +424,8 @@ int salad_attn_backward(const void* q, const void* k, const void* v, const void*
   if (B < 1 || N < 1 || num_heads < 1) return SALAD_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
   if (block != 128) return SALAD_ERR_UNSUPPORTED;
-  if (num_heads > 65535 || (long long)B * num_heads > 65535 ||
-      (long long)B * num_heads * ((N + 127) / 128) >= (1ll << 31))
+  // (the reductions run B*Hh + 1 rows of CTAs: at most 65535)
+  if ((long long)B * num_heads > 65534 || (long long)B * num_heads * ((N + 127) / 128) >= (1ll << 31))
     return SALAD_ERR_UNSUPPORTED;
   const void* p16[] = {q, k, v, out, dout, w_proj, dq, dk, dv};
   for (const void* ptr : p16)
