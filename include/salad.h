@@ -257,7 +257,7 @@ int salad_attn_backward(const void* q, const void* k, const void* v, const void*
  *   workspace  DEVICE, >= salad_topk_workspace_bytes(B, N, Hh, d, block), 4-byte
  *              aligned (the block means).
  * Rows are per (b, h): pass the mask to salad_attn_forward_bh.  Never
- * synchronises.  Errors: INVALID_ARG, UNSUPPORTED (d, nb > 2048, sizes),
+ * synchronises.  Errors: INVALID_ARG, UNSUPPORTED (d, nb > 2048, B*Hh > 65535, sizes),
  * WORKSPACE, CUDA.
  */
 /*

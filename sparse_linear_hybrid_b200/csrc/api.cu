@@ -603,7 +603,9 @@ int salad_build_topk_mask(const void* q, const void* k, int B, int N, int num_he
   const long long nb = ((long long)N + block - 1) / block;
   if (nb > kTopkMaxBlocks) return SALAD_ERR_UNSUPPORTED;
   const long long kk = keep < nb ? keep : nb;
-  if ((long long)B * num_heads * nb * kk >= (1ll << 31) || (long long)B * N * num_heads * d >= (1ll << 40))
+  // (the pooling launches B*Hh rows of CTAs: at most 65535)
+  if ((long long)B * num_heads > 65535 || (long long)B * num_heads * nb * kk >= (1ll << 31) ||
+      (long long)B * N * num_heads * d >= (1ll << 40))
     return SALAD_ERR_UNSUPPORTED;
   if (!aligned(q, 4) || !aligned(k, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(workspace, 4))
     return SALAD_ERR_INVALID_ARG;

@@ -150,6 +150,7 @@ def test_topk_mask_argument_errors(L):
     assert topk(L, N=0) == sl.SALAD_ERR_INVALID_ARG
     assert topk(L, d=96) == sl.SALAD_ERR_UNSUPPORTED
     assert topk(L, N=2049 * 64) == sl.SALAD_ERR_UNSUPPORTED          # more than 2048 blocks per row
+    assert topk(L, B=40000, N=64) == sl.SALAD_ERR_UNSUPPORTED        # B * Hh above 65535
     assert topk(L, row_ptr=FAKE + 2) == sl.SALAD_ERR_INVALID_ARG     # misaligned
     assert topk(L, ws_bytes=16) == sl.SALAD_ERR_WORKSPACE
     # two fp32 block means per (b, h, block, feature)
