@@ -87,6 +87,7 @@ struct AttnShared {
   volatile int abort_flag;
   float xmax[2][2][128];     // per exchange parity, per half: partial row maxima
   float xsum[2][2][128];     // per exchange parity, per half: partial row sums
+  float xlse[2][2][128];     // the same of the unrounded p (log-sum-exp output)
   float xden[2][2][128];     // per exchange parity, per half: partial relu(q) . z
   alignas(16) float zs[2][128];  // per item slot: z of the item's (b, h)
   int k_edge[2];             // tile blocks: per K ring stage, which grid edges its box sticks out of
@@ -729,7 +730,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (im.w < 0) break;
       const uint32_t q_addr = sbase + C::OFF_Q0 + slot * C::Q_BYTES;
       float m_ref = -INFINITY;  // running reference max (raw score units), same in both halves
-      float l = 0.f;            // this half's share of the row sum
+      float l = 0.f;            // this half's share of the row sum (of the bf16-rounded p)
+      float le = 0.f;           // the same sum of the unrounded p, for the log-sum-exp output
       KeyIter it = item_iter(im, col_idx);  // read only when BLK == 64 (which rows use a tile)
       int j = 0;
       for (; j < im.n; ++j) {
@@ -800,12 +802,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             rescale = true;
           }
         }
-        // p = 2^(s * c - m_ref * c) in pairs; rows that do not use the tile write zeros
+        // p = 2^(s * c - m_ref * c) in pairs; rows that do not use the tile write zeros.
+        // The row sum adds the bf16-rounded p that the PV product consumes, so O / l
+        // is a weighted mean with exactly the weights O was formed with: the rounding
+        // of a dominant key's p (up to 2^8 under the lazy rescale) cancels in O / l.
         uint32_t pk[HC / 2];
-        float rs;
+        float rs, rse = 0.f;
         {
           const uint64_t nmb2 = f32x2_pack(-m_ref * scale_log2, -m_ref * scale_log2);
           uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // 0.0f pairs
+          uint64_t acce = 0;
 #pragma unroll
           for (int i = 0; i < HC / 2; ++i) {
             const uint64_t x =
@@ -820,24 +826,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               p0 = ex2_approx(x0);
               p1 = ex2_approx(x1);
             }
-            const uint64_t pp = f32x2_pack(p0, p1);
+            pk[i] = pack_bf16x2(p0, p1);
+            if (lse_out != nullptr) acce = f32x2_add(acce, f32x2_pack(p0, p1));
+            const uint64_t pp = f32x2_pack(bf16_lo_to_f32(pk[i]), bf16_hi_to_f32(pk[i]));
             if ((i & 3) == 0) acc0 = f32x2_add(acc0, pp);
             if ((i & 3) == 1) acc1 = f32x2_add(acc1, pp);
             if ((i & 3) == 2) acc2 = f32x2_add(acc2, pp);
             if ((i & 3) == 3) acc3 = f32x2_add(acc3, pp);
-            pk[i] = pack_bf16x2(p0, p1);
           }
           const uint64_t a = f32x2_add(f32x2_add(acc0, acc1), f32x2_add(acc2, acc3));
           float a0, a1;
           f32x2_unpack(a, a0, a1);
           rs = a0 + a1;
+          f32x2_unpack(acce, a0, a1);
+          rse = a0 + a1;
         }
         if (!use) {
 #pragma unroll
           for (int i = 0; i < HC / 2; ++i) pk[i] = 0u;
           rs = 0.f;
+          rse = 0.f;
         }
         l = l * alpha + rs;
+        le = le * alpha + rse;
         // the P buffer and O were last read / written by the PV of global tile tt-1
         // (O is rescaled only within an item: an item's first tile has a reference
         // that starts at -inf)
@@ -946,10 +957,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the row sum and relu(q) . z of both halves
       sh->xsum[xc & 1][hf][r] = l;
+      sh->xlse[xc & 1][hf][r] = le;
       sh->xden[xc & 1][hf][r] = den_h;
       mbar_arrive(&sh->xbar[quarter]);
       if (!mbar_wait_warp(&sh->xbar[quarter], (uint32_t)(xc & 1), limit_ns)) { ok = false; break; }
       l += sh->xsum[xc & 1][hf ^ 1][r];
+      le += sh->xlse[xc & 1][hf ^ 1][r];
       const float gd = im.lin ? im.g / ((sh->xden[xc & 1][0][r] + sh->xden[xc & 1][1][r]) + eps) : 0.f;
       ++xc;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -958,7 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // sum_j exp(scale s_j) = 2^(m_ref * scale * log2 e) * l
         if (lse_out != nullptr && hf == 0 && im.qtile * 128 + r < N)
           lse_out[(size_t)im.bh * N + im.qtile * 128 + r] =
-              l > 0.f ? (m_ref * scale_log2 + log2f(l)) * 0.6931471805599453f : -INFINITY;
+              le > 0.f ? (m_ref * scale_log2 + log2f(le)) * 0.6931471805599453f : -INFINITY;
       }
       // U lands in the S slot after this item's tiles
       const int su = sj & 1;

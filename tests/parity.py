@@ -2,12 +2,14 @@
 and the comparison against the oracle.
 
 Tolerance (the layer's stated bar for bf16 inputs with fp32 accumulation):
-max-abs error <= 2e-2 and relative L2 error <= 5e-3 against the fp64 oracle.
+max-abs error <= 2e-2 and relative L2 error <= 5e-3 against the fp64 oracle,
+applied as stated to every element whose bf16 rounding leaves room for it.
 The output is stored as bf16 (one round-to-nearest-even), which by itself moves
-a value by up to half a bf16 ulp: 1.6e-2 at |out| in [4, 8) and 3.1e-2 at
-|out| >= 8.  The max-abs bound is therefore applied to the error beyond that
-final rounding: |gpu - ref| <= 2e-2 + ulp_bf16(ref) / 2.  The plain max-abs
-error is reported alongside.
+a value by up to half a bf16 ulp: 2^-6 = 1.56e-2 at |out| in [4, 8), 2^-5 =
+3.1e-2 at |out| in [8, 16).  Below 8 the plain bound therefore leaves the
+kernel DELTA = 2e-2 - 2^-6 = 4.4e-3 of error before that final rounding.  Only
+where |ref| >= 8, and the rounding alone can exceed 2e-2, is the bound widened,
+to half an ulp plus the same DELTA: bound(ref) = max(2e-2, ulp_bf16(ref)/2 + DELTA).
 """
 from __future__ import annotations
 
@@ -18,6 +20,7 @@ import salad_inputs as si
 
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
+DELTA = MAX_ABS - 2.0 ** -6   # error allowed before the final rounding where the plain bound binds
 
 
 def to_dev(bits: np.ndarray) -> torch.Tensor:
@@ -38,16 +41,25 @@ def half_ulp_bf16(x: np.ndarray) -> np.ndarray:
     return np.ldexp(1.0, e - 9)
 
 
+def bound(ref: np.ndarray) -> np.ndarray:
+    """Per-element max-abs bound: 2e-2, except where the bf16 rounding of the
+    output alone can exceed it (|ref| >= 8)."""
+    return np.maximum(MAX_ABS, half_ulp_bf16(ref) + DELTA)
+
+
 def compare(got: np.ndarray, ref: np.ndarray):
     """Returns (ok, stats) for bf16-derived `got` against fp64 `ref`."""
     mask = ~np.isnan(ref)
     g, r = got[mask], ref[mask]
     err = np.abs(g - r)
+    big = np.abs(r) >= 8.0
     stats = dict(max_abs=float(err.max()) if err.size else 0.0,
+                 max_abs_below_8=float(err[~big].max()) if (~big).any() else 0.0,
+                 n_above_8=int(big.sum()),
+                 max_excess_above_8=float((err[big] - half_ulp_bf16(r[big])).max()) if big.any() else 0.0,
                  rel_l2=float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300)),
-                 max_excess=float((err - half_ulp_bf16(r)).max()) if err.size else 0.0,
                  n=int(err.size), finite=bool(np.all(np.isfinite(g))))
-    ok = stats["finite"] and stats["max_excess"] <= MAX_ABS and stats["rel_l2"] <= REL_L2
+    ok = stats["finite"] and bool(np.all(err <= bound(r))) and stats["rel_l2"] <= REL_L2
     return ok, stats
 
 
