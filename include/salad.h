@@ -45,7 +45,8 @@ typedef enum {
   SALAD_ERR_CAPACITY = -3,       /* col_idx too small for the mask (see nnz_out) */
   SALAD_ERR_WORKSPACE = -4,      /* workspace smaller than salad_workspace_bytes() */
   SALAD_ERR_CUDA = -5,           /* a CUDA runtime/driver call or launch failed */
-  SALAD_ERR_DEVICE_TIMEOUT = -6  /* a kernel gave up waiting (see salad_check_status) */
+  SALAD_ERR_DEVICE_TIMEOUT = -6, /* a kernel gave up waiting (see salad_check_status) */
+  SALAD_ERR_OUT_OF_MEMORY = -7   /* the device had no memory left for the static scratch */
 } salad_status;
 
 /*
@@ -327,9 +328,9 @@ int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, in
                           size_t workspace_bytes, salad_stream_t stream);
 
 /* Size of the static device scratch behind salad_attn_forward_static: 32 MiB.
- * The scratch grows with B*Hh, not with N: at d = 128 it covers any N up to
- * B*Hh = 250 (about 1,000 at d = 64); the 12-head 32,760-token layer needs 20 MB,
- * the 40-head 75,600-token one 21 MB. */
+ * The scratch grows with B*Hh, not with N (salad_workspace_bytes): for any N it
+ * covers B*Hh <= 254 at d = 128 and B*Hh <= 1008 at d = 64.  The 12-head
+ * 32,760-token layer needs 20 MB, the 40-head 75,600-token one 21 MB. */
 #define SALAD_STATIC_SCRATCH_BYTES (32u << 20)
 
 /*
@@ -345,22 +346,36 @@ int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, in
  * device array of SALAD_STATIC_SCRATCH_BYTES that every GPU loading the
  * library holds until the process exits.  It calls no cudaMalloc, cudaFree or
  * allocating library routine.
- *   - The first call on a device looks up the array's device address on that
- *     device (once, cached); make that first call before any stream capture.
+ *   - Each call asks the runtime for the array's device address on the
+ *     current device.  The first call on a device loads the library's device
+ *     code there, and with it the driver maps the 32 MiB array: make that first
+ *     call before any stream capture, and before the engine reserves its memory
+ *     pool.  If the device has no memory left for the array the call returns
+ *     SALAD_ERR_OUT_OF_MEMORY.  After a context reset (cudaDeviceReset) the next
+ *     call maps the array again, in the new context.
  *   - Every call shares the one array, which keeps the previous call's
- *     contents; the call clears the status word it needs at zero.  Calls that
- *     may overlap on the GPU (other streams, other threads) race on the array:
- *     serialise them.
- *   - Device time-outs are recorded in the array's status word, which
- *     salad_check_status cannot see; an output produced after a time-out is
- *     invalid.
+ *     contents.  Calls that may overlap on the GPU (other streams, other
+ *     threads) race on the array: serialise them.
+ *   - A device time-out is recorded in the array's status word and stays there
+ *     until salad_check_status_static reads and clears it; an output produced
+ *     by a call that timed out is invalid.
  * Errors: as salad_attn_forward; WORKSPACE when salad_workspace_bytes(B, N,
- * num_heads, d) exceeds SALAD_STATIC_SCRATCH_BYTES; CUDA when the scratch
- * address cannot be obtained.
+ * num_heads, d) exceeds SALAD_STATIC_SCRATCH_BYTES; OUT_OF_MEMORY as above;
+ * CUDA when the scratch address cannot be obtained.
  */
 int salad_attn_forward_static(const void* q, const void* k, const void* v, int B, int N, int num_heads, int d,
                               int block, const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj,
                               const float* gate, float softmax_scale, float eps, void* out, salad_stream_t stream);
+
+/*
+ * salad_check_status for salad_attn_forward_static, whose status word lives in
+ * the static scratch of the current device: synchronises `stream`, then reads
+ * and clears that word.  Returns SALAD_ERR_DEVICE_TIMEOUT if a kernel of an
+ * earlier static call on this device gave up on a bounded wait, SALAD_ERR_CUDA
+ * if the stream reports an error, SALAD_OK otherwise.  (No counterpart on the
+ * SALAD pages either.)
+ */
+int salad_check_status_static(salad_stream_t stream);
 
 /*
  * The linear-branch state alone (summary section 2.1: ReLU linear attention),

@@ -30,6 +30,7 @@ SALAD_ERR_CAPACITY = -3
 SALAD_ERR_WORKSPACE = -4
 SALAD_ERR_CUDA = -5
 SALAD_ERR_DEVICE_TIMEOUT = -6
+SALAD_ERR_OUT_OF_MEMORY = -7
 
 
 class SaladError(RuntimeError):
@@ -94,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.salad_linear_state.restype = i
         L.salad_check_status.argtypes = [p, p]
         L.salad_check_status.restype = i
+        L.salad_check_status_static.argtypes = [p]
+        L.salad_check_status_static.restype = i
         L.salad_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.salad_set_wait_limit_ns.restype = None
         L.salad_set_max_ctas.argtypes = [i]

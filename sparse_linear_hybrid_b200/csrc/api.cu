@@ -674,6 +674,7 @@ const char* salad_status_string(int status) {
     case SALAD_ERR_WORKSPACE: return "workspace too small";
     case SALAD_ERR_CUDA: return "CUDA error";
     case SALAD_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case SALAD_ERR_OUT_OF_MEMORY: return "device out of memory for the static scratch";
     default: return "unknown status";
   }
 }

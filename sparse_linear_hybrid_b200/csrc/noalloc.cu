@@ -9,31 +9,30 @@
 // status word, the linear-branch state [S | z] and the split partial sums)
 // lives in the file-scope array below, which every GPU that loads the library
 // holds until the process exits.
-#include <mutex>
-
 #include "internal.h"
 
 namespace {
 
+// Zero-initialised when the module is loaded on a device, so its status word
+// starts at 0; afterwards only salad_check_status_static clears it.
 static __device__ __align__(256) uint8_t g_static_scratch[SALAD_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
 // Device address of the static scratch on the current device.  Host code only
-// sees a host-side stand-in under the array's name, so the address is looked
-// up once per device, with that device current, and cached.
+// sees a host-side stand-in under the array's name, so the address is asked of
+// the runtime with the device current.  It is asked on every call rather than
+// cached: a context that is reset and created again loads the module anew, at
+// an address a cached value would not follow.  The first lookup on a device
+// loads the module, which maps the array's memory; the runtime reports a
+// failure to map it as an allocation error.
 int scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SALAD_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return SALAD_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e == cudaErrorMemoryAllocation) {
+    (void)cudaGetLastError();  // not sticky: clear it so the caller's next call is unaffected
+    return SALAD_ERR_OUT_OF_MEMORY;
   }
-  *out = g_scratch_addr[dev];
+  if (e != cudaSuccess || p == nullptr) return SALAD_ERR_CUDA;
+  *out = p;
   return SALAD_OK;
 }
 
@@ -49,10 +48,17 @@ extern "C" int salad_attn_forward_static(const void* q, const void* k, const voi
   void* scratch = nullptr;
   const int st = scratch_address(&scratch);
   if (st != SALAD_OK) return st;
-  // the array keeps the previous call's contents; only the status word must
-  // start at zero (every other byte the forward reads it first writes)
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), s) != cudaSuccess) return SALAD_ERR_CUDA;
+  // The array keeps the previous call's contents.  Every byte the forward reads
+  // it first writes, except the status word, which records a time-out until
+  // salad_check_status_static reads and clears it (as the workspace forward's
+  // does until salad_check_status).
   return salad_attn_forward(q, k, v, B, N, num_heads, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale,
                             eps, out, scratch, SALAD_STATIC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int salad_check_status_static(salad_stream_t stream) {
+  void* scratch = nullptr;
+  const int st = scratch_address(&scratch);
+  if (st != SALAD_OK) return st;
+  return salad_check_status(scratch, stream);
 }

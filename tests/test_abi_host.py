@@ -307,3 +307,23 @@ def test_validate_mask():
     badp[3] = badp[2] - 1                                         # row_ptr decreasing
     assert sl.validate_mask(badp, ci, 4) in (2, 3)
     assert sl.validate_mask(np.array([0, 0, 0], dtype=np.int32), np.zeros(0, dtype=np.int32), 4) == -1
+
+
+STATIC_MAX_BH = {128: 254, 64: 1008}  # the limits include/salad.h states for SALAD_STATIC_SCRATCH_BYTES
+
+
+def test_static_scratch_limit_matches_the_stated_figure(L):
+    cap = 32 << 20
+    for d, bh in STATIC_MAX_BH.items():
+        for N in (64, 1000, 32760, 75600, 1_000_000):
+            # the stated maximum fits whatever N is, one more (b, h) does not
+            assert L.salad_workspace_bytes(1, N, bh, d) <= cap, (d, N)
+            assert L.salad_workspace_bytes(1, N, bh + 1, d) > cap, (d, N)
+            assert L.salad_workspace_bytes(2, N, bh // 2, d) <= cap, (d, N)
+    header = open(HEADER).read()
+    assert "B*Hh <= 254 at d = 128" in header and "B*Hh <= 1008 at d = 64" in header
+
+
+def test_static_status_reader_and_out_of_memory_status_are_exported(L):
+    assert L.salad_status_string(sl.SALAD_ERR_OUT_OF_MEMORY).decode().startswith("device out of memory")
+    assert hasattr(L, "salad_check_status_static")
