@@ -35,3 +35,12 @@ def test_kept_pairs_flops_is_the_token_pair_count():
             for J in ci[rp[h * nb + I]:rp[h * nb + I + 1]]:
                 pairs += ni * min(wl.block, wl.N - J * wl.block)
     assert bench.kept_pairs_flops(rp, ci, wl) == 4.0 * wl.d * pairs * wl.B
+
+
+def test_peak_fractions_three_denominators():
+    f = bench.peak_fractions(1000.0, 1671.5, 148, 1965.0)
+    assert abs(f["measured"] - 1000 / 1671.5) < 1e-4
+    assert abs(f["datasheet"] - 1000 / 2250) < 1e-4
+    assert abs(f["sm_clock_peak_tflops"] - 148 * 1965e6 * 8192 / 1e12) < 0.1
+    assert abs(f["sm_clock"] - 1000 / (148 * 1965e6 * 8192 / 1e12)) < 1e-4
+    assert "sm_clock" not in bench.peak_fractions(1000.0, 1671.5, 148, None)

@@ -1,9 +1,18 @@
 """The backward pass of the sparse branch on the GPU (salad_attn_backward_sparse)
 against the oracle's backward with every gate 0 (then the layer is the sparse
-branch alone and out is its output): dq, dk and dv within rel-L2 1e-2 and a
-max-abs error of 3e-2 of the largest reference value (bf16 operands P and dS,
-fp32 accumulation; D_i from the bf16 output), at ragged shapes, both head
-widths, a full window and a 9,360-token grid."""
+branch alone and out is its output), at ragged shapes, both head widths, a full
+window and a 9,360-token grid; then the whole layer's backward.
+
+Tolerances, from the arithmetic: P and dS enter the tensor-core products as bf16
+(relative 2^-9 each, about 4e-3 together), D_i comes from the bf16 output, and
+everything accumulates in fp32.  The error of a gradient row therefore scales
+with that row's own size, not the tensor's largest value:
+  - dq, dk, dv: per row (one token of one head) ||got - ref|| <= 2e-2 ||ref_row||
+    + 2e-3 x (the RMS of the row norms), the second term for rows whose
+    gradient nearly vanishes; and rel-L2 <= 1e-2 over the tensor;
+  - dW, dgate: per element |got - ref| <= 1e-2 |ref| + 1e-3 max|ref|, and
+    rel-L2 <= 1e-2.
+"""
 import numpy as np
 import pytest
 import torch
@@ -17,10 +26,29 @@ pytestmark = pytest.mark.gpu
 
 
 def check(got, ref, name):
+    """Per-row bound for a [B, N, Hh, d] gradient (module docstring)."""
+    assert np.all(np.isfinite(got)), name
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    d = ref.shape[-1]
+    rn = np.linalg.norm(ref.reshape(-1, d), axis=1)
+    en = np.linalg.norm((got - ref).reshape(-1, d), axis=1)
+    floor = 2e-3 * np.sqrt(np.mean(rn ** 2))
+    worst = float(np.max(en / (2e-2 * rn + floor)))
+    print(name, dict(rel_l2=rel, worst_row_ratio=worst))
+    assert rel <= 1e-2 and worst <= 1.0, (name, rel, worst)
+
+
+def check_elements(got, ref, name):
+    """Per-element bound for dW and dgate (module docstring)."""
+    assert np.all(np.isfinite(got)), name
     err = np.abs(got - ref)
     rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
-    assert np.all(np.isfinite(got)), name
-    assert rel <= 1e-2 and err.max() <= 3e-2 * np.abs(ref).max(), (name, rel, err.max(), np.abs(ref).max())
+    lim = 1e-2 * np.abs(ref) + 1e-3 * np.abs(ref).max()
+    print(name, dict(rel_l2=rel, worst_ratio=float(np.max(err / np.maximum(lim, 1e-300)))))
+    if np.abs(ref).max() == 0:
+        assert np.all(got == 0), name
+    else:
+        assert rel <= 1e-2 and np.all(err <= lim), (name, rel, float(np.max(err / lim)))
 
 
 @pytest.mark.parametrize("B,T,H,W,Hh,d,window", [
@@ -56,7 +84,7 @@ def test_backward_matches_oracle(B, T, H, W, Hh, d, window):
 def test_layer_backward_matches_oracle(B, T, H, W, Hh, d, window):
     """The whole layer's gradients (salad_attn_backward) with gates in (0, 1) and,
     where there are several branches, one gate 0, against the oracle: dq, dk, dv
-    as above; dW and dgate within rel-L2 1e-2."""
+    per row and dW, dgate per element (module docstring)."""
     wl = si.Workload("lbw", B=B, Hh=Hh, d=d, T=T, H=H, W=W, block=128, window=window, seed=73)
     inp = si.make_inputs(wl, v_mean=0.5)
     if B * Hh > 1:
@@ -77,6 +105,4 @@ def test_layer_backward_matches_oracle(B, T, H, W, Hh, d, window):
     for name in ("dq", "dk", "dv"):
         check(got[name].cpu().numpy().astype(np.float64), ref[name], name)
     for name in ("dw", "dgate"):
-        g = got[name].cpu().numpy().astype(np.float64)
-        diff = np.linalg.norm(g - ref[name])
-        assert np.all(np.isfinite(g)) and diff <= 1e-2 * np.linalg.norm(ref[name]), (name, diff)
+        check_elements(got[name].cpu().numpy().astype(np.float64), ref[name], name)
