@@ -327,6 +327,27 @@ int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, in
                           const float* gate, float softmax_scale, float eps, void* out, void* workspace,
                           size_t workspace_bytes, salad_stream_t stream);
 
+/*
+ * salad_attn_forward on a range of heads: q, k, v and out are full
+ * [B][N][heads_total][d] tensors, and the call reads and writes heads
+ * [head_begin, head_begin + head_count) of them only.  The layer's (b, h) units
+ * are independent (every head has its own mask rows, linear-branch state and
+ * output; SALAD summary section 2.1), so a head-parallel job runs one range per
+ * GPU with no exchange in the forward pass; the other heads of out are left
+ * untouched.
+ *   row_ptr, col_idx  the mask of the range's heads (head_count rows of blocks,
+ *                     as salad_build_block_mask builds it from their windows).
+ *   gate              DEVICE fp32 [B][head_count]: the range's gates.
+ *   workspace         >= salad_workspace_bytes(B, N, head_count, d).
+ * Everything else as salad_attn_forward (d, block, alignment, eps, stream).
+ * Errors: INVALID_ARG also when the range does not lie inside [0, heads_total);
+ * UNSUPPORTED when heads_total > 65535; otherwise as salad_attn_forward.
+ */
+int salad_attn_forward_heads(const void* q, const void* k, const void* v, int B, int N, int heads_total,
+                             int head_begin, int head_count, int d, int block, const int32_t* row_ptr,
+                             const int32_t* col_idx, const void* w_proj, const float* gate, float softmax_scale,
+                             float eps, void* out, void* workspace, size_t workspace_bytes, salad_stream_t stream);
+
 /* Size of the static device scratch behind salad_attn_forward_static: 32 MiB.
  * The scratch grows with B*Hh, not with N (salad_workspace_bytes): for any N it
  * covers B*Hh <= 254 at d = 128 and B*Hh <= 1008 at d = 64.  The 12-head
@@ -421,6 +442,19 @@ void salad_set_max_ctas(int max_ctas);
  * to stop.  Host-global setting; it changes no result.
  */
 void salad_set_phase_events(void* before_linear, void* before_attention, void* after_attention);
+
+/*
+ * Profiling hook, live only in the profiling build of the library (compiled
+ * with -DSALAD_PROFILE: `python -m sparse_linear_hybrid_b200.build --profile`,
+ * which writes libsalad_profile.so); the normal build returns
+ * SALAD_ERR_UNSUPPORTED and records nothing.  Later attention launches write
+ * phase stamps (event code << 56 | SM clock) into `device_buffer`: per CTA,
+ * 4 recording threads x 8192 uint64 words, for as many CTAs as `bytes` holds
+ * (unused words keep what the caller put there).  NULL stops the recording.
+ * sparse_linear_hybrid_b200/profile_phases.py reads them back as cycles per
+ * phase.  Host-global setting; it changes no result.
+ */
+int salad_profile_set_buffer(void* device_buffer, size_t bytes);
 
 const char* salad_status_string(int status);
 

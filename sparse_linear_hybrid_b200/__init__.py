@@ -7,7 +7,8 @@ raise if the library is missing or a tensor is not on a CUDA device.
 
 The entry points mirror ``include/salad.h``:
     mask_num_blocks, build_block_mask, validate_mask, tile_num_blocks, build_tile_mask, build_topk_mask,
-    workspace_bytes, attn_forward, attn_forward_lse, attn_forward_tiles, attn_forward_static, attn_backward_sparse,
+    workspace_bytes, attn_forward, attn_forward_lse, attn_forward_heads, attn_forward_tiles, attn_forward_static,
+    attn_backward_sparse,
     attn_backward, gate_forward, linear_state, check_status, set_wait_limit_ns, set_max_ctas, set_phase_events,
     status_string
 """
@@ -43,10 +44,13 @@ def lib() -> ctypes.CDLL:
     """Load libsalad.so (raises when it has not been built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+        # SALAD_LIBRARY selects another build of the same library (the profiling
+        # build, libsalad_profile.so); by default the in-tree libsalad.so
+        path = os.environ.get("SALAD_LIBRARY") or LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
                                "`python -m sparse_linear_hybrid_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
+        L = ctypes.CDLL(path)
         i, p, f, sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
         L.salad_mask_num_blocks.argtypes = [i, i, i, i, ctypes.POINTER(i)]
         L.salad_mask_num_blocks.restype = i
@@ -68,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.salad_attn_forward_bh.restype = i
         L.salad_attn_forward_lse.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p, f, f, i, p, p, p, sz, p]
         L.salad_attn_forward_lse.restype = i
+        L.salad_attn_forward_heads.argtypes = [p, p, p, i, i, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
+        L.salad_attn_forward_heads.restype = i
         L.salad_backward_workspace_bytes.argtypes = [i, i, i]
         L.salad_backward_workspace_bytes.restype = sz
         L.salad_attn_backward_sparse.argtypes = [p, p, p, p, p, p, i, i, i, i, i, p, p, p, p, i, f, p, p, p, p, sz,
@@ -103,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.salad_set_max_ctas.restype = None
         L.salad_set_phase_events.argtypes = [p, p, p]
         L.salad_set_phase_events.restype = None
+        L.salad_profile_set_buffer.argtypes = [p, sz]
+        L.salad_profile_set_buffer.restype = i
         L.salad_status_string.argtypes = [i]
         L.salad_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -252,6 +260,28 @@ def attn_forward_lse(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, softma
         _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(lse, torch.float32, "lse"),
         _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "salad_attn_forward_lse")
     return out, lse
+
+
+def attn_forward_heads(q, k, v, head_begin: int, head_count: int, row_ptr, col_idx, w_proj, gate, block: int,
+                       softmax_scale: float = 0.0, eps: float = 1e-6, out=None, workspace=None,
+                       stream=None) -> torch.Tensor:
+    """attn_forward on heads [head_begin, head_begin + head_count) of full
+    [B, N, Hh, d] tensors (one rank's share of a head-parallel layer): the mask
+    holds the range's heads, gate is fp32 [B, head_count]; out (full shape) is
+    written on those heads only."""
+    B, N, Hh, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = new_workspace(B, N, head_count, d, q.device)
+    _check(lib().salad_attn_forward_heads(
+        _dev_ptr(q, torch.bfloat16, "q"), _dev_ptr(k, torch.bfloat16, "k"), _dev_ptr(v, torch.bfloat16, "v"),
+        B, N, Hh, int(head_begin), int(head_count), d, block, _dev_ptr(row_ptr, torch.int32, "row_ptr"),
+        _dev_ptr(col_idx, torch.int32, "col_idx"), _dev_ptr(w_proj, torch.bfloat16, "w_proj"),
+        _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps),
+        _dev_ptr(out, torch.bfloat16, "out"), _dev_ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream)), "salad_attn_forward_heads")
+    return out
 
 
 def _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh):

@@ -20,6 +20,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libsalad.so")
+# the profiling build: the attention kernel writes phase stamps (SALAD_PROFILE)
+PROF_OBJ = os.path.join(ROOT, "_build", "profile")
+PROF_LIB = os.path.join(HERE, "libsalad_profile.so")
 SOURCES = ["api.cu", "mask.cu", "linear.cu", "attn.cu", "noalloc.cu", "topk.cu", "gate.cu", "bwd.cu", "bwd_linear.cu"]
 HEADERS = ["ptx.cuh", "internal.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -34,13 +37,13 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, verbose):
-    obj = os.path.join(OBJ, os.path.splitext(src)[0] + ".o")
+def _compile(src, verbose, profile=False):
+    obj = os.path.join(PROF_OBJ if profile else OBJ, os.path.splitext(src)[0] + ".o")
     deps = [os.path.join(CSRC, src)] + [os.path.join(CSRC, h) for h in HEADERS] + \
         [os.path.join(ROOT, "include", "salad.h")]
     if not _stale(obj, deps):
         return obj, ""
-    cmd = [NVCC, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+    cmd = [NVCC, *FLAGS, *(["-DSALAD_PROFILE"] if profile else []), "-c", os.path.join(CSRC, src), "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -49,27 +52,31 @@ def _compile(src, verbose):
     return obj, res.stderr
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, profile: bool = False) -> str:
+    """Builds libsalad.so (or, with profile=True, libsalad_profile.so with the
+    attention kernel's phase stamps compiled in)."""
+    obj_dir, lib = (PROF_OBJ, PROF_LIB) if profile else (OBJ, LIB)
+    os.makedirs(obj_dir, exist_ok=True)
     if force:
-        for f in os.listdir(OBJ):
+        for f in os.listdir(obj_dir):
             if f.endswith(".o"):
-                os.remove(os.path.join(OBJ, f))
+                os.remove(os.path.join(obj_dir, f))
     with cf.ThreadPoolExecutor(len(SOURCES)) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, verbose, profile), SOURCES))
     objs = [o for o, _ in results]
     if verbose:
         for _, log in results:
             sys.stderr.write(log)
-    if force or _stale(LIB, objs):
-        cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB, *objs]
+    if force or _stale(lib, objs):
+        cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", lib, *objs]
         subprocess.check_call(cmd)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--profile", action="store_true", help="the profiling build (libsalad_profile.so)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose))
+    print(build(a.force, a.verbose, a.profile))

@@ -55,9 +55,13 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
 }
 
 // [B][N][Hh][d] bf16 viewed as a 3-D tensor (Hh*d, N, B); box (64, rows, 1).
-bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int Hh, int d, uint32_t rows) {
+// With Hh_total > Hh the view is Hh consecutive heads of a tensor that holds
+// Hh_total heads per token (`base` already points at the first of them).
+bool make_bnhd_map(CUtensorMap* m, const void* base, int B, int N, int Hh, int d, uint32_t rows,
+                   int Hh_total = 0) {
+  const uint64_t row = (uint64_t)(Hh_total > 0 ? Hh_total : Hh) * d * 2;
   const uint64_t dims[3] = {(uint64_t)Hh * d, (uint64_t)N, (uint64_t)B};
-  const uint64_t strides[2] = {(uint64_t)Hh * d * 2, (uint64_t)N * Hh * d * 2};
+  const uint64_t strides[2] = {row, (uint64_t)N * row};
   const uint32_t box[3] = {64, rows, 1};
   return make_map(m, base, 3, dims, strides, box);
 }
@@ -94,9 +98,10 @@ int check_common(const void* k, const void* v, int B, int N, int Hh, int d, void
 // The linear-branch kernels.  Forward (S_out == nullptr): z and (S W)^T into the
 // workspace.  State export: S and z into S_out / z_out.
 int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const float* gate, const void* w_proj,
-               float* S_out, float* z_out, uint8_t* ws, const WorkspaceLayout& L, cudaStream_t s) {
+               float* S_out, float* z_out, uint8_t* ws, const WorkspaceLayout& L, cudaStream_t s, int Hh_total = 0) {
   CUtensorMap tk, tv;
-  if (!make_bnhd_map(&tk, k, B, N, Hh, d, 64) || !make_bnhd_map(&tv, v, B, N, Hh, d, 64)) return SALAD_ERR_CUDA;
+  if (!make_bnhd_map(&tk, k, B, N, Hh, d, 64, Hh_total) || !make_bnhd_map(&tv, v, B, N, Hh, d, 64, Hh_total))
+    return SALAD_ERR_CUDA;
   LinearArgs la{};
   la.tm_k = &tk;
   la.tm_v = &tv;
@@ -213,8 +218,11 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
                       const int32_t* row_ptr, const int32_t* col_idx, const void* w_proj, const float* gate,
                       float softmax_scale, float eps, void* out, void* workspace, size_t workspace_bytes,
                       salad_stream_t stream, int mask_per_bh, const TileGeom* tiles = nullptr,
-                      float* lse = nullptr) {
+                      float* lse = nullptr, int head_begin = 0, int heads_total = 0) {
+  // heads_total > 0: q, k, v and out hold heads_total heads per token and the
+  // call runs heads [head_begin, head_begin + num_heads) of them
   if (!q || !row_ptr || !col_idx || !w_proj || !gate || !out) return SALAD_ERR_INVALID_ARG;
+  const int Ht = heads_total > 0 ? heads_total : num_heads;
   int st = check_common(k, v, B, N, num_heads, d, workspace, workspace_bytes);
   if (st != SALAD_OK) return st;
   if (block != 64 && block != 128) return SALAD_ERR_UNSUPPORTED;
@@ -222,10 +230,17 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
       !aligned(row_ptr, 4) || !aligned(col_idx, 4))
     return SALAD_ERR_INVALID_ARG;
   if (!std::isfinite(eps) || eps < 0.f || !std::isfinite(softmax_scale)) return SALAD_ERR_INVALID_ARG;
-  const size_t tensor_bytes = (size_t)B * N * num_heads * d * 2;
+  const size_t tensor_bytes = (size_t)B * N * Ht * d * 2;
   if (overlaps(out, tensor_bytes, q, tensor_bytes) || overlaps(out, tensor_bytes, k, tensor_bytes) ||
       overlaps(out, tensor_bytes, v, tensor_bytes))
     return SALAD_ERR_INVALID_ARG;
+  // the first head of the range, as byte offsets into the tensors (16-byte
+  // aligned: d is 64 or 128)
+  const size_t h0 = (size_t)head_begin * d;
+  q = static_cast<const uint16_t*>(q) + h0;
+  k = static_cast<const uint16_t*>(k) + h0;
+  v = static_cast<const uint16_t*>(v) + h0;
+  out = static_cast<uint16_t*>(out) + h0;
   const long long qtiles = tiles ? (long long)(tiles->T / tiles->bt) * tiles->nh * tiles->nw : (N + 127) / 128;
   if (qtiles * B * num_heads >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
 
@@ -234,7 +249,7 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   if (!record(g_ev_linear, s)) return SALAD_ERR_CUDA;
-  st = run_linear(k, v, B, N, num_heads, d, gate, w_proj, nullptr, nullptr, ws, L, s);
+  st = run_linear(k, v, B, N, num_heads, d, gate, w_proj, nullptr, nullptr, ws, L, s, Ht);
   if (st != SALAD_OK) return st;
 
   CUtensorMap tq, tk, tv, to, tt;
@@ -245,9 +260,10 @@ int attn_forward_impl(const void* q, const void* k, const void* v, int B, int N,
   const bool maps_ok =
       tiles ? make_tile_map(&tq, q, B, *tiles, num_heads, d) && make_tile_map(&tk, k, B, *tiles, num_heads, d) &&
                   make_tile_map(&tv, v, B, *tiles, num_heads, d) && make_tile_map(&to, out, B, *tiles, num_heads, d)
-            : make_bnhd_map(&tq, q, B, N, num_heads, d, 128) && make_bnhd_map(&tk, k, B, N, num_heads, d, block) &&
-                  make_bnhd_map(&tv, v, B, N, num_heads, d, block) &&
-                  make_bnhd_map(&to, out, B, N, num_heads, d, 128);
+            : make_bnhd_map(&tq, q, B, N, num_heads, d, 128, Ht) &&
+                  make_bnhd_map(&tk, k, B, N, num_heads, d, block, Ht) &&
+                  make_bnhd_map(&tv, v, B, N, num_heads, d, block, Ht) &&
+                  make_bnhd_map(&to, out, B, N, num_heads, d, 128, Ht);
   if (!maps_ok || !make_map(&tt, ws + L.off_t, 3, t_dims, t_strides, t_box)) return SALAD_ERR_CUDA;
 
   AttnArgs aa{};
@@ -307,6 +323,18 @@ int salad_attn_forward_lse(const void* q, const void* k, const void* v, int B, i
   if (!lse || !aligned(lse, 4)) return SALAD_ERR_INVALID_ARG;
   return attn_forward_impl(q, k, v, B, N, num_heads, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
                            out, workspace, workspace_bytes, stream, mask_per_bh ? 1 : 0, nullptr, lse);
+}
+
+int salad_attn_forward_heads(const void* q, const void* k, const void* v, int B, int N, int heads_total,
+                             int head_begin, int head_count, int d, int block, const int32_t* row_ptr,
+                             const int32_t* col_idx, const void* w_proj, const float* gate, float softmax_scale,
+                             float eps, void* out, void* workspace, size_t workspace_bytes, salad_stream_t stream) {
+  if (heads_total < 1 || head_begin < 0 || head_count < 1 || head_count > heads_total ||
+      head_begin > heads_total - head_count)
+    return SALAD_ERR_INVALID_ARG;
+  if (heads_total > 65535) return SALAD_ERR_UNSUPPORTED;
+  return attn_forward_impl(q, k, v, B, N, head_count, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
+                           out, workspace, workspace_bytes, stream, 0, nullptr, nullptr, head_begin, heads_total);
 }
 
 size_t salad_backward_workspace_bytes(int B, int N, int num_heads) {
@@ -658,6 +686,12 @@ int salad_check_status(void* workspace, salad_stream_t stream) {
 void salad_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns.store(limit_ns); }
 
 void salad_set_max_ctas(int max_ctas) { g_max_ctas.store(max_ctas > 0 ? max_ctas : 0); }
+
+int salad_profile_set_buffer(void* device_buffer, size_t bytes) {
+  if (device_buffer != nullptr && (reinterpret_cast<uintptr_t>(device_buffer) % 8) != 0)
+    return SALAD_ERR_INVALID_ARG;
+  return set_profile_buffer(device_buffer, device_buffer ? bytes : 0);
+}
 
 void salad_set_phase_events(void* before_linear, void* before_attention, void* after_attention) {
   g_ev_linear.store(before_linear);

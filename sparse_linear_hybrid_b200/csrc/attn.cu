@@ -59,6 +59,37 @@ constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 constexpr int kThreads = 384;
 
+// Phase stamps of the profiling build (-DSALAD_PROFILE, off by default): four
+// recording threads per CTA -- the leader, the tcgen05 issuer, the V producer
+// and the first thread of softmax warp 2 -- write (event code << 56 | clock64)
+// into their own run of kProfEvents words of a buffer the host hands over
+// (salad_profile_set_buffer); sparse_linear_hybrid_b200/profile_phases.py turns
+// them into cycles per phase.  The normal build compiles none of it.
+#ifdef SALAD_PROFILE
+constexpr int kProfEvents = 8192;
+constexpr int kProfRecorders = 4;
+__device__ uint64_t* g_prof_buf = nullptr;
+__device__ int g_prof_ctas = 0;  // CTAs the buffer has room for
+#define SALAD_PROF(code)                                                                           \
+  do {                                                                                             \
+    if (prof_ != nullptr && prof_n_ < kProfEvents)                                                 \
+      prof_[prof_n_++] = ((uint64_t)(code) << 56) | ((uint64_t)clock64() & 0x00FFFFFFFFFFFFFFull); \
+  } while (0)
+#else
+#define SALAD_PROF(code) \
+  do {                   \
+  } while (0)
+#endif
+// event codes
+enum : int {
+  kPfLdItem = 1, kPfLdKWait = 2, kPfLdKGot = 3,
+  kPfSWait = 10, kPfSReady = 11, kPfSIssued = 12, kPfQCopied = 13, kPfUWait = 14, kPfUIssued = 15,
+  kPfPvWait = 20, kPfPvP = 21, kPfPvV = 22, kPfPvIssued = 23,
+  kPfVWait = 30, kPfVGot = 31,
+  kPfSmWait = 40, kPfSmS = 41, kPfSmLoaded = 42, kPfSmMax = 43, kPfSmXchg = 44, kPfSmExp = 45, kPfSmPv = 46,
+  kPfSmP = 47, kPfEpBegin = 50, kPfEpRelu = 51, kPfEpSums = 52, kPfEpU = 53, kPfEpEnd = 54,
+};
+
 // A work item as the leader hands it to the other roles (through shared
 // memory, so that no other role reads the mask or the gate from global memory
 // on its way into an item).
@@ -343,6 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+#ifdef SALAD_PROFILE
+  uint64_t* prof_ = nullptr;
+  int prof_n_ = 0;
+  {
+    const int rec = warp == 0 ? 0 : warp == 1 ? 1 : warp == 10 ? 2 : warp == 2 ? 3 : -1;
+    if (rec >= 0 && lane == 0 && g_prof_buf != nullptr && (int)blockIdx.x < g_prof_ctas)
+      prof_ = g_prof_buf + ((size_t)blockIdx.x * kProfRecorders + rec) * kProfEvents;
+  }
+#endif
 
   if (warp == 0) {
     // ============================ leader and TMA producer of Q and K
@@ -355,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // next K ring entry: wait for its stage, expect its bytes
       auto k_stage = [&](int edge) -> uint8_t* {
         const int s = kj & 1;
+        SALAD_PROF(kPfLdKWait);
         // the stage is free once the product that read entry kj - 2 is done.  With
         // T in the rings every K entry feeds exactly one S slot use (S or U) in the
         // same order, so that product's own completion barrier tells; otherwise
@@ -363,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  ? (kj < 2 || mbar_wait(&sh->s_full[s], (uint32_t)(((kj - 2) >> 1) & 1), limit_ns))
                                  : mbar_wait(&sh->k_empty[s], ((kj >> 1) & 1) ^ 1, limit_ns);
         if (sh->abort_flag || !free_ok) return nullptr;
+        SALAD_PROF(kPfLdKGot);
         if constexpr (TILES) sh->k_edge[s] = edge;  // read by the MMA thread after k_full
         mbar_arrive_expect_tx(&sh->k_full[s], C::KV_BYTES);
         return smem + C::OFF_K0 + s * C::KV_BYTES;
@@ -373,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // hand the next item to the other roles
         if (sh->abort_flag || !mbar_wait(&sh->item_empty[slot], ph ^ 1, limit_ns)) { ok = false; break; }
         const int w = (int)atomicAdd(work_ctr, 1u);
+        SALAD_PROF(kPfLdItem);
         Item im;
         if (w < num_items) {
           im = make_item<BLK, TILES>(w, qtiles, heads, N, nblocks, row_ptr, col_idx, gate, mask_per_bh);
@@ -475,7 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int col, bits;
         while (it.next(col, bits)) {
           const int s = vj & 1;
+          SALAD_PROF(kPfVWait);
           if (!v_stage_free(s)) { ok = false; break; }
+          SALAD_PROF(kPfVGot);
           if (s) {
             is_tlo1 = false;
             tile1 = gtile;
@@ -566,9 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // `gv0` (P from tensor memory; operands waited for here)
       auto issue_pv = [&](int gt, int gv, bool first) -> bool {
         const int s = gt & 1, vs = gv & 1;
-        if (sh->abort_flag || !mbar_wait(&sh->p_full[s], (uint32_t)((gt >> 1) & 1), limit_ns) ||
-            !mbar_wait(&sh->v_full[vs], (uint32_t)((gv >> 1) & 1), limit_ns))
-          return false;
+        SALAD_PROF(kPfPvWait);
+        if (sh->abort_flag || !mbar_wait(&sh->p_full[s], (uint32_t)((gt >> 1) & 1), limit_ns)) return false;
+        SALAD_PROF(kPfPvP);
+        if (!mbar_wait(&sh->v_full[vs], (uint32_t)((gv >> 1) & 1), limit_ns)) return false;
+        SALAD_PROF(kPfPvV);
         pf_seen = gt;
         tc_fence_after();
         const uint32_t vt = sbase + C::OFF_V0 + vs * C::KV_BYTES;
@@ -579,16 +626,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ts(tmem + C::TM_O, pt + kk * 8, bd, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
         }
         mma_commit(&sh->pv_done[s]);  // also frees the V stage
+        SALAD_PROF(kPfPvIssued);
         return true;
       };
       // S = Q K^T into the next S slot (K tile kj of the ring; Q from tensor memory)
       auto issue_s = [&]() -> bool {
         const int s = sj & 1, ks = kj & 1;
+        SALAD_PROF(kPfSWait);
         if (sh->abort_flag || !mbar_wait(&sh->k_full[ks], (uint32_t)((kj >> 1) & 1), limit_ns)) return false;
         const int prev = s ? slot_tile1 : slot_tile0;
         const bool implied = prev >= 0 && prev <= pf_seen;
         if (sj >= 2 && !implied && !mbar_wait(&sh->s_free[s], (uint32_t)(((sj - 2) >> 1) & 1), limit_ns))
           return false;
+        SALAD_PROF(kPfSReady);
         if (s) {
           slot_tile1 = st;
         } else {
@@ -614,6 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         q_last = sj;
         ++kj;
         ++sj;
+        SALAD_PROF(kPfSIssued);
         return true;
       };
       // U = relu(Q) [T_hi ; T_lo] of the item in Q buffer `qb` (K = 2d: relu(Q)
@@ -629,6 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (sh->abort_flag || !t_ok || !mbar_wait(&sh->q_relu[qb], (uint32_t)((qseq >> 1) & 1), limit_ns))
           return false;
         if (sj >= 2 && !mbar_wait(&sh->s_free[s], (uint32_t)(((sj - 2) >> 1) & 1), limit_ns)) return false;
+        SALAD_PROF(kPfUWait);
         if (s) {
           slot_tile1 = -1;
         } else {
@@ -656,6 +708,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         q_last = sj;
         ++sj;
+        SALAD_PROF(kPfUIssued);
         return true;
       };
       for (;;) {
@@ -685,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             tmem_cp_128x256b(tmem + C::TM_Q + kk * 8, sw128_desc(q_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024));
+          SALAD_PROF(kPfQCopied);
         }
         if (n >= 1 && !issue_s()) { ok = false; break; }
         for (int j = 1; j < n && ok; ++j) {
@@ -745,7 +799,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int s = sj & 1;
         const bool aborted = __shfl_sync(0xffffffffu, sh->abort_flag != 0, 0);
+        SALAD_PROF(kPfSmWait);
         if (aborted || !mbar_wait_warp(&sh->s_full[s], (uint32_t)((sj >> 1) & 1), limit_ns)) { ok = false; break; }
+        SALAD_PROF(kPfSmS);
         tc_fence_after();
         uint32_t sr[HC];
 #pragma unroll
@@ -756,6 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->s_free[s]);
+        SALAD_PROF(kPfSmLoaded);
 
         const bool use = ((bits >> half) & 1) != 0;           // warp-uniform
         const int valid = vtile - hf * HC;  // real keys among this thread's columns (raster blocks)
@@ -784,6 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mt = fmaxf(m0, m1);
         }
+        SALAD_PROF(kPfSmMax);
         // both halves of the row agree on the tile maximum (one barrier phase per
         // exchange; a bounded wait, so a time-out on either side cannot hang its partner)
         sh->xmax[xc & 1][hf][r] = mt;
@@ -791,6 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_warp(&sh->xbar[quarter], (uint32_t)(xc & 1), limit_ns)) { ok = false; break; }
         mt = fmaxf(mt, sh->xmax[xc & 1][hf ^ 1][r]);
         ++xc;
+        SALAD_PROF(kPfSmXchg);
         float alpha = 1.f;
         bool rescale = false;
         if (use) {
@@ -849,6 +908,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l = l * alpha + rs;
         le = le * alpha + rse;
+        SALAD_PROF(kPfSmExp);
         // the P buffer and O were last read / written by the PV of global tile tt-1
         // (O is rescaled only within an item: an item's first tile has a reference
         // that starts at -inf)
@@ -859,6 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_after();
+        SALAD_PROF(kPfSmPv);
         if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
@@ -879,11 +940,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->p_full[tt & 1]);
+        SALAD_PROF(kPfSmP);
         ++sj;
         ++tt;
       }
       if (!ok) break;
       const int n = j;
+      SALAD_PROF(kPfEpBegin);
       // relu(Q) over the Q columns of tensor memory for U, each thread its half of
       // its row, and this half's share of relu(q) . z on the way; the arrive
       // happens for every item, so the barrier keeps count of items
@@ -948,6 +1011,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->q_relu[slot]);
+      SALAD_PROF(kPfEpRelu);
       if (n >= 1) {
         if (!mbar_wait_warp(&sh->pv_done[(tt - 1) & 1], (uint32_t)(((tt - 1) >> 1) & 1), limit_ns)) {
           ok = false;
@@ -965,6 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       le += sh->xlse[xc & 1][hf ^ 1][r];
       const float gd = im.lin ? im.g / ((sh->xden[xc & 1][0][r] + sh->xden[xc & 1][1][r]) + eps) : 0.f;
       ++xc;
+      SALAD_PROF(kPfEpSums);
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       if constexpr (!TILES) {
         // the row's log-sum-exp (natural log) of the sparse softmax, for training:
@@ -979,6 +1044,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_warp(&sh->s_full[su], (uint32_t)((sj >> 1) & 1), limit_ns)) { ok = false; break; }
         tc_fence_after();
       }
+      SALAD_PROF(kPfEpU);
       // out = O / l + g U / den for this half's features -> bf16 staging in the Q buffer
       const uint32_t tm_u = su ? C::TM_S1 : C::TM_S0;
 #pragma unroll
@@ -1019,6 +1085,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (im.lin) mbar_arrive(&sh->s_free[su]);
         mbar_arrive(&sh->staged[slot]);
       }
+      SALAD_PROF(kPfEpEnd);
       if (im.lin) ++sj;
       ++seq;
     }
@@ -1065,6 +1132,23 @@ cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+// The profiling build's buffer: kProfRecorders x kProfEvents uint64 stamps per
+// CTA, for the first bytes / (8 * kProfRecorders * kProfEvents) CTAs.
+int set_profile_buffer(void* dev, size_t bytes) {
+#ifdef SALAD_PROFILE
+  const int ctas = (int)(bytes / (sizeof(uint64_t) * kProfRecorders * kProfEvents));
+  uint64_t* p = static_cast<uint64_t*>(dev);
+  if (cudaMemcpyToSymbol(g_prof_buf, &p, sizeof(p)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_prof_ctas, &ctas, sizeof(ctas)) != cudaSuccess)
+    return SALAD_ERR_CUDA;
+  return SALAD_OK;
+#else
+  (void)dev;
+  (void)bytes;
+  return SALAD_ERR_UNSUPPORTED;
+#endif
+}
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s) {
   if (a.tiles.bt > 0) return a.d == 64 ? launch_attn_t<64, 128, true>(a, s) : launch_attn_t<128, 128, true>(a, s);

@@ -100,6 +100,9 @@ struct AttnArgs {
   uint64_t wait_limit_ns;
 };
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+// Profiling build only (SALAD_PROFILE): the attention kernel's phase-stamp
+// buffer; SALAD_ERR_UNSUPPORTED in the normal build.
+int set_profile_buffer(void* dev, size_t bytes);
 
 // Backward pass of the sparse branch (bwd.cu); raster blocks of 128 tokens.
 struct BwdArgs {
