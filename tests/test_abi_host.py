@@ -327,3 +327,18 @@ def test_static_scratch_limit_matches_the_stated_figure(L):
 def test_static_status_reader_and_out_of_memory_status_are_exported(L):
     assert L.salad_status_string(sl.SALAD_ERR_OUT_OF_MEMORY).decode().startswith("device out of memory")
     assert hasattr(L, "salad_check_status_static")
+
+
+def test_head_range_forward_argument_errors(L):
+    def call(**kw):
+        a = dict(B=1, N=256, Ht=4, h0=0, hc=2, d=64, block=64)
+        a.update(kw)
+        return L.salad_attn_forward_heads(p(FAKE), p(FAKE + 0x10000000), p(FAKE + 0x20000000), a["B"], a["N"],
+                                          a["Ht"], a["h0"], a["hc"], a["d"], a["block"], p(FAKE), p(FAKE), p(FAKE),
+                                          p(FAKE), 0.0, 1e-6, p(FAKE + 0x30000000), p(0x40000000), 1 << 30, None)
+    assert call(h0=-1) == sl.SALAD_ERR_INVALID_ARG
+    assert call(hc=0) == sl.SALAD_ERR_INVALID_ARG
+    assert call(h0=3, hc=2) == sl.SALAD_ERR_INVALID_ARG        # past the last head
+    assert call(Ht=0) == sl.SALAD_ERR_INVALID_ARG
+    assert call(d=96) == sl.SALAD_ERR_UNSUPPORTED
+    assert call(Ht=70000, hc=1) == sl.SALAD_ERR_UNSUPPORTED
