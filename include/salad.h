@@ -328,6 +328,23 @@ int salad_attn_forward_bh(const void* q, const void* k, const void* v, int B, in
                           size_t workspace_bytes, salad_stream_t stream);
 
 /*
+ * The transpose of a block mask, for the backward pass (its dk and dv walk
+ * the query blocks that keep a key block).  For every group g (a head, or a
+ * (b, h) for a mask with rows per (b, h)) and key block J, t_col_idx lists in
+ * ascending order the query blocks I whose row (g, I) keeps J.
+ *   row_ptr, col_idx  DEVICE, groups*nb rows with ascending columns (as the mask
+ *                     builders write them).
+ *   t_row_ptr         DEVICE int32 [groups*nb + 1], written.
+ *   t_col_idx         DEVICE int32 [nnz], nnz = row_ptr[groups*nb] (a
+ *                     transpose keeps every pair), written.
+ * Asynchronous on `stream`; deterministic.  The window masks are symmetric and
+ * are their own transpose.  Errors: INVALID_ARG (null, misaligned, non-positive
+ * sizes), UNSUPPORTED (groups > 65535 or groups*nb*nb >= 2^31), CUDA.
+ */
+int salad_transpose_block_mask(const int32_t* row_ptr, const int32_t* col_idx, int groups, int nb,
+                               int32_t* t_row_ptr, int32_t* t_col_idx, salad_stream_t stream);
+
+/*
  * salad_attn_forward on a range of heads: q, k, v and out are full
  * [B][N][heads_total][d] tensors, and the call reads and writes heads
  * [head_begin, head_begin + head_count) of them only.  The layer's (b, h) units

@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.salad_build_tile_mask.argtypes = [i, i, i, i, i, i, i, p, p, p, ctypes.c_int64,
                                             ctypes.POINTER(ctypes.c_int64), p]
         L.salad_build_tile_mask.restype = i
+        L.salad_transpose_block_mask.argtypes = [p, p, i, i, p, p, p]
+        L.salad_transpose_block_mask.restype = i
         L.salad_validate_mask.argtypes = [p, p, ctypes.c_int64, i, ctypes.POINTER(ctypes.c_int64)]
         L.salad_validate_mask.restype = i
         L.salad_workspace_bytes.argtypes = [i, i, i, i]
@@ -284,15 +286,28 @@ def attn_forward_heads(q, k, v, head_begin: int, head_count: int, row_ptr, col_i
     return out
 
 
-def _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh):
+def transpose_block_mask(row_ptr, col_idx, groups: int, nb: int, stream=None):
+    """The transposed mask on the GPU (salad_transpose_block_mask): for every
+    group (head, or (b, h)) and key block J, the ascending query blocks whose
+    row keeps J.  Returns (t_row_ptr, t_col_idx), int32 CUDA tensors."""
+    t_row_ptr = torch.empty(groups * nb + 1, dtype=torch.int32, device=row_ptr.device)
+    t_col_idx = torch.empty(max(1, col_idx.numel()), dtype=torch.int32, device=row_ptr.device)
+    _check(lib().salad_transpose_block_mask(
+        _dev_ptr(row_ptr, torch.int32, "row_ptr"), _dev_ptr(col_idx, torch.int32, "col_idx"), int(groups), int(nb),
+        _dev_ptr(t_row_ptr, torch.int32, "t_row_ptr"), _dev_ptr(t_col_idx, torch.int32, "t_col_idx"),
+        _stream(stream)), "salad_transpose_block_mask")
+    return t_row_ptr, t_col_idx[:col_idx.numel()]
+
+
+def _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh, groups=0, nb=0):
     """The transposed mask the backward walks for dk and dv: given, or the mask
-    itself for the symmetric window masks (rows per head).  A mask with rows
-    per (b, h) (Top-K) is not symmetric, so its transpose must be given."""
+    itself for the symmetric window masks (rows per head), or built on the GPU
+    for a mask with rows per (b, h) (Top-K), which is not symmetric."""
     if (t_row_ptr is None) != (t_col_idx is None):
         raise ValueError("give both t_row_ptr and t_col_idx, or neither")
     if t_row_ptr is None:
         if mask_per_bh:
-            raise ValueError("a mask with rows per (b, h) needs its transpose (t_row_ptr, t_col_idx)")
+            return transpose_block_mask(row_ptr, col_idx, groups, nb)
         return row_ptr, col_idx
     return t_row_ptr, t_col_idx
 
@@ -305,7 +320,8 @@ def attn_backward_sparse(q, k, v, o, dout, lse, row_ptr, col_idx, block: int = 1
     the transposed mask defaults to the mask itself, which is right for the
     symmetric window masks; a mask with rows per (b, h) needs its transpose."""
     B, N, Hh, d = q.shape
-    t_row_ptr, t_col_idx = _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh)
+    t_row_ptr, t_col_idx = _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh, B * Hh,
+                                            (N + block - 1) // block)
     grads = [torch.empty(B, N, Hh, d, dtype=torch.float32, device=q.device) for _ in range(3)]
     if workspace is None:
         workspace = torch.zeros(lib().salad_backward_workspace_bytes(B, N, Hh), dtype=torch.uint8, device=q.device)
@@ -328,7 +344,8 @@ def attn_backward(q, k, v, out, dout, lse, row_ptr, col_idx, w_proj, gate, block
     dv [B, N, Hh, d], dw [d, d] and dgate [B, Hh].  out and lse come from
     attn_forward_lse on the same inputs."""
     B, N, Hh, d = q.shape
-    t_row_ptr, t_col_idx = _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh)
+    t_row_ptr, t_col_idx = _transposed_mask(row_ptr, col_idx, t_row_ptr, t_col_idx, mask_per_bh, B * Hh,
+                                            (N + block - 1) // block)
     res = {n: torch.empty(B, N, Hh, d, dtype=torch.float32, device=q.device) for n in ("dq", "dk", "dv")}
     res["dw"] = torch.empty(d, d, dtype=torch.float32, device=q.device)
     res["dgate"] = torch.empty(B, Hh, dtype=torch.float32, device=q.device)

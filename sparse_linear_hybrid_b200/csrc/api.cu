@@ -562,6 +562,19 @@ int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B,
                            eps, out, workspace, workspace_bytes, stream, 0, &g);
 }
 
+int salad_transpose_block_mask(const int32_t* row_ptr, const int32_t* col_idx, int groups, int nb,
+                               int32_t* t_row_ptr, int32_t* t_col_idx, salad_stream_t stream) {
+  if (!row_ptr || !col_idx || !t_row_ptr || !t_col_idx || groups < 1 || nb < 1) return SALAD_ERR_INVALID_ARG;
+  if (!aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(t_row_ptr, 4) || !aligned(t_col_idx, 4))
+    return SALAD_ERR_INVALID_ARG;
+  // (one CTA row per group; every pair must be addressable by an int32 offset)
+  if (groups > 65535 || (long long)groups * nb * nb >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
+  return launch_mask_transpose(row_ptr, col_idx, groups, nb, t_row_ptr, t_col_idx,
+                               reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SALAD_OK
+             : SALAD_ERR_CUDA;
+}
+
 int salad_validate_mask(const int32_t* row_ptr, const int32_t* col_idx, int64_t rows, int nb, int64_t* bad_row) {
   if (bad_row) *bad_row = -1;
   if (!row_ptr || rows < 0 || nb < 1) return SALAD_ERR_INVALID_ARG;

@@ -27,6 +27,9 @@ cudaError_t launch_mask_count(const MaskGrid& g, const WindowTable& win, int32_t
 cudaError_t launch_mask_scan(int32_t* row_ptr, int n, cudaStream_t s);
 cudaError_t launch_mask_fill(const MaskGrid& g, const WindowTable& win, const int32_t* row_ptr, int32_t* col_idx,
                              cudaStream_t s);
+// The transposed mask of `groups` x nb rows (count, scan, fill).
+cudaError_t launch_mask_transpose(const int32_t* row_ptr, const int32_t* col_idx, int groups, int nb,
+                                  int32_t* t_row_ptr, int32_t* t_col_idx, cudaStream_t s);
 
 // Workspace layout of the forward pass (byte offsets from the workspace base).
 struct WorkspaceLayout {

@@ -133,6 +133,63 @@ cudaError_t launch_mask_count(const MaskGrid& g, const WindowTable& win, int32_t
   return cudaGetLastError();
 }
 
+namespace {
+
+// ---------------------------------------------------------------- transpose
+// The transposed mask: for every group g (a head, or a (b, h) of a mask with
+// rows per (b, h)) and key block J, the ascending query blocks I whose row
+// keeps J.  One warp per column (g, J) walks the query blocks 32 at a time and
+// tests membership by binary search in each row's ascending list; a ballot
+// counts (first pass) or places (second pass) the hits in order, so the result
+// is deterministic and needs no sort.
+__device__ __forceinline__ bool row_keeps(const int32_t* row_ptr, const int32_t* col_idx, int r, int J) {
+  int lo = row_ptr[r], hi = row_ptr[r + 1];  // [lo, hi)
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int c = col_idx[mid];
+    if (c == J) return true;
+    if (c < J) {
+      lo = mid + 1;
+    } else {
+      hi = mid;
+    }
+  }
+  return false;
+}
+
+template <bool FILL>
+__global__ void __launch_bounds__(128) mask_t_kernel(const int32_t* __restrict__ row_ptr,
+                                                     const int32_t* __restrict__ col_idx, int nb,
+                                                     int32_t* __restrict__ t_row_ptr, int32_t* __restrict__ t_col_idx) {
+  const int lane = threadIdx.x & 31;
+  const int J = blockIdx.x * 4 + (threadIdx.x >> 5), g = blockIdx.y;
+  if (J >= nb) return;
+  int pos = FILL ? t_row_ptr[(size_t)g * nb + J] : 0;
+  for (int I0 = 0; I0 < nb; I0 += 32) {
+    const int I = I0 + lane;
+    const bool has = I < nb && row_keeps(row_ptr, col_idx, g * nb + I, J);
+    const uint32_t m = __ballot_sync(0xffffffffu, has);
+    if (FILL && has) t_col_idx[pos + __popc(m & ((1u << lane) - 1u))] = I;
+    pos += __popc(m);
+  }
+  if (!FILL && lane == 0) t_row_ptr[(size_t)g * nb + J + 1] = pos;  // counts, then the scan
+}
+
+}  // namespace
+
+cudaError_t launch_mask_transpose(const int32_t* row_ptr, const int32_t* col_idx, int groups, int nb,
+                                  int32_t* t_row_ptr, int32_t* t_col_idx, cudaStream_t s) {
+  const dim3 grid((nb + 3) / 4, groups);
+  mask_t_kernel<false><<<grid, 128, 0, s>>>(row_ptr, col_idx, nb, t_row_ptr, nullptr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  mask_scan_kernel<<<1, 1024, 0, s>>>(t_row_ptr, groups * nb);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  mask_t_kernel<true><<<grid, 128, 0, s>>>(row_ptr, col_idx, nb, t_row_ptr, t_col_idx);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mask_scan(int32_t* row_ptr, int n, cudaStream_t s) {
   mask_scan_kernel<<<1, 1024, 0, s>>>(row_ptr, n);
   return cudaGetLastError();

@@ -268,12 +268,15 @@ def test_backward_argument_errors(L):
     assert L.salad_layer_backward_workspace_bytes(1, 256, 2, 96) == 0
 
 
-def test_backward_binding_needs_the_transpose_of_a_per_bh_mask():
+def test_backward_binding_builds_or_takes_the_transpose_of_a_per_bh_mask():
     import torch
     x = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
     idx = torch.zeros(2, dtype=torch.int32)
-    with pytest.raises(ValueError):
+    # without a transpose, a mask with rows per (b, h) gets one built by the
+    # library's kernels, which take device tensors only (no CPU path)
+    with pytest.raises(TypeError, match="CUDA tensor"):
         sl.attn_backward_sparse(x, x, x, x, x, torch.zeros(1, 1, 128), idx, idx, mask_per_bh=True)
+    # half a transpose is refused
     with pytest.raises(ValueError):
         sl.attn_backward(x, x, x, x, x, torch.zeros(1, 1, 128), idx, idx, x, torch.zeros(1, 1), t_row_ptr=idx)
 
@@ -342,3 +345,13 @@ def test_head_range_forward_argument_errors(L):
     assert call(Ht=0) == sl.SALAD_ERR_INVALID_ARG
     assert call(d=96) == sl.SALAD_ERR_UNSUPPORTED
     assert call(Ht=70000, hc=1) == sl.SALAD_ERR_UNSUPPORTED
+
+
+def test_transpose_mask_argument_errors(L):
+    T = L.salad_transpose_block_mask
+    assert T(None, p(FAKE), 1, 4, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_INVALID_ARG
+    assert T(p(FAKE), p(FAKE), 0, 4, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_INVALID_ARG
+    assert T(p(FAKE), p(FAKE), 1, 0, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_INVALID_ARG
+    assert T(p(FAKE + 2), p(FAKE), 1, 4, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_INVALID_ARG
+    assert T(p(FAKE), p(FAKE), 70000, 4, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_UNSUPPORTED
+    assert T(p(FAKE), p(FAKE), 1, 50000, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_UNSUPPORTED
