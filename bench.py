@@ -114,6 +114,13 @@ def kept_pairs_flops(row_ptr: np.ndarray, col_idx: np.ndarray, wl: si.Workload) 
     return 4.0 * wl.d * pairs * (1 if mask_per_bh(wl) else wl.B)
 
 
+def layer_backward_linear_flops(wl: si.Workload) -> float:
+    """Counted FLOPs of the layer backward's linear branch, projection and gate:
+    about 7 d^2 multiply-adds per token per (b, h) for the row and per-key terms
+    and the dS contraction, plus d^2 per token for dW (2 FLOPs each)."""
+    return 2.0 * 8.0 * wl.d * wl.d * wl.N * wl.B * wl.Hh
+
+
 def block_flops(row_ptr, col_idx, wl, pairs):
     nb = wl.nb
     sizes = block_sizes(wl)
@@ -302,6 +309,14 @@ class RankGroup:
         if self._dist is not None:
             self._dist.barrier()
 
+    def sum_over_ranks(self, x: float) -> float:
+        if self._dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self._dist.all_reduce(t, op=self._dist.ReduceOp.SUM)
+        return float(t.item())
+
     def max_over_ranks(self, x: float) -> float:
         if self._dist is None:
             return x
@@ -316,25 +331,39 @@ class RankGroup:
             self._dist = None
 
 
+def rank_heads(wl: si.Workload, rank: int, world: int) -> tuple[int, int]:
+    """Head split (--split heads): rank r's contiguous range (head_begin,
+    head_count) of the workload's heads; all ranks share one layer (strong
+    scaling) and exchange nothing in the forward pass."""
+    from sparse_linear_hybrid_b200.heads import head_ranges
+    return head_ranges(wl.Hh, world)[rank]
+
+
 def rank_workload(wl: si.Workload, rank: int) -> si.Workload:
     """Weak scaling: every rank runs its own batch of the workload (same shapes,
     its own seed)."""
     return wl.with_(seed=wl.seed + 1000 * rank)
 
 
+def job_tflops(steps: int, job_flops_per_step: float, total_ms: float) -> float:
+    """Throughput of the whole job: the kept work of all ranks per step, over the
+    slowest rank's time for the steps."""
+    return steps * job_flops_per_step / (total_ms / 1e3) / 1e12
+
+
 def whole_job_tflops(world: int, steps: int, flops_per_step: float, total_ms: float) -> float:
-    """Throughput of the whole job: the work of all ranks over the slowest rank's time."""
-    return world * steps * flops_per_step / (total_ms / 1e3) / 1e12
+    """The same with replicas: every rank did flops_per_step each step."""
+    return job_tflops(steps, world * flops_per_step, total_ms)
 
 
-def config_of(wl: si.Workload, flops: float, nnz: int, world: int):
+def config_of(wl: si.Workload, flops: float, nnz: int, world: int, split: str = "replicas"):
     rows = wl.B * wl.Hh * wl.nb if wl.topk else wl.Hh * wl.nb
     mask = {"topk_keep": wl.topk} if wl.topk else {"window_thw": list(wl.window)}
     blocks = {"tile_thw": list(wl.tile), "blocks_per_head": wl.nb} if wl.tile else {}
     return {"workload": wl.name, "B": wl.B, "heads": wl.Hh, "d": wl.d,
             "grid_THW": [wl.T, wl.H, wl.W], "tokens": wl.N, "block": wl.block, **blocks,
             **mask, "block_sparsity": round(1 - nnz / (rows * wl.nb), 5),
-            "kept_gflop_per_step": round(flops / 1e9, 3), "parallelism": f"replicas{world}",
+            "kept_gflop_per_step": round(flops / 1e9, 3), "parallelism": f"{split}{world}",
             "l2": "flushed between steps (256 MB write outside the timed events)"}
 
 
@@ -478,7 +507,7 @@ def run_reference(args, wl):
 
 
 # --------------------------------------------------------------------------- GPU leg
-def run_e2e(args, inputs, out, flush, step, flops, world, max_over_ranks, barrier):
+def run_e2e(args, inputs, out, flush, step, flops_job, max_over_ranks, barrier):
     """Same metric end to end: every step copies its inputs (`inputs`: name ->
     device tensor) from pinned host memory, runs the C-ABI forward and copies
     the output back, all between the CUDA events.  Two untimed warm-up steps
@@ -502,7 +531,7 @@ def run_e2e(args, inputs, out, flush, step, flops, world, max_over_ranks, barrie
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev[2:]))
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = out_h.numel() * out_h.element_size()
-    return {"value": round(world * ke * flops / (e2e_ms / 1e3) / 1e12, 3), "unit": UNIT,
+    return {"value": round(job_tflops(ke, flops_job, e2e_ms), 3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms / ke, 3),
             "steps": ke}
 
@@ -517,6 +546,7 @@ def run_salad(args, wl):
     import torch
 
     import sparse_linear_hybrid_b200 as sl
+    from sparse_linear_hybrid_b200.heads import gather_heads
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -524,8 +554,14 @@ def run_salad(args, wl):
     ranks = RankGroup("nccl", dev)
     barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
-    my_wl = rank_workload(wl, rank)
+    split_heads = args.split == "heads"
+    if split_heads and (wl.topk or wl.tile or wl.itads):
+        raise SystemExit("--split heads runs the window-mask workloads with raster blocks")
+    # replicas: every rank its own batch (its own seed); heads: one layer, each
+    # rank its range of heads of the same inputs
+    my_wl = wl if split_heads else rank_workload(wl, rank)
     inp = si.make_inputs(my_wl)
+    h0, hc = rank_heads(wl, rank, world) if split_heads else (0, wl.Hh)
 
     def up(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -541,14 +577,18 @@ def run_salad(args, wl):
         topk.run()
         mask_ms = topk.device_ms()
     else:
-        row_ptr, col_idx = build_window_mask(sl, wl, inp.windows, dev)
+        wins = inp.windows[h0:h0 + hc]
+        row_ptr, col_idx = build_window_mask(sl, wl, wins, dev)
         # the mask build once more into the same buffers, on the device clock (the
         # first call above also sizes col_idx and loads the kernels)
-        mask_ms = time_block_mask(wl, inp.windows, row_ptr, col_idx)
+        mask_ms = time_block_mask(wl, wins, row_ptr, col_idx)
     rp_h, ci_h = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
-    flops = kept_pairs_flops(rp_h, ci_h, wl)
+    flops = kept_pairs_flops(rp_h, ci_h, wl)            # this rank's kept work per step
+    flops_job = ranks.sum_over_ranks(flops) if split_heads else world * flops
     nnz = int(rp_h[-1])
-    ws = sl.new_workspace(wl.B, wl.N, wl.Hh, wl.d, dev)
+    nnz_job = int(ranks.sum_over_ranks(nnz)) if split_heads else nnz
+    ws = sl.new_workspace(wl.B, wl.N, hc, wl.d, dev)
+    gate_used = gate[:, h0:h0 + hc].contiguous() if split_heads else gate
     out = torch.empty_like(q)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
@@ -574,7 +614,11 @@ def run_salad(args, wl):
         e2e_inputs = dict(q=q, k=k, v=v, w=w, **gdev)
 
     def forward(rp, ci, g):
-        if wl.tile:
+        if split_heads:
+            sl.attn_forward_heads(q, k, v, h0, hc, rp, ci, w, g, wl.block, out=out, workspace=ws)
+            if args.gather:
+                gather_heads(out, rank, world)
+        elif wl.tile:
             sl.attn_forward_tiles(q, k, v, (wl.T, wl.H, wl.W), wl.tile, rp, ci, w, g, out=out, workspace=ws)
         else:
             sl.attn_forward(q, k, v, rp, ci, w, g, wl.block, out=out, workspace=ws, mask_per_bh=topk is not None)
@@ -584,7 +628,7 @@ def run_salad(args, wl):
             topk.run()
         if gate_step is not None:
             gate_step()
-        forward(row_ptr, col_idx, gate)
+        forward(row_ptr, col_idx, gate_used)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -643,7 +687,9 @@ def run_salad(args, wl):
     unflushed_ms = statistics.median(a.elapsed_time(b) for a, b in uev)
     total_ms = max_over_ranks(sum(step_ms))
     ms_per_step = total_ms / K
-    value = whole_job_tflops(world, K, flops, total_ms)
+    # the whole job's kept work per step (replicas: every rank its own batch;
+    # heads: the ranks' ranges of one layer) over the slowest rank's time
+    value = job_tflops(K, flops_job, total_ms)
 
     peaks = load_peaks()
     timed_s = sum(step_ms) / 1e3
@@ -678,13 +724,13 @@ def run_salad(args, wl):
     # from pinned memory, the forward, D2H of the output, all inside the events
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, e2e_inputs, out, flush, step, flops, world, max_over_ranks, barrier)
+        e2e = run_e2e(args, e2e_inputs, out, flush, step, flops_job, max_over_ranks, barrier)
 
     dense = None
     if not args.no_dense:
         dwl = wl.with_(window=(wl.T, wl.H, wl.W), topk=0)
-        drp, dci = build_window_mask(sl, dwl, dwl.windows(), dev)
-        zero_gate = torch.zeros_like(gate)
+        drp, dci = build_window_mask(sl, dwl, dwl.windows()[h0:h0 + hc], dev)
+        zero_gate = torch.zeros_like(gate_used)
         dflops = kept_pairs_flops(drp.cpu().numpy(), dci.cpu().numpy(), dwl)
         dev_ev = [(E(), E()) for _ in range(5)]
         for i in range(6):
@@ -704,7 +750,7 @@ def run_salad(args, wl):
     # its output and log-sum-exp from a gate-0 forward, a seeded dout, K timed
     # steps with the L2 flush between them (not part of the headline step)
     backward = None
-    if not args.no_backward and not wl.tile and not wl.topk and wl.block == 128:
+    if not args.no_backward and not wl.tile and not wl.topk and wl.block == 128 and not split_heads:
         zero_gate = torch.zeros_like(gate)
         o_sp, lse = sl.attn_forward_lse(q, k, v, row_ptr, col_idx, w, zero_gate, wl.block, workspace=ws)
         g_bits = si.f32_to_bf16_bits(np.random.default_rng(my_wl.seed + 99).standard_normal(
@@ -730,7 +776,35 @@ def run_salad(args, wl):
                     "frac": round(bflops / (bms / 1e3) / 1e12 / peak, 4),
                     "algorithmic": "2.5 x the forward's kept FLOPs (the S, dP, dV, dK and dQ products; the two "
                                    "kernels each recompute S and dP, so 3.5 x is executed)", "steps": kb}
-        del o_sp, lse, dout, bws
+        # the whole layer's backward (both branches, the projection and the gate)
+        # on the workload's own gates: a forward with the log-sum-exp, then
+        # salad_attn_backward, K timed steps with the L2 flush between them
+        out_l, lse_l = sl.attn_forward_lse(q, k, v, row_ptr, col_idx, w, gate, wl.block, workspace=ws)
+        lws = torch.zeros(sl.lib().salad_layer_backward_workspace_bytes(wl.B, wl.N, wl.Hh, wl.d), dtype=torch.uint8,
+                          device=dev)
+        lev = [(E(), E()) for _ in range(kb)]
+        for i in range(3 + kb):
+            flush.zero_()
+            if i >= 3:
+                lev[i - 3][0].record()
+            sl.attn_backward(q, k, v, out_l, dout, lse_l, row_ptr, col_idx, w, gate, workspace=lws)
+            if i >= 3:
+                lev[i - 3][1].record()
+        torch.cuda.synchronize()
+        if sl.check_status(lws) != sl.SALAD_OK:
+            raise RuntimeError("device status after the layer backward steps")
+        lms = statistics.median(a.elapsed_time(b) for a, b in lev)
+        lin_flops = layer_backward_linear_flops(wl)
+        lflops = 2.5 * flops + lin_flops
+        backward["layer"] = {
+            "what": "dq, dk, dv, dW, dgate of the whole layer (salad_attn_backward: the linear state, the row "
+                    "kernel, the sparse branch, the reductions and the per-key terms)",
+            "ms_per_step_p50": round(lms, 4), "tflops": round(lflops / (lms / 1e3) / 1e12, 2),
+            "frac": round(lflops / (lms / 1e3) / 1e12 / peak, 4),
+            "algorithmic": "2.5 x the forward's kept FLOPs + 16 d^2 per token per (b,h) for the linear branch, "
+                           "projection and gate", "gflop_linear_part": round(lin_flops / 1e9, 2),
+            "workspace_mb": round(lws.numel() / 1e6, 1), "steps": kb}
+        del o_sp, lse, dout, bws, out_l, lse_l, lws
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -746,8 +820,11 @@ def run_salad(args, wl):
         line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
                 "ms_per_step_unflushed_p50": round(unflushed_ms, 4),
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {**config_of(wl, flops, nnz, world), **(gate_desc or {})},
+                "scaling": "strong" if split_heads else "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {**config_of(wl, flops_job / (1 if split_heads else world), nnz_job, world,
+                                       "heads" if split_heads else "replicas"), **(gate_desc or {}),
+                           **({"heads_per_rank": hc, "gather": bool(args.gather)} if split_heads else {})},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": (3 + (2 if wl.topk else 0) + (2 if wl.itads else 0)) * K,
                 "clocks": clk, "kernels": kernels, "dense": dense, "backward": backward,
@@ -771,6 +848,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle forward budget for cpu_baseline")
+    ap.add_argument("--split", choices=["replicas", "heads"], default="replicas",
+                    help="multi-GPU: every rank its own batch (weak scaling), or the ranks split one layer's "
+                         "heads (strong scaling)")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --split heads: all-gather the output's heads to every rank in each step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -24,6 +24,16 @@ def main():
     res = {"rank": rank, "world": world}
     g.barrier()
     res["max"] = g.max_over_ranks(10.0 + rank)
+    # head split: the ranks' ranges of one layer, their kept work adds up to the layer's
+    import oracle
+    lay = si.TINY.with_(Hh=5, seed=3)
+    linp = si.make_inputs(lay)
+    h0, hc = bench.rank_heads(lay, rank, world)
+    rp, ci = oracle.block_mask(lay.T, lay.H, lay.W, lay.block, linp.windows[h0:h0 + hc])
+    res["heads"] = [h0, hc]
+    res["flops_sum"] = g.sum_over_ranks(bench.kept_pairs_flops(rp, ci, lay))
+    frp, fci = oracle.block_mask(lay.T, lay.H, lay.W, lay.block, linp.windows)
+    res["flops_layer"] = bench.kept_pairs_flops(frp, fci, lay)
     wl = bench.rank_workload(si.TINY, rank)
     inp = si.make_inputs(wl)
     res["seed"] = wl.seed

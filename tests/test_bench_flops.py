@@ -44,3 +44,8 @@ def test_peak_fractions_three_denominators():
     assert abs(f["sm_clock_peak_tflops"] - 148 * 1965e6 * 8192 / 1e12) < 0.1
     assert abs(f["sm_clock"] - 1000 / (148 * 1965e6 * 8192 / 1e12)) < 1e-4
     assert "sm_clock" not in bench.peak_fractions(1000.0, 1671.5, 148, None)
+
+
+def test_layer_backward_linear_flops():
+    wl = si.WORKLOADS["wan1.3b-32760tok-90pct"]
+    assert bench.layer_backward_linear_flops(wl) == 16 * 128 * 128 * 32760 * 12

@@ -44,6 +44,9 @@ def test_two_ranks_over_gloo():
     assert sorted(res) == [0, 1] and all(r["world"] == 2 for r in res.values())
     # max over ranks reaches every rank
     assert res[0]["max"] == res[1]["max"] == 11.0
+    # head split: contiguous ranges of the 5 heads; their kept work sums to the layer's
+    assert res[0]["heads"] == [0, 3] and res[1]["heads"] == [3, 2]
+    assert res[0]["flops_sum"] == res[1]["flops_sum"] == res[0]["flops_layer"]
     # weak scaling: same shapes, own seed, different data
     assert res[0]["q_shape"] == res[1]["q_shape"]
     assert res[0]["seed"] != res[1]["seed"] and res[0]["q_sum"] != res[1]["q_sum"]
@@ -58,3 +61,5 @@ def test_whole_job_throughput_is_all_ranks_work_over_the_slowest_time():
     # 2 ranks x 10 steps x 1 TFLOP in 1 s (the max over ranks) = 20 TFLOP/s
     assert bench.whole_job_tflops(2, 10, 1e12, 1000.0) == 20.0
     assert bench.whole_job_tflops(1, 5, 2e12, 500.0) == 20.0
+    # a head split: one layer of 3 TFLOP per step shared by the ranks, 10 steps in 1 s
+    assert bench.job_tflops(10, 3e12, 1000.0) == 30.0
