@@ -225,9 +225,15 @@ int salad_attn_backward_sparse(const void* q, const void* k, const void* v, cons
  *   dw         DEVICE fp32 [d][d];  dgate DEVICE fp32 [B][Hh] (written).
  *   workspace  DEVICE, >= salad_layer_backward_workspace_bytes(B, N, Hh, d),
  *              256-byte aligned, status word first (zero it once).
- * Other arguments as salad_attn_backward_sparse.  The linear branch's terms are
- * fp32 CUDA-core arithmetic in a fixed order (deterministic).  Errors:
- * INVALID_ARG, UNSUPPORTED (d, block != 128, B*Hh > 65534), WORKSPACE, CUDA.
+ * Other arguments as salad_attn_backward_sparse.  The linear branch runs on the
+ * tensor cores through T = S W: a_i T and dout_i T^T per row, M = sum_i a_i^T
+ * (g / den_i) dout_i over the rows, dS = M W^T and dW = sum over (b, h) of S^T M;
+ * every operand that is not already bf16 (T, (g / den_i) dout_i, dS) enters as
+ * bf16 hi + lo halves, accumulation is fp32 and every sum runs in a fixed order
+ * (deterministic).  The workspace is O(B Hh (N + d^2)), about 30 MB for
+ * 32,760 tokens x 12 heads of d = 128.  Errors: INVALID_ARG, UNSUPPORTED (d,
+ * block != 128, B*Hh > 65535), WORKSPACE, CUDA; a stalled wait sets the status
+ * word's time-out bit (salad_check_status).
  */
 size_t salad_layer_backward_workspace_bytes(int B, int N, int num_heads, int d);
 int salad_attn_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,

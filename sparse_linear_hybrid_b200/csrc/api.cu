@@ -96,9 +96,11 @@ int check_common(const void* k, const void* v, int B, int N, int Hh, int d, void
 }
 
 // The linear-branch kernels.  Forward (S_out == nullptr): z and (S W)^T into the
-// workspace.  State export: S and z into S_out / z_out.
+// workspace.  State export: S and z into S_out / z_out, with with_t also (S W)^T
+// into the workspace.
 int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const float* gate, const void* w_proj,
-               float* S_out, float* z_out, uint8_t* ws, const WorkspaceLayout& L, cudaStream_t s, int Hh_total = 0) {
+               float* S_out, float* z_out, uint8_t* ws, const WorkspaceLayout& L, cudaStream_t s, int Hh_total = 0,
+               bool with_t = false) {
   CUtensorMap tk, tv;
   if (!make_bnhd_map(&tk, k, B, N, Hh, d, 64, Hh_total) || !make_bnhd_map(&tv, v, B, N, Hh, d, 64, Hh_total))
     return SALAD_ERR_CUDA;
@@ -111,6 +113,7 @@ int run_linear(const void* k, const void* v, int B, int N, int Hh, int d, const 
   la.t_op = reinterpret_cast<uint16_t*>(ws + L.off_t);
   la.z = S_out ? z_out : reinterpret_cast<float*>(ws + L.off_z);
   la.S_out = S_out;
+  la.with_t = with_t;
   la.work_ctr = reinterpret_cast<uint32_t*>(ws + L.off_status) + 1;
   la.B = B;
   la.N = N;
@@ -404,29 +407,28 @@ int salad_attn_backward_sparse(const void* q, const void* k, const void* v, cons
 namespace {
 // Workspace of the layer backward (byte offsets; every region 256-byte aligned).
 struct LayerBwdLayout {
-  WorkspaceLayout fwd;  // the forward's workspace (status word at 0, the state export's partials)
-  size_t off_S, off_z, off_lse2, off_dvec, off_o, off_dy, off_du, off_dden, off_yg, off_partial, off_dS, off_dz, total;
-  int splits, npad;
+  WorkspaceLayout fwd;  // the forward's workspace (status word at 0, (S W)^T, the state's partials)
+  size_t off_S, off_z, off_lse2, off_dvec, off_mpart, off_dzpart, off_dgpart, off_dwpart, off_ds, off_dz, total;
+  int splits, tiles_per_split, npad;
 };
 LayerBwdLayout layer_bwd_layout(int B, int N, int heads, int d) {
   LayerBwdLayout L{};
   L.fwd = workspace_layout(B, N, heads, d);
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t BH = (size_t)B * heads, rows = (size_t)B * N * heads;
+  const size_t BH = (size_t)B * heads;
   L.npad = (N + 127) / 128 * 128;
-  L.splits = 8;
+  linear_backward_splits((int)BH, N, d, &L.splits, &L.tiles_per_split);
+  const size_t S = (size_t)L.splits;
   size_t o = up(L.fwd.total);
   L.off_S = o;       o += up(BH * d * d * 4);
   L.off_z = o;       o += up(BH * d * 4);
   L.off_lse2 = o;    o += up(BH * L.npad * 4);
   L.off_dvec = o;    o += up(BH * L.npad * 4);
-  L.off_o = o;       o += up(rows * d * 4);
-  L.off_dy = o;      o += up(rows * d * 4);
-  L.off_du = o;      o += up(rows * d * 4);
-  L.off_dden = o;    o += up(BH * N * 4);
-  L.off_yg = o;      o += up(BH * N * 4);
-  L.off_partial = o; o += up((size_t)2 * L.splits * BH * d * d * 4);
-  L.off_dS = o;      o += up(BH * d * d * 4);
+  L.off_mpart = o;   o += up(S * BH * d * d * 4);
+  L.off_dzpart = o;  o += up(S * BH * d * 4);
+  L.off_dgpart = o;  o += up(S * BH * 4);
+  L.off_dwpart = o;  o += up(BH * (d / 16) * d * d * 4);
+  L.off_ds = o;      o += up(BH * d * 2 * d * 2);
   L.off_dz = o;      o += up(BH * d * 4);
   L.total = o;
   return L;
@@ -452,8 +454,8 @@ int salad_attn_backward(const void* q, const void* k, const void* v, const void*
   if (B < 1 || N < 1 || num_heads < 1) return SALAD_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SALAD_ERR_UNSUPPORTED;
   if (block != 128) return SALAD_ERR_UNSUPPORTED;
-  // (the reductions run B*Hh + 1 rows of CTAs: at most 65535)
-  if ((long long)B * num_heads > 65534 || (long long)B * num_heads * ((N + 127) / 128) >= (1ll << 31))
+  // (the streaming kernels run B*Hh rows of CTAs: at most 65535)
+  if ((long long)B * num_heads > 65535 || (long long)B * num_heads * ((N + 127) / 128) >= (1ll << 31))
     return SALAD_ERR_UNSUPPORTED;
   const void* p16[] = {q, k, v, out, dout, w_proj, dq, dk, dv};
   for (const void* ptr : p16)
@@ -467,15 +469,27 @@ int salad_attn_backward(const void* q, const void* k, const void* v, const void*
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
-  // 1. the linear branch's state S, z (fp32)
-  int st = run_linear(k, v, B, N, num_heads, d, nullptr, w_proj, F(L.off_S), F(L.off_z), ws, L.fwd, s);
+  // 1. the linear branch's state S, z (fp32) and T = S W (bf16 hi + lo)
+  int st = run_linear(k, v, B, N, num_heads, d, nullptr, w_proj, F(L.off_S), F(L.off_z), ws, L.fwd, s, 0, true);
   if (st != SALAD_OK) return st;
+  CUtensorMap tq, tk, tv, tdo, tt, tds;
+  const int BH = B * num_heads;
+  const uint64_t op_dims[3] = {(uint64_t)2 * d, (uint64_t)d, (uint64_t)BH};
+  const uint64_t op_strides[2] = {(uint64_t)2 * d * 2, (uint64_t)d * 2 * d * 2};
+  const uint32_t op_box[3] = {64, (uint32_t)d, 1};
+  if (!make_bnhd_map(&tq, q, B, N, num_heads, d, 128) || !make_bnhd_map(&tk, k, B, N, num_heads, d, 128) ||
+      !make_bnhd_map(&tv, v, B, N, num_heads, d, 128) || !make_bnhd_map(&tdo, dout, B, N, num_heads, d, 128) ||
+      !make_map(&tt, ws + L.fwd.off_t, 3, op_dims, op_strides, op_box) ||
+      !make_map(&tds, ws + L.off_ds, 3, op_dims, op_strides, op_box))
+    return SALAD_ERR_CUDA;
   LinBwdArgs la{};
-  la.q = static_cast<const uint16_t*>(q);
-  la.k = static_cast<const uint16_t*>(k);
-  la.v = static_cast<const uint16_t*>(v);
+  la.tm_q = &tq;
+  la.tm_do = &tdo;
+  la.tm_k = &tk;
+  la.tm_v = &tv;
+  la.tm_t = &tt;
+  la.tm_ds = &tds;
   la.out = static_cast<const uint16_t*>(out);
-  la.dout = static_cast<const uint16_t*>(dout);
   la.w = static_cast<const uint16_t*>(w_proj);
   la.lse = lse;
   la.gate = gate;
@@ -488,13 +502,11 @@ int salad_attn_backward(const void* q, const void* k, const void* v, const void*
   la.dgate = dgate;
   la.lse2 = F(L.off_lse2);
   la.dvec = F(L.off_dvec);
-  la.o_s = F(L.off_o);
-  la.dy_s = F(L.off_dy);
-  la.du_s = F(L.off_du);
-  la.dden_s = F(L.off_dden);
-  la.yg_s = F(L.off_yg);
-  la.partial = F(L.off_partial);
-  la.dS = F(L.off_dS);
+  la.m_part = F(L.off_mpart);
+  la.dz_part = F(L.off_dzpart);
+  la.dg_part = F(L.off_dgpart);
+  la.dw_part = F(L.off_dwpart);
+  la.ds_op = reinterpret_cast<uint16_t*>(ws + L.off_ds);
   la.dz = F(L.off_dz);
   la.B = B;
   la.N = N;
@@ -502,14 +514,15 @@ int salad_attn_backward(const void* q, const void* k, const void* v, const void*
   la.d = d;
   la.npad = L.npad;
   la.splits = L.splits;
+  la.tiles_per_split = L.tiles_per_split;
   la.eps = eps;
+  la.status = reinterpret_cast<uint32_t*>(ws + L.fwd.off_status);
+  la.wait_limit_ns = g_wait_limit_ns.load();
   // 2. per-row terms of the linear branch, D_i and lse2; dq starts as the linear branch's part
   if (launch_linear_backward_rows(la, s) != cudaSuccess) return SALAD_ERR_CUDA;
-  // 3. the sparse branch: dq += ..., dk and dv written
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_bnhd_map(&tq, q, B, N, num_heads, d, 128) || !make_bnhd_map(&tk, k, B, N, num_heads, d, 128) ||
-      !make_bnhd_map(&tv, v, B, N, num_heads, d, 128) || !make_bnhd_map(&tdo, dout, B, N, num_heads, d, 128))
-    return SALAD_ERR_CUDA;
+  // 3. dS, dz, dW, dgate
+  if (launch_linear_backward_state(la, s) != cudaSuccess) return SALAD_ERR_CUDA;
+  // 4. the sparse branch: dq += ..., dk and dv written
   BwdArgs ba{};
   ba.tm_q = &tq;
   ba.tm_k = &tk;
@@ -540,8 +553,8 @@ int salad_attn_backward(const void* q, const void* k, const void* v, const void*
   ba.wait_limit_ns = g_wait_limit_ns.load();
   ba.full = 1;
   if (launch_backward(ba, s) != cudaSuccess) return SALAD_ERR_CUDA;
-  // 4. dS, dz, dW, dgate, then the linear parts of dk and dv
-  return launch_linear_backward_tail(la, s) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
+  // 5. the linear parts of dk and dv
+  return launch_linear_backward_keys(la, s) == cudaSuccess ? SALAD_OK : SALAD_ERR_CUDA;
 }
 
 int salad_attn_forward_tiles(const void* q, const void* k, const void* v, int B, int T, int H, int W, int bt,

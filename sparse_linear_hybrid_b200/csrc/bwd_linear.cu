@@ -1,333 +1,857 @@
-// Backward pass of the linear branch, its projection and the gate (the rest of
-// the layer's gradients next to the sparse branch's in bwd.cu).  Per (b, h),
-// with S and z the branch's state, a_i = relu(q_i), den_i = a_i.z + eps,
-// o_i = a_i^T S / den_i, y_i = o_i W and G = dL/dout:
-//   dgate      = sum_i G_i.y_i
-//   dy_i       = g G_i,  dW += sum_i o_i^T dy_i  (over every (b, h))
-//   do_i       = dy_i W^T,  du_i = do_i / den_i,  dden_i = -(do_i.o_i) / den_i
-//   dS         = sum_i a_i du_i^T,   dz = sum_i dden_i a_i
-//   dq_i      += [q_i > 0] (S du_i + dden_i z)
-//   dk_j      += [k_j > 0] (dS v_j + dz),   dv_j += dS^T relu(k_j)
-// and, for the sparse branch, D_i = G_i.(out_i - g y_i) (its output is out
-// minus the linear term).  fp32 CUDA-core arithmetic in a fixed order:
-//   lin_rows_kernel    per 128 query rows of a (b, h), one thread per feature,
-//                      S, S^T, W, W^T in shared memory: the per-row terms; it
-//                      writes dq (the sparse backward then adds its part), D_i,
-//                      lse_i in base 2, and o, dy, du, dden, G.y for the sums
-//   lin_outer_kernel   split sums of a_i du_i^T (dS) and o_i dy_i^T (dW), 16 x 16
-//                      threads each owning a block of the d x d result
-//   lin_vec_kernel     dz and dgate per (b, h): eight row groups, added in order
-//   lin_reduce_kernel  the splits (and, for dW, the (b, h)) in order
-//   lin_keys_kernel    per 128 key rows: the linear parts of dk and dv
+// Backward pass of the linear branch, its projection and the gate, on the
+// tensor cores (the sparse branch's gradients are in bwd.cu).  SALAD summary
+// section 2.1 defines the branch: per (b, h), with the state S, z of linear.cu,
+// a_i = relu(q_i), den_i = a_i.z + eps, o_i = a_i S / den_i, out_i gets g o_i W.
+// With T = S W (the projected state of the forward), G_i = dL/dout_i and
+//   P1_i = a_i T,  P2_i = G_i T^T                          (row products)
+//   yg_i = G_i.P1_i / den_i  (= G_i.(o_i W)),  s_i = g / den_i,  dden_i = -g yg_i / den_i
+// the gradients are
+//   dgate = sum_i yg_i
+//   dq_i  = [q_i > 0] (s_i P2_i + dden_i z)       (the sparse branch's part is added later)
+//   M     = sum_i a_i^T (s_i G_i)                 (d x d)
+//   dS    = M W^T,  dz = sum_i dden_i a_i,  dW = sum over (b, h) of S^T M
+//   dk_j += [k_j > 0] (v_j dS^T + dz),  dv_j += relu(k_j) dS
+// and the sparse branch's D_i = G_i.out_i - g yg_i (its output is out_i - g o_i W).
+// These follow from dy_i = g G_i, do_i = dy_i W^T, du_i = do_i / den_i:
+// do_i.o_i = g yg_i, S du_i = s_i T G_i, sum_i a_i du_i^T = M W^T and
+// sum_i o_i^T dy_i = S^T M.
+//
+//   lin_rows_kernel        grid (splits, B*Hh): each CTA streams 128-row tiles of
+//                          one (b, h) through a two-stage TMA ring; one thread
+//                          issues P1 = A [T_hi; T_lo] and P2 = G [T_hi; T_lo]^T
+//                          into tensor memory, four warps turn each row into dq,
+//                          D_i, lse2, dden_i and the row of X = s_i G_i (bf16 hi +
+//                          lo), and M += A^T X_hi + A^T X_lo accumulates in tensor
+//                          memory across the CTA's tiles.  Per split: M, dz, dgate.
+//   lin_state_grad_kernel  the splits in order: dS = M W^T as bf16 hi + lo operand
+//                          halves, dz, dgate, and S^T M over 16 rows of S and M
+//   lin_dw_kernel          dW: those partials in (b, h) then row-block order
+//   lin_keys_kernel        grid (splits, B*Hh): per 128 key rows, V [dS_hi; dS_lo]^T
+//                          and relu(K) [dS_hi; dS_lo] in double-buffered tensor
+//                          memory, added to the sparse branch's dk and dv.
+// Every sum runs in a fixed order, so the gradients do not vary run to run.
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace salad {
 namespace {
 
-constexpr int kOuterThreads = 256;
-constexpr int kOuterRows = 32;  // rows staged per step of lin_outer_kernel
-constexpr int kVecGroups = 8;
+constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kLog2eL = 1.4426950408889634f;
 
-__device__ __forceinline__ float bf16f(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
-
-// Fixed-order tree sum over the D threads of the block.
+// Shared layout of both streaming kernels: an operand of d x d bf16 hi + lo
+// halves (T or dS: 2d/64 chunks of [d rows x 64 columns], 128-byte swizzle),
+// then two stages of two 128-row tiles.
 template <int D>
-__device__ float tree_sum(float v, float* red) {
-  red[threadIdx.x] = v;
-  __syncthreads();
-#pragma unroll
-  for (int s = D / 2; s > 0; s >>= 1) {
-    if ((int)threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
-    __syncthreads();
-  }
-  const float r = red[0];
-  __syncthreads();
-  return r;
+struct LinBwdCfg {
+  static constexpr int BOX = 128 * 128;                 // [128 rows x 64 columns] bf16
+  static constexpr int TILE = (D / 64) * BOX;           // a 128 x D tile
+  static constexpr int OP_CH = D * 128;                 // [D rows x 64 columns] bf16
+  static constexpr int OP_BYTES = 2 * (D / 64) * OP_CH;  // hi chunks, then lo chunks
+  static constexpr int STAGES = 2;
+  static constexpr int OFF_STAGE = OP_BYTES;            // stage s: first tile, then second tile
+  static constexpr int OFF_XLO = OFF_STAGE + STAGES * 2 * TILE;  // rows kernel only
+  static constexpr int ROWS_OFF_BAR = OFF_XLO + TILE;
+  static constexpr int KEYS_OFF_BAR = OFF_XLO;
+  static constexpr uint32_t IDESC_NN = idesc_bf16(128, D, false, false);  // both K-major
+  static constexpr uint32_t IDESC_NT = idesc_bf16(128, D, false, true);   // B MN-major
+  static constexpr uint32_t IDESC_TT = idesc_bf16(128, D, true, true);    // A and B MN-major
+  static constexpr uint32_t TMEM_COLS = D == 128 ? 512 : 256;
+  // CTAs one SM holds: shared memory allows one at d = 128, two at d = 64.
+  static constexpr int CTAS_PER_SM = D == 128 ? 1 : 2;
+};
+
+struct RowShared {
+  uint64_t full[2], empty[2];
+  uint64_t op_full, relu, p_full, p_free, x_full, x_free, dd_bar, m_done, drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  float zs[128];
+  float dden[2][128];
+  float red[4];
+};
+
+struct KeyShared {
+  uint64_t full[2], empty[2];
+  uint64_t op_full, relu, acc_full[2], acc_free[2], drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  float dzs[128];
+};
+
+template <int D>
+constexpr int rows_smem() { return LinBwdCfg<D>::ROWS_OFF_BAR + (int)sizeof(RowShared) + 1024; }
+template <int D>
+constexpr int keys_smem() { return LinBwdCfg<D>::KEYS_OFF_BAR + (int)sizeof(KeyShared) + 1024; }
+static_assert(rows_smem<128>() <= 232448, "rows kernel shared memory");
+static_assert(keys_smem<128>() <= 232448, "keys kernel shared memory");
+
+template <typename Sh>
+__device__ __forceinline__ void record_timeout(Sh* sh, uint32_t* status) {
+  sh->abort_flag = 1;
+  atomicOr(status, kStatusTimeout);
 }
 
-template <int D>
-__global__ void __launch_bounds__(D) lin_rows_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ out,
-                                                     const uint16_t* __restrict__ dout, const float* __restrict__ lse,
-                                                     const uint16_t* __restrict__ w, const float* __restrict__ gate,
-                                                     const float* __restrict__ S, const float* __restrict__ z, int N,
-                                                     int heads, int npad, float eps, float* __restrict__ dq,
-                                                     float* __restrict__ lse2, float* __restrict__ dvec,
-                                                     float* __restrict__ o_s, float* __restrict__ dy_s,
-                                                     float* __restrict__ du_s, float* __restrict__ dden_s,
-                                                     float* __restrict__ yg_s) {
-  extern __shared__ float lin_smem[];
-  float* Ss = lin_smem;            // [D][D]: S[c][e]
-  float* St = Ss + D * D;          // [D][D]: S[e][c]
-  uint16_t* Ws = reinterpret_cast<uint16_t*>(St + D * D);  // [D][D] bf16: W[e][f]
-  uint16_t* Wt = Ws + D * D;                                // [D][D] bf16: W[f][e]
-  float* zs = reinterpret_cast<float*>(Wt + D * D);         // [D]
-  float* a = zs + D;               // [D] per row
-  float* o = a + D;
-  float* dy = o + D;
-  float* du = dy + D;
-  float* red = du + D;
-  const int t = threadIdx.x, bh = blockIdx.y, b = bh / heads, h = bh % heads;
-  const float g = gate[bh];
-  for (int x = t; x < D * D; x += D) {
-    const int r = x / D, c = x % D;
-    const float sv = S[(size_t)bh * D * D + x];
-    Ss[x] = sv;
-    St[c * D + r] = sv;
-    Ws[x] = w[x];
-    Wt[c * D + r] = w[x];
-  }
-  zs[t] = z[(size_t)bh * D + t];
-  __syncthreads();
-  const int r0 = blockIdx.x * 128, r1 = min(N, r0 + 128);
-  for (int i = r0; i < r1; ++i) {
-    const size_t off = (((size_t)b * N + i) * heads + h) * D;
-    const size_t ri = (size_t)bh * N + i;
-    const float qv = bf16f(q[off + t]);
-    const float Gt = bf16f(dout[off + t]);
-    a[t] = qv > 0.f ? qv : 0.f;
-    __syncthreads();
-    const float den = eps + tree_sum<D>(a[t] * zs[t], red);
-    float u = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) u = fmaf(a[c], Ss[c * D + t], u);
-    const float ot = u / den;
-    o[t] = ot;
-    __syncthreads();
-    float y = 0.f;
-#pragma unroll 8
-    for (int e = 0; e < D; ++e) y = fmaf(o[e], bf16f(Ws[e * D + t]), y);
-    const float yg = tree_sum<D>(Gt * y, red);
-    const float Dval = tree_sum<D>(Gt * (bf16f(out[off + t]) - g * y), red);
-    dy[t] = g * Gt;
-    __syncthreads();
-    float dov = 0.f;
-#pragma unroll 8
-    for (int f = 0; f < D; ++f) dov = fmaf(bf16f(Wt[f * D + t]), dy[f], dov);
-    const float dden = -tree_sum<D>(dov * ot, red) / den;
-    du[t] = dov / den;
-    __syncthreads();
-    float dA = dden * zs[t];
-#pragma unroll 8
-    for (int e = 0; e < D; ++e) dA = fmaf(St[e * D + t], du[e], dA);
-    dq[off + t] = qv > 0.f ? dA : 0.f;
-    o_s[off + t] = ot;
-    dy_s[off + t] = dy[t];
-    du_s[off + t] = du[t];
-    if (t == 0) {
-      dden_s[ri] = dden;
-      yg_s[ri] = yg;
-      dvec[(size_t)bh * npad + i] = Dval;
-      lse2[(size_t)bh * npad + i] = lse[ri] * kLog2eL;
-    }
-    __syncthreads();
-  }
-  // pad rows of the last tile: no probability mass, no D
-  if (blockIdx.x == gridDim.x - 1)
-    for (int i = N + t; i < npad; i += D) {
-      lse2[(size_t)bh * npad + i] = INFINITY;
-      dvec[(size_t)bh * npad + i] = 0.f;
-    }
+// Bounded wait taken by a whole warp, false (in every lane) once the CTA is
+// aborting or the wait timed out, so the warp never diverges around it.
+template <typename Sh>
+__device__ __forceinline__ bool warp_wait(Sh* sh, uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (__any_sync(0xffffffffu, sh->abort_flag != 0)) return false;
+  return mbar_wait_warp(bar, parity, limit_ns);
 }
 
-// Split sums of x_i y_i^T over the rows of a split: product 0 is
-// relu(q_i) du_i^T (dS), product 1 is o_i dy_i^T (dW); fp32 partials
-// [2][splits][B*Hh][D][D].
+__device__ __forceinline__ uint32_t relu2(uint32_t v) {
+  const uint32_t neg = ((v >> 15) & 0x00010001u) * 0xFFFFu;  // 0xFFFF in each negative half
+  return v & ~neg;
+}
+
+// Row r of a 128-row tile (D / 64 boxes): ReLU in place; returns sum_c relu(x_c) z_c.
 template <int D>
-__global__ void __launch_bounds__(kOuterThreads) lin_outer_kernel(const uint16_t* __restrict__ q,
-                                                                  const float* __restrict__ o_s,
-                                                                  const float* __restrict__ dy_s,
-                                                                  const float* __restrict__ du_s, int N, int heads,
-                                                                  int rows_per_split, float* __restrict__ partial) {
-  constexpr int M = D / 16;  // the M x M block of the result each thread owns
-  __shared__ float xs[kOuterRows][D];
-  __shared__ float ys[kOuterRows][D];
-  const int split = blockIdx.x, bh = blockIdx.y, prod = blockIdx.z, b = bh / heads, h = bh % heads;
-  const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
-  float acc[M][M];
+__device__ __forceinline__ float relu_row(uint32_t tile, int r, const float* z) {
+  float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-  for (int i = 0; i < M; ++i)
+  for (int ch = 0; ch < D / 64; ++ch)
 #pragma unroll
-    for (int j = 0; j < M; ++j) acc[i][j] = 0.f;
-  const int n0 = split * rows_per_split, n1 = min(N, n0 + rows_per_split);
-  for (int c0 = n0; c0 < n1; c0 += kOuterRows) {
-    const int nr = min(kOuterRows, n1 - c0);
-    for (int x = threadIdx.x; x < kOuterRows * D; x += kOuterThreads) {
-      const int r = x / D, f = x % D;
-      float xv = 0.f, yv = 0.f;
-      if (r < nr) {
-        const size_t off = (((size_t)b * N + c0 + r) * heads + h) * D + f;
-        if (prod == 0) {
-          const float qv = bf16f(q[off]);
-          xv = qv > 0.f ? qv : 0.f;
-          yv = du_s[off];
-        } else {
-          xv = o_s[off];
-          yv = dy_s[off];
+    for (int p = 0; p < 8; ++p) {
+      const uint32_t addr = tile + ch * LinBwdCfg<D>::BOX + sw128_offset((uint32_t)r, (uint32_t)p);
+      uint32_t x[4];
+      ld_shared_v4(addr, x[0], x[1], x[2], x[3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[i] = relu2(x[i]);
+      st_shared_v4(addr, x[0], x[1], x[2], x[3]);
+      if (z != nullptr) {
+        const int c = ch * 64 + p * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          d0 = fmaf(bf16_lo_to_f32(x[i]), z[c + 2 * i], d0);
+          d1 = fmaf(bf16_hi_to_f32(x[i]), z[c + 2 * i + 1], d1);
         }
       }
-      xs[r][f] = xv;
-      ys[r][f] = yv;
     }
-    __syncthreads();
-    for (int r = 0; r < nr; ++r) {
-      float xr[M], yr[M];
+  return d0 + d1;
+}
+
+// The 32 bf16 of columns 32 cc ... 32 cc + 31 of row r of a tile, as 16 pairs.
+template <int D>
+__device__ __forceinline__ void tile_cols32(uint32_t tile, int r, int cc, uint32_t (&x)[16]) {
 #pragma unroll
-      for (int i = 0; i < M; ++i) {
-        xr[i] = xs[r][ti * M + i];
-        yr[i] = ys[r][tj * M + i];
+  for (int j = 0; j < 4; ++j)
+    ld_shared_v4(tile + (cc / 2) * LinBwdCfg<D>::BOX + sw128_offset((uint32_t)r, (uint32_t)((cc % 2) * 4 + j)),
+                 x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+}
+
+// ------------------------------------------------------------------ rows
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    lin_rows_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_t, const uint16_t* __restrict__ out,
+                    const float* __restrict__ lse, const float* __restrict__ gate, const float* __restrict__ zvec,
+                    int N, int heads, int npad, int tiles_per_split, float eps, float* __restrict__ dq,
+                    float* __restrict__ lse2, float* __restrict__ dvec, float* __restrict__ m_part,
+                    float* __restrict__ dz_part, float* __restrict__ dg_part, uint32_t* status, uint64_t limit_ns) {
+  using C = LinBwdCfg<D>;
+  const int split = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
+  const int b = bh / heads, h = bh % heads;
+  const int ntiles = (N + 127) / 128;
+  const int t_begin = split * tiles_per_split;
+  const int n_tiles = min(ntiles, t_begin + tiles_per_split) - t_begin;  // >= 1 by construction
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  RowShared* sh = reinterpret_cast<RowShared*>(smem + C::ROWS_OFF_BAR);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 1 + 4);  // the MMA commit and the four row warps
+    }
+    mbar_init(&sh->op_full, 1);
+    mbar_init(&sh->relu, 4);
+    mbar_init(&sh->p_full, 1);
+    mbar_init(&sh->p_free, 4);
+    mbar_init(&sh->x_full, 4);
+    mbar_init(&sh->x_free, 1);
+    mbar_init(&sh->dd_bar, 128);
+    mbar_init(&sh->m_done, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_do);
+    tma_prefetch_map(&tm_t);
+  }
+  if (threadIdx.x < D) sh->zs[threadIdx.x] = zvec[(size_t)bh * D + threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  constexpr uint32_t TM_P1 = 0, TM_P2 = D, TM_M = 2 * D;
+  const uint32_t op = sbase;  // T hi | lo
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sh->op_full, C::OP_BYTES);
+#pragma unroll
+      for (int ch = 0; ch < 2 * D / 64; ++ch) tma_load_3d(smem + ch * C::OP_CH, &tm_t, &sh->op_full, ch * 64, 0, bh);
+      int issued = 0;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->empty[s], ph ^ 1, limit_ns)) {
+          record_timeout(sh, status);
+          break;
+        }
+        uint8_t* at = smem + C::OFF_STAGE + s * 2 * C::TILE;
+        mbar_arrive_expect_tx(&sh->full[s], 2 * C::TILE);
+        const int row0 = (t_begin + it) * 128;
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) {
+          tma_load_3d(at + ch * C::BOX, &tm_q, &sh->full[s], h * D + ch * 64, row0, b);
+          tma_load_3d(at + C::TILE + ch * C::BOX, &tm_do, &sh->full[s], h * D + ch * 64, row0, b);
+        }
+        issued = it + 1;
+      }
+      if (sh->abort_flag) {
+        // let every copy this thread started land before the CTA can exit
+        mbar_wait(&sh->op_full, 0, kDrainNs);
+        for (int it = (issued > 2 ? issued - 2 : 0); it < issued; ++it)
+          mbar_wait(&sh->full[it & 1], (it >> 1) & 1, kDrainNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&sh->op_full, 0, limit_ns);
+      if (!ok) record_timeout(sh, status);
+      for (int it = 0; it < n_tiles && ok; ++it) {
+        const int s = it & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->relu, it & 1, limit_ns) ||
+            (it > 0 && !mbar_wait(&sh->p_free, (it - 1) & 1, limit_ns))) {
+          record_timeout(sh, status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t at = sbase + C::OFF_STAGE + s * 2 * C::TILE, gt = at + C::TILE;
+        // P1 = A T: B rows are f (N), K = c runs along them (K-major)
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = sw128_desc(at + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(op + (hl * (D / 64) + kk / 4) * C::OP_CH + (kk % 4) * 32, 16, 1024);
+            mma_bf16_ss(tmem + TM_P1, a, bd, C::IDESC_NN, (hl | kk) ? 1u : 0u);
+          }
+        // P2 = G T^T: the same rows f are now K, c runs along them (MN-major)
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = sw128_desc(gt + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(op + hl * (D / 64) * C::OP_CH + kk * 2048, C::OP_CH, 1024);
+            mma_bf16_ss(tmem + TM_P2, a, bd, C::IDESC_NT, (hl | kk) ? 1u : 0u);
+          }
+        mma_commit(&sh->p_full);
+        if (sh->abort_flag || !mbar_wait(&sh->x_full, it & 1, limit_ns)) {
+          record_timeout(sh, status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // M += A^T X: K = the 128 rows of the tile, A^T and X both MN-major.
+        // At d = 64 the second 64-wide half of A^T reads the G tile and lands in
+        // accumulator rows 64..127, which are never read.
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = sw128_desc(at + kk * 2048, C::BOX, 1024);
+            const uint64_t bd = sw128_desc((hl ? sbase + C::OFF_XLO : gt) + kk * 2048, C::BOX, 1024);
+            mma_bf16_ss(tmem + TM_M, a, bd, C::IDESC_TT, (it | hl | kk) ? 1u : 0u);
+          }
+        mma_commit(&sh->empty[s]);
+        mma_commit(&sh->x_free);
+      }
+      if (ok) {
+        mma_commit(&sh->m_done);
+      } else {
+        mma_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0, kDrainNs);
+      }
+    }
+  } else {
+    // ---------------- row warps 2..5: thread (quarter, lane) owns row 32 quarter + lane
+    const int t = threadIdx.x - 64;
+    const int quarter = warp & 3, r = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float g = gate[bh];
+    float dg_acc = 0.f, dz_acc = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_tiles; ++it) {
+      const int s = it & 1;
+      const uint32_t ph = (it >> 1) & 1;
+      const uint32_t at = sbase + C::OFF_STAGE + s * 2 * C::TILE, gt = at + C::TILE, xlo = sbase + C::OFF_XLO;
+      const int row = (t_begin + it) * 128 + r;
+      // 1. ReLU of the row of q in place, den
+      if (!warp_wait(sh, &sh->full[s], ph, limit_ns)) {
+        ok = false;
+        break;
+      }
+      const float den = relu_row<D>(at, r, sh->zs) + eps;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->relu);
+      // 2. yg and G.out from P1
+      if (!warp_wait(sh, &sh->p_full, it & 1, limit_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool live = row < N;
+      const uint16_t* orow = out + (((size_t)b * N + (live ? row : 0)) * heads + h) * D;
+      float yg0 = 0.f, yg1 = 0.f, go0 = 0.f, go1 = 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t p1[32], gx[16];
+        tmem_ld32(lane_base + TM_P1 + cc * 32, p1);
+        uint4 ov[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          ov[j] = live ? __ldg(reinterpret_cast<const uint4*>(orow + cc * 32) + j) : make_uint4(0, 0, 0, 0);
+        tile_cols32<D>(gt, r, cc, gx);
+        tmem_ld_wait();
+        const uint32_t* ow = reinterpret_cast<const uint32_t*>(ov);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float ga = bf16_lo_to_f32(gx[i]), gb = bf16_hi_to_f32(gx[i]);
+          yg0 = fmaf(ga, __uint_as_float(p1[2 * i]), yg0);
+          yg1 = fmaf(gb, __uint_as_float(p1[2 * i + 1]), yg1);
+          go0 = fmaf(ga, bf16_lo_to_f32(ow[i]), go0);
+          go1 = fmaf(gb, bf16_hi_to_f32(ow[i]), go1);
+        }
+      }
+      const float yg = (yg0 + yg1) / den;
+      const float dden = -g * yg / den;
+      const float sg = g / den;
+      // 3. the row of X = s_i G_i as bf16 hi (over G) and lo (its own buffer)
+      if (it > 0 && !warp_wait(sh, &sh->x_free, (it - 1) & 1, limit_ns)) {
+        ok = false;
+        break;
       }
 #pragma unroll
-      for (int i = 0; i < M; ++i)
+      for (int ch = 0; ch < D / 64; ++ch)
 #pragma unroll
-        for (int j = 0; j < M; ++j) acc[i][j] = fmaf(xr[i], yr[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-  float* dst = partial + (((size_t)prod * gridDim.x + split) * gridDim.y + bh) * D * D;
+        for (int p = 0; p < 8; ++p) {
+          const uint32_t off = ch * C::BOX + sw128_offset((uint32_t)r, (uint32_t)p);
+          uint32_t x[4], hi[4], lo[4];
+          ld_shared_v4(gt + off, x[0], x[1], x[2], x[3]);
 #pragma unroll
-  for (int i = 0; i < M; ++i)
+          for (int i = 0; i < 4; ++i) {
+            const float v0 = sg * bf16_lo_to_f32(x[i]), v1 = sg * bf16_hi_to_f32(x[i]);
+            hi[i] = pack_bf16x2(v0, v1);
+            lo[i] = pack_bf16x2(v0 - bf16_lo_to_f32(hi[i]), v1 - bf16_hi_to_f32(hi[i]));
+          }
+          st_shared_v4(gt + off, hi[0], hi[1], hi[2], hi[3]);
+          st_shared_v4(xlo + off, lo[0], lo[1], lo[2], lo[3]);
+        }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->x_full);
+      // 4. dq = [q > 0] (s_i P2 + dden z)
+      float* dqrow = dq + (((size_t)b * N + (live ? row : 0)) * heads + h) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t p2[32], ax[16];
+        tmem_ld32(lane_base + TM_P2 + cc * 32, p2);
+        tile_cols32<D>(at, r, cc, ax);
+        tmem_ld_wait();
+        float v[32];
 #pragma unroll
-    for (int j = 0; j < M; ++j) dst[(ti * M + i) * D + tj * M + j] = acc[i][j];
-}
-
-// dz[bh][c] = sum_i dden_i relu(q_ic) and dgate[bh] = sum_i yg_i: eight groups of
-// D threads take every eighth row, the groups are added in order.
-template <int D>
-__global__ void __launch_bounds__(D * kVecGroups) lin_vec_kernel(const uint16_t* __restrict__ q,
-                                                                 const float* __restrict__ dden_s,
-                                                                 const float* __restrict__ yg_s, int N, int heads,
-                                                                 float* __restrict__ dz, float* __restrict__ dgate) {
-  __shared__ float gz[kVecGroups][D];
-  __shared__ float gg[kVecGroups];
-  const int bh = blockIdx.x, b = bh / heads, h = bh % heads;
-  const int c = threadIdx.x % D, grp = threadIdx.x / D;
-  float acc = 0.f, accg = 0.f;
-#pragma unroll 4
-  for (int i = grp; i < N; i += kVecGroups) {
-    const float qv = bf16f(q[(((size_t)b * N + i) * heads + h) * D + c]);
-    const float dd = dden_s[(size_t)bh * N + i];
-    if (qv > 0.f) acc = fmaf(dd, qv, acc);
-    if (c == 0) accg += yg_s[(size_t)bh * N + i];
-  }
-  gz[grp][c] = acc;
-  if (c == 0) gg[grp] = accg;
-  __syncthreads();
-  if (grp == 0) {
-    float s = 0.f;
+        for (int i = 0; i < 16; ++i) {
+          const int c = cc * 32 + 2 * i;
+          v[2 * i] = (ax[i] & 0xFFFFu) ? fmaf(sg, __uint_as_float(p2[2 * i]), dden * sh->zs[c]) : 0.f;
+          v[2 * i + 1] = (ax[i] >> 16) ? fmaf(sg, __uint_as_float(p2[2 * i + 1]), dden * sh->zs[c + 1]) : 0.f;
+        }
+        if (live) {
 #pragma unroll
-    for (int k = 0; k < kVecGroups; ++k) s += gz[k][c];
-    dz[(size_t)bh * D + c] = s;
-    if (c == 0) {
-      float sg = 0.f;
-#pragma unroll
-      for (int k = 0; k < kVecGroups; ++k) sg += gg[k];
-      dgate[bh] = sg;
-    }
-  }
-}
-
-// dS[bh] = the splits of product 0 in order; dW = product 1 over the splits of
-// each (b, h) in order, the (b, h) in order.
-template <int D>
-__global__ void __launch_bounds__(256) lin_reduce_kernel(const float* __restrict__ partial, int splits, int BH,
-                                                         float* __restrict__ dS, float* __restrict__ dw) {
-  const int e = blockIdx.x * 256 + threadIdx.x;
-  if (e >= D * D) return;
-  const int bh = blockIdx.y;
-  if (bh < BH) {
-    float s = 0.f;
-    for (int k = 0; k < splits; ++k) s += partial[(((size_t)0 * splits + k) * BH + bh) * D * D + e];
-    dS[(size_t)bh * D * D + e] = s;
-  } else {
-    float s = 0.f;
-    for (int x = 0; x < BH; ++x) {
-      float sb = 0.f;
-      for (int k = 0; k < splits; ++k) sb += partial[(((size_t)1 * splits + k) * BH + x) * D * D + e];
-      s += sb;
-    }
-    dw[e] = s;
-  }
-}
-
-// The linear parts of dk and dv for 128 key rows of a (b, h), added to the
-// sparse branch's.
-template <int D>
-__global__ void __launch_bounds__(D) lin_keys_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-                                                     const float* __restrict__ dS, const float* __restrict__ dz, int N,
-                                                     int heads, float* __restrict__ dk, float* __restrict__ dv) {
-  extern __shared__ float lin_smem[];
-  float* Ds = lin_smem;      // [D][D]: dS[c][e]
-  float* Dt = Ds + D * D;    // [D][D]: dS[e][c]
-  float* kr = Dt + D * D;    // [D] relu(k_j)
-  float* vr = kr + D;        // [D] v_j
-  const int t = threadIdx.x, bh = blockIdx.y, b = bh / heads, h = bh % heads;
-  for (int x = t; x < D * D; x += D) {
-    const float sv = dS[(size_t)bh * D * D + x];
-    Ds[x] = sv;
-    Dt[(x % D) * D + x / D] = sv;
-  }
-  const float dzt = dz[(size_t)bh * D + t];
-  __syncthreads();
-  const int r0 = blockIdx.x * 128, r1 = min(N, r0 + 128);
-  for (int j = r0; j < r1; ++j) {
-    const size_t off = (((size_t)b * N + j) * heads + h) * D;
-    const float kv = bf16f(k[off + t]);
-    kr[t] = kv > 0.f ? kv : 0.f;
-    vr[t] = bf16f(v[off + t]);
-    __syncthreads();
-    float tk = dzt, tv = 0.f;
+          for (int j = 0; j < 8; ++j)
+            reinterpret_cast<float4*>(dqrow + cc * 32)[j] =
+                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->p_free);
+      // 5. per-row outputs for the sparse backward, dgate, and dz over the tile's rows
+      if (live) {
+        dvec[(size_t)bh * npad + row] = go0 + go1 - g * yg;
+        lse2[(size_t)bh * npad + row] = lse[(size_t)bh * N + row] * kLog2eL;
+      } else if (row < npad) {
+        dvec[(size_t)bh * npad + row] = 0.f;  // pad rows: no probability mass
+        lse2[(size_t)bh * npad + row] = INFINITY;
+      }
+      dg_acc += yg;
+      sh->dden[it & 1][r] = dden;
+      mbar_arrive(&sh->dd_bar);
+      if (!warp_wait(sh, &sh->dd_bar, it & 1, limit_ns)) {
+        ok = false;
+        break;
+      }
+      if (t < D) {
+        const uint32_t col = at + (t / 64) * C::BOX + (uint32_t)(t % 8) * 2;
+        const uint32_t piece = (uint32_t)((t % 64) / 8);
+        float z0 = 0.f, z1 = 0.f;
 #pragma unroll 8
-    for (int e = 0; e < D; ++e) {
-      tk = fmaf(Dt[e * D + t], vr[e], tk);  // (dS v_j)_t
-      tv = fmaf(Ds[e * D + t], kr[e], tv);  // (dS^T relu(k_j))_t
+        for (int i = 0; i < 128; i += 2) {
+          uint16_t a0, a1;
+          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(a0) : "r"(col + sw128_offset((uint32_t)i, piece)));
+          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(a1) : "r"(col + sw128_offset((uint32_t)i + 1, piece)));
+          z0 = fmaf(__uint_as_float((uint32_t)a0 << 16), sh->dden[it & 1][i], z0);
+          z1 = fmaf(__uint_as_float((uint32_t)a1 << 16), sh->dden[it & 1][i + 1], z1);
+        }
+        dz_acc += z0 + z1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->empty[s]);
     }
-    if (kv > 0.f) dk[off + t] += tk;
-    dv[off + t] += tv;
-    __syncthreads();
+    if (!ok) record_timeout(sh, status);
+    ok = __all_sync(0xffffffffu, ok);
+    // dgate: fixed-order sum over the 128 threads (shuffle tree, then the four warps in order)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dg_acc += __shfl_xor_sync(0xffffffffu, dg_acc, o);
+    const size_t part = (size_t)split * BH + bh;
+    if (lane == 0) sh->red[warp - 2] = dg_acc;
+    if (ok) {
+      if (t < D) dz_part[part * D + t] = dz_acc;
+      if (warp_wait(sh, &sh->m_done, 0, limit_ns)) {
+        tc_fence_after();
+        if (quarter * 32 < D) {
+          float* mrow = m_part + (part * D + quarter * 32 + lane) * D;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t m[32];
+            tmem_ld32(lane_base + TM_M + cc * 32, m);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              reinterpret_cast<float4*>(mrow + cc * 32)[j] =
+                  make_float4(__uint_as_float(m[4 * j]), __uint_as_float(m[4 * j + 1]),
+                              __uint_as_float(m[4 * j + 2]), __uint_as_float(m[4 * j + 3]));
+          }
+        }
+      } else {
+        record_timeout(sh, status);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  // dgate partial: the four row warps' sums in order
+  if (threadIdx.x == 64 && !sh->abort_flag)
+    dg_part[(size_t)split * BH + bh] = (sh->red[0] + sh->red[1]) + (sh->red[2] + sh->red[3]);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
+// ------------------------------------------------------------------ keys
 template <int D>
-cudaError_t launch_lin_rows_t(const LinBwdArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)(2 * D * D + 6 * D) * sizeof(float) + (size_t)2 * D * D * sizeof(uint16_t);
-  cudaError_t e = cudaFuncSetAttribute(lin_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+__global__ void __launch_bounds__(192, 1)
+    lin_keys_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_ds, const float* __restrict__ dz, int N, int heads,
+                    int tiles_per_split, float* __restrict__ dk, float* __restrict__ dv, uint32_t* status,
+                    uint64_t limit_ns) {
+  using C = LinBwdCfg<D>;
+  const int split = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / heads, h = bh % heads;
+  const int ntiles = (N + 127) / 128;
+  const int t_begin = split * tiles_per_split;
+  const int n_tiles = min(ntiles, t_begin + tiles_per_split) - t_begin;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  KeyShared* sh = reinterpret_cast<KeyShared*>(smem + C::KEYS_OFF_BAR);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 1 + 4);
+      mbar_init(&sh->acc_full[s], 1);
+      mbar_init(&sh->acc_free[s], 4);
+    }
+    mbar_init(&sh->op_full, 1);
+    mbar_init(&sh->relu, 4);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_v);
+    tma_prefetch_map(&tm_ds);
+  }
+  if (threadIdx.x < D) sh->dzs[threadIdx.x] = dz[(size_t)bh * D + threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const uint32_t op = sbase;  // dS hi | lo, rows c
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sh->op_full, C::OP_BYTES);
+#pragma unroll
+      for (int ch = 0; ch < 2 * D / 64; ++ch) tma_load_3d(smem + ch * C::OP_CH, &tm_ds, &sh->op_full, ch * 64, 0, bh);
+      int issued = 0;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->empty[s], ph ^ 1, limit_ns)) {
+          record_timeout(sh, status);
+          break;
+        }
+        uint8_t* kt = smem + C::OFF_STAGE + s * 2 * C::TILE;
+        mbar_arrive_expect_tx(&sh->full[s], 2 * C::TILE);
+        const int row0 = (t_begin + it) * 128;
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) {
+          tma_load_3d(kt + ch * C::BOX, &tm_k, &sh->full[s], h * D + ch * 64, row0, b);
+          tma_load_3d(kt + C::TILE + ch * C::BOX, &tm_v, &sh->full[s], h * D + ch * 64, row0, b);
+        }
+        issued = it + 1;
+      }
+      if (sh->abort_flag) {
+        mbar_wait(&sh->op_full, 0, kDrainNs);
+        for (int it = (issued > 2 ? issued - 2 : 0); it < issued; ++it)
+          mbar_wait(&sh->full[it & 1], (it >> 1) & 1, kDrainNs);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(&sh->op_full, 0, limit_ns);
+      if (!ok) record_timeout(sh, status);
+      for (int it = 0; it < n_tiles && ok; ++it) {
+        const int s = it & 1, buf = it & 1;
+        if (sh->abort_flag || !mbar_wait(&sh->relu, it & 1, limit_ns) ||
+            !mbar_wait(&sh->acc_free[buf], ((it >> 1) & 1) ^ 1, limit_ns)) {
+          record_timeout(sh, status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kt = sbase + C::OFF_STAGE + s * 2 * C::TILE, vt = kt + C::TILE;
+        const uint32_t acc_k = tmem + buf * 2 * D, acc_v = acc_k + D;
+        // v_j dS^T: B rows are c (N), K = e runs along them (K-major)
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = sw128_desc(vt + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(op + (hl * (D / 64) + kk / 4) * C::OP_CH + (kk % 4) * 32, 16, 1024);
+            mma_bf16_ss(acc_k, a, bd, C::IDESC_NN, (hl | kk) ? 1u : 0u);
+          }
+        // relu(k_j) dS: the rows c are K, e runs along them (MN-major)
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = sw128_desc(kt + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(op + hl * (D / 64) * C::OP_CH + kk * 2048, C::OP_CH, 1024);
+            mma_bf16_ss(acc_v, a, bd, C::IDESC_NT, (hl | kk) ? 1u : 0u);
+          }
+        mma_commit(&sh->acc_full[buf]);
+        mma_commit(&sh->empty[s]);
+      }
+      if (!ok) {
+        mma_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0, kDrainNs);
+      }
+    }
+  } else {
+    // ---------------- row warps: ReLU of the next tile, then this tile's rows of dk, dv
+    const int quarter = warp & 3, r = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    if (n_tiles > 0) {
+      if (!warp_wait(sh, &sh->full[0], 0, limit_ns)) {
+        ok = false;
+      } else {
+        relu_row<D>(sbase + C::OFF_STAGE, r, nullptr);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->relu);
+      }
+    }
+    for (int it = 0; it < n_tiles && ok; ++it) {
+      const int s = it & 1, buf = it & 1;
+      if (it + 1 < n_tiles) {
+        const int s1 = (it + 1) & 1;
+        if (!warp_wait(sh, &sh->full[s1], ((it + 1) >> 1) & 1, limit_ns)) {
+          ok = false;
+          break;
+        }
+        relu_row<D>(sbase + C::OFF_STAGE + s1 * 2 * C::TILE, r, nullptr);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->relu);
+      }
+      if (!warp_wait(sh, &sh->acc_full[buf], (it >> 1) & 1, limit_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t kt = sbase + C::OFF_STAGE + s * 2 * C::TILE;
+      const int row = (t_begin + it) * 128 + r;
+      const bool live = row < N;
+      const size_t off = (((size_t)b * N + (live ? row : 0)) * heads + h) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ak[32], av[32], kx[16];
+        tmem_ld32(lane_base + buf * 2 * D + cc * 32, ak);
+        tmem_ld32(lane_base + buf * 2 * D + D + cc * 32, av);
+        tile_cols32<D>(kt, r, cc, kx);
+        float4 ok4[8], ov4[8];
+        float4* dkr = reinterpret_cast<float4*>(dk + off + cc * 32);
+        float4* dvr = reinterpret_cast<float4*>(dv + off + cc * 32);
+        if (live) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            ok4[j] = dkr[j];
+            ov4[j] = dvr[j];
+          }
+        }
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int c = cc * 32 + 4 * j;
+            const uint32_t m0 = kx[2 * j], m1 = kx[2 * j + 1];
+            float4 a = ok4[j];
+            a.x += (m0 & 0xFFFFu) ? __uint_as_float(ak[4 * j]) + sh->dzs[c] : 0.f;
+            a.y += (m0 >> 16) ? __uint_as_float(ak[4 * j + 1]) + sh->dzs[c + 1] : 0.f;
+            a.z += (m1 & 0xFFFFu) ? __uint_as_float(ak[4 * j + 2]) + sh->dzs[c + 2] : 0.f;
+            a.w += (m1 >> 16) ? __uint_as_float(ak[4 * j + 3]) + sh->dzs[c + 3] : 0.f;
+            dkr[j] = a;
+            float4 e = ov4[j];
+            e.x += __uint_as_float(av[4 * j]);
+            e.y += __uint_as_float(av[4 * j + 1]);
+            e.z += __uint_as_float(av[4 * j + 2]);
+            e.w += __uint_as_float(av[4 * j + 3]);
+            dvr[j] = e;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sh->acc_free[buf]);
+        mbar_arrive(&sh->empty[s]);
+      }
+    }
+    if (!ok) record_timeout(sh, status);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ state gradients
+// grid (B*Hh, D/16), 256 threads.  CTA (bh, blk) owns rows c in [16 blk, 16 blk + 16)
+// of M: it sums their split partials in split order, writes those rows of dS =
+// M W^T as bf16 hi + lo halves ds_op[bh][c][e] (hi), ds_op[bh][c][D + e] (lo), the
+// operand layout of lin_keys_kernel, and the partial S^T M over its 16 rows,
+// dw_part[bh][blk][e][f] = sum_{c in blk} S[c][e] M[c][f].  CTA (bh, 0) also sums
+// dz and dgate.
+template <int D>
+__global__ void __launch_bounds__(256) lin_state_grad_kernel(const float* __restrict__ m_part,
+                                                             const float* __restrict__ dz_part,
+                                                             const float* __restrict__ dg_part,
+                                                             const float* __restrict__ S, const uint16_t* __restrict__ w,
+                                                             int splits, uint16_t* __restrict__ ds_op,
+                                                             float* __restrict__ dz, float* __restrict__ dgate,
+                                                             float* __restrict__ dw_part) {
+  extern __shared__ float sg_smem[];
+  float* Ms = sg_smem;                                           // [16][D]
+  float* Ss = Ms + 16 * D;                                       // [16][D]
+  uint16_t* Wt = reinterpret_cast<uint16_t*>(Ss + 16 * D);       // [D][D]: Wt[f][e] = W[e][f]
+  const int bh = blockIdx.x, blk = blockIdx.y, BH = gridDim.x, t = threadIdx.x;
+  const int c0 = blk * 16;
+  for (int x = t; x < D * D; x += 256) Wt[(x % D) * D + x / D] = w[x];
+  for (int x = t; x < 16 * D; x += 256) {
+    const size_t e = ((size_t)bh * D + c0) * D + x;
+    float acc = 0.f;
+    int sp = 0;
+    for (; sp + 4 <= splits; sp += 4) {
+      float a[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = m_part[(size_t)(sp + i) * BH * D * D + e];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc += a[i];
+    }
+    for (; sp < splits; ++sp) acc += m_part[(size_t)sp * BH * D * D + e];
+    Ms[x] = acc;
+    Ss[x] = S[e];
+  }
+  if (blk == 0) {
+    if (t < D) {
+      float acc = 0.f;
+      for (int sp = 0; sp < splits; ++sp) acc += dz_part[((size_t)sp * BH + bh) * D + t];
+      dz[(size_t)bh * D + t] = acc;
+    } else if (t == D) {
+      float acc = 0.f;
+      for (int sp = 0; sp < splits; ++sp) acc += dg_part[(size_t)sp * BH + bh];
+      dgate[bh] = acc;
+    }
+  }
+  __syncthreads();
+  constexpr int G = 256 / D;     // thread groups: 2 (d = 128) or 4 (d = 64)
+  const int col = t % D, grp = t / D;
+  // dS rows: thread (e = col, grp) owns rows grp * (16 / G) ...
+  {
+    constexpr int R = 16 / G;
+    float acc[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int f = 0; f < D; ++f) {
+      const float wv = __uint_as_float((uint32_t)Wt[f * D + col] << 16);
+#pragma unroll
+      for (int i = 0; i < R; ++i) acc[i] = fmaf(Ms[(grp * R + i) * D + f], wv, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const uint16_t hi = (uint16_t)(pack_bf16x2(acc[i], 0.f) & 0xFFFFu);
+      const float rest = acc[i] - __uint_as_float((uint32_t)hi << 16);
+      const uint16_t lo = (uint16_t)(pack_bf16x2(rest, 0.f) & 0xFFFFu);
+      uint16_t* row = ds_op + ((size_t)bh * D + c0 + grp * R + i) * (2 * D);
+      row[col] = hi;
+      row[D + col] = lo;
+    }
+  }
+  // S^T M over the 16 rows: thread (f = col, grp) owns e in [grp * D / G, +D / G)
+  {
+    constexpr int E = D / G;
+    float acc[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) acc[i] = 0.f;
+#pragma unroll 2
+    for (int rr = 0; rr < 16; ++rr) {
+      const float mv = Ms[rr * D + col];
+#pragma unroll
+      for (int i = 0; i < E; ++i) acc[i] = fmaf(Ss[rr * D + grp * E + i], mv, acc[i]);
+    }
+    float* dst = dw_part + (((size_t)bh * (D / 16) + blk) * D + grp * E) * D + col;
+#pragma unroll
+    for (int i = 0; i < E; ++i) dst[(size_t)i * D] = acc[i];
+  }
+}
+
+// dW[x] = the partials of lin_state_grad_kernel in (b, h), then row-block order.
+__global__ void __launch_bounds__(256) lin_dw_kernel(const float* __restrict__ dw_part, int parts, int DD,
+                                                     float* __restrict__ dw) {
+  const int x = blockIdx.x * 256 + threadIdx.x;
+  if (x >= DD) return;
+  float acc = 0.f;
+  int p = 0;
+  for (; p + 8 <= parts; p += 8) {
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = dw_part[(size_t)(p + i) * DD + x];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc += a[i];
+  }
+  for (; p < parts; ++p) acc += dw_part[(size_t)p * DD + x];
+  dw[x] = acc;
+}
+
+template <int D>
+cudaError_t launch_rows_t(const LinBwdArgs& a, cudaStream_t s) {
+  constexpr int smem = rows_smem<D>();
+  cudaError_t e = cudaFuncSetAttribute(lin_rows_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  lin_rows_kernel<D><<<dim3(a.npad / 128, a.B * a.heads), D, smem, s>>>(
-      a.q, a.out, a.dout, a.lse, a.w, a.gate, a.S, a.z, a.N, a.heads, a.npad, a.eps, a.dq, a.lse2, a.dvec, a.o_s,
-      a.dy_s, a.du_s, a.dden_s, a.yg_s);
+  lin_rows_kernel<D><<<dim3(a.splits, a.B * a.heads), 192, smem, s>>>(
+      *a.tm_q, *a.tm_do, *a.tm_t, a.out, a.lse, a.gate, a.z, a.N, a.heads, a.npad, a.tiles_per_split, a.eps, a.dq,
+      a.lse2, a.dvec, a.m_part, a.dz_part, a.dg_part, a.status, a.wait_limit_ns);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_lin_tail_t(const LinBwdArgs& a, cudaStream_t s) {
+cudaError_t launch_tail_t(const LinBwdArgs& a, cudaStream_t s) {
   const int BH = a.B * a.heads;
-  const int rps = (a.N + a.splits - 1) / a.splits;
-  lin_outer_kernel<D><<<dim3(a.splits, BH, 2), kOuterThreads, 0, s>>>(a.q, a.o_s, a.dy_s, a.du_s, a.N, a.heads, rps,
-                                                                     a.partial);
-  cudaError_t e = cudaGetLastError();
+  const size_t sg_smem = (size_t)32 * D * sizeof(float) + (size_t)D * D * sizeof(uint16_t);
+  cudaError_t e = cudaFuncSetAttribute(lin_state_grad_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sg_smem);
   if (e != cudaSuccess) return e;
-  lin_vec_kernel<D><<<BH, D * kVecGroups, 0, s>>>(a.q, a.dden_s, a.yg_s, a.N, a.heads, a.dz, a.dgate);
+  lin_state_grad_kernel<D><<<dim3(BH, D / 16), 256, sg_smem, s>>>(a.m_part, a.dz_part, a.dg_part, a.S, a.w,
+                                                                 a.splits, a.ds_op, a.dz, a.dgate, a.dw_part);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  lin_reduce_kernel<D><<<dim3((D * D + 255) / 256, BH + 1), 256, 0, s>>>(a.partial, a.splits, BH, a.dS, a.dw);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t smem = (size_t)(2 * D * D + 2 * D) * sizeof(float);
-  if ((e = cudaFuncSetAttribute(lin_keys_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-      cudaSuccess)
-    return e;
-  lin_keys_kernel<D><<<dim3(a.npad / 128, BH), D, smem, s>>>(a.k, a.v, a.dS, a.dz, a.N, a.heads, a.dk, a.dv);
+  lin_dw_kernel<<<(D * D + 255) / 256, 256, 0, s>>>(a.dw_part, BH * (D / 16), D * D, a.dw);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_keys_t(const LinBwdArgs& a, cudaStream_t s) {
+  constexpr int smem = keys_smem<D>();
+  cudaError_t e = cudaFuncSetAttribute(lin_keys_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  lin_keys_kernel<D><<<dim3(a.splits, a.B * a.heads), 192, smem, s>>>(*a.tm_k, *a.tm_v, *a.tm_ds, a.dz, a.N,
+                                                                      a.heads, a.tiles_per_split, a.dk, a.dv,
+                                                                      a.status, a.wait_limit_ns);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_linear_backward_rows(const LinBwdArgs& a, cudaStream_t s) {
-  return a.d == 64 ? launch_lin_rows_t<64>(a, s) : launch_lin_rows_t<128>(a, s);
+void linear_backward_splits(int BH, int N, int d, int* splits, int* tiles_per_split) {
+  const int ntiles = (N + 127) / 128;
+  const int slots = 148 * (d == 128 ? LinBwdCfg<128>::CTAS_PER_SM : LinBwdCfg<64>::CTAS_PER_SM);
+  // the fewest splits whose cost (waves x tiles per CTA) is within 5% of the best
+  long long best = -1;
+  int best_s = 1;
+  const int top = ntiles < 512 ? ntiles : 512;
+  long long cost[513];
+  for (int s = 1; s <= top; ++s) {
+    const long long waves = ((long long)BH * s + slots - 1) / slots;
+    cost[s] = waves * ((ntiles + s - 1) / s);
+    if (best < 0 || cost[s] < best) best = cost[s];
+  }
+  for (int s = 1; s <= top; ++s)
+    if (cost[s] * 100 <= best * 105) {
+      best_s = s;
+      break;
+    }
+  const int tps = (ntiles + best_s - 1) / best_s;
+  *tiles_per_split = tps;
+  *splits = (ntiles + tps - 1) / tps;  // every split owns at least one tile
 }
 
-cudaError_t launch_linear_backward_tail(const LinBwdArgs& a, cudaStream_t s) {
-  return a.d == 64 ? launch_lin_tail_t<64>(a, s) : launch_lin_tail_t<128>(a, s);
+cudaError_t launch_linear_backward_rows(const LinBwdArgs& a, cudaStream_t s) {
+  return a.d == 64 ? launch_rows_t<64>(a, s) : launch_rows_t<128>(a, s);
+}
+
+cudaError_t launch_linear_backward_state(const LinBwdArgs& a, cudaStream_t s) {
+  return a.d == 64 ? launch_tail_t<64>(a, s) : launch_tail_t<128>(a, s);
+}
+
+cudaError_t launch_linear_backward_keys(const LinBwdArgs& a, cudaStream_t s) {
+  return a.d == 64 ? launch_keys_t<64>(a, s) : launch_keys_t<128>(a, s);
 }
 
 }  // namespace salad

@@ -52,6 +52,7 @@ struct LinearArgs {
   uint16_t* t_op;           // forward: (S W)^T hi | lo, bf16 [B*Hh][d][2d]
   float* z;                 // fp32 [B*Hh][d]
   float* S_out;             // state export: fp32 [B*Hh][d][d]; null in the forward
+  bool with_t = false;      // with S_out: also (S W)^T into t_op (the layer backward)
   uint32_t* work_ctr;       // zeroed here for the attention kernel that follows
   int B, N, heads, d, splits, chunks_per_split;
   uint32_t* status;
@@ -127,18 +128,30 @@ cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s);
 
 // Backward pass of the linear branch, projection and gate (bwd_linear.cu).
 struct LinBwdArgs {
-  const uint16_t *q, *k, *v, *out, *dout, *w;  // bf16
-  const float *lse, *gate, *S, *z;             // S fp32 [B*Hh][d][d], z [B*Hh][d]
+  const CUtensorMap *tm_q, *tm_do, *tm_k, *tm_v;  // box (64, 128, 1)
+  const CUtensorMap* tm_t;                         // box (64, d, 1) over (S W)^T hi | lo (the forward's layout)
+  const CUtensorMap* tm_ds;                        // box (64, d, 1) over ds_op
+  const uint16_t *out, *w;                         // bf16
+  const float *lse, *gate, *S, *z;                 // S fp32 [B*Hh][d][d], z [B*Hh][d]
   float *dq, *dk, *dv, *dw, *dgate;
-  float *lse2, *dvec;                          // [B*Hh][npad], read by the sparse backward
-  float *o_s, *dy_s, *du_s;                    // fp32 [B][N][Hh][d] scratch
-  float *dden_s, *yg_s;                        // fp32 [B*Hh][N] scratch
-  float *partial, *dS, *dz;                    // [2][splits][B*Hh][d][d], [B*Hh][d][d], [B*Hh][d]
-  int B, N, heads, d, npad, splits;
+  float *lse2, *dvec;                              // [B*Hh][npad], read by the sparse backward
+  float *m_part, *dz_part, *dg_part;               // [splits][B*Hh][d][d], [splits][B*Hh][d], [splits][B*Hh]
+  float* dw_part;                                  // [B*Hh][d/16][d][d]
+  uint16_t* ds_op;                                 // bf16 [B*Hh][d][2d]: dS hi | lo, rows c
+  float* dz;                                       // [B*Hh][d]
+  int B, N, heads, d, npad, splits, tiles_per_split;
   float eps;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
 };
+// Splits of the streaming kernels: CTAs per (b, h) and 128-row tiles per CTA.
+void linear_backward_splits(int BH, int N, int d, int* splits, int* tiles_per_split);
+// dq (linear part), D_i, lse2 and the per-split M, dz, dgate.
 cudaError_t launch_linear_backward_rows(const LinBwdArgs& a, cudaStream_t s);
-cudaError_t launch_linear_backward_tail(const LinBwdArgs& a, cudaStream_t s);
+// dS operand, dz, dgate, dW.
+cudaError_t launch_linear_backward_state(const LinBwdArgs& a, cudaStream_t s);
+// dk, dv += the linear parts.
+cudaError_t launch_linear_backward_keys(const LinBwdArgs& a, cudaStream_t s);
 
 // Dynamic gate and branch dropping (gate.cu).
 struct GateArgs {

@@ -10,9 +10,9 @@
 // operands MN-major and the fp32 accumulator in tensor memory.  The CTA writes
 // its partial S and z in fp32.
 // linear_finalize_kernel: fixed-order sum of the partials (deterministic), then
-// either S and z in fp32 (the state export) or z in fp32 plus the projected
-// state S W as bf16 hi + lo halves in the B operand layout the attention
-// epilogue feeds to the tensor cores.
+// z in fp32 with S in fp32 (the state export), the projected state S W as bf16
+// hi + lo halves in the B operand layout the attention epilogue feeds to the
+// tensor cores (the forward), or both (the layer backward).
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -243,16 +243,17 @@ __global__ void __launch_bounds__(192, 1)
 
 // grid (B*Hh, D/ROWS), 256 threads.  CTA (bh, g) owns features c in
 // [ROWS*g, ROWS*g + ROWS): it sums their split partials in split order (float4
-// loads, coalesced along e), a fixed order, so results do not vary run to run.
-//   EXPORT:  S_out[bh][c][e] and z_out[bh][c] in fp32 (salad_linear_state).
-//   forward: z_out[bh][c] in fp32 and the projected state T = S W,
+// loads, coalesced along e), a fixed order, so results do not vary run to run,
+// and writes z_out[bh][c] in fp32 and
+//   WRITE_S: S_out[bh][c][e] in fp32 (salad_linear_state, the layer backward).
+//   WRITE_T: the projected state T = S W,
 //            T[c][f] = sum_e S[c][e] W[e][f], transposed and split into bf16
 //            hi + lo halves: t_op[bh][f][c] = hi(T[c][f]), t_op[bh][f][D+c] =
 //            lo(T[c][f]).  That is the K-major B operand of the attention
 //            epilogue's U = relu(q) T, so the projection is applied to the state
 //            once per (b, h) instead of to every query row:
 //            (relu(q) S / den) W = relu(q) (S W) / den.
-template <int D, bool EXPORT>
+template <int D, bool WRITE_S, bool WRITE_T>
 __global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __restrict__ partial,
                                                               const float* __restrict__ gate,
                                                               const uint16_t* __restrict__ w,
@@ -266,9 +267,9 @@ __global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __res
   const int bh = blockIdx.x, g = blockIdx.y, BH = gridDim.x;
   if (gate != nullptr && gate[bh] == 0.0f) return;
   __shared__ __align__(16) float acc[ROWS][D];
-  __shared__ __align__(16) uint16_t wsm[EXPORT ? 8 : D * D];
+  __shared__ __align__(16) uint16_t wsm[WRITE_T ? D * D : 8];
   const int t = threadIdx.x, rr = t / E4, e4 = (t % E4) * 4;
-  if constexpr (!EXPORT) {
+  if constexpr (WRITE_T) {
     // W into shared memory first: its loads are in flight with the partials'
     uint4 wv[WV / 256];
 #pragma unroll
@@ -315,13 +316,14 @@ __global__ void __launch_bounds__(256) linear_finalize_kernel(const float* __res
     for (; q < splits; ++q) z += zsrc[(size_t)q * split_stride];
     z_out[(size_t)bh * D + ROWS * g + t] = z;
   }
-  if constexpr (EXPORT) {
+  if constexpr (WRITE_S) {
     float* dst = S_out + ((size_t)bh * D + ROWS * g + rr) * D + e4;  // S_out is only 4-byte aligned
     dst[0] = s.x;
     dst[1] = s.y;
     dst[2] = s.z;
     dst[3] = s.w;
-  } else {
+  }
+  if constexpr (WRITE_T) {
     *reinterpret_cast<float4*>(&acc[rr][e4]) = s;
     __syncthreads();
     // thread (f, fg): T rows ROWS*g + fg*RPT + k, column f
@@ -369,12 +371,15 @@ cudaError_t launch_linear_t(const LinearArgs& a, cudaStream_t s) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const dim3 fgrid(BH, D / (256 / (D / 4)));
-  if (a.S_out != nullptr)
-    linear_finalize_kernel<D, true><<<fgrid, 256, 0, s>>>(a.partial, a.gate, nullptr, nullptr, a.z, a.S_out,
-                                                         a.splits);
+  if (a.S_out != nullptr && a.with_t)
+    linear_finalize_kernel<D, true, true><<<fgrid, 256, 0, s>>>(a.partial, a.gate, a.w, a.t_op, a.z, a.S_out,
+                                                               a.splits);
+  else if (a.S_out != nullptr)
+    linear_finalize_kernel<D, true, false><<<fgrid, 256, 0, s>>>(a.partial, a.gate, nullptr, nullptr, a.z,
+                                                                a.S_out, a.splits);
   else
-    linear_finalize_kernel<D, false><<<fgrid, 256, 0, s>>>(a.partial, a.gate, a.w, a.t_op, a.z, nullptr,
-                                                          a.splits);
+    linear_finalize_kernel<D, false, true><<<fgrid, 256, 0, s>>>(a.partial, a.gate, a.w, a.t_op, a.z, nullptr,
+                                                                a.splits);
   return cudaGetLastError();
 }
 

@@ -259,7 +259,7 @@ def test_backward_argument_errors(L):
     assert layer(w=0) == sl.SALAD_ERR_INVALID_ARG
     assert layer(eps=-1.0) == sl.SALAD_ERR_INVALID_ARG
     assert layer(block=64) == sl.SALAD_ERR_UNSUPPORTED
-    assert layer(B=40000) == sl.SALAD_ERR_UNSUPPORTED          # B * Hh above 65534
+    assert layer(B=40000) == sl.SALAD_ERR_UNSUPPORTED          # B * Hh above 65535
     assert layer(B=32768) == sl.SALAD_ERR_UNSUPPORTED          # B * Hh = 65536
     assert layer(ws=0x40000000 + 16) == sl.SALAD_ERR_INVALID_ARG
     assert layer(ws_bytes=1024) == sl.SALAD_ERR_WORKSPACE
