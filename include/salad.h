@@ -46,7 +46,8 @@ typedef enum {
   SALAD_ERR_WORKSPACE = -4,      /* workspace smaller than salad_workspace_bytes() */
   SALAD_ERR_CUDA = -5,           /* a CUDA runtime/driver call or launch failed */
   SALAD_ERR_DEVICE_TIMEOUT = -6, /* a kernel gave up waiting (see salad_check_status) */
-  SALAD_ERR_OUT_OF_MEMORY = -7   /* the device had no memory left for the static scratch */
+  SALAD_ERR_OUT_OF_MEMORY = -7,  /* the device had no memory left for the static scratch */
+  SALAD_ERR_BAD_MASK = -8        /* checking build (SALAD_DEBUG): a kernel skipped a malformed mask row */
 } salad_status;
 
 /*
@@ -437,8 +438,12 @@ int salad_linear_state(const void* k, const void* v, int B, int N, int num_heads
 /*
  * Synchronises `stream`, then reads and clears the workspace status word.
  * Returns SALAD_ERR_DEVICE_TIMEOUT if a kernel of an earlier call gave up on a
- * bounded wait (its output is then invalid), SALAD_ERR_CUDA if the stream
- * reports an error, SALAD_OK otherwise.
+ * bounded wait (its output is then invalid), SALAD_ERR_BAD_MASK if a kernel of
+ * the checking build (compiled with SALAD_DEBUG: libsalad_debug.so) found a
+ * malformed mask row (a decreasing or out-of-range row_ptr, a column outside
+ * [0, nb) or not ascending) and read it as an empty row, SALAD_ERR_CUDA if the
+ * stream reports an error, SALAD_OK otherwise.  Release builds take mask rows
+ * as given: check masks from elsewhere with salad_validate_mask first.
  */
 int salad_check_status(void* workspace, salad_stream_t stream);
 

@@ -32,6 +32,7 @@ SALAD_ERR_WORKSPACE = -4
 SALAD_ERR_CUDA = -5
 SALAD_ERR_DEVICE_TIMEOUT = -6
 SALAD_ERR_OUT_OF_MEMORY = -7
+SALAD_ERR_BAD_MASK = -8
 
 
 class SaladError(RuntimeError):
@@ -45,7 +46,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         # SALAD_LIBRARY selects another build of the same library (the profiling
-        # build, libsalad_profile.so); by default the in-tree libsalad.so
+        # build libsalad_profile.so, the checking build libsalad_debug.so); by
+        # default the in-tree libsalad.so
         path = os.environ.get("SALAD_LIBRARY") or LIB_PATH
         if not os.path.exists(path):
             raise RuntimeError(f"{path} is missing: build it with "

@@ -1,6 +1,6 @@
 """Build libsalad.so in-tree with nvcc for sm_100a.
 
-    python -m sparse_linear_hybrid_b200.build [--force] [--verbose]
+    python -m sparse_linear_hybrid_b200.build [--force] [--verbose] [--profile | --debug]
 
 Each translation unit compiles in parallel to an object under _build/, then one
 shared library is linked next to this file.  The CUDA runtime is linked
@@ -20,9 +20,16 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libsalad.so")
-# the profiling build: the attention kernel writes phase stamps (SALAD_PROFILE)
-PROF_OBJ = os.path.join(ROOT, "_build", "profile")
-PROF_LIB = os.path.join(HERE, "libsalad_profile.so")
+# variants: (object directory, library, extra nvcc flags)
+#   profile: the attention kernel writes phase stamps (SALAD_PROFILE)
+#   debug:   kernels check every mask row before using it (SALAD_DEBUG)
+VARIANTS = {
+    "release": (OBJ, LIB, []),
+    "profile": (os.path.join(OBJ, "profile"), os.path.join(HERE, "libsalad_profile.so"), ["-DSALAD_PROFILE"]),
+    "debug": (os.path.join(OBJ, "debug"), os.path.join(HERE, "libsalad_debug.so"), ["-DSALAD_DEBUG"]),
+}
+PROF_LIB = VARIANTS["profile"][1]
+DEBUG_LIB = VARIANTS["debug"][1]
 SOURCES = ["api.cu", "mask.cu", "linear.cu", "attn.cu", "noalloc.cu", "topk.cu", "gate.cu", "bwd.cu", "bwd_linear.cu"]
 HEADERS = ["ptx.cuh", "internal.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -37,13 +44,14 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, verbose, profile=False):
-    obj = os.path.join(PROF_OBJ if profile else OBJ, os.path.splitext(src)[0] + ".o")
+def _compile(src, verbose, variant="release"):
+    obj_dir, _, extra = VARIANTS[variant]
+    obj = os.path.join(obj_dir, os.path.splitext(src)[0] + ".o")
     deps = [os.path.join(CSRC, src)] + [os.path.join(CSRC, h) for h in HEADERS] + \
         [os.path.join(ROOT, "include", "salad.h")]
     if not _stale(obj, deps):
         return obj, ""
-    cmd = [NVCC, *FLAGS, *(["-DSALAD_PROFILE"] if profile else []), "-c", os.path.join(CSRC, src), "-o", obj]
+    cmd = [NVCC, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -52,17 +60,21 @@ def _compile(src, verbose, profile=False):
     return obj, res.stderr
 
 
-def build(force: bool = False, verbose: bool = False, profile: bool = False) -> str:
-    """Builds libsalad.so (or, with profile=True, libsalad_profile.so with the
-    attention kernel's phase stamps compiled in)."""
-    obj_dir, lib = (PROF_OBJ, PROF_LIB) if profile else (OBJ, LIB)
+def build(force: bool = False, verbose: bool = False, profile: bool = False, debug: bool = False) -> str:
+    """Builds libsalad.so, or with profile=True libsalad_profile.so (the
+    attention kernel's phase stamps compiled in), or with debug=True
+    libsalad_debug.so (mask rows checked on the device before use)."""
+    if profile and debug:
+        raise ValueError("one variant at a time")
+    variant = "profile" if profile else "debug" if debug else "release"
+    obj_dir, lib, _ = VARIANTS[variant]
     os.makedirs(obj_dir, exist_ok=True)
     if force:
         for f in os.listdir(obj_dir):
             if f.endswith(".o"):
                 os.remove(os.path.join(obj_dir, f))
     with cf.ThreadPoolExecutor(len(SOURCES)) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose, profile), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, verbose, variant), SOURCES))
     objs = [o for o, _ in results]
     if verbose:
         for _, log in results:
@@ -78,5 +90,6 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--profile", action="store_true", help="the profiling build (libsalad_profile.so)")
+    ap.add_argument("--debug", action="store_true", help="the checking build (libsalad_debug.so)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.profile))
+    print(build(a.force, a.verbose, a.profile, a.debug))

@@ -582,7 +582,7 @@ int salad_transpose_block_mask(const int32_t* row_ptr, const int32_t* col_idx, i
     return SALAD_ERR_INVALID_ARG;
   // (one CTA row per group; every pair must be addressable by an int32 offset)
   if (groups > 65535 || (long long)groups * nb * nb >= (1ll << 31)) return SALAD_ERR_UNSUPPORTED;
-  return launch_mask_transpose(row_ptr, col_idx, groups, nb, t_row_ptr, t_col_idx,
+  return launch_mask_transpose(row_ptr, col_idx, groups, nb, t_row_ptr, t_col_idx, nullptr,
                                reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SALAD_OK
              : SALAD_ERR_CUDA;
@@ -706,7 +706,8 @@ int salad_check_status(void* workspace, salad_stream_t stream) {
   if (word == 0) return SALAD_OK;
   if (cudaMemsetAsync(dev, 0, sizeof(word), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
     return SALAD_ERR_CUDA;
-  return (word & kStatusTimeout) ? SALAD_ERR_DEVICE_TIMEOUT : SALAD_ERR_CUDA;
+  if (word & kStatusTimeout) return SALAD_ERR_DEVICE_TIMEOUT;
+  return (word & kStatusBadMask) ? SALAD_ERR_BAD_MASK : SALAD_ERR_CUDA;
 }
 
 void salad_set_wait_limit_ns(uint64_t limit_ns) { g_wait_limit_ns.store(limit_ns); }
@@ -734,6 +735,7 @@ const char* salad_status_string(int status) {
     case SALAD_ERR_WORKSPACE: return "workspace too small";
     case SALAD_ERR_CUDA: return "CUDA error";
     case SALAD_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case SALAD_ERR_BAD_MASK: return "a kernel skipped a malformed mask row (checking build)";
     case SALAD_ERR_OUT_OF_MEMORY: return "device out of memory for the static scratch";
     default: return "unknown status";
   }

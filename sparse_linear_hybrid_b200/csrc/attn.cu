@@ -221,7 +221,8 @@ __device__ __forceinline__ KeyIter make_iter(const int32_t* row_ptr, const int32
 
 template <int BLK, bool TILES>
 __device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, int nb, const int32_t* row_ptr,
-                                          const int32_t* col_idx, const float* gate, int mask_per_bh) {
+                                          const int32_t* col_idx, const float* gate, int mask_per_bh,
+                                          int mask_rows, uint32_t* status) {
   Item im;
   im.w = w;
   im.bh = w / qtiles;
@@ -232,6 +233,18 @@ __device__ __forceinline__ Item make_item(int w, int qtiles, int heads, int N, i
   im.lin = im.g != 0.0f;
   // the mask's rows are per head, or per (b, h) for a data-dependent mask
   KeyIter it = make_iter<BLK>(row_ptr, col_idx, mask_per_bh ? im.bh : im.h, nb, im.qtile);
+  {
+    // debug builds: a malformed row of the item reads as no kept key blocks
+    const int r0 = (mask_per_bh ? im.bh : im.h) * nb + (BLK == 128 ? im.qtile : 2 * im.qtile);
+    bool ok = debug_row_ok(row_ptr, col_idx, r0, mask_rows, nb, true, status);
+    if (BLK != 128 && 2 * im.qtile + 1 < nb) ok = debug_row_ok(row_ptr, col_idx, r0 + 1, mask_rows, nb, true, status) && ok;
+    if (!ok) {
+      it.a = col_idx;
+      it.na = 0;
+      it.b = nullptr;
+      it.nb = 0;
+    }
+  }
   im.ra = (int)(it.a - col_idx);
   im.na = it.na;
   im.rb = it.b ? (int)(it.b - col_idx) : 0;
@@ -314,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = AttnCfg<D, BLK>;
   static_assert(!TILES || BLK == 128, "a tile block fills one 128-row query tile");
   const int nblocks = TILES ? qtiles : (N + BLK - 1) / BLK;  // key blocks per mask row
+  const int mask_rows = (mask_per_bh ? num_items / qtiles : heads) * nblocks;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -418,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         SALAD_PROF(kPfLdItem);
         Item im;
         if (w < num_items) {
-          im = make_item<BLK, TILES>(w, qtiles, heads, N, nblocks, row_ptr, col_idx, gate, mask_per_bh);
+          im = make_item<BLK, TILES>(w, qtiles, heads, N, nblocks, row_ptr, col_idx, gate, mask_per_bh, mask_rows,
+                                     status);
         } else {
           im.w = -1;
         }

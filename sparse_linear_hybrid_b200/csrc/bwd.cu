@@ -136,7 +136,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x % nb, bh = blockIdx.x / nb, b = bh / heads, h = bh % heads;
   const int mrow = (mask_per_bh ? bh : h) * nb + qt;
-  const int c0 = row_ptr[mrow], n = row_ptr[mrow + 1] - c0;
+  const int mask_rows = (mask_per_bh ? (int)(gridDim.x / nb) : heads) * nb;
+  const int c0 = row_ptr[mrow];
+  const int n = debug_row_ok(row_ptr, col_idx, mrow, mask_rows, nb, true, status) ? row_ptr[mrow + 1] - c0 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->fixed_full, 1);
@@ -322,7 +324,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = blockIdx.x % nb, bh = blockIdx.x / nb, b = bh / heads, h = bh % heads;
   const int mrow = (mask_per_bh ? bh : h) * nb + kt;
-  const int c0 = t_row_ptr[mrow], n = t_row_ptr[mrow + 1] - c0;
+  const int mask_rows = (mask_per_bh ? (int)(gridDim.x / nb) : heads) * nb;
+  const int c0 = t_row_ptr[mrow];
+  const int n =
+      debug_row_ok(t_row_ptr, t_col_idx, mrow, mask_rows, nb, true, status) ? t_row_ptr[mrow + 1] - c0 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->fixed_full, 1);

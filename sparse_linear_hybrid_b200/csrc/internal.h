@@ -28,8 +28,9 @@ cudaError_t launch_mask_scan(int32_t* row_ptr, int n, cudaStream_t s);
 cudaError_t launch_mask_fill(const MaskGrid& g, const WindowTable& win, const int32_t* row_ptr, int32_t* col_idx,
                              cudaStream_t s);
 // The transposed mask of `groups` x nb rows (count, scan, fill).
+// status: a device word for debug builds' kStatusBadMask bit, or null.
 cudaError_t launch_mask_transpose(const int32_t* row_ptr, const int32_t* col_idx, int groups, int nb,
-                                  int32_t* t_row_ptr, int32_t* t_col_idx, cudaStream_t s);
+                                  int32_t* t_row_ptr, int32_t* t_col_idx, uint32_t* status, cudaStream_t s);
 
 // Workspace layout of the forward pass (byte offsets from the workspace base).
 struct WorkspaceLayout {
@@ -186,5 +187,31 @@ constexpr int kTopkMaxBlocks = 2048;  // the selection keeps one row of scores p
 
 // Status word bits written by kernels.
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBadMask = 2u;  // debug builds: a malformed mask row was skipped
+
+#ifdef __CUDACC__
+// Debug builds (SALAD_DEBUG) check a CSR row of a block mask before a kernel
+// indexes with it: 0 <= row_ptr[r] <= row_ptr[r + 1] <= row_ptr[rows] and, with
+// cols, every column in [0, nb) and strictly ascending.  A bad row sets
+// kStatusBadMask (where the call has a status word) and the caller treats it as
+// empty, so no access follows from it; the kernel goes on with the other rows.  Release builds take every row
+// as given (the host validates masks with salad_validate_mask).
+__device__ __forceinline__ bool debug_row_ok(const int32_t* row_ptr, const int32_t* col_idx, int r, int rows,
+                                             int nb, bool cols, uint32_t* status) {
+#ifdef SALAD_DEBUG
+  const int32_t lo = row_ptr[r], hi = row_ptr[r + 1], total = row_ptr[rows];
+  bool ok = r >= 0 && r < rows && 0 <= lo && lo <= hi && hi <= total;
+  for (int32_t i = lo; cols && ok && i < hi; ++i) {
+    const int32_t c = col_idx[i];
+    ok = c >= 0 && c < nb && (i == lo || c > col_idx[i - 1]);
+  }
+  if (!ok && status != nullptr) atomicOr(status, kStatusBadMask);
+  return ok;
+#else
+  (void)row_ptr, (void)col_idx, (void)r, (void)rows, (void)nb, (void)cols, (void)status;
+  return true;
+#endif
+}
+#endif
 
 }  // namespace salad

@@ -160,14 +160,18 @@ __device__ __forceinline__ bool row_keeps(const int32_t* row_ptr, const int32_t*
 template <bool FILL>
 __global__ void __launch_bounds__(128) mask_t_kernel(const int32_t* __restrict__ row_ptr,
                                                      const int32_t* __restrict__ col_idx, int nb,
-                                                     int32_t* __restrict__ t_row_ptr, int32_t* __restrict__ t_col_idx) {
+                                                     int32_t* __restrict__ t_row_ptr, int32_t* __restrict__ t_col_idx,
+                                                     uint32_t* status) {
   const int lane = threadIdx.x & 31;
   const int J = blockIdx.x * 4 + (threadIdx.x >> 5), g = blockIdx.y;
   if (J >= nb) return;
+  const int rows = (int)gridDim.y * nb;
   int pos = FILL ? t_row_ptr[(size_t)g * nb + J] : 0;
   for (int I0 = 0; I0 < nb; I0 += 32) {
     const int I = I0 + lane;
-    const bool has = I < nb && row_keeps(row_ptr, col_idx, g * nb + I, J);
+    // (debug builds: a row whose range is malformed is searched as empty)
+    const bool has = I < nb && debug_row_ok(row_ptr, col_idx, g * nb + I, rows, nb, false, status) &&
+                     row_keeps(row_ptr, col_idx, g * nb + I, J);
     const uint32_t m = __ballot_sync(0xffffffffu, has);
     if (FILL && has) t_col_idx[pos + __popc(m & ((1u << lane) - 1u))] = I;
     pos += __popc(m);
@@ -178,15 +182,15 @@ __global__ void __launch_bounds__(128) mask_t_kernel(const int32_t* __restrict__
 }  // namespace
 
 cudaError_t launch_mask_transpose(const int32_t* row_ptr, const int32_t* col_idx, int groups, int nb,
-                                  int32_t* t_row_ptr, int32_t* t_col_idx, cudaStream_t s) {
+                                  int32_t* t_row_ptr, int32_t* t_col_idx, uint32_t* status, cudaStream_t s) {
   const dim3 grid((nb + 3) / 4, groups);
-  mask_t_kernel<false><<<grid, 128, 0, s>>>(row_ptr, col_idx, nb, t_row_ptr, nullptr);
+  mask_t_kernel<false><<<grid, 128, 0, s>>>(row_ptr, col_idx, nb, t_row_ptr, nullptr, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   mask_scan_kernel<<<1, 1024, 0, s>>>(t_row_ptr, groups * nb);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  mask_t_kernel<true><<<grid, 128, 0, s>>>(row_ptr, col_idx, nb, t_row_ptr, t_col_idx);
+  mask_t_kernel<true><<<grid, 128, 0, s>>>(row_ptr, col_idx, nb, t_row_ptr, t_col_idx, status);
   return cudaGetLastError();
 }
 

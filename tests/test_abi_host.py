@@ -42,6 +42,20 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+@pytest.mark.parametrize("variant", ["debug", "profile"])
+def test_checking_and_profiling_builds_export_the_same_symbols(variant):
+    """The SALAD_DEBUG and SALAD_PROFILE variants build from the same sources and
+    export the same C ABI; the status the checking build adds is documented."""
+    from sparse_linear_hybrid_b200 import build
+    path = build.build(debug=variant == "debug", profile=variant == "profile")
+    V = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(V, name), (variant, name)
+    V.salad_status_string.restype = ctypes.c_char_p
+    assert b"malformed mask row" in V.salad_status_string(sl.SALAD_ERR_BAD_MASK)
+    assert "SALAD_ERR_BAD_MASK = -8" in open(HEADER).read()
+
+
 FAKE = 0x100000  # 16-byte aligned, never dereferenced by argument checks
 
 
