@@ -425,7 +425,7 @@ LayerBwdLayout layer_bwd_layout(int B, int N, int heads, int d) {
   L.off_lse2 = o;    o += up(BH * L.npad * 4);
   L.off_dvec = o;    o += up(BH * L.npad * 4);
   L.off_mpart = o;   o += up(S * BH * d * d * 4);
-  L.off_dzpart = o;  o += up(S * BH * d * 4);
+  L.off_dzpart = o;  o += up(S * BH * 256 * 4);  // [splits][B*Hh][256/d row groups][d]
   L.off_dgpart = o;  o += up(S * BH * 4);
   L.off_dwpart = o;  o += up(BH * (d / 16) * d * d * 4);
   L.off_ds = o;      o += up(BH * d * 2 * d * 2);

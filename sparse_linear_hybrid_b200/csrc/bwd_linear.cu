@@ -131,6 +131,22 @@ __device__ __forceinline__ float relu_row(uint32_t tile, int r, const float* z) 
   return d0 + d1;
 }
 
+// ReLU in place on columns [half D / 2, half D / 2 + D / 2) of row r of a
+// 128-row tile.
+template <int D>
+__device__ __forceinline__ void relu_half_row(uint32_t tile, int r, int half) {
+#pragma unroll
+  for (int pp = 0; pp < D / 16; ++pp) {
+    const int piece = half * (D / 16) + pp;  // 16-byte piece of the row: chunk piece / 8
+    const uint32_t addr = tile + (piece / 8) * LinBwdCfg<D>::BOX + sw128_offset((uint32_t)r, (uint32_t)(piece % 8));
+    uint32_t x[4];
+    ld_shared_v4(addr, x[0], x[1], x[2], x[3]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = relu2(x[i]);
+    st_shared_v4(addr, x[0], x[1], x[2], x[3]);
+  }
+}
+
 // The 32 bf16 of columns 32 cc ... 32 cc + 31 of row r of a tile, as 16 pairs.
 template <int D>
 __device__ __forceinline__ void tile_cols32(uint32_t tile, int r, int cc, uint32_t (&x)[16]) {
@@ -292,13 +308,24 @@ __global__ void __launch_bounds__(192, 1)
     const int quarter = warp & 3, r = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float g = gate[bh];
-    float dg_acc = 0.f, dz_acc = 0.f;
+    // dz: thread t sums the column pair (2 pr, 2 pr + 1) over row group rg of every tile
+    constexpr int PAIRS = D / 2, RG = 128 / PAIRS, RPG = 128 / RG;
+    const int pr = t % PAIRS, rg = t / PAIRS;
+    float dg_acc = 0.f, dz_acc0 = 0.f, dz_acc1 = 0.f;
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
       const int s = it & 1;
       const uint32_t ph = (it >> 1) & 1;
       const uint32_t at = sbase + C::OFF_STAGE + s * 2 * C::TILE, gt = at + C::TILE, xlo = sbase + C::OFF_XLO;
       const int row = (t_begin + it) * 128 + r;
+      // the row of the output, for D_i: its loads are in flight during the waits below
+      const bool live = row < N;
+      uint4 ov[D / 8];
+      {
+        const uint4* orow = reinterpret_cast<const uint4*>(out + (((size_t)b * N + (live ? row : 0)) * heads + h) * D);
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) ov[j] = live ? __ldg(orow + j) : make_uint4(0, 0, 0, 0);
+      }
       // 1. ReLU of the row of q in place, den
       if (!warp_wait(sh, &sh->full[s], ph, limit_ns)) {
         ok = false;
@@ -314,20 +341,14 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
-      const bool live = row < N;
-      const uint16_t* orow = out + (((size_t)b * N + (live ? row : 0)) * heads + h) * D;
       float yg0 = 0.f, yg1 = 0.f, go0 = 0.f, go1 = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t p1[32], gx[16];
         tmem_ld32(lane_base + TM_P1 + cc * 32, p1);
-        uint4 ov[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          ov[j] = live ? __ldg(reinterpret_cast<const uint4*>(orow + cc * 32) + j) : make_uint4(0, 0, 0, 0);
         tile_cols32<D>(gt, r, cc, gx);
         tmem_ld_wait();
-        const uint32_t* ow = reinterpret_cast<const uint32_t*>(ov);
+        const uint32_t* ow = reinterpret_cast<const uint32_t*>(&ov[cc * 4]);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float ga = bf16_lo_to_f32(gx[i]), gb = bf16_hi_to_f32(gx[i]);
@@ -404,19 +425,21 @@ __global__ void __launch_bounds__(192, 1)
         ok = false;
         break;
       }
-      if (t < D) {
-        const uint32_t col = at + (t / 64) * C::BOX + (uint32_t)(t % 8) * 2;
-        const uint32_t piece = (uint32_t)((t % 64) / 8);
+      {
+        // column pair (2 pr, 2 pr + 1): chunk pr / 32, 16-byte piece (pr % 32) / 4, word pr % 4
+        const uint32_t col = at + (pr / 32) * C::BOX + (uint32_t)(pr % 4) * 4;
+        const uint32_t piece = (uint32_t)((pr % 32) / 4);
         float z0 = 0.f, z1 = 0.f;
 #pragma unroll 8
-        for (int i = 0; i < 128; i += 2) {
-          uint16_t a0, a1;
-          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(a0) : "r"(col + sw128_offset((uint32_t)i, piece)));
-          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(a1) : "r"(col + sw128_offset((uint32_t)i + 1, piece)));
-          z0 = fmaf(__uint_as_float((uint32_t)a0 << 16), sh->dden[it & 1][i], z0);
-          z1 = fmaf(__uint_as_float((uint32_t)a1 << 16), sh->dden[it & 1][i + 1], z1);
+        for (int i = rg * RPG; i < (rg + 1) * RPG; ++i) {
+          uint32_t a2;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(a2) : "r"(col + sw128_offset((uint32_t)i, piece)));
+          const float dd = sh->dden[it & 1][i];
+          z0 = fmaf(bf16_lo_to_f32(a2), dd, z0);
+          z1 = fmaf(bf16_hi_to_f32(a2), dd, z1);
         }
-        dz_acc += z0 + z1;
+        dz_acc0 += z0;
+        dz_acc1 += z1;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->empty[s]);
@@ -429,7 +452,8 @@ __global__ void __launch_bounds__(192, 1)
     const size_t part = (size_t)split * BH + bh;
     if (lane == 0) sh->red[warp - 2] = dg_acc;
     if (ok) {
-      if (t < D) dz_part[part * D + t] = dz_acc;
+      dz_part[(part * RG + rg) * D + 2 * pr] = dz_acc0;
+      dz_part[(part * RG + rg) * D + 2 * pr + 1] = dz_acc1;
       if (warp_wait(sh, &sh->m_done, 0, limit_ns)) {
         tc_fence_after();
         if (quarter * 32 < D) {
@@ -465,7 +489,7 @@ __global__ void __launch_bounds__(192, 1)
 
 // ------------------------------------------------------------------ keys
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     lin_keys_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_ds, const float* __restrict__ dz, int N, int heads,
                     int tiles_per_split, float* __restrict__ dk, float* __restrict__ dv, uint32_t* status,
@@ -486,12 +510,12 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sh->full[s], 1);
-      mbar_init(&sh->empty[s], 1 + 4);
+      mbar_init(&sh->empty[s], 1 + 8);  // the MMA commit and the eight row warps
       mbar_init(&sh->acc_full[s], 1);
-      mbar_init(&sh->acc_free[s], 4);
+      mbar_init(&sh->acc_free[s], 8);
     }
     mbar_init(&sh->op_full, 1);
-    mbar_init(&sh->relu, 4);
+    mbar_init(&sh->relu, 8);
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_mbar_init();
@@ -581,15 +605,17 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ---------------- row warps: ReLU of the next tile, then this tile's rows of dk, dv
-    const int quarter = warp & 3, r = quarter * 32 + lane;
+    // ---------------- row warps 2..9: ReLU of the next tile, then this tile's rows of
+    // dk, dv; warp w takes row 32 (w % 4) + lane (its TMEM lane quarter) and the
+    // column half (w - 2) / 4
+    const int quarter = warp & 3, r = quarter * 32 + lane, half = (warp - 2) >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
     if (n_tiles > 0) {
       if (!warp_wait(sh, &sh->full[0], 0, limit_ns)) {
         ok = false;
       } else {
-        relu_row<D>(sbase + C::OFF_STAGE, r, nullptr);
+        relu_half_row<D>(sbase + C::OFF_STAGE, r, half);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->relu);
@@ -603,7 +629,7 @@ __global__ void __launch_bounds__(192, 1)
           ok = false;
           break;
         }
-        relu_row<D>(sbase + C::OFF_STAGE + s1 * 2 * C::TILE, r, nullptr);
+        relu_half_row<D>(sbase + C::OFF_STAGE + s1 * 2 * C::TILE, r, half);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->relu);
@@ -618,7 +644,7 @@ __global__ void __launch_bounds__(192, 1)
       const bool live = row < N;
       const size_t off = (((size_t)b * N + (live ? row : 0)) * heads + h) * D;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = half * (D / 64); cc < (half + 1) * (D / 64); ++cc) {
         uint32_t ak[32], av[32], kx[16];
         tmem_ld32(lane_base + buf * 2 * D + cc * 32, ak);
         tmem_ld32(lane_base + buf * 2 * D + D + cc * 32, av);
@@ -711,8 +737,10 @@ __global__ void __launch_bounds__(256) lin_state_grad_kernel(const float* __rest
   }
   if (blk == 0) {
     if (t < D) {
+      constexpr int RG = 256 / D;  // row groups of the rows kernel's dz partials
       float acc = 0.f;
-      for (int sp = 0; sp < splits; ++sp) acc += dz_part[((size_t)sp * BH + bh) * D + t];
+      for (int sp = 0; sp < splits; ++sp)
+        for (int g = 0; g < RG; ++g) acc += dz_part[(((size_t)sp * BH + bh) * RG + g) * D + t];
       dz[(size_t)bh * D + t] = acc;
     } else if (t == D) {
       float acc = 0.f;
@@ -811,7 +839,7 @@ cudaError_t launch_keys_t(const LinBwdArgs& a, cudaStream_t s) {
   constexpr int smem = keys_smem<D>();
   cudaError_t e = cudaFuncSetAttribute(lin_keys_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  lin_keys_kernel<D><<<dim3(a.splits, a.B * a.heads), 192, smem, s>>>(*a.tm_k, *a.tm_v, *a.tm_ds, a.dz, a.N,
+  lin_keys_kernel<D><<<dim3(a.splits, a.B * a.heads), 320, smem, s>>>(*a.tm_k, *a.tm_v, *a.tm_ds, a.dz, a.N,
                                                                       a.heads, a.tiles_per_split, a.dk, a.dv,
                                                                       a.status, a.wait_limit_ns);
   return cudaGetLastError();

@@ -136,7 +136,7 @@ struct LinBwdArgs {
   const float *lse, *gate, *S, *z;                 // S fp32 [B*Hh][d][d], z [B*Hh][d]
   float *dq, *dk, *dv, *dw, *dgate;
   float *lse2, *dvec;                              // [B*Hh][npad], read by the sparse backward
-  float *m_part, *dz_part, *dg_part;               // [splits][B*Hh][d][d], [splits][B*Hh][d], [splits][B*Hh]
+  float *m_part, *dz_part, *dg_part;               // [splits][B*Hh][d][d], [splits][B*Hh][256/d][d], [splits][B*Hh]
   float* dw_part;                                  // [B*Hh][d/16][d][d]
   uint16_t* ds_op;                                 // bf16 [B*Hh][d][2d]: dS hi | lo, rows c
   float* dz;                                       // [B*Hh][d]
