@@ -19,9 +19,11 @@
 //                    dP^T = V dO^T, one thread per key row forms P^T and dS^T
 //                    (bf16, written over the columns of S^T and dP^T it has
 //                    read), dV += P^T dO and dK += dS^T Q
-// Warp roles, 192 threads: warp 0 lane 0 issues the TMA loads and the MMAs in
+// Warp roles, 320 threads: warp 0 lane 0 issues the TMA loads and the MMAs in
 // program order (K/V or Q/dO tiles in a 2-deep ring), warp 1 owns the tensor
-// memory, warps 2-5 take one row each (TMEM lane quarter = warp % 4).  Every
+// memory, warps 2-9 take one row each (TMEM lane quarter = warp % 4) and one
+// half of its 128 columns (warp (w - 2) / 4); the exponentials of one pair in
+// four run on the FMA pipe (exp2_fma_x2), the rest on the MUFU.  Every
 // barrier wait is bounded; on a time-out the kernel records it and drains.
 // Gradients are written in fp32.
 #include "internal.h"
@@ -30,14 +32,19 @@
 namespace salad {
 namespace {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;  // producer/issuer, TMEM owner, eight row warps
 constexpr uint64_t kBwdDrainNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdShared {
   uint64_t fixed_full;    // the CTA's fixed tiles (Q and dO, or K and V)
-  uint64_t ring_full[2];  // the streamed tiles (K and V, or Q, dO and the row vectors)
-  uint64_t sdp_full;      // S and dP of the current tile are in tensor memory
+  uint64_t ring_full[2];  // dK/dV kernel: the streamed tiles (Q, dO and the row vectors)
+  uint64_t k_full[3];     // dQ kernel: the K ring (three stages)
+  uint64_t v_full[2];     // dQ kernel: the V ring (two stages)
+  uint64_t sdp_full;      // dK/dV kernel: S^T and dP^T of the current tile are in tensor memory
+  uint64_t dp_full;       // dQ kernel: dP of the current tile is in tensor memory
+  uint64_t s_full[2];     // dQ kernel: S of the current tile is in tensor memory ([0] used)
+  uint64_t s_read;        // dQ kernel: the row warps have read S of the current tile
   uint64_t ds_full;       // the four row warps have written dS (and P^T) of the tile
   uint64_t mm_done;       // the gradient products of the tile have completed
   uint64_t drain;
@@ -57,9 +64,15 @@ struct BwdCfg {
   static constexpr int SMEM_USED = OFF_BAR + (int)sizeof(BwdShared) + 1024;
   // at least 120 KB so that one CTA (and its 512 TMEM columns) owns the SM
   static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
+  // dQ kernel: Q and dO, then a three-stage K ring and a two-stage V ring (K_j is
+  // read by S_j and the dQ product, V_j only by dP_j, which completes earlier)
+  static constexpr int DQ_OFF_K = 2 * TILE;
+  static constexpr int DQ_OFF_V = 5 * TILE;
+  static constexpr int DQ_OFF_BAR = 7 * TILE;
+  static constexpr int DQ_SMEM = DQ_OFF_BAR + (int)sizeof(BwdShared) + 1024;
   static constexpr uint32_t IDESC_SS = idesc_bf16(128, 128, false, false);  // X Y^T, both K-major
   static constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);      // A (tmem) x B (MN-major)
-  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(SMEM <= 232448 && DQ_SMEM <= 232448, "shared memory budget");
 };
 
 // 128 x 128 product X Y^T of two K-major 128 x D tiles in shared memory.
@@ -73,14 +86,62 @@ __device__ __forceinline__ void mma_xyt(uint32_t d_tmem, uint32_t x, uint32_t y)
   }
 }
 
-// D += A B with A = 128 x 128 bf16 in tensor memory (columns a_tmem ...), B a
-// 128 x D tile in shared memory read as an MN-major operand.
+// 128 x 128 product X Y^T with X (128 x D bf16) in tensor memory from column
+// x_tmem and Y a K-major 128 x D tile in shared memory: one shared operand per
+// MMA instead of two.
 template <int D>
-__device__ __forceinline__ void mma_grad(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool accumulate) {
+__device__ __forceinline__ void mma_tyt(uint32_t d_tmem, uint32_t x_tmem, uint32_t y) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b + kk * 2048, 16384, 1024), BwdCfg<D>::IDESC_G,
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_bf16_ts(d_tmem, x_tmem + kk * 8, sw128_desc(y + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+                BwdCfg<D>::IDESC_SS, kk > 0 ? 1u : 0u);
+}
+
+// A 128 x D bf16 tile of shared memory (K-major, 128-byte swizzle) into tensor
+// memory columns [t, t + D / 2): row i to lane i; ordered with the MMAs issued
+// later by the same thread.
+template <int D>
+__device__ __forceinline__ void copy_tile_to_tmem(uint32_t t, uint32_t tile) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    tmem_cp_128x256b(t + kk * 8, sw128_desc(tile + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024));
+}
+
+// D += A B with A = 128 x 128 bf16 in tensor memory, B a 128 x D tile in shared
+// memory read as an MN-major operand.  A's K = 128 pairs of columns sit at
+// a_tmem + [0, 64) (split = false) or, written by two column halves each into
+// its own range, at a_tmem + [0, 32) and a_tmem + [64, 96) (split = true).
+template <int D>
+__device__ __forceinline__ void mma_grad(uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool accumulate,
+                                         bool split) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t a = a_tmem + (split && kk >= 4 ? 64 + (kk - 4) * 8 : kk * 8);
+    mma_bf16_ts(d_tmem, a, sw128_desc(b + kk * 2048, 16384, 1024), BwdCfg<D>::IDESC_G,
                 (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// p = 2^(s * c - l) for the 32 values of a row chunk, 0 from column `valid` on;
+// one pair in four on the FMA pipe.
+__device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[32], float c, float l, int col0, int valid,
+                                          float* p) {
+  const uint64_t c2 = f32x2_pack(c, c), nl = f32x2_pack(-l, -l);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nl);
+    float p0, p1;
+    if ((i & 3) == 3) {
+      exp2_fma_x2(x, p0, p1);
+    } else {
+      float x0, x1;
+      f32x2_unpack(x, x0, x1);
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    p[2 * i] = col0 + 2 * i < valid ? p0 : 0.f;
+    p[2 * i + 1] = col0 + 2 * i + 1 < valid ? p1 : 0.f;
+  }
 }
 
 __device__ __forceinline__ void bwd_timeout(BwdShared* sh, uint32_t* status) {
@@ -128,10 +189,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                   int heads, int nb, int npad, int mask_per_bh, float scale, float scale_log2, uint32_t* status,
                   uint64_t limit_ns, int accumulate) {
   using C = BwdCfg<D>;
-  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 384;
+  // S [0,128), dP [128,256) (dS as bf16 over its own dP: columns [0,32) and
+  // [64,96), one range per column half), dQ [256,256+D), then Q and dO as bf16
+  // A operands: [384,384+D/2) and [448,448+D/2)
+  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_Q = 384, TM_DO = 448;
   extern __shared__ uint8_t bwd_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~uintptr_t(1023));
-  BwdShared* sh = reinterpret_cast<BwdShared*>(smem + C::OFF_BAR);
+  BwdShared* sh = reinterpret_cast<BwdShared*>(smem + C::DQ_OFF_BAR);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x % nb, bh = blockIdx.x / nb, b = bh / heads, h = bh % heads;
@@ -142,10 +206,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->fixed_full, 1);
-    mbar_init(&sh->ring_full[0], 1);
-    mbar_init(&sh->ring_full[1], 1);
-    mbar_init(&sh->sdp_full, 1);
-    mbar_init(&sh->ds_full, 4);
+    for (int st = 0; st < 3; ++st) mbar_init(&sh->k_full[st], 1);
+    for (int st = 0; st < 2; ++st) mbar_init(&sh->v_full[st], 1);
+    mbar_init(&sh->dp_full, 1);
+    mbar_init(&sh->s_full[0], 1);
+    mbar_init(&sh->s_read, 8);
+    mbar_init(&sh->ds_full, 8);
     mbar_init(&sh->mm_done, 1);
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
@@ -164,18 +230,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       bool ok = true;
-      int loads = 0;  // ring loads issued
-      auto load_kv = [&](int j) {
-        const int s = j & 1, col = col_idx[c0 + j];
-        uint8_t* dst = smem + C::OFF_RING + s * 2 * C::TILE;
-        mbar_arrive_expect_tx(&sh->ring_full[s], 2 * C::TILE);
+      int kl = 0, vl = 0;  // K and V loads issued
+      auto load_k = [&](int j) {
+        const int st = j % 3, col = col_idx[c0 + j];
+        mbar_arrive_expect_tx(&sh->k_full[st], C::TILE);
 #pragma unroll
-        for (int ch = 0; ch < C::DCH; ++ch) {
-          tma_load_3d(dst + ch * 16384, &tm_k, &sh->ring_full[s], h * D + ch * 64, col * 128, b);
-          tma_load_3d(dst + C::TILE + ch * 16384, &tm_v, &sh->ring_full[s], h * D + ch * 64, col * 128, b);
-        }
-        ++loads;
+        for (int ch = 0; ch < C::DCH; ++ch)
+          tma_load_3d(smem + C::DQ_OFF_K + st * C::TILE + ch * 16384, &tm_k, &sh->k_full[st], h * D + ch * 64,
+                      col * 128, b);
+        ++kl;
       };
+      auto load_v = [&](int j) {
+        const int st = j & 1, col = col_idx[c0 + j];
+        mbar_arrive_expect_tx(&sh->v_full[st], C::TILE);
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch)
+          tma_load_3d(smem + C::DQ_OFF_V + st * C::TILE + ch * 16384, &tm_v, &sh->v_full[st], h * D + ch * 64,
+                      col * 128, b);
+        ++vl;
+      };
+      auto k_tile = [&](int j) { return sbase + C::DQ_OFF_K + (j % 3) * C::TILE; };
+      auto v_tile = [&](int j) { return sbase + C::DQ_OFF_V + (j & 1) * C::TILE; };
+      auto wait_k = [&](int j) { return mbar_wait(&sh->k_full[j % 3], (uint32_t)((j / 3) & 1), limit_ns); };
+      auto wait_v = [&](int j) { return mbar_wait(&sh->v_full[j & 1], (uint32_t)((j >> 1) & 1), limit_ns); };
       mbar_arrive_expect_tx(&sh->fixed_full, 2 * C::TILE);
 #pragma unroll
       for (int ch = 0; ch < C::DCH; ++ch) {
@@ -183,37 +260,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_3d(smem + C::OFF_FIX + C::TILE + ch * 16384, &tm_do, &sh->fixed_full, h * D + ch * 64, qt * 128,
                     b);
       }
-      for (int j = 0; j < n && j < 2; ++j) load_kv(j);
+      for (int j = 0; j < n && j < 3; ++j) load_k(j);
+      for (int j = 0; j < n && j < 2; ++j) load_v(j);
+      // Q and dO go to tensor memory once, so that S = Q K^T and dP = dO V^T read
+      // one shared operand each.  Schedule: S_{j+1} as soon as the row warps have
+      // read S_j (while they form dS_j over dP_j), then dQ += dS_j K_j and
+      // dP_{j+1} (after the dQ product, in issue order) while they take the
+      // exponentials of S_{j+1}.  K_{j+3} refills K_j's stage once the dQ product
+      // has read it, V_{j+2} refills V_j's once dP_j is done.
       ok = mbar_wait(&sh->fixed_full, 0, limit_ns);
       if (ok && n >= 1) {
-        ok = mbar_wait(&sh->ring_full[0], 0, limit_ns);
+        ok = wait_k(0) && wait_v(0);
         if (ok) {
           tc_fence_after();
-          const uint32_t kt = sbase + C::OFF_RING;
-          mma_xyt<D>(tmem + TM_S, q_s, kt);
-          mma_xyt<D>(tmem + TM_DP, do_s, kt + C::TILE);
-          mma_commit(&sh->sdp_full);
+          copy_tile_to_tmem<D>(tmem + TM_Q, q_s);
+          copy_tile_to_tmem<D>(tmem + TM_DO, do_s);
+          mma_tyt<D>(tmem + TM_S, tmem + TM_Q, k_tile(0));
+          mma_commit(&sh->s_full[0]);
+          mma_tyt<D>(tmem + TM_DP, tmem + TM_DO, v_tile(0));
+          mma_commit(&sh->dp_full);
         }
       }
       for (int j = 0; ok && j < n; ++j) {
-        const int s = j & 1;
+        if (j + 1 < n) {
+          // S_{j+1} over S_j once the row warps have read it
+          if (sh->abort_flag || !mbar_wait(&sh->s_read, (uint32_t)(j & 1), limit_ns) || !wait_k(j + 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tyt<D>(tmem + TM_S, tmem + TM_Q, k_tile(j + 1));
+          mma_commit(&sh->s_full[0]);
+        }
         if (sh->abort_flag || !mbar_wait(&sh->ds_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
         tc_fence_after();
-        mma_grad<D>(tmem + TM_DQ, tmem + TM_DS, sbase + C::OFF_RING + s * 2 * C::TILE, j > 0);
+        mma_grad<D>(tmem + TM_DQ, tmem + TM_DP, k_tile(j), j > 0, true);
         mma_commit(&sh->mm_done);
+        // dP_j completed before the row warps formed dS_j: V_j's stage is free
+        if (j + 2 < n) load_v(j + 2);
         if (j + 1 < n) {
-          const int s1 = (j + 1) & 1;
-          if (!mbar_wait(&sh->ring_full[s1], (uint32_t)(((j + 1) >> 1) & 1), limit_ns)) { ok = false; break; }
+          // dP_{j+1} over dS_j, after the dQ product that reads it (issue order)
+          if (!wait_v(j + 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kt = sbase + C::OFF_RING + s1 * 2 * C::TILE;
-          mma_xyt<D>(tmem + TM_S, q_s, kt);
-          mma_xyt<D>(tmem + TM_DP, do_s, kt + C::TILE);
-          mma_commit(&sh->sdp_full);
+          mma_tyt<D>(tmem + TM_DP, tmem + TM_DO, v_tile(j + 1));
+          mma_commit(&sh->dp_full);
         }
-        if (j + 2 < n) {
-          // stage s is free once the dQ product of tile j has read its K
+        if (j + 3 < n) {
+          // K_j's stage is free once the dQ product of tile j has read it
           if (!mbar_wait(&sh->mm_done, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
-          load_kv(j + 2);
+          load_k(j + 3);
         }
       }
       if (!ok) {
@@ -223,38 +318,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       // every copy this thread started lands before the CTA exits
       mbar_wait(&sh->fixed_full, 0, kBwdDrainNs);
-      for (int i = (loads > 2 ? loads - 2 : 0); i < loads; ++i)
-        mbar_wait(&sh->ring_full[i & 1], (uint32_t)((i >> 1) & 1), kBwdDrainNs);
+      for (int i = (kl > 3 ? kl - 3 : 0); i < kl; ++i)
+        mbar_wait(&sh->k_full[i % 3], (uint32_t)((i / 3) & 1), kBwdDrainNs);
+      for (int i = (vl > 2 ? vl - 2 : 0); i < vl; ++i)
+        mbar_wait(&sh->v_full[i & 1], (uint32_t)((i >> 1) & 1), kBwdDrainNs);
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------------- one thread per query row
-    const int quarter = warp & 3, r = quarter * 32 + lane;
+    // and column half: keys [64 half, 64 half + 64) of each key tile
+    const int quarter = warp & 3, r = quarter * 32 + lane, half = (warp - 2) >> 2;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const float l2 = lse2[(size_t)bh * npad + qt * 128 + r];
     const float Dr = dvec[(size_t)bh * npad + qt * 128 + r];
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int valid = min(128, N - col_idx[c0 + j] * 128);  // real keys of the tile
-      if (!mbar_wait_warp(&sh->sdp_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
-      // (S and dP of tile j were committed after the dQ product of tile j - 1, so
-      // that product, the last reader of the dS columns, has completed too)
+      // P of the row from S_j (fp32, kept in registers), then S_j is released
+      const uint32_t s_addr = lane_addr + TM_S;
+      if (!mbar_wait_warp(&sh->s_full[0], (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32], pr[32], dsp[16];
-        tmem_ld32(lane_addr + TM_S + c * 32, sr);
-        tmem_ld32(lane_addr + TM_DP + c * 32, pr);
+      float p[64];
+      {
+        uint32_t sr0[32], sr1[32];  // both chunks of this half, one wait
+        tmem_ld32(s_addr + (2 * half) * 32, sr0);
+        tmem_ld32(s_addr + (2 * half + 1) * 32, sr1);
+        tmem_ld_wait();
+        exp_chunk(sr0, scale_log2, l2, (2 * half) * 32, valid, p);
+        exp_chunk(sr1, scale_log2, l2, (2 * half + 1) * 32, valid, p + 32);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->s_read);
+      // dS = P (dP - D) over this half's own dP columns, read first
+      if (!mbar_wait_warp(&sh->dp_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+      tc_fence_after();
+      {
+        uint32_t pr[2][32];
+        tmem_ld32(lane_addr + TM_DP + (2 * half) * 32, pr[0]);
+        tmem_ld32(lane_addr + TM_DP + (2 * half + 1) * 32, pr[1]);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k0 = c * 32 + 2 * i;
-          const float p0 = k0 < valid ? ex2_approx(__uint_as_float(sr[2 * i]) * scale_log2 - l2) : 0.f;
-          const float p1 = k0 + 1 < valid ? ex2_approx(__uint_as_float(sr[2 * i + 1]) * scale_log2 - l2) : 0.f;
-          dsp[i] = pack_bf16x2(p0 * (__uint_as_float(pr[2 * i]) - Dr), p1 * (__uint_as_float(pr[2 * i + 1]) - Dr));
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t dsp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            dsp[i] = pack_bf16x2(p[cc * 32 + 2 * i] * (__uint_as_float(pr[cc][2 * i]) - Dr),
+                                 p[cc * 32 + 2 * i + 1] * (__uint_as_float(pr[cc][2 * i + 1]) - Dr));
+          tmem_st16(lane_addr + TM_DP + 64 * half + 16 * cc, dsp);
         }
-        tmem_st16(lane_addr + TM_DS + c * 16, dsp);
-        tmem_st_wait();
       }
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->ds_full);
@@ -267,7 +380,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int row = qt * 128 + r;
       float* dst = dq + (((size_t)b * N + row) * heads + h) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t g[32];
         if (n >= 1) {
           tmem_ld32(lane_addr + TM_DQ + c * 32, g);
@@ -314,8 +427,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     float* __restrict__ dv, int N, int heads, int nb, int npad, int mask_per_bh, float scale,
                     float scale_log2, uint32_t* status, uint64_t limit_ns) {
   using C = BwdCfg<D>;
-  // S^T [0,128) (P^T as bf16 over its first 64 columns), dP^T [128,256) (dS^T
-  // over its first 64), dV [256,256+D), dK [384,384+D)
+  // S^T [0,128) (P^T as bf16 over its columns [0,32) and [64,96), one range per
+  // column half), dP^T [128,256) (dS^T likewise), dV [256,256+D), dK [384,384+D)
   constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 384;
   extern __shared__ uint8_t bwd_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -334,7 +447,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sh->ring_full[0], 1);
     mbar_init(&sh->ring_full[1], 1);
     mbar_init(&sh->sdp_full, 1);
-    mbar_init(&sh->ds_full, 4);
+    mbar_init(&sh->ds_full, 8);
     mbar_init(&sh->mm_done, 1);
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
@@ -391,8 +504,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (sh->abort_flag || !mbar_wait(&sh->ds_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qs = sbase + C::OFF_RING + s * 2 * C::TILE;
-        mma_grad<D>(tmem + TM_DV, tmem + TM_S, qs + C::TILE, j > 0);  // dV += P^T dO
-        mma_grad<D>(tmem + TM_DK, tmem + TM_DP, qs, j > 0);          // dK += dS^T Q
+        mma_grad<D>(tmem + TM_DV, tmem + TM_S, qs + C::TILE, j > 0, true);  // dV += P^T dO
+        mma_grad<D>(tmem + TM_DK, tmem + TM_DP, qs, j > 0, true);          // dK += dS^T Q
         mma_commit(&sh->mm_done);
         if (j + 1 < n) {
           // S^T and dP^T of the next tile overwrite P^T and dS^T: issued after
@@ -421,7 +534,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------------- one thread per key row
-    const int quarter = warp & 3, r = quarter * 32 + lane;
+    // and column half: query rows [64 half, 64 half + 64) of each query tile
+    const int quarter = warp & 3, r = quarter * 32 + lane, half = (warp - 2) >> 2;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -432,27 +546,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const float* l2v = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * C::VEC);
       const float* dvv = l2v + 128;
+      uint32_t sr2[2][32], pr2[2][32];  // this half's chunks of S^T and dP^T, one wait
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32], pr[32];
-        tmem_ld32(lane_addr + TM_S + c * 32, sr);
-        tmem_ld32(lane_addr + TM_DP + c * 32, pr);
-        tmem_ld_wait();
+      for (int cc = 0; cc < 2; ++cc) {
+        tmem_ld32(lane_addr + TM_S + (2 * half + cc) * 32, sr2[cc]);
+        tmem_ld32(lane_addr + TM_DP + (2 * half + cc) * 32, pr2[cc]);
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * half + cc;
+        const uint32_t(&sr)[32] = sr2[cc];
+        const uint32_t(&pr)[32] = pr2[cc];
         uint32_t pp[16], dsp[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int q0 = c * 32 + 2 * i;
-          const float p0 = ex2_approx(__uint_as_float(sr[2 * i]) * scale_log2 - l2v[q0]);
-          const float p1 = ex2_approx(__uint_as_float(sr[2 * i + 1]) * scale_log2 - l2v[q0 + 1]);
+          const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                       f32x2_pack(scale_log2, scale_log2), f32x2_pack(-l2v[q0], -l2v[q0 + 1]));
+          float p0, p1;
+          if ((i & 3) == 3) {
+            exp2_fma_x2(x, p0, p1);  // one pair in four on the FMA pipe
+          } else {
+            float x0, x1;
+            f32x2_unpack(x, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
           pp[i] = pack_bf16x2(p0, p1);
           dsp[i] = pack_bf16x2(p0 * (__uint_as_float(pr[2 * i]) - dvv[q0]),
                                p1 * (__uint_as_float(pr[2 * i + 1]) - dvv[q0 + 1]));
         }
-        // columns [16c, 16c + 16) of each region: already read by this thread
-        tmem_st16(lane_addr + TM_S + c * 16, pp);
-        tmem_st16(lane_addr + TM_DP + c * 16, dsp);
-        tmem_st_wait();
+        // this half's packed columns, inside the range it has already read:
+        // [64 half + 16 cc, + 16) of each region
+        tmem_st16(lane_addr + TM_S + 64 * half + 16 * cc, pp);
+        tmem_st16(lane_addr + TM_DP + 64 * half + 16 * cc, dsp);
       }
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->ds_full);
@@ -469,7 +599,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         float* dst = (part == 0 ? dv : dk) + off;
         const float mul = part == 0 ? 1.f : scale;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
           uint32_t g[32];
           if (n >= 1) {
             tmem_ld32(lane_addr + (part == 0 ? TM_DV : TM_DK) + c * 32, g);
@@ -510,9 +640,9 @@ cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   const int grid = a.B * a.heads * a.nb;
-  e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::DQ_SMEM);
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<grid, kBwdThreads, C::SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.row_ptr, a.col_idx,
+  bwd_dq_kernel<D><<<grid, kBwdThreads, C::DQ_SMEM, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.row_ptr, a.col_idx,
                                                       a.lse2, a.dvec, a.dq, a.N, a.heads, a.nb, a.npad,
                                                       a.mask_per_bh, a.scale, a.scale_log2, a.status,
                                                       a.wait_limit_ns, a.full);
