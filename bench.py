@@ -46,10 +46,10 @@ FLUSH_BYTES = 256 << 20
 # from an ncu capture (see profiles/), keyed by the kernel sources it was taken
 # on; stale entries are ignored.
 NCU_TRAFFIC = {
-    "wan1.3b-32760tok-90pct": {"source": "613b0b110525a10e", "bytes": 303_341_568 + 84_111_616},
-    "wan1.3b-32760tok-tiles1x32x4": {"source": "613b0b110525a10e", "bytes": 303_325_440 + 83_893_248},
-    "wan1.3b-32760tok-topk26": {"source": "613b0b110525a10e", "bytes": 303_766_528 + 85_206_528},
-    "wan1.3b-32760tok-90pct-itads": {"source": "613b0b110525a10e", "bytes": 303_142_144 + 84_182_272},
+    "wan1.3b-32760tok-90pct": {"source": "3c09ac19706bfa90", "bytes": 303_178_496 + 84_154_368},
+    "wan1.3b-32760tok-tiles1x32x4": {"source": "3c09ac19706bfa90", "bytes": 303_182_336 + 83_957_504},
+    "wan1.3b-32760tok-topk26": {"source": "3c09ac19706bfa90", "bytes": 304_167_168 + 84_824_320},
+    "wan1.3b-32760tok-90pct-itads": {"source": "3c09ac19706bfa90", "bytes": 302_995_200 + 83_959_808},
 }
 
 
