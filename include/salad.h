@@ -202,6 +202,45 @@ int salad_attn_forward_lse(const void* q, const void* k, const void* v, int B, i
  * rounded to bf16 as operands), fp32 elsewhere.  Never synchronises.
  * Errors: INVALID_ARG, UNSUPPORTED (d, block), WORKSPACE, CUDA.
  */
+/*
+ * salad_attn_forward on inputs and output in HOST memory, for a caller whose
+ * tensors live on the host: the host-to-device copies of one chunk of heads
+ * run while the chunk before it computes and the one before that copies its
+ * output back.  The layer's (b, h) units are independent (SALAD summary section
+ * 2.1: every head has its own mask rows, linear-branch state and output), so a
+ * chunk (one batch element, heads [h0, h0 + heads_per_chunk)) is a complete
+ * forward of its own (salad_attn_forward_heads on it).
+ *   q_host, k_host, v_host  HOST bf16 [B][N][Hh][d], read; out_host HOST bf16
+ *                  [B][N][Hh][d], written.  Page-locked memory (cudaHostAlloc
+ *                  or cudaHostRegister) for the copies to overlap; pageable
+ *                  memory works but serialises them.
+ *   q_dev, k_dev, v_dev, out_dev  DEVICE bf16 [B][N][Hh][d], 16-byte aligned:
+ *                  the staging copies (they hold the inputs and the output
+ *                  afterwards).  The library allocates nothing.
+ *   row_ptr, col_idx, w_proj, gate  DEVICE, as salad_attn_forward (a per-head
+ *                  raster mask from salad_build_block_mask).
+ *   heads_per_chunk  > 0, or 0 for about six chunks per batch element (at 12
+ *                  heads, 32,760 tokens: 6.43 ms per call against 5.45 ms for
+ *                  the input copies alone and 8.2 ms with one chunk).
+ *   workspace      >= salad_workspace_bytes(1, N, heads_per_chunk, d) (chunks
+ *                  run one after another on `stream` and share it).
+ *   stream         the forwards; copy_in, copy_out  two other streams for the
+ *                  copies.  The copies wait for the work queued on `stream`
+ *                  before the call, and `stream` waits for the last output copy:
+ *                  synchronising `stream` (or an event recorded on it after the
+ *                  call) covers the whole call.
+ * Arithmetic, rounding and results as salad_attn_forward_heads per chunk.
+ * Errors: INVALID_ARG (null, misaligned device buffers, equal streams),
+ * UNSUPPORTED (block, d, Hh > 65535), WORKSPACE, CUDA; otherwise as
+ * salad_attn_forward.
+ */
+int salad_attn_forward_host(const void* q_host, const void* k_host, const void* v_host, void* out_host, int B,
+                            int N, int num_heads, int d, int block, const int32_t* row_ptr, const int32_t* col_idx,
+                            const void* w_proj, const float* gate, float softmax_scale, float eps,
+                            int heads_per_chunk, void* q_dev, void* k_dev, void* v_dev, void* out_dev,
+                            void* workspace, size_t workspace_bytes, salad_stream_t stream,
+                            salad_stream_t copy_in, salad_stream_t copy_out);
+
 size_t salad_backward_workspace_bytes(int B, int N, int num_heads);
 int salad_attn_backward_sparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
                                const float* lse, int B, int N, int num_heads, int d, int block,

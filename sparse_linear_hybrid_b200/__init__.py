@@ -78,6 +78,9 @@ def lib() -> ctypes.CDLL:
         L.salad_attn_forward_lse.restype = i
         L.salad_attn_forward_heads.argtypes = [p, p, p, i, i, i, i, i, i, i, p, p, p, p, f, f, p, p, sz, p]
         L.salad_attn_forward_heads.restype = i
+        L.salad_attn_forward_host.argtypes = [p, p, p, p, i, i, i, i, i, p, p, p, p, f, f, i, p, p, p, p, p, sz, p, p,
+                                              p]
+        L.salad_attn_forward_host.restype = i
         L.salad_backward_workspace_bytes.argtypes = [i, i, i]
         L.salad_backward_workspace_bytes.restype = sz
         L.salad_attn_backward_sparse.argtypes = [p, p, p, p, p, p, i, i, i, i, i, p, p, p, p, i, f, p, p, p, p, sz,
@@ -144,6 +147,19 @@ def _dev_ptr(t: torch.Tensor, dtype, name: str) -> ctypes.c_void_p:
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t: torch.Tensor, dtype, name: str) -> ctypes.c_void_p:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+_copy_streams = {}
 
 
 def mask_num_blocks(T: int, H: int, W: int, block: int) -> int:
@@ -367,6 +383,41 @@ def attn_backward(q, k, v, out, dout, lse, row_ptr, col_idx, w_proj, gate, block
         float(eps), f32("dq"), f32("dk"), f32("dv"), f32("dw"), f32("dgate"),
         _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "salad_attn_backward")
     return res
+
+
+def attn_forward_host(q, k, v, row_ptr, col_idx, w_proj, gate, block: int, out=None, staging=None,
+                      heads_per_chunk: int = 0, softmax_scale: float = 0.0, eps: float = 1e-6, workspace=None,
+                      stream=None, copy_streams=None, device=None):
+    """The layer forward on host tensors (see salad_attn_forward_host): q, k, v
+    bf16 CPU [B, N, Hh, d] (pinned for the copies to overlap the compute), the
+    mask, w_proj and gate on the GPU.  `staging` is (q_dev, k_dev, v_dev, out_dev)
+    bf16 CUDA tensors of the same shape (allocated when None); `copy_streams` two
+    CUDA streams for the copies (two per device are kept for reuse when None).
+    Returns the host output tensor (pinned when allocated here)."""
+    B, N, Hh, d = q.shape
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    if staging is None:
+        staging = tuple(torch.empty(q.shape, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    if copy_streams is None:
+        key = dev.index if dev.index is not None else torch.cuda.current_device()
+        if key not in _copy_streams:
+            _copy_streams[key] = (torch.cuda.Stream(device=key), torch.cuda.Stream(device=key))
+        copy_streams = _copy_streams[key]
+    hpc = int(heads_per_chunk) if heads_per_chunk > 0 else (Hh + 5) // 6
+    if workspace is None:
+        workspace = new_workspace(1, N, min(hpc, Hh), d, dev)
+    h = lambda t, n: _host_ptr(t, torch.bfloat16, n)  # noqa: E731
+    g = lambda t, n: _dev_ptr(t, torch.bfloat16, n)  # noqa: E731
+    _check(lib().salad_attn_forward_host(
+        h(q, "q"), h(k, "k"), h(v, "v"), h(out, "out"), B, N, Hh, d, int(block),
+        _dev_ptr(row_ptr, torch.int32, "row_ptr"), _dev_ptr(col_idx, torch.int32, "col_idx"),
+        g(w_proj, "w_proj"), _dev_ptr(gate, torch.float32, "gate"), float(softmax_scale), float(eps),
+        int(heads_per_chunk), g(staging[0], "q_dev"), g(staging[1], "k_dev"), g(staging[2], "v_dev"),
+        g(staging[3], "out_dev"), _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _stream(stream), _stream(copy_streams[0]), _stream(copy_streams[1])), "salad_attn_forward_host")
+    return out
 
 
 def attn_forward_tiles(q, k, v, grid, tile, row_ptr, col_idx, w_proj, gate, softmax_scale: float = 0.0,

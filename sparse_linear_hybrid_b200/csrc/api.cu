@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 
@@ -338,6 +339,86 @@ int salad_attn_forward_heads(const void* q, const void* k, const void* v, int B,
   if (heads_total > 65535) return SALAD_ERR_UNSUPPORTED;
   return attn_forward_impl(q, k, v, B, N, head_count, d, block, row_ptr, col_idx, w_proj, gate, softmax_scale, eps,
                            out, workspace, workspace_bytes, stream, 0, nullptr, nullptr, head_begin, heads_total);
+}
+
+int salad_attn_forward_host(const void* q_host, const void* k_host, const void* v_host, void* out_host, int B,
+                            int N, int num_heads, int d, int block, const int32_t* row_ptr, const int32_t* col_idx,
+                            const void* w_proj, const float* gate, float softmax_scale, float eps,
+                            int heads_per_chunk, void* q_dev, void* k_dev, void* v_dev, void* out_dev,
+                            void* workspace, size_t workspace_bytes, salad_stream_t stream,
+                            salad_stream_t copy_in, salad_stream_t copy_out) {
+  if (!q_host || !k_host || !v_host || !out_host || !q_dev || !k_dev || !v_dev || !out_dev || !row_ptr ||
+      !col_idx || !w_proj || !gate || !workspace)
+    return SALAD_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || num_heads < 1 || heads_per_chunk < 0) return SALAD_ERR_INVALID_ARG;
+  if (block != 64 && block != 128) return SALAD_ERR_UNSUPPORTED;
+  if (num_heads > 65535) return SALAD_ERR_UNSUPPORTED;
+  // about six chunks per batch element: measured best at 12 heads (the last
+  // chunk's compute and output copy are the part the copies cannot hide)
+  int hpc = heads_per_chunk > 0 ? heads_per_chunk : (num_heads + 5) / 6;
+  if (hpc > num_heads) hpc = num_heads;
+  if (workspace_bytes < salad_workspace_bytes(1, N, hpc, d)) return SALAD_ERR_WORKSPACE;
+  const void* p16[] = {q_dev, k_dev, v_dev, out_dev};
+  for (const void* ptr : p16)
+    if (!aligned(ptr, 16)) return SALAD_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t c_in = reinterpret_cast<cudaStream_t>(copy_in), c_out = reinterpret_cast<cudaStream_t>(copy_out);
+  if (c_in == s || c_out == s || c_in == c_out) return SALAD_ERR_INVALID_ARG;
+  const int nb = (N + block - 1) / block;
+  const int chunks_per_b = (num_heads + hpc - 1) / hpc;
+  const int chunks = B * chunks_per_b;
+  // events ordering the three streams: the copies wait for the work queued on
+  // `stream` before the call, each chunk's forward for its inputs, each chunk's
+  // output copy for its forward, and `stream` for the last output copy
+  std::vector<cudaEvent_t> ev(2 * (size_t)chunks + 2, nullptr);
+  int st = SALAD_OK;
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      e = nullptr;
+      st = SALAD_ERR_CUDA;
+      break;
+    }
+  const size_t pitch = (size_t)num_heads * d * 2;
+  auto bytes_at = [&](const void* base, size_t off) { return static_cast<const uint8_t*>(base) + off; };
+  auto wbytes_at = [&](void* base, size_t off) { return static_cast<uint8_t*>(base) + off; };
+  if (st == SALAD_OK &&
+      (cudaEventRecord(ev[0], s) != cudaSuccess || cudaStreamWaitEvent(c_in, ev[0], 0) != cudaSuccess ||
+       cudaStreamWaitEvent(c_out, ev[0], 0) != cudaSuccess))
+    st = SALAD_ERR_CUDA;
+  for (int c = 0; c < chunks && st == SALAD_OK; ++c) {
+    const int b = c / chunks_per_b, h0 = (c % chunks_per_b) * hpc;
+    const int hc = h0 + hpc <= num_heads ? hpc : num_heads - h0;
+    const size_t batch_off = (size_t)b * N * pitch, off = batch_off + (size_t)h0 * d * 2;
+    const size_t width = (size_t)hc * d * 2;
+    const void* src[3] = {q_host, k_host, v_host};
+    void* dst[3] = {q_dev, k_dev, v_dev};
+    for (int t = 0; t < 3 && st == SALAD_OK; ++t)
+      if (cudaMemcpy2DAsync(wbytes_at(dst[t], off), pitch, bytes_at(src[t], off), pitch, width, (size_t)N,
+                            cudaMemcpyHostToDevice, c_in) != cudaSuccess)
+        st = SALAD_ERR_CUDA;
+    if (st != SALAD_OK) break;
+    if (cudaEventRecord(ev[1 + 2 * c], c_in) != cudaSuccess || cudaStreamWaitEvent(s, ev[1 + 2 * c], 0) != cudaSuccess) {
+      st = SALAD_ERR_CUDA;
+      break;
+    }
+    // the chunk's forward: batch element b, heads [h0, h0 + hc) of the full tensors
+    st = attn_forward_impl(bytes_at(q_dev, batch_off), bytes_at(k_dev, batch_off), bytes_at(v_dev, batch_off), 1, N,
+                           hc, d, block, row_ptr + (size_t)h0 * nb, col_idx, w_proj, gate + (size_t)b * num_heads + h0,
+                           softmax_scale, eps, wbytes_at(out_dev, batch_off), workspace, workspace_bytes, stream, 0,
+                           nullptr, nullptr, h0, num_heads);
+    if (st != SALAD_OK) break;
+    if (cudaEventRecord(ev[2 + 2 * c], s) != cudaSuccess || cudaStreamWaitEvent(c_out, ev[2 + 2 * c], 0) != cudaSuccess ||
+        cudaMemcpy2DAsync(wbytes_at(out_host, off), pitch, bytes_at(out_dev, off), pitch, width, (size_t)N,
+                          cudaMemcpyDeviceToHost, c_out) != cudaSuccess)
+      st = SALAD_ERR_CUDA;
+  }
+  // `stream` waits for the last output copy, so synchronising it covers the call
+  if (st == SALAD_OK && (cudaEventRecord(ev.back(), c_out) != cudaSuccess ||
+                         cudaStreamWaitEvent(s, ev.back(), 0) != cudaSuccess))
+    st = SALAD_ERR_CUDA;
+  for (auto e : ev)
+    if (e != nullptr) cudaEventDestroy(e);  // released once the work recorded on it completes
+  return st;
 }
 
 size_t salad_backward_workspace_bytes(int B, int N, int num_heads) {

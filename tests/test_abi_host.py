@@ -369,3 +369,22 @@ def test_transpose_mask_argument_errors(L):
     assert T(p(FAKE + 2), p(FAKE), 1, 4, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_INVALID_ARG
     assert T(p(FAKE), p(FAKE), 70000, 4, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_UNSUPPORTED
     assert T(p(FAKE), p(FAKE), 1, 50000, p(FAKE), p(FAKE), None) == sl.SALAD_ERR_UNSUPPORTED
+
+
+def test_host_buffer_forward_argument_errors(L):
+    """salad_attn_forward_host checks its arguments before any CUDA call."""
+    def call(**kw):
+        a = dict(B=1, N=256, H=2, d=64, block=64, hpc=0, ws_bytes=1 << 30, dev=FAKE + 0x30000000, s=0x1000,
+                 cin=0x2000, cout=0x3000, q=FAKE)
+        a.update(kw)
+        return L.salad_attn_forward_host(p(a["q"]), p(FAKE), p(FAKE), p(FAKE), a["B"], a["N"], a["H"], a["d"],
+                                         a["block"], p(FAKE), p(FAKE), p(FAKE), p(FAKE), 0.0, 1e-6, a["hpc"],
+                                         p(a["dev"]), p(FAKE), p(FAKE), p(FAKE), p(0x40000000), a["ws_bytes"],
+                                         p(a["s"]), p(a["cin"]), p(a["cout"]))
+    assert call(q=0) == sl.SALAD_ERR_INVALID_ARG
+    assert call(hpc=-1) == sl.SALAD_ERR_INVALID_ARG
+    assert call(block=96) == sl.SALAD_ERR_UNSUPPORTED
+    assert call(ws_bytes=1024) == sl.SALAD_ERR_WORKSPACE
+    assert call(dev=FAKE + 8) == sl.SALAD_ERR_INVALID_ARG      # staging not 16-byte aligned
+    assert call(cin=0x1000) == sl.SALAD_ERR_INVALID_ARG        # a copy stream equal to the compute stream
+    assert call(cin=0x2000, cout=0x2000) == sl.SALAD_ERR_INVALID_ARG
