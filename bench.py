@@ -356,6 +356,19 @@ def whole_job_tflops(world: int, steps: int, flops_per_step: float, total_ms: fl
     return job_tflops(steps, world * flops_per_step, total_ms)
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (reported beside the oracle's core count)."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def config_of(wl: si.Workload, flops: float, nnz: int, world: int, split: str = "replicas"):
     rows = wl.B * wl.Hh * wl.nb if wl.topk else wl.Hh * wl.nb
     mask = {"topk_keep": wl.topk} if wl.topk else {"window_thw": list(wl.window)}
@@ -451,8 +464,8 @@ def reference_line(args, wl, world, cores, m, n_blocks, t_lin, flops_step, nnz, 
             "kept_flop_fraction_per_step": round(sum(flops_list) / len(flops_list) / flops_step, 6),
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(wl, flops_step, nnz, world),
-            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": desc},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "cpu": cpu_model(),
+                             "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -828,7 +841,8 @@ def run_salad(args, wl):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, desc, _, _ = oracle_sample_rate(wl, inp, rp_h, ci_h, budget_s=args.cpu_seconds)
-        cpu = {"value": round(rate, 6), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = {"value": round(rate, 6), "unit": UNIT, "cores": cores, "cpu": cpu_model(), "kind": "oracle",
+               "sample": desc}
 
     clk = clocks.summary()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
