@@ -43,9 +43,9 @@ struct BwdShared {
   uint64_t v_full[2];     // dQ kernel: the V ring (two stages)
   uint64_t sdp_full;      // dK/dV kernel: S^T and dP^T of the current tile are in tensor memory
   uint64_t dp_full;       // dQ kernel: dP of the current tile is in tensor memory
-  uint64_t s_full[2];     // dQ kernel: S of the current tile is in tensor memory ([0] used)
+  uint64_t s_full;        // dQ kernel: S of the current tile is in tensor memory
   uint64_t s_read;        // dQ kernel: the row warps have read S of the current tile
-  uint64_t ds_full;       // the four row warps have written dS (and P^T) of the tile
+  uint64_t ds_full;       // the eight row warps have written dS (and P^T) of the tile
   uint64_t mm_done;       // the gradient products of the tile have completed
   uint64_t drain;
   uint32_t tmem_base;
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int st = 0; st < 3; ++st) mbar_init(&sh->k_full[st], 1);
     for (int st = 0; st < 2; ++st) mbar_init(&sh->v_full[st], 1);
     mbar_init(&sh->dp_full, 1);
-    mbar_init(&sh->s_full[0], 1);
+    mbar_init(&sh->s_full, 1);
     mbar_init(&sh->s_read, 8);
     mbar_init(&sh->ds_full, 8);
     mbar_init(&sh->mm_done, 1);
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           copy_tile_to_tmem<D>(tmem + TM_Q, q_s);
           copy_tile_to_tmem<D>(tmem + TM_DO, do_s);
           mma_tyt<D>(tmem + TM_S, tmem + TM_Q, k_tile(0));
-          mma_commit(&sh->s_full[0]);
+          mma_commit(&sh->s_full);
           mma_tyt<D>(tmem + TM_DP, tmem + TM_DO, v_tile(0));
           mma_commit(&sh->dp_full);
         }
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tc_fence_after();
           mma_tyt<D>(tmem + TM_S, tmem + TM_Q, k_tile(j + 1));
-          mma_commit(&sh->s_full[0]);
+          mma_commit(&sh->s_full);
         }
         if (sh->abort_flag || !mbar_wait(&sh->ds_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
         tc_fence_after();
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int valid = min(128, N - col_idx[c0 + j] * 128);  // real keys of the tile
       // P of the row from S_j (fp32, kept in registers), then S_j is released
       const uint32_t s_addr = lane_addr + TM_S;
-      if (!mbar_wait_warp(&sh->s_full[0], (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+      if (!mbar_wait_warp(&sh->s_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
       tc_fence_after();
       float p[64];
       {
