@@ -17,13 +17,16 @@
 //   bwd_dkdv_kernel  one CTA per (key tile, b, h), over the query tiles whose
 //                    rows keep it (the transposed mask): S^T = K Q^T and
 //                    dP^T = V dO^T, one thread per key row forms P^T and dS^T
-//                    (bf16, written over the columns of S^T and dP^T it has
-//                    read), dV += P^T dO and dK += dS^T Q
+//                    (bf16, written over the columns of S^T it has read),
+//                    dV += P^T dO and dK += dS^T Q.  dP^T of the next tile
+//                    runs as soon as dP^T is in the row warps' registers, and
+//                    the products of the first query half while the row warps
+//                    form the second.
 // Warp roles, 320 threads: warp 0 lane 0 issues the TMA loads and the MMAs in
 // program order (K/V or Q/dO tiles in a 2-deep ring), warp 1 owns the tensor
-// memory, warps 2-9 take one row each (TMEM lane quarter = warp % 4) and one
-// half of its 128 columns (warp (w - 2) / 4); the exponentials of one pair in
-// four run on the FMA pipe (exp2_fma_x2), the rest on the MUFU.  Every
+// memory, warps 2-9 take one row each (TMEM lane quarter = warp % 4) and 64 of
+// its 128 columns (warp (w - 2) / 4 picks which); the exponentials of one pair
+// in four run on the FMA pipe (exp2_fma_x2), the rest on the MUFU.  Every
 // barrier wait is bounded; on a time-out the kernel records it and drains.
 // Gradients are written in fp32.
 #include "internal.h"
@@ -41,11 +44,13 @@ struct BwdShared {
   uint64_t ring_full[2];  // dK/dV kernel: the streamed tiles (Q, dO and the row vectors)
   uint64_t k_full[3];     // dQ kernel: the K ring (three stages)
   uint64_t v_full[2];     // dQ kernel: the V ring (two stages)
-  uint64_t sdp_full;      // dK/dV kernel: S^T and dP^T of the current tile are in tensor memory
-  uint64_t dp_full;       // dQ kernel: dP of the current tile is in tensor memory
-  uint64_t s_full;        // dQ kernel: S of the current tile is in tensor memory
+  uint64_t dp_full;       // dP (dQ kernel) or dP^T (dK/dV kernel) of the current tile is in tensor memory
+  uint64_t s_full;        // S (dQ kernel) or S^T (dK/dV kernel) of the current tile is in tensor memory
   uint64_t s_read;        // dQ kernel: the row warps have read S of the current tile
-  uint64_t ds_full;       // the eight row warps have written dS (and P^T) of the tile
+  uint64_t dp_read;       // dK/dV kernel: the row warps have read dP^T of the current tile
+  uint64_t ds_h[2];       // dK/dV kernel: P^T and dS^T of one query half of the current tile are written
+  uint64_t grads_done;    // dK/dV kernel: the gradient products of the last tile have completed
+  uint64_t ds_full;       // dQ kernel: the eight row warps have written dS of the tile
   uint64_t mm_done;       // the gradient products of the tile have completed
   uint64_t drain;
   uint32_t tmem_base;
@@ -120,6 +125,19 @@ __device__ __forceinline__ void mma_grad(uint32_t d_tmem, uint32_t a_tmem, uint3
     mma_bf16_ts(d_tmem, a, sw128_desc(b + kk * 2048, 16384, 1024), BwdCfg<D>::IDESC_G,
                 (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+// D += A_h B_h over query half h of a tile (dK/dV kernel): A_h = 128 x 64 bf16 in
+// tensor memory, its K = 64 query columns packed in pairs at a_tmem + [0, 16)
+// (queries [0, 32) of the half) and a_tmem + [32, 48) (queries [32, 64)); B_h =
+// rows [64 h, 64 h + 64) of a 128 x D tile in shared memory read as an MN-major
+// operand (b_half = B + 8192 h).
+template <int D>
+__device__ __forceinline__ void mma_grad_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_half, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    mma_bf16_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1), sw128_desc(b_half + kk * 2048, 16384, 1024),
+                BwdCfg<D>::IDESC_G, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // p = 2^(s * c - l) for the 32 values of a row chunk, 0 from column `valid` on;
@@ -427,8 +445,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     float* __restrict__ dv, int N, int heads, int nb, int npad, int mask_per_bh, float scale,
                     float scale_log2, uint32_t* status, uint64_t limit_ns) {
   using C = BwdCfg<D>;
-  // S^T [0,128) (P^T as bf16 over its columns [0,32) and [64,96), one range per
-  // column half), dP^T [128,256) (dS^T likewise), dV [256,256+D), dK [384,384+D)
+  // S^T [0,128), dP^T [128,256), dV [256,256+D), dK [384,384+D).  Each row warp
+  // owns 32 query columns of each query half (columns [64 h + 32 e, + 32) of S^T
+  // and dP^T, e = (warp - 2) / 4) and writes P^T and dS^T of those queries as
+  // bf16 pairs over the S^T columns it has read: P^T at [64 h + 32 e, + 16),
+  // dS^T at [64 h + 32 e + 16, + 16).
   constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 384;
   extern __shared__ uint8_t bwd_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -446,8 +467,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sh->fixed_full, 1);
     mbar_init(&sh->ring_full[0], 1);
     mbar_init(&sh->ring_full[1], 1);
-    mbar_init(&sh->sdp_full, 1);
-    mbar_init(&sh->ds_full, 8);
+    mbar_init(&sh->s_full, 1);
+    mbar_init(&sh->dp_full, 1);
+    mbar_init(&sh->dp_read, 8);
+    mbar_init(&sh->ds_h[0], 8);
+    mbar_init(&sh->ds_h[1], 8);
+    mbar_init(&sh->grads_done, 1);
     mbar_init(&sh->mm_done, 1);
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
@@ -495,30 +520,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
           const uint32_t qs = sbase + C::OFF_RING;
           mma_xyt<D>(tmem + TM_S, k_s, qs);
+          mma_commit(&sh->s_full);
           mma_xyt<D>(tmem + TM_DP, v_s, qs + C::TILE);
-          mma_commit(&sh->sdp_full);
+          mma_commit(&sh->dp_full);
         }
       }
+      // Per tile: dP^T_{j+1} as soon as the row warps hold dP^T_j in registers;
+      // the gradient products of query half 0 while they form half 1; then those
+      // of half 1 and S^T_{j+1}, which overwrites the P^T / dS^T they read (the
+      // tensor cores run them in issue order).
       for (int j = 0; ok && j < n; ++j) {
-        const int s = j & 1;
-        if (sh->abort_flag || !mbar_wait(&sh->ds_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qs = sbase + C::OFF_RING + s * 2 * C::TILE;
-        mma_grad<D>(tmem + TM_DV, tmem + TM_S, qs + C::TILE, j > 0, true);  // dV += P^T dO
-        mma_grad<D>(tmem + TM_DK, tmem + TM_DP, qs, j > 0, true);          // dK += dS^T Q
-        mma_commit(&sh->mm_done);
+        const uint32_t qs = sbase + C::OFF_RING + (j & 1) * 2 * C::TILE;
+        const uint32_t qn = sbase + C::OFF_RING + ((j + 1) & 1) * 2 * C::TILE;
         if (j + 1 < n) {
-          // S^T and dP^T of the next tile overwrite P^T and dS^T: issued after
-          // the products that read them, which the tensor cores run in order
-          const int s1 = (j + 1) & 1;
-          if (!mbar_wait(&sh->ring_full[s1], (uint32_t)(((j + 1) >> 1) & 1), limit_ns)) { ok = false; break; }
+          if (sh->abort_flag || !mbar_wait(&sh->dp_read, (uint32_t)(j & 1), limit_ns) ||
+              !mbar_wait(&sh->ring_full[(j + 1) & 1], (uint32_t)(((j + 1) >> 1) & 1), limit_ns)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t qn = sbase + C::OFF_RING + s1 * 2 * C::TILE;
-          mma_xyt<D>(tmem + TM_S, k_s, qn);
           mma_xyt<D>(tmem + TM_DP, v_s, qn + C::TILE);
-          mma_commit(&sh->sdp_full);
+          mma_commit(&sh->dp_full);
+        }
+        for (int ph = 0; ph < 2; ++ph) {
+          if (sh->abort_flag || !mbar_wait(&sh->ds_h[ph], (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+          tc_fence_after();
+          const bool acc = j > 0 || ph > 0;
+          mma_grad_half<D>(tmem + TM_DV, tmem + TM_S + 64 * ph, qs + C::TILE + ph * 8192, acc);  // dV += P^T dO
+          mma_grad_half<D>(tmem + TM_DK, tmem + TM_S + 64 * ph + 16, qs + ph * 8192, acc);       // dK += dS^T Q
+        }
+        if (!ok) break;
+        mma_commit(j + 1 < n ? &sh->mm_done : &sh->grads_done);
+        if (j + 1 < n) {
+          mma_xyt<D>(tmem + TM_S, k_s, qn);
+          mma_commit(&sh->s_full);
         }
         if (j + 2 < n) {
+          // the stage of tile j is free once its gradient products have read it
           if (!mbar_wait(&sh->mm_done, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
           load_q(j + 2);
         }
@@ -534,34 +572,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------------- one thread per key row
-    // and column half: query rows [64 half, 64 half + 64) of each query tile
+    // and 32 query columns of each query half: [64 ph + 32 half, + 32)
     const int quarter = warp & 3, r = quarter * 32 + lane, half = (warp - 2) >> 2;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int s = j & 1;
-      if (!mbar_wait_warp(&sh->sdp_full, (uint32_t)(j & 1), limit_ns)) { ok = false; break; }
+      if (!mbar_wait_warp(&sh->s_full, (uint32_t)(j & 1), limit_ns) ||
+          !mbar_wait_warp(&sh->dp_full, (uint32_t)(j & 1), limit_ns)) {
+        ok = false;
+        break;
+      }
       // the row vectors of this query tile landed with its tiles (ring_full of stage s)
       if (!mbar_wait_warp(&sh->ring_full[s], (uint32_t)((j >> 1) & 1), limit_ns)) { ok = false; break; }
       tc_fence_after();
       const float* l2v = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * C::VEC);
       const float* dvv = l2v + 128;
-      uint32_t sr2[2][32], pr2[2][32];  // this half's chunks of S^T and dP^T, one wait
+      uint32_t sr2[2][32], pr2[2][32];  // this thread's chunks of S^T and dP^T, one wait
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        tmem_ld32(lane_addr + TM_S + (2 * half + cc) * 32, sr2[cc]);
-        tmem_ld32(lane_addr + TM_DP + (2 * half + cc) * 32, pr2[cc]);
+      for (int ph = 0; ph < 2; ++ph) {
+        tmem_ld32(lane_addr + TM_S + 64 * ph + 32 * half, sr2[ph]);
+        tmem_ld32(lane_addr + TM_DP + 64 * ph + 32 * half, pr2[ph]);
       }
       tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->dp_read);  // dP^T_j is in registers: its columns are free
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * half + cc;
-        const uint32_t(&sr)[32] = sr2[cc];
-        const uint32_t(&pr)[32] = pr2[cc];
+      for (int ph = 0; ph < 2; ++ph) {
+        const uint32_t(&sr)[32] = sr2[ph];
+        const uint32_t(&pr)[32] = pr2[ph];
         uint32_t pp[16], dsp[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int q0 = c * 32 + 2 * i;
+          const int q0 = 64 * ph + 32 * half + 2 * i;
           const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
                                        f32x2_pack(scale_log2, scale_log2), f32x2_pack(-l2v[q0], -l2v[q0 + 1]));
           float p0, p1;
@@ -577,17 +621,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dsp[i] = pack_bf16x2(p0 * (__uint_as_float(pr[2 * i]) - dvv[q0]),
                                p1 * (__uint_as_float(pr[2 * i + 1]) - dvv[q0 + 1]));
         }
-        // this half's packed columns, inside the range it has already read:
-        // [64 half + 16 cc, + 16) of each region
-        tmem_st16(lane_addr + TM_S + 64 * half + 16 * cc, pp);
-        tmem_st16(lane_addr + TM_DP + 64 * half + 16 * cc, dsp);
+        tmem_st16(lane_addr + TM_S + 64 * ph + 32 * half, pp);
+        tmem_st16(lane_addr + TM_S + 64 * ph + 32 * half + 16, dsp);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->ds_h[ph]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->ds_full);
     }
-    if (ok && n >= 1) ok = mbar_wait_warp(&sh->mm_done, (uint32_t)((n - 1) & 1), limit_ns);
+    if (ok && n >= 1) ok = mbar_wait_warp(&sh->grads_done, 0, limit_ns);
     if (!ok) {
       bwd_timeout(sh, status);
     } else {
