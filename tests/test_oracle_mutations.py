@@ -17,6 +17,7 @@ FWD = ["tests/test_oracle_forward.py"]
 GATE = ["tests/test_oracle_gate.py"]
 BWD = ["tests/test_oracle_backward.py"]
 TILE = ["tests/test_oracle_tiles.py"]
+TOPK = ["tests/test_oracle_topk.py"]
 
 # (name, text in the source, replacement, occurrences replaced, pin files)
 MUTANTS = [
@@ -42,6 +43,18 @@ MUTANTS = [
     ("tiles: y window one short", "llabs(y - y2) <= wh && llabs(x - x2) <= ww",
      "llabs(y - y2) < wh && llabs(x - x2) <= ww", 1, TILE),
     ("tiles: boxes numbered column-major", "xi = (int)(I % nw);", "xi = (int)((I / nh) % nw);", 1, TILE),
+    ("topk: keeps the lowest scores", "if (x->score > y->score) return -1;\n    if (x->score < y->score) return 1;",
+     "if (x->score < y->score) return -1;\n    if (x->score > y->score) return 1;", 1, TOPK),
+    ("topk: ties keep the larger block", "return (x->j > y->j) - (x->j < y->j);",
+     "return (x->j < y->j) - (x->j > y->j);", 1, TOPK),
+    # (on the key side: the query mean of a row scales all of that row's scores
+    # alike, so the same mistake there leaves the ranking unchanged)
+    ("topk: partial key block averaged over the block size", "km[(int64_t)I * d + c] = sk / (float)(t1 - t0);",
+     "km[(int64_t)I * d + c] = sk / (float)blk;", 1, TOPK),
+    ("lse: running maximum left out", "l > 0.0 ? m + log(l) : -INFINITY;", "l > 0.0 ? log(l) : -INFINITY;", 1, BWD),
+    ("backward: relu derivative dropped in dq", "if (!(qi[c] > 0.0)) continue;", "if (0) continue;", 1, BWD),
+    ("backward: dk without the relu mask", "if (kj[c] > 0.0) {", "if (1) {", 1, BWD),
+    ("backward: dz left out of dk", "double t = dzb[c];", "double t = 0.0;", 1, BWD),
 ]
 
 
