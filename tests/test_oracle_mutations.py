@@ -30,6 +30,12 @@ MUTANTS = [
     ("forward: eps dropped", "lin[e] = u / (dn + eps);", "lin[e] = u / dn;", 1, FWD),
     ("forward: W transposed", "y += lin[c] * W[c * d + e];", "y += lin[c] * W[e * d + c];", 1, FWD),
     ("forward: gate dropped", "out[ooff + e] = acc[e] + g * y;", "out[ooff + e] = acc[e] + y;", 1, FWD),
+    ("forward: relu of k dropped in the state", "pk[c] = kv > 0.0 ? kv : 0.0;", "pk[c] = kv;", 1, FWD),
+    ("forward: relu of q dropped", "const double pq = qi[c] > 0.0 ? qi[c] : 0.0;", "const double pq = qi[c];", 2, FWD),
+    ("forward: softmax not normalised", "acc[c] /= den;", "acc[c] /= 1.0;", 1, FWD),
+    ("forward: last kept block of a row skipped",
+     "for (int32_t r = r0; r < r1; ++r) {\n            block_tokens(geom, N, blk, col_idx[r], slot_tok);",
+     "for (int32_t r = r0; r < r1 - 1; ++r) {\n            block_tokens(geom, N, blk, col_idx[r], slot_tok);", 1, FWD),
     ("gate: sum for mean", "logit += w_x[(size_t)h * d + f] * (sum / N);",
      "logit += w_x[(size_t)h * d + f] * sum;", 1, GATE),
     ("gate: sigmoid sign", "1.0 / (1.0 + exp(-logit))", "1.0 / (1.0 + exp(logit))", 1, GATE),
