@@ -270,7 +270,7 @@ int salad_attn_backward_sparse(const void* q, const void* k, const void* v, cons
  * (g / den_i) dout_i over the rows, dS = M W^T and dW = sum over (b, h) of S^T M;
  * every operand that is not already bf16 (T, (g / den_i) dout_i, dS) enters as
  * bf16 hi + lo halves, accumulation is fp32 and every sum runs in a fixed order
- * (deterministic).  The workspace is O(B Hh (N + d^2)), about 30 MB for
+ * (deterministic).  The workspace is O(B Hh (N + d^2)), about 40 MB for
  * 32,760 tokens x 12 heads of d = 128.  Errors: INVALID_ARG, UNSUPPORTED (d,
  * block != 128, B*Hh > 65535), WORKSPACE, CUDA; a stalled wait sets the status
  * word's time-out bit (salad_check_status).
